@@ -1,0 +1,383 @@
+"""Pins of the CPU oracle against facts the pages and the mathematics fix.
+
+Each test ties one oracle function to something other than the oracle itself:
+numbers printed on the pages (tests/golden/, each file carries its citation),
+closed forms, convexity, a numerical derivative, brute force over all subsets,
+or hand-derived routing outcomes. No GPU is involved.
+"""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle as O
+
+
+def _load(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------------------
+# Scaled dot-product attention: the pages' worked examples
+# ---------------------------------------------------------------------------
+
+def test_sdpa_three_token_example(golden_dir):
+    g = _load(golden_dir, "attention_3token.json")
+    half = 0.5 * 10 ** -g["decimals"] + 1e-12
+    A, Out = O.sdpa(np.array(g["Q"]), np.array(g["K"]), np.array(g["V"]))
+    S = np.array(g["Q"]) @ np.array(g["K"]).T / math.sqrt(2)
+    assert np.max(np.abs(S - np.array(g["S_scaled"]))) <= half
+    assert np.max(np.abs(A - np.array(g["A"]))) <= half
+    assert np.max(np.abs(Out - np.array(g["O"]))) <= half
+
+
+def test_sdpa_causal_example(golden_dir):
+    g = _load(golden_dir, "attention_causal.json")
+    half = 0.5 * 10 ** -g["decimals"] + 1e-12
+    mask = np.tril(np.ones((3, 3), bool))
+    A, Out = O.sdpa(np.array(g["Q"]), np.array(g["K"]), np.array(g["V"]), mask)
+    assert np.max(np.abs(A[1, :2] - np.array(g["A_row2_visible"]))) <= half
+    assert A[0, 0] == 1.0 and A[1, 2] == 0.0
+    assert np.max(np.abs(Out - np.array(g["O_causal"]))) <= half
+
+
+def test_attend_over_token_sets_reproduces_examples(golden_dir):
+    """attend() over S = all tokens gives O; over S = prefix {0..i} gives O_causal."""
+    g = _load(golden_dir, "attention_3token.json")
+    c = _load(golden_dir, "attention_causal.json")
+    half = 0.5e-3 + 1e-12
+    K, V = np.array(g["K"], float), np.array(g["V"], float)
+    for i, q in enumerate(np.array(g["Q"], float)):
+        o, lse = O.attend(q, K, V, np.arange(3))
+        assert np.max(np.abs(o - np.array(g["O"][i]))) <= half
+        s = K @ q / math.sqrt(2)
+        assert abs(lse - math.log(np.exp(s).sum())) < 1e-12
+        o_c, _ = O.attend(q, K, V, np.arange(i + 1))
+        assert np.max(np.abs(o_c - np.array(c["O_causal"][i]))) <= half
+
+
+def test_softmax_saturation_through_attend(golden_dir):
+    """The softmax weights printed for scores [1,0,-1] and [11.3,0,-11.3]: feed
+    keys that produce those scaled scores and one-hot values, so o = weights."""
+    g = _load(golden_dir, "softmax_saturation.json")
+    d = 4
+    for case in g["cases"]:
+        scores = np.array(case["scores"])
+        q = np.zeros(d); q[0] = math.sqrt(d)          # q.k/sqrt(d) = k[0]
+        K = np.zeros((3, d)); K[:, 0] = scores
+        V = np.eye(d)[:3]
+        o, _ = O.attend(q, K, V, np.arange(3))
+        w = np.array(case["weights"])
+        tol = case["abs_tol"]
+        assert np.max(np.abs(o[:2] - w[:2])) <= tol
+        assert abs(o[2] - w[2]) <= case.get("abs_tol_last", tol)
+        assert o[3] == 0.0
+
+
+# ---------------------------------------------------------------------------
+# The combine identity: the online-softmax table
+# ---------------------------------------------------------------------------
+
+def test_combine_reproduces_online_softmax_table(golden_dir):
+    g = _load(golden_dir, "online_softmax_table.json")
+    half = 0.5e-3 + 1e-12
+    Q = np.array([[1, 0], [0, 1], [1, 1]], float)
+    V = np.array([[1, 0], [0, 2], [3, 3]], float)
+    q = np.array(g["query"], float)
+    s = Q @ q / math.sqrt(2)                       # K = Q in the example
+    assert np.max(np.abs(s - np.array(g["scaled_scores"]))) <= half
+    # block 1 on its own: log mass m + log l, normalised output o / l
+    b1 = g["blocks"][0]
+    F1, avg1 = O.combine_log_masses(s[b1], V[b1])
+    a1 = g["after_block1"]
+    assert abs(F1 - (a1["m"] + math.log(a1["l"]))) <= half * 2
+    assert np.max(np.abs(avg1 - np.array(a1["o"]) / a1["l"])) <= half
+    # block 2 is one token: its log mass is its score, its state its value
+    b2 = g["blocks"][1]
+    F2, avg2 = O.combine_log_masses(s[b2], V[b2])
+    # combine the two block states: this is the table's second row
+    F, avg = O.combine_log_masses(np.array([F1, F2]), np.stack([avg1, avg2]))
+    a2 = g["after_block2"]
+    assert abs(math.exp(a1["m"] - a2["m"]) - g["rescale_factor"]) <= half
+    assert abs(F - (a2["m"] + math.log(a2["l"]))) <= 2 * half
+    assert np.max(np.abs(avg - np.array(a2["o"]) / a2["l"])) <= half
+    assert np.max(np.abs(avg - np.array(g["final"]))) <= half
+
+
+def test_merge_of_unequal_children_matches_worked_example(golden_dir):
+    """Summaries of {tok1, tok2} and {tok3} at q_r = token 3's query, merged by
+    the tree's rule, give the page's numbers: F = m + log l from the online-softmax
+    table, and khat = (row 3 of A) applied to K."""
+    g = _load(golden_dir, "attention_3token.json")
+    t = _load(golden_dir, "online_softmax_table.json")
+    K = np.array(g["K"], float)
+    qhat = np.array([[1.0, 1.0]])
+    kh_a, bh_a = O.summarise_chunk(qhat, K[:2])
+    kh_b, bh_b = O.summarise_chunk(qhat, K[2:])
+    kh, bh = O.merge_children(qhat, np.stack([kh_a, kh_b]), np.stack([bh_a, bh_b]))
+    F = bh[0] + qhat[0] @ kh[0] / math.sqrt(2)
+    a2 = t["after_block2"]
+    assert abs(F - (a2["m"] + math.log(a2["l"]))) <= 2e-3
+    A3 = np.array(g["A"][2])
+    assert np.max(np.abs(kh[0] - A3 @ K)) <= 2e-3
+    # and it equals the direct summary of all three keys
+    kd, bd = O.summarise_chunk(qhat, K)
+    assert np.allclose(kh, kd, rtol=0, atol=1e-14) and np.allclose(bh, bd, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# Tangent-plane summaries: closed forms, convexity, gradient
+# ---------------------------------------------------------------------------
+
+def _rand_chunk(rng, C=16, d=8, R=5, scale=1.0):
+    Kc = rng.standard_normal((C, d)) * scale
+    qhat = rng.standard_normal((R, d)) * math.sqrt(d)
+    return qhat, Kc
+
+
+def test_summary_of_identical_keys_is_that_key_and_log_C():
+    rng = np.random.default_rng(1)
+    d, C, R = 6, 7, 3                    # C != R so an axis mix-up shows
+    k = rng.standard_normal(d)
+    qhat = rng.standard_normal((R, d)) * 3
+    kh, bh = O.summarise_chunk(qhat, np.tile(k, (C, 1)))
+    assert np.allclose(kh, np.tile(k, (R, 1)), atol=1e-13)
+    assert np.allclose(bh, math.log(C), atol=1e-13)
+
+
+def test_summary_of_a_single_key():
+    rng = np.random.default_rng(2)
+    qhat, Kc = _rand_chunk(rng, C=1, d=5, R=4)
+    kh, bh = O.summarise_chunk(qhat, Kc)
+    assert np.allclose(kh, np.tile(Kc[0], (4, 1)), atol=1e-14)
+    assert np.allclose(bh, 0.0, atol=1e-13)
+
+
+def test_tangent_is_exact_at_its_reference_query():
+    rng = np.random.default_rng(3)
+    qhat, Kc = _rand_chunk(rng, C=32, d=16, R=6, scale=2.0)
+    kh, bh = O.summarise_chunk(qhat, Kc)
+    for r in range(qhat.shape[0]):
+        t = O.tangent_planes(qhat[r], kh, bh)[r]
+        assert abs(t - O.chunk_log_mass(qhat[r], Kc)) < 1e-12
+
+
+def test_max_of_planes_is_a_lower_bound_of_the_log_mass():
+    """LSE is convex, so each tangent plane lies below F_C everywhere."""
+    rng = np.random.default_rng(4)
+    qhat, Kc = _rand_chunk(rng, C=24, d=12, R=8, scale=1.5)
+    kh, bh = O.summarise_chunk(qhat, Kc)
+    qs = rng.standard_normal((10_000, 12)) * 4.0
+    est = np.array([O.node_score(q, kh, bh) for q in qs])
+    true = O.chunk_log_mass(qs, Kc)
+    assert np.all(est <= true + 1e-12)
+    assert np.mean(true - est) > 1e-3     # and not trivially equal
+
+
+def test_node_score_is_exact_at_every_reference_query():
+    """At q = q_r plane r touches F_C and every other plane lies below it, so the
+    max-of-planes estimate equals the true log mass there (and no less)."""
+    rng = np.random.default_rng(7)
+    qhat, Kc = _rand_chunk(rng, C=16, d=8, R=6, scale=2.0)
+    kh, bh = O.summarise_chunk(qhat, Kc)
+    for r in range(6):
+        assert abs(O.node_score(qhat[r], kh, bh) - O.chunk_log_mass(qhat[r], Kc)) < 1e-12
+    planes = O.tangent_planes(qhat[0], kh, bh)
+    assert np.min(planes) < np.max(planes) - 1e-3
+
+
+def test_compressed_key_is_the_gradient_of_the_log_mass():
+    """d F_C / d q at q_r equals khat_r / sqrt(d) (central differences)."""
+    rng = np.random.default_rng(5)
+    qhat, Kc = _rand_chunk(rng, C=20, d=10, R=4)
+    kh, _ = O.summarise_chunk(qhat, Kc)
+    h = 1e-5
+    for r in range(4):
+        grad = np.zeros(10)
+        for i in range(10):
+            e = np.zeros(10); e[i] = h
+            grad[i] = (O.chunk_log_mass(qhat[r] + e, Kc) - O.chunk_log_mass(qhat[r] - e, Kc)) / (2 * h)
+        assert np.allclose(grad, kh[r] / math.sqrt(10), rtol=1e-6, atol=1e-8)
+
+
+def test_chunk_log_mass_against_a_plain_loop():
+    rng = np.random.default_rng(6)
+    q = rng.standard_normal(9)
+    Kc = rng.standard_normal((11, 9)) * 2
+    total = 0.0
+    for j in range(11):
+        total += math.exp(sum(q[i] * Kc[j, i] for i in range(9)) / 3.0)
+    assert abs(O.chunk_log_mass(q, Kc) - math.log(total)) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# Upper levels: merge == direct summary of the raw keys
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("C,L,n_tokens", [(4, 3, 64), (4, 3, 93), (3, 4, 200), (2, 1, 9)])
+def test_every_level_equals_the_direct_summary(C, L, n_tokens):
+    rng = np.random.default_rng(10 + C + L)
+    d, R = 8, 5
+    K = rng.standard_normal((n_tokens, d)) * 1.5 + rng.standard_normal(d)
+    qhat = rng.standard_normal((R, d)) * 2
+    tree = O.build_tree(K, qhat, C, L, n_tokens)
+    for lvl in range(1, L + 1):
+        span = C ** lvl
+        kh, bh = tree.nodes[lvl]
+        assert kh.shape[0] == (C * (n_tokens // C)) // span == tree.n_nodes(lvl)
+        for i in range(kh.shape[0]):
+            kd, bd = O.summarise_chunk(qhat, K[i * span:(i + 1) * span])
+            assert np.allclose(kh[i], kd, rtol=1e-10, atol=1e-12)
+            assert np.allclose(bh[i], bd, rtol=1e-10, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Top-p selection: brute force, special cases, tie rule
+# ---------------------------------------------------------------------------
+
+def test_top_p_is_the_minimal_subset_by_brute_force():
+    rng = np.random.default_rng(20)
+    for trial in range(300):
+        n = int(rng.integers(1, 11))
+        sigma = rng.standard_normal(n) * rng.uniform(0.1, 4)
+        ids = rng.permutation(50)[:n]
+        p = float(rng.uniform(0.05, 0.999))
+        sel = O.top_p_prefix(sigma, ids, p)
+        pi = np.exp(sigma - sigma.max()); pi /= pi.sum()
+        # smallest cardinality of ANY subset whose mass reaches p
+        best = None
+        for k in range(1, n + 1):
+            if any(sum(pi[list(c)]) >= p for c in itertools.combinations(range(n), k)):
+                best = k
+                break
+        assert sel.m == best, (trial, sel.m, best)
+        # the kept set is the top-m by score and reaches p
+        kept_pos = [int(np.nonzero(ids == k)[0][0]) for k in sel.kept]
+        assert pi[kept_pos].sum() >= p - 1e-15
+        if sel.m < n:
+            assert min(sigma[kept_pos]) >= max(np.delete(sigma, kept_pos))
+
+
+def test_top_p_special_cases():
+    ids = np.arange(4)
+    assert O.top_p_prefix(np.array([0.3, -1.0, 2.0, 0.0]), ids, 1.0).m == 4
+    assert O.top_p_prefix(np.array([0.3, -1.0, 2.0, 0.0]), ids, 1.5).m == 4
+    one = O.top_p_prefix(np.array([0.0, 30.0, 0.0, 0.0]), ids, 0.99)
+    assert one.m == 1 and list(one.kept) == [1]
+    flat = O.top_p_prefix(np.zeros(4), np.array([7, 3, 9, 5]), 0.5)
+    assert flat.m == 2 and list(flat.kept) == [3, 5]      # ties: lower index first
+    flat = O.top_p_prefix(np.zeros(4), np.array([7, 3, 9, 5]), 0.51)
+    assert flat.m == 3 and list(flat.kept) == [3, 5, 7]
+    assert O.top_p_prefix(np.zeros(0), np.zeros(0, int), 0.9).m == 0
+
+
+# ---------------------------------------------------------------------------
+# Routing: hand-built trees, invariants, p = 1 equals dense attention
+# ---------------------------------------------------------------------------
+
+def test_route_follows_a_single_strong_key_by_hand():
+    """C=2, L=2, N=11: level-1 nodes 0..4 (tokens 0..9), level-2 nodes 0..1
+    (tokens 0..3, 4..7), level-1 node 4 is an orphan, token 10 is the tail.
+    One strong key at token 5: the route keeps level-2 node 1, then level-1
+    node 2, so S = {0} u {4, 5} u {10}."""
+    d = 2
+    K = np.zeros((11, d)); K[5] = [3.0, 0.0]
+    tree = O.build_tree(K, np.array([[1.0, 0.0]]), chunk=2, levels=2, n_tokens=11)
+    tr = O.route(np.array([10.0, 0.0]), tree, p=0.9)
+    assert list(tr.levels[2].candidates) == [0, 1]
+    assert list(tr.levels[2].topp.kept) == [1]
+    assert list(tr.levels[1].candidates) == [2, 3, 4]          # children of 1 + orphan 4
+    assert list(tr.levels[1].topp.kept) == [2]
+    assert list(tr.tokens) == [0, 4, 5, 10]
+
+
+def test_route_on_flat_keys_breaks_ties_by_index_by_hand():
+    """All keys zero: every node's score is log(tokens under it). Level 2: two
+    equal nodes, p=0.5 keeps node 0. Level 1: children {0,1} + orphan {4}, each
+    of mass 1/3; p=0.5 keeps {0,1}. S = {0,1,2,3} u {10}."""
+    K = np.zeros((11, 2))
+    tree = O.build_tree(K, np.array([[1.0, 0.0], [0.0, 1.0]]), 2, 2, 11)
+    tr = O.route(np.array([1.0, -2.0]), tree, p=0.5)
+    assert np.allclose(tr.levels[2].sigma, math.log(4))
+    assert list(tr.levels[2].topp.kept) == [0]
+    assert list(tr.levels[1].candidates) == [0, 1, 4]
+    assert list(tr.levels[1].topp.kept) == [0, 1]
+    assert list(tr.tokens) == [0, 1, 2, 3, 10]
+
+
+def _random_tree(seed, n_tokens=1000, C=4, L=3, d=8, R=4):
+    rng = np.random.default_rng(seed)
+    K = rng.standard_normal((n_tokens, d)) * 1.3
+    V = rng.standard_normal((n_tokens, d))
+    qhat = rng.standard_normal((R, d)) * 2
+    return rng, K, V, O.build_tree(K, qhat, C, L, n_tokens)
+
+
+@pytest.mark.parametrize("n_tokens", [1000, 1027, 64, 63, 3, 1])
+def test_route_set_invariants(n_tokens):
+    rng, K, V, tree = _random_tree(30 + n_tokens, n_tokens=n_tokens)
+    C, L = tree.chunk, tree.levels
+    for _ in range(20):
+        q = rng.standard_normal(8) * 3
+        tr = O.route(q, tree, p=float(rng.uniform(0.3, 0.95)))
+        S = set(tr.tokens.tolist())
+        assert 0 in S
+        assert set(range(tree.n_built, n_tokens)) <= S
+        assert max(S) < n_tokens
+        for lvl in range(1, L + 1):
+            lt = tr.levels[lvl]
+            kept = set(lt.topp.kept.tolist())
+            assert kept <= set(lt.candidates.tolist())
+            n_par = tree.n_nodes(lvl + 1)
+            for i in kept:
+                parent = i // C
+                if parent < n_par:
+                    assert parent in set(tr.levels[lvl + 1].topp.kept.tolist())
+            # candidates: every node whose parent was kept, and every orphan
+            expect = [i for i in range(tree.n_nodes(lvl))
+                      if i // C >= n_par or (lvl < L and i // C in set(tr.levels[lvl + 1].expanded.tolist()))]
+            assert sorted(lt.candidates.tolist()) == expect
+        # S is exactly sink + tail + tokens of kept chunks
+        expect_S = {0} | set(range(tree.n_built, n_tokens))
+        for c in tr.leaf_chunks:
+            expect_S |= set(range(c * C, (c + 1) * C))
+        assert S == expect_S
+
+
+@pytest.mark.parametrize("n_tokens", [1000, 1027, 70, 5])
+def test_route_at_p1_equals_dense_attention(n_tokens):
+    rng, K, V, tree = _random_tree(50 + n_tokens, n_tokens=n_tokens)
+    for _ in range(5):
+        q = rng.standard_normal(8) * 3
+        tr = O.route(q, tree, p=1.0)
+        assert list(tr.tokens) == list(range(n_tokens))
+        o, lse = O.attend(q, K, V, tr.tokens)
+        _, dense = O.sdpa(q[None], K[:n_tokens], V[:n_tokens])
+        assert np.max(np.abs(o - dense[0])) < 1e-12
+
+
+def test_forced_expansion_uses_the_given_kept_set():
+    rng, K, V, tree = _random_tree(70, n_tokens=1000)
+    q = rng.standard_normal(8) * 3
+    forced = {3: np.array([1, 2])}
+    tr = O.route(q, tree, p=0.6, forced_kept=forced)
+    C = tree.chunk
+    n2 = tree.n_nodes(2)
+    expect = sorted([c for k in (1, 2) for c in range(k * C, k * C + C)] +
+                    list(range(C * tree.n_nodes(3), n2)))
+    assert sorted(tr.levels[2].candidates.tolist()) == expect
+
+
+def test_bf16_decode_is_exact():
+    vals = np.array([1.0, -2.5, 0.15625, 3.0e38, -1.0e-38, 0.0], np.float32)
+    bits = (vals.view(np.uint32) >> 16).astype(np.uint16)     # these values are bf16-exact
+    assert np.array_equal(O.bf16_bits_to_f64(bits), vals.astype(np.float64)) or \
+        np.allclose(O.bf16_bits_to_f64(bits), vals.astype(np.float64), rtol=2 ** -8)
+    assert O.bf16_bits_to_f64(np.array([0x3F80], np.uint16))[0] == 1.0
+    assert O.bf16_bits_to_f64(np.array([0xC020], np.uint16))[0] == -2.5
+    assert O.bf16_bits_to_f64(np.array([0x0000], np.uint16))[0] == 0.0
