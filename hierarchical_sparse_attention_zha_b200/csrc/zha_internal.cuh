@@ -1,0 +1,179 @@
+// zha_internal.cuh -- geometry, layouts and device helpers shared by the
+// kernels and the C-ABI host code of libzha (not part of the public ABI).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "zha.h"
+
+#define ZHA_MAX_LEVELS 8
+#define ZHA_MAX_REF 32
+#define ZHA_MAX_CHUNK 128
+
+namespace zha {
+
+// ---------------------------------------------------------------------------
+// Geometry of one tree configuration, passed by value to kernels.
+// ---------------------------------------------------------------------------
+struct Geom {
+  int32_t hkv, hq, group, d, chunk, levels, nref, node_floats;
+  int32_t kv_bf16;
+  float scale;                           // 1 / sqrt(d)
+  int64_t max_tokens;
+  int64_t cap[ZHA_MAX_LEVELS + 2];       // node capacity per KV head, index by level
+  int64_t off[ZHA_MAX_LEVELS + 2];       // float offset of level l's [hkv][cap][node] block
+};
+
+// C^l, saturating at a value above any token count.
+__host__ __device__ inline int64_t span_of(int32_t chunk, int32_t level) {
+  int64_t s = 1;
+  for (int i = 0; i < level; ++i) {
+    if (s > (int64_t(1) << 40)) return int64_t(1) << 50;
+    s *= chunk;
+  }
+  return s;
+}
+
+// Nodes of level l that exist when N_b tokens are covered by complete chunks.
+__host__ __device__ inline int64_t nodes_at(int64_t nb, int32_t chunk, int32_t level) {
+  return nb / span_of(chunk, level);
+}
+
+__host__ __device__ inline int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+__host__ __device__ inline int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ inline int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+// ---------------------------------------------------------------------------
+// Route workspace layout: per level, sigma [B][Hq][n_l] float and (unless the
+// caller passes its own buffer) kept bitmaps [B][Hq][W_l] uint32, plus the
+// compacted kept parents [B][Hq][n_max] int32 used to enumerate candidates.
+// ---------------------------------------------------------------------------
+struct RouteLayout {
+  int64_t n[ZHA_MAX_LEVELS + 2];         // nodes per level at n_tokens
+  int64_t words[ZHA_MAX_LEVELS + 2];     // bitmap words per head per level
+  int64_t sig_off[ZHA_MAX_LEVELS + 2];   // float offsets into sigma region
+  int64_t bits_off[ZHA_MAX_LEVELS + 2];  // word offsets into the bitmap region
+  int64_t sig_floats, bits_words, kp_ints;
+  int64_t bytes;                          // total workspace (bitmaps included)
+  int64_t bytes_no_bits;                  // when the caller supplies the bitmaps
+};
+
+inline RouteLayout route_layout(const Geom& g, int32_t batch, int64_t n_tokens) {
+  RouteLayout r{};
+  const int64_t nb = int64_t(g.chunk) * (n_tokens / g.chunk);
+  const int64_t heads = int64_t(batch) * g.hq;
+  int64_t sig = 0, bits = 0, nmax = 0;
+  for (int l = 1; l <= g.levels; ++l) {
+    r.n[l] = nodes_at(nb, g.chunk, l);
+    r.words[l] = (r.n[l] + 31) / 32;
+    r.sig_off[l] = sig;
+    r.bits_off[l] = bits;
+    sig += round_up(heads * r.n[l], 64);
+    bits += heads * r.words[l];
+    if (l >= 2 && r.n[l] > nmax) nmax = r.n[l];
+  }
+  r.sig_floats = sig;
+  r.bits_words = bits;
+  r.kp_ints = round_up(heads * (nmax > 0 ? nmax : 1), 64);
+  r.bytes_no_bits = round_up(sig * 4, 256) + round_up(r.kp_ints * 4, 256);
+  r.bytes = r.bytes_no_bits + round_up(bits * 4, 256);
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// Attend workspace: one partial state per (query head, range of W chunks) plus
+// one for the sink-and-tail pass; each slot is [m, l, 0, 0, o[d]] floats.
+// ---------------------------------------------------------------------------
+constexpr int kAttendRangeTokens = 1024;
+
+inline int32_t attend_range_chunks(int32_t chunk) {
+  int32_t w = kAttendRangeTokens / chunk;
+  return w < 1 ? 1 : w;
+}
+
+struct AttendLayout {
+  int64_t n_chunks, n_ranges, slots_per_head, slot_floats, bytes;
+  int32_t range_chunks;
+};
+
+inline AttendLayout attend_layout(const Geom& g, int32_t batch, int64_t n_tokens) {
+  AttendLayout a{};
+  const int64_t nb = int64_t(g.chunk) * (n_tokens / g.chunk);
+  a.n_chunks = nb / g.chunk;
+  a.range_chunks = attend_range_chunks(g.chunk);
+  a.n_ranges = (a.n_chunks + a.range_chunks - 1) / a.range_chunks;
+  a.slots_per_head = a.n_ranges + 1;
+  a.slot_floats = g.d + 4;
+  a.bytes = round_up(int64_t(batch) * g.hq * a.slots_per_head * a.slot_floats * 4, 256);
+  return a;
+}
+
+// ---------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// EPL consecutive elements of a row, starting at element `e0`, widened to fp32.
+// The row start is 16-byte aligned; e0 is a multiple of EPL.
+template <int EPL>
+__device__ __forceinline__ void load_slice(const float* row, int e0, float (&out)[EPL]) {
+  if constexpr (EPL == 4) {
+    float4 v = *reinterpret_cast<const float4*>(row + e0);
+    out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+  } else if constexpr (EPL == 2) {
+    float2 v = *reinterpret_cast<const float2*>(row + e0);
+    out[0] = v.x; out[1] = v.y;
+  } else {
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) out[i] = row[e0 + i];
+  }
+}
+
+template <int EPL>
+__device__ __forceinline__ void load_slice(const __nv_bfloat16* row, int e0, float (&out)[EPL]) {
+  if constexpr (EPL == 8) {
+    uint4 v = *reinterpret_cast<const uint4*>(row + e0);
+    out[0] = __uint_as_float(v.x << 16); out[1] = __uint_as_float(v.x & 0xffff0000u);
+    out[2] = __uint_as_float(v.y << 16); out[3] = __uint_as_float(v.y & 0xffff0000u);
+    out[4] = __uint_as_float(v.z << 16); out[5] = __uint_as_float(v.z & 0xffff0000u);
+    out[6] = __uint_as_float(v.w << 16); out[7] = __uint_as_float(v.w & 0xffff0000u);
+  } else if constexpr (EPL == 4) {
+    uint2 v = *reinterpret_cast<const uint2*>(row + e0);
+    out[0] = __uint_as_float(v.x << 16); out[1] = __uint_as_float(v.x & 0xffff0000u);
+    out[2] = __uint_as_float(v.y << 16); out[3] = __uint_as_float(v.y & 0xffff0000u);
+  } else if constexpr (EPL == 2) {
+    uint32_t v = *reinterpret_cast<const uint32_t*>(row + e0);
+    out[0] = __uint_as_float(v << 16); out[1] = __uint_as_float(v & 0xffff0000u);
+  } else {
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) out[i] = __bfloat162float(row[e0 + i]);
+  }
+}
+
+// Monotone map float -> uint32 (ascending floats give ascending keys).
+__device__ __forceinline__ uint32_t float_order_key(float f) {
+  uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float order_key_float(uint32_t k) {
+  uint32_t u = (k & 0x80000000u) ? (k & 0x7fffffffu) : ~k;
+  return __uint_as_float(u);
+}
+
+}  // namespace zha
+
+// Launch bookkeeping shared by the host wrappers.
+void zha_count_launch();

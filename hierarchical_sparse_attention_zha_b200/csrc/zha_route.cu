@@ -1,0 +1,505 @@
+// zha_route.cu -- per-level top-p routing of decode queries through the trees.
+//
+// Citations: [ZHA: 무엇과 다른가 / 전제와 한계] = page "ZHA는 KV 캐시를 트리로 요약해
+// 어텐션 비용을 준(sub)이차로 낮춘다" (onedev.kr/papers/1556): a node's log mass for
+// a future query is estimated by the maximum of its R tangent planes (무엇과 다른가);
+// routing runs top-p per level -- sort the candidates by score, keep the minimal
+// prefix holding estimated mass p, pass the kept nodes' children and the
+// parentless chunks down (전제와 한계).
+//
+// Per level l = L..1 the host launches two kernels:
+//   score_kernel  -- one warp per candidate node (the union over the query heads
+//                    of a KV head), the node's R planes held in registers, one
+//                    score per query head that has the node as candidate;
+//   select_kernel -- one CTA per query head: softmax over its candidates, radix
+//                    select of the cut on the key (score desc, node index asc)
+//                    with fixed-point mass histograms, kept bitmap (and at
+//                    level 1 the ascending chunk list).
+#include "zha_internal.cuh"
+
+namespace zha {
+
+constexpr int kScoreThreads = 256;
+constexpr int kScoreTile = 32;       // nodes per score CTA
+constexpr int kScoreQBlock = 64;     // query heads per score CTA (u64 masks)
+constexpr int kSelectThreads = 512;
+constexpr int kSelectCache = 16384;  // candidate scores cached in shared memory
+constexpr double kMassScale = 1099511627776.0;  // 2^40: fixed-point unit of probability
+
+// ---------------------------------------------------------------------------
+// Scoring. A candidate of level l for query head (b, h) of KV head g is a node n
+// with n >= C * n_{l+1} (an orphan; every node at the top level) or whose parent
+// n / C is kept by (b, h) at level l+1. sigma = max_r (q . khat_r / sqrt(d) + bhat_r).
+// ---------------------------------------------------------------------------
+
+// v[RP] partial sums per lane -> lane L holds the full sum of value L >> (5 - log2 RP).
+template <int RP>
+__device__ __forceinline__ float transpose_reduce(float (&v)[RP]) {
+  const int lane = threadIdx.x & 31;
+  int count = RP;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    if (count > 1) {
+      const int half = count >> 1;
+      const bool upper = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < RP / 2; ++i) {
+        if (i < half) {
+          const float send = upper ? v[i] : v[i + half];
+          const float keep = upper ? v[i + half] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      count = half;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+    }
+  }
+  return v[0];
+}
+
+template <int RP>
+__device__ __forceinline__ int reduced_index() {
+  constexpr int LOG = RP == 1 ? 0 : RP == 2 ? 1 : RP == 4 ? 2 : RP == 8 ? 3 : RP == 16 ? 4 : 5;
+  return (threadIdx.x & 31) >> (5 - LOG);
+}
+
+template <int D, int RP>
+__global__ void __launch_bounds__(kScoreThreads)
+score_kernel(Geom G, int level, int64_t n_nodes, int64_t n_par, int32_t batch,
+             const float* __restrict__ Q, const uint32_t* __restrict__ kept_up, int64_t words_up,
+             float* __restrict__ sigma, const float* __restrict__ store) {
+  constexpr int EPL = D / 32;
+  __shared__ unsigned long long s_mask[kScoreTile];
+  __shared__ uint32_t s_kw[kScoreQBlock][2];
+  const int g = blockIdx.y;
+  const int64_t n0 = int64_t(blockIdx.x) * kScoreTile;
+  const int GQ = G.group;
+  const int qn_total = batch * GQ;
+  const int qb0 = blockIdx.z * kScoreQBlock;
+  const int nq = min(kScoreQBlock, qn_total - qb0);
+  const int C = G.chunk, R = G.nref;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t orphan0 = int64_t(C) * n_par;
+  const int64_t p_lo = n0 / C;
+  const int64_t w_lo = p_lo >> 5;
+
+  if (tid < nq && n0 < orphan0) {
+    const int qi = qb0 + tid;
+    const int b = qi / GQ, h = g * GQ + qi % GQ;
+    const uint32_t* kw = kept_up + (int64_t(b) * G.hq + h) * words_up;
+    s_kw[tid][0] = kw[w_lo];
+    s_kw[tid][1] = (w_lo + 1 < words_up) ? kw[w_lo + 1] : 0u;
+  }
+  __syncthreads();
+  if (tid < kScoreTile) {
+    const int64_t n = n0 + tid;
+    unsigned long long m = 0ull;
+    if (n < n_nodes) {
+      if (n >= orphan0) {
+        m = nq == 64 ? ~0ull : ((1ull << nq) - 1ull);
+      } else {
+        const int64_t p = n / C;
+        const int slot = int((p >> 5) - w_lo);
+        const int bit = int(p & 31);
+        for (int s = 0; s < nq; ++s) m |= (unsigned long long)((s_kw[s][slot] >> bit) & 1u) << s;
+      }
+    }
+    s_mask[tid] = m;
+  }
+  __syncthreads();
+
+  for (int t = warp; t < kScoreTile; t += kScoreThreads / 32) {
+    unsigned long long m = s_mask[t];
+    if (m == 0ull) continue;
+    const int64_t n = n0 + t;
+    const float* rec = store + G.off[level] + (int64_t(g) * G.cap[level] + n) * G.node_floats;
+    float kr[RP][EPL];
+#pragma unroll
+    for (int r = 0; r < RP; ++r) {
+      if (r < R) {
+        load_slice<EPL>(rec + r * D, EPL * lane, kr[r]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) kr[r][e] = 0.f;
+      }
+    }
+    const int rl = reduced_index<RP>();
+    const float bl = rl < R ? rec[R * D + rl] : 0.f;
+    while (m) {
+      const int s = __ffsll(m) - 1;
+      m &= m - 1ull;
+      const int qi = qb0 + s;
+      const int b = qi / GQ, h = g * GQ + qi % GQ;
+      float q[EPL];
+      load_slice<EPL>(Q + (int64_t(b) * G.hq + h) * D, EPL * lane, q);
+      float v[RP];
+#pragma unroll
+      for (int r = 0; r < RP; ++r) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) a += q[e] * kr[r][e];
+        v[r] = a;
+      }
+      const float dot = transpose_reduce<RP>(v);
+      const float tr = rl < R ? dot * G.scale + bl : -INFINITY;
+      const float sg = warp_max(tr);
+      if (lane == 0) sigma[(int64_t(b) * G.hq + h) * n_nodes + n] = sg;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Block-wide helpers for the select kernel (blockDim = kSelectThreads).
+// ---------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ T warp_incl_scan(T v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    T n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
+// Exclusive prefix over threads in thread order; returns this thread's offset
+// and writes the block total to *total. `tmp` holds >= 33 elements.
+template <typename T>
+__device__ T block_excl_scan(T v, T* tmp, T* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const T incl = warp_incl_scan(v);
+  if (lane == 31) tmp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    T w = lane < nw ? tmp[lane] : T(0);
+    T wi = warp_incl_scan(w);
+    if (lane < nw) tmp[lane] = wi - w;
+    if (lane == 31) tmp[32] = wi;
+  }
+  __syncthreads();
+  const T out = tmp[warp] + incl - v;
+  *total = tmp[32];
+  __syncthreads();
+  return out;
+}
+
+__device__ float block_max(float v, float* tmp) {
+  v = warp_max(v);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if (lane == 0) tmp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    float w = lane < nw ? tmp[lane] : -INFINITY;
+    w = warp_max(w);
+    if (lane == 0) tmp[32] = w;
+  }
+  __syncthreads();
+  const float r = tmp[32];
+  __syncthreads();
+  return r;
+}
+
+__device__ float block_sum(float v, float* tmp) {
+  v = warp_sum(v);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  if (lane == 0) tmp[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    float w = lane < nw ? tmp[lane] : 0.f;
+    w = warp_sum(w);
+    if (lane == 0) tmp[32] = w;
+  }
+  __syncthreads();
+  const float r = tmp[32];
+  __syncthreads();
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// Selection for one query head at one level.
+// ---------------------------------------------------------------------------
+struct SelectArgs {
+  int level;
+  int64_t n_nodes, n_par;
+  const uint32_t* kept_up;   // level l+1 bitmaps, [B*Hq][words_up] (null at the top)
+  int64_t words_up;
+  uint32_t* kept_here;       // level l bitmaps, [B*Hq][words_here]
+  int64_t words_here;
+  const float* sigma;        // [B*Hq][n_nodes]
+  int32_t* kp;               // scratch [B*Hq][kp_stride]
+  int64_t kp_stride;
+  unsigned long long p_fixed;
+  int keep_all;
+  int32_t* chunk_ids;        // level 1 only
+  int32_t* n_chunks;
+  int32_t max_sel;
+  int32_t* status;
+};
+
+__global__ void __launch_bounds__(kSelectThreads)
+select_kernel(Geom G, SelectArgs a) {
+  extern __shared__ float4 smem_v4[];
+  unsigned long long* hist = reinterpret_cast<unsigned long long*>(smem_v4);  // [nwarps][256]
+  float* s_sig = reinterpret_cast<float*>(hist + (kSelectThreads / 32) * 256);
+  __shared__ float s_f[33];
+  __shared__ unsigned long long s_u[33];
+  __shared__ uint32_t s_w[33];
+  __shared__ uint32_t s_bucket;
+  __shared__ unsigned long long s_before;
+
+  const int bh = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  const int C = G.chunk;
+  uint32_t* bits = a.kept_here + int64_t(bh) * a.words_here;
+  for (int64_t w = tid; w < a.words_here; w += blockDim.x) bits[w] = 0u;
+
+  // Kept parents of this head, ascending (compaction of the level-(l+1) bitmap).
+  int32_t* kp = a.kp + int64_t(bh) * a.kp_stride;
+  uint32_t n_kp = 0;
+  if (a.kept_up != nullptr && a.words_up > 0) {
+    const uint32_t* up = a.kept_up + int64_t(bh) * a.words_up;
+    for (int64_t w0 = 0; w0 < a.words_up; w0 += blockDim.x) {
+      const int64_t w = w0 + tid;
+      const uint32_t word = w < a.words_up ? up[w] : 0u;
+      uint32_t tot;
+      uint32_t pos = n_kp + block_excl_scan<uint32_t>(__popc(word), s_w, &tot);
+      uint32_t x = word;
+      while (x) {
+        const int bit = __ffs(x) - 1;
+        x &= x - 1u;
+        kp[pos++] = int32_t(w * 32 + bit);
+      }
+      n_kp += tot;
+    }
+  }
+  __syncthreads();   // kp visible to the block (global memory, same CTA)
+
+  const int64_t orphan0 = int64_t(C) * a.n_par;
+  const int64_t n_child = int64_t(n_kp) * C;
+  const int64_t n_c = n_child + (a.n_nodes - orphan0);
+  auto node_of = [&](int64_t i) -> int64_t {
+    return i < n_child ? int64_t(kp[i / C]) * C + i % C : orphan0 + (i - n_child);
+  };
+  const float* sig = a.sigma + int64_t(bh) * a.n_nodes;
+  const bool cached = n_c <= kSelectCache;
+  if (cached)
+    for (int64_t i = tid; i < n_c; i += blockDim.x) s_sig[i] = sig[node_of(i)];
+  __syncthreads();
+  auto sigma_of = [&](int64_t i) -> float { return cached ? s_sig[i] : sig[node_of(i)]; };
+
+  // Softmax statistics over the candidates.
+  float mx = -INFINITY;
+  for (int64_t i = tid; i < n_c; i += blockDim.x) mx = fmaxf(mx, sigma_of(i));
+  mx = block_max(mx, s_f);
+  float z = 0.f;
+  for (int64_t i = tid; i < n_c; i += blockDim.x) z += expf(sigma_of(i) - mx);
+  z = block_sum(z, s_f);
+  const float inv_z = 1.f / z;
+  auto mass_of = [&](float s) -> unsigned long long {
+    return __float2ull_rn(expf(s - mx) * inv_z * float(kMassScale));
+  };
+
+  // Cut: smallest key (score desc, index asc) whose cumulative mass reaches p.
+  bool keep_all = a.keep_all != 0 || n_c == 0;
+  uint32_t key_cut = 0xffffffffu;
+  unsigned long long t_keep = 0;
+  if (!keep_all) {
+    unsigned long long tm = 0;
+    for (int64_t i = tid; i < n_c; i += blockDim.x) tm += mass_of(sigma_of(i));
+    unsigned long long total;
+    block_excl_scan<unsigned long long>(tm, s_u, &total);
+    if (total < a.p_fixed) keep_all = true;
+  }
+  if (!keep_all) {
+    uint32_t prefix = 0, pmask = 0;
+    unsigned long long before = 0;
+    unsigned long long* wh = hist + warp * 256;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      for (int k = lane; k < 256; k += 32) wh[k] = 0ull;
+      __syncthreads();
+      for (int64_t i = tid; i < n_c; i += blockDim.x) {
+        const float s = sigma_of(i);
+        const uint32_t key = ~float_order_key(s);
+        if ((key & pmask) == prefix) atomicAdd(&wh[(key >> shift) & 255u], mass_of(s));
+      }
+      __syncthreads();
+      // bucket totals into warp 0's histogram
+      for (int k = tid; k < 256; k += blockDim.x) {
+        unsigned long long v = 0;
+        for (int w = 0; w < nw; ++w) v += hist[w * 256 + k];
+        hist[k] = v;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane owns buckets [8*lane, 8*lane+8)
+        unsigned long long loc[8], run = 0;
+        for (int k = 0; k < 8; ++k) { loc[k] = hist[8 * lane + k]; run += loc[k]; }
+        unsigned long long incl = warp_incl_scan<unsigned long long>(run);
+        unsigned long long excl = incl - run;
+        // first bucket whose inclusive cumulative mass reaches p
+        int found = -1;
+        unsigned long long acc = before + excl, acc_before = 0;
+        for (int k = 0; k < 8; ++k) {
+          if (found < 0 && acc + loc[k] >= a.p_fixed) { found = 8 * lane + k; acc_before = acc; }
+          acc += loc[k];
+        }
+        const unsigned ball = __ballot_sync(0xffffffffu, found >= 0);
+        const int src = ball ? __ffs(ball) - 1 : 31;
+        const int fb = __shfl_sync(0xffffffffu, found, src);
+        const unsigned long long ab = __shfl_sync(0xffffffffu, acc_before, src);
+        if (lane == 0) {
+          s_bucket = fb < 0 ? 255u : uint32_t(fb);
+          s_before = fb < 0 ? before : ab;
+        }
+      }
+      __syncthreads();
+      prefix |= s_bucket << shift;
+      pmask |= 255u << shift;
+      before = s_before;
+      __syncthreads();
+    }
+    key_cut = prefix;
+    const unsigned long long pi_cut = mass_of(order_key_float(~key_cut));
+    const unsigned long long need = a.p_fixed > before ? a.p_fixed - before : 0ull;
+    t_keep = pi_cut > 0 ? (need + pi_cut - 1) / pi_cut : 0ull;
+  }
+
+  // Keep flags in candidate order (ascending node index): thread-contiguous
+  // ranges so that ties at the cut are taken lowest index first.
+  const int64_t per = (n_c + blockDim.x - 1) / blockDim.x;
+  const int64_t i_lo = min64(n_c, per * tid), i_hi = min64(n_c, i_lo + per);
+  uint32_t my_ties = 0;
+  if (!keep_all)
+    for (int64_t i = i_lo; i < i_hi; ++i) my_ties += (~float_order_key(sigma_of(i)) == key_cut);
+  uint32_t tie_total;
+  uint32_t tie_rank = block_excl_scan<uint32_t>(my_ties, s_w, &tie_total);
+  uint32_t my_kept = 0;
+  {
+    uint32_t tr = tie_rank;
+    for (int64_t i = i_lo; i < i_hi; ++i) {
+      bool k = keep_all;
+      if (!k) {
+        const uint32_t key = ~float_order_key(sigma_of(i));
+        k = key < key_cut || (key == key_cut && tr++ < t_keep);
+      }
+      my_kept += k;
+    }
+  }
+  uint32_t kept_total;
+  uint32_t pos = block_excl_scan<uint32_t>(my_kept, s_w, &kept_total);
+  {
+    uint32_t tr = tie_rank;
+    for (int64_t i = i_lo; i < i_hi; ++i) {
+      bool k = keep_all;
+      if (!k) {
+        const uint32_t key = ~float_order_key(sigma_of(i));
+        k = key < key_cut || (key == key_cut && tr++ < t_keep);
+      }
+      if (k) {
+        const int64_t node = node_of(i);
+        atomicOr(&bits[node >> 5], 1u << (node & 31));
+        if (a.chunk_ids != nullptr && pos < uint32_t(a.max_sel))
+          a.chunk_ids[int64_t(bh) * a.max_sel + pos] = int32_t(node);
+        ++pos;
+      }
+    }
+  }
+  if (a.chunk_ids != nullptr && tid == 0) {
+    a.n_chunks[bh] = int32_t(kept_total);
+    if (kept_total > uint32_t(a.max_sel) && a.status != nullptr)
+      atomicOr(a.status, ZHA_DEV_SELECTION_TRUNCATED);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host launcher: levels L..1, score then select.
+// ---------------------------------------------------------------------------
+template <int D, int RP>
+static cudaError_t launch_score_t(const Geom& G, int level, int64_t n_nodes, int64_t n_par,
+                                  int32_t batch, const float* Q, const uint32_t* kept_up,
+                                  int64_t words_up, float* sigma, const float* store,
+                                  cudaStream_t s) {
+  const int qn = batch * G.group;
+  dim3 grid(unsigned((n_nodes + kScoreTile - 1) / kScoreTile), unsigned(G.hkv),
+            unsigned((qn + kScoreQBlock - 1) / kScoreQBlock));
+  score_kernel<D, RP><<<grid, kScoreThreads, 0, s>>>(G, level, n_nodes, n_par, batch, Q, kept_up,
+                                                     words_up, sigma, store);
+  zha_count_launch();
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_score_d(const Geom& G, int level, int64_t n_nodes, int64_t n_par,
+                                  int32_t batch, const float* Q, const uint32_t* kept_up,
+                                  int64_t words_up, float* sigma, const float* store,
+                                  cudaStream_t s) {
+  const int R = G.nref;
+#define ZHA_SCORE_CASE(RP)                                                                      \
+  if (R <= RP)                                                                                  \
+    return launch_score_t<D, RP>(G, level, n_nodes, n_par, batch, Q, kept_up, words_up, sigma, \
+                                 store, s);
+  ZHA_SCORE_CASE(1)
+  ZHA_SCORE_CASE(2)
+  ZHA_SCORE_CASE(4)
+  ZHA_SCORE_CASE(8)
+  ZHA_SCORE_CASE(16)
+  ZHA_SCORE_CASE(32)
+#undef ZHA_SCORE_CASE
+  return cudaErrorInvalidValue;
+}
+
+size_t select_smem_bytes() {
+  return size_t(kSelectThreads / 32) * 256 * sizeof(unsigned long long) +
+         size_t(kSelectCache) * sizeof(float);
+}
+
+cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n_tokens, float p,
+                         int32_t* chunk_ids, int32_t* n_chunks, int32_t max_sel, uint32_t* bits,
+                         float* sigma, int32_t* kp, const RouteLayout& lay, int32_t* status,
+                         const float* store, cudaStream_t s) {
+  const size_t smem = select_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem));
+  if (e != cudaSuccess) return e;
+  const int heads = batch * G.hq;
+  SelectArgs a{};
+  a.p_fixed = (unsigned long long)ceil(double(p) * kMassScale);
+  if (a.p_fixed == 0) a.p_fixed = 1;
+  a.keep_all = p >= 1.0f;
+  a.kp = kp;
+  int64_t kp_stride = lay.kp_ints / (heads > 0 ? heads : 1);
+  a.kp_stride = kp_stride;
+  a.max_sel = max_sel;
+  a.status = status;
+  for (int level = G.levels; level >= 1; --level) {
+    const int64_t n_nodes = lay.n[level];
+    const int64_t n_par = level < G.levels ? lay.n[level + 1] : 0;
+    const uint32_t* up = level < G.levels ? bits + lay.bits_off[level + 1] : nullptr;
+    const int64_t words_up = level < G.levels ? lay.words[level + 1] : 0;
+    float* sg = sigma + lay.sig_off[level];
+    if (n_nodes > 0) {
+      e = G.d == 128 ? launch_score_d<128>(G, level, n_nodes, n_par, batch, Q, up, words_up, sg,
+                                           store, s)
+                     : launch_score_d<64>(G, level, n_nodes, n_par, batch, Q, up, words_up, sg,
+                                          store, s);
+      if (e != cudaSuccess) return e;
+    }
+    a.level = level;
+    a.n_nodes = n_nodes;
+    a.n_par = n_par;
+    a.kept_up = up;
+    a.words_up = words_up;
+    a.kept_here = bits + lay.bits_off[level];
+    a.words_here = lay.words[level];
+    a.sigma = sg;
+    a.chunk_ids = level == 1 ? chunk_ids : nullptr;
+    a.n_chunks = level == 1 ? n_chunks : nullptr;
+    select_kernel<<<heads, kSelectThreads, smem, s>>>(G, a);
+    zha_count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace zha

@@ -1,0 +1,229 @@
+"""Python binding of libzha (the C ABI in include/zha.h).
+
+Argument marshalling only: every step of the hot path runs in the library's
+CUDA kernels. Tensors are torch CUDA tensors (PyTorch supplies device memory
+and streams); their data pointers and the current stream are handed to the C
+calls. Importing this module raises if libzha.so has not been built -- there is
+no fallback implementation.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, byref, c_char_p, c_float, c_int32, c_int64, c_size_t, c_uint64, c_void_p
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libzha.so")
+
+ZHA_OK = 0
+ZHA_ERR_INVALID = -1
+ZHA_ERR_CAPACITY = -2
+ZHA_ERR_STATE = -3
+ZHA_ERR_CUDA = -4
+ZHA_ERR_UNSUPPORTED = -6
+ZHA_F32 = 0
+ZHA_BF16 = 1
+ZHA_DEV_SELECTION_TRUNCATED = 1
+ZHA_DEV_BAD_SELECTION = 2
+
+
+class ZhaError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+class Config(ctypes.Structure):
+    _fields_ = [
+        ("n_kv_heads", c_int32), ("n_q_heads", c_int32), ("head_dim", c_int32),
+        ("chunk", c_int32), ("levels", c_int32), ("n_ref", c_int32),
+        ("kv_dtype", c_int32), ("reserved", c_int32), ("max_tokens", c_int64),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m "
+            "hierarchical_sparse_attention_zha_b200.build` (there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = c_void_p
+    sig = {
+        "zha_abi_version": (c_int32, []),
+        "zha_status_str": (c_char_p, [c_int32]),
+        "zha_last_error": (c_char_p, []),
+        "zha_launch_count": (c_uint64, []),
+        "zha_tree_bytes": (c_size_t, [POINTER(Config)]),
+        "zha_tree_create": (c_int32, [POINTER(Config), P, c_size_t, P, POINTER(P)]),
+        "zha_tree_destroy": (None, [P]),
+        "zha_tree_built_tokens": (c_int64, [P]),
+        "zha_tree_level_layout": (c_int32, [P, c_int32, POINTER(c_int64), POINTER(c_int64),
+                                            POINTER(c_int32)]),
+        "zha_build": (c_int32, [P, P, c_int64, c_int64, P]),
+        "zha_append_chunk": (c_int32, [P, P, c_int64, c_int64, P]),
+        "zha_route_workspace_bytes": (c_size_t, [POINTER(Config), c_int32, c_int64]),
+        "zha_route_kept_words": (c_size_t, [POINTER(Config), c_int32, c_int64]),
+        "zha_route": (c_int32, [P, P, c_int32, c_int64, c_float, P, P, c_int32, P, P, c_size_t,
+                                P, P]),
+        "zha_attend_workspace_bytes": (c_size_t, [POINTER(Config), c_int32, c_int64]),
+        "zha_sparse_attend": (c_int32, [P, P, P, P, c_int64, c_int64, c_int32, P, P, c_int32, P,
+                                        P, P, c_size_t, P, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def status_str(status: int) -> str:
+    return lib.zha_status_str(status).decode()
+
+
+def last_error() -> str:
+    return lib.zha_last_error().decode()
+
+
+def launch_count() -> int:
+    return int(lib.zha_launch_count())
+
+
+def check(status: int, what: str) -> None:
+    if status != ZHA_OK:
+        raise ZhaError(status, f"{what}: {status_str(status)}: {last_error()}")
+
+
+def ptr(t: torch.Tensor | None):
+    return None if t is None else c_void_p(t.data_ptr())
+
+
+def stream_ptr(stream: torch.cuda.Stream | None = None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return c_void_p(s.cuda_stream)
+
+
+def make_config(n_kv_heads: int, n_q_heads: int, head_dim: int, chunk: int, levels: int,
+                n_ref: int, kv_dtype: torch.dtype, max_tokens: int) -> Config:
+    dt = {torch.float32: ZHA_F32, torch.bfloat16: ZHA_BF16}[kv_dtype]
+    return Config(n_kv_heads, n_q_heads, head_dim, chunk, levels, n_ref, dt, 0, max_tokens)
+
+
+def tree_bytes(cfg: Config) -> int:
+    return int(lib.zha_tree_bytes(byref(cfg)))
+
+
+def route_workspace_bytes(cfg: Config, batch: int, n_tokens: int) -> int:
+    return int(lib.zha_route_workspace_bytes(byref(cfg), batch, n_tokens))
+
+
+def route_kept_words(cfg: Config, batch: int, n_tokens: int) -> int:
+    return int(lib.zha_route_kept_words(byref(cfg), batch, n_tokens))
+
+
+def attend_workspace_bytes(cfg: Config, batch: int, n_tokens: int) -> int:
+    return int(lib.zha_attend_workspace_bytes(byref(cfg), batch, n_tokens))
+
+
+def _bytes_tensor(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(1, (nbytes + 255) // 256) * 64, dtype=torch.float32, device=device)
+
+
+class Tree:
+    """One summary store (all KV heads) plus its C handle.
+
+    ``ref_q``: float32 CUDA tensor [n_kv_heads, n_ref, head_dim], kept alive here.
+    """
+
+    def __init__(self, cfg: Config, ref_q: torch.Tensor):
+        if not (ref_q.is_cuda and ref_q.dtype == torch.float32 and ref_q.is_contiguous()):
+            raise ValueError("ref_q must be a contiguous float32 CUDA tensor")
+        if tuple(ref_q.shape) != (cfg.n_kv_heads, cfg.n_ref, cfg.head_dim):
+            raise ValueError("ref_q shape does not match the config")
+        self.cfg = cfg
+        self.ref_q = ref_q
+        self.device = ref_q.device
+        nbytes = tree_bytes(cfg)
+        if nbytes == 0:
+            check(ZHA_ERR_INVALID, "zha_tree_bytes")
+        self.store = _bytes_tensor(nbytes, self.device)
+        handle = c_void_p()
+        check(lib.zha_tree_create(byref(cfg), ptr(self.store), self.store.numel() * 4, ptr(ref_q),
+                                  byref(handle)), "zha_tree_create")
+        self.handle = handle
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h is not None and h.value:
+            lib.zha_tree_destroy(h)
+            self.handle = None
+
+    @property
+    def built_tokens(self) -> int:
+        return int(lib.zha_tree_built_tokens(self.handle))
+
+    def _kv(self, K: torch.Tensor) -> None:
+        want = torch.float32 if self.cfg.kv_dtype == ZHA_F32 else torch.bfloat16
+        if not (K.is_cuda and K.dtype == want and K.is_contiguous() and K.dim() == 3
+                and K.shape[0] == self.cfg.n_kv_heads and K.shape[2] == self.cfg.head_dim):
+            raise ValueError(f"cache must be a contiguous {want} CUDA tensor [Hkv, ld, d]")
+
+    def build(self, K: torch.Tensor, n_tokens: int, stream=None) -> None:
+        self._kv(K)
+        check(lib.zha_build(self.handle, ptr(K), K.shape[1], n_tokens, stream_ptr(stream)),
+              "zha_build")
+
+    def append_chunk(self, K: torch.Tensor, n_tokens: int, stream=None) -> None:
+        self._kv(K)
+        check(lib.zha_append_chunk(self.handle, ptr(K), K.shape[1], n_tokens, stream_ptr(stream)),
+              "zha_append_chunk")
+
+    def level(self, level: int) -> tuple[torch.Tensor, torch.Tensor]:
+        """Views of level `level`'s summaries: khat [Hkv, cap, R, d], bhat [Hkv, cap, R]."""
+        off, cap, nf = c_int64(), c_int64(), c_int32()
+        check(lib.zha_tree_level_layout(self.handle, level, byref(off), byref(cap), byref(nf)),
+              "zha_tree_level_layout")
+        H, R, d = self.cfg.n_kv_heads, self.cfg.n_ref, self.cfg.head_dim
+        blk = self.store[off.value: off.value + H * cap.value * nf.value].view(H, cap.value, nf.value)
+        return blk[:, :, : R * d].reshape(H, cap.value, R, d), blk[:, :, R * d: R * d + R]
+
+    def route(self, Q: torch.Tensor, n_tokens: int, p: float, max_sel: int,
+              chunk_ids: torch.Tensor | None = None, n_chunks: torch.Tensor | None = None,
+              kept_bits: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+              status: torch.Tensor | None = None, stream=None):
+        B = Q.shape[0]
+        if chunk_ids is None:
+            chunk_ids = torch.empty(B, self.cfg.n_q_heads, max_sel, dtype=torch.int32, device=self.device)
+        if n_chunks is None:
+            n_chunks = torch.empty(B, self.cfg.n_q_heads, dtype=torch.int32, device=self.device)
+        if ws is None:
+            ws = _bytes_tensor(route_workspace_bytes(self.cfg, B, n_tokens), self.device)
+        check(lib.zha_route(self.handle, ptr(Q), B, n_tokens, p, ptr(chunk_ids), ptr(n_chunks),
+                            max_sel, ptr(kept_bits), ptr(ws), ws.numel() * ws.element_size(),
+                            ptr(status), stream_ptr(stream)), "zha_route")
+        return chunk_ids, n_chunks
+
+    def sparse_attend(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, n_tokens: int,
+                      chunk_ids: torch.Tensor, n_chunks: torch.Tensor,
+                      out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                      ws: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                      stream=None):
+        self._kv(K)
+        self._kv(V)
+        B = Q.shape[0]
+        if out is None:
+            out = torch.empty(B, self.cfg.n_q_heads, self.cfg.head_dim, dtype=torch.float32,
+                              device=self.device)
+        if lse is None:
+            lse = torch.empty(B, self.cfg.n_q_heads, dtype=torch.float32, device=self.device)
+        if ws is None:
+            ws = _bytes_tensor(attend_workspace_bytes(self.cfg, B, n_tokens), self.device)
+        check(lib.zha_sparse_attend(self.handle, ptr(Q), ptr(K), ptr(V), K.shape[1], n_tokens, B,
+                                    ptr(chunk_ids), ptr(n_chunks), chunk_ids.shape[-1], ptr(out),
+                                    ptr(lse), ptr(ws), ws.numel() * ws.element_size(), ptr(status),
+                                    stream_ptr(stream)), "zha_sparse_attend")
+        return out, lse

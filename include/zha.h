@@ -1,0 +1,189 @@
+/*
+ * zha.h -- C ABI of the ZHA decode hot path on B200 (sm_100a): tree-summarised
+ * KV-cache attention.
+ *
+ * Citations name a page by its title and a section on it:
+ *   [ZHA: <section>]  page "ZHA는 KV 캐시를 트리로 요약해 어텐션 비용을 준(sub)이차로
+ *                     낮춘다" (onedev.kr/papers/1556);
+ *   [Attention: <section>]  page "Attention"
+ *                     (zzong2006.github.io/machine_learning/nlp/attention-function).
+ *
+ * The method: every contiguous key chunk of C tokens gets, at each of R
+ * reference queries q_r, a tangent plane t_r(q) = q.khat_r/sqrt(d) + bhat_r of
+ * its log attention mass; level l >= 2 nodes merge C children the same way.
+ * At decode time each query head is routed level by level with top-p over the
+ * planes' maximum, and exact softmax attention runs over the gathered leaf
+ * tokens, the sink (token 0) and the in-progress tail [ZHA: 무엇과 다른가,
+ * 전제와 한계]. One tree per KV head serves its GQA query heads.
+ *
+ * Conventions for every call:
+ *  - All pointers named d_* are DEVICE pointers owned by the caller (the library
+ *    allocates no device memory). They must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Calls enqueue work and return; none synchronises the device.
+ *  - Return value: ZHA_OK, or a negative zha_status when the host-side checks
+ *    reject the arguments (nothing is launched then) or a launch fails
+ *    (ZHA_ERR_CUDA). zha_last_error() gives a message for the calling thread.
+ *  - Conditions only the device can see are OR-ed into *d_status (int32,
+ *    ZHA_DEV_* bits) where the call takes one; the caller zeroes it and reads it
+ *    after synchronising.
+ *  - Layouts: K and V caches are [n_kv_heads][ld][head_dim] (element type
+ *    zha_config.kv_dtype, ld >= tokens used); queries Q are float32
+ *    [batch][n_q_heads][head_dim]; query head h uses KV head h / (n_q_heads /
+ *    n_kv_heads) [Attention: "Key·value head 를 나눠 쓰거나 압축한다"];
+ *    reference queries are float32 [n_kv_heads][n_ref][head_dim].
+ *  - No call is thread-safe against another call on the same tree unless the
+ *    caller orders them (same stream or events).
+ */
+#ifndef ZHA_H
+#define ZHA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ZHA_ABI_VERSION 1
+
+typedef enum {
+    ZHA_OK = 0,
+    ZHA_ERR_INVALID = -1,     /* bad argument: null pointer, size, alignment, range */
+    ZHA_ERR_CAPACITY = -2,    /* a caller buffer (store, workspace, max_sel) is too small */
+    ZHA_ERR_STATE = -3,       /* the tree's built prefix does not match n_tokens */
+    ZHA_ERR_CUDA = -4,        /* a CUDA launch or query failed (see zha_last_error) */
+    ZHA_ERR_UNSUPPORTED = -6  /* a configuration this build does not implement */
+} zha_status;
+
+/* Bits OR-ed into *d_status by device code. */
+#define ZHA_DEV_SELECTION_TRUNCATED 1 /* zha_route: a head kept more than max_sel chunks; its list holds the first max_sel (ascending) and d_n_chunks the true count */
+#define ZHA_DEV_BAD_SELECTION 2       /* zha_sparse_attend: a chunk list had an id out of range, was not strictly ascending, or a count above max_sel; the offending entries were skipped */
+
+typedef enum { ZHA_F32 = 0, ZHA_BF16 = 1 } zha_dtype;
+
+typedef struct {
+    int32_t n_kv_heads;  /* KV heads = trees, >= 1 */
+    int32_t n_q_heads;   /* query heads, a multiple of n_kv_heads */
+    int32_t head_dim;    /* d: 64 or 128 */
+    int32_t chunk;       /* C: tokens per level-1 chunk, 2..128 */
+    int32_t levels;      /* L: summary levels, 1..8; level l covers C^l tokens */
+    int32_t n_ref;       /* R: reference queries per tree, 1..32 */
+    int32_t kv_dtype;    /* zha_dtype of the K and V caches */
+    int32_t reserved;    /* must be 0 */
+    int64_t max_tokens;  /* tokens the summary store must cover, >= 1 */
+} zha_config;
+
+typedef struct zha_tree zha_tree; /* opaque host handle; holds no device memory */
+
+/* ABI version of the loaded library (ZHA_ABI_VERSION). */
+int32_t zha_abi_version(void);
+
+/* Static text for a zha_status. */
+const char* zha_status_str(int32_t status);
+
+/* Message describing the last failed call made by the calling thread. */
+const char* zha_last_error(void);
+
+/* Number of kernels this library has launched in the process so far. */
+uint64_t zha_launch_count(void);
+
+/* Bytes of device memory the summary store of `cfg` needs (0 if cfg is
+ * invalid). Layout, level-major: for l = 1..L, float32
+ * [n_kv_heads][floor(max_tokens / C^l)][node_floats], each node holding
+ * khat [n_ref][head_dim] then bhat [n_ref], padded to node_floats =
+ * n_ref*head_dim + round_up(n_ref, 4). [ZHA: 무엇과 다른가] */
+size_t zha_tree_bytes(const zha_config* cfg);
+
+/* Create a host handle over a caller-owned store (>= zha_tree_bytes bytes,
+ * 256-byte aligned) and reference queries d_ref_q [n_kv_heads][n_ref][head_dim]
+ * float32, which must stay valid while the tree is used. The tree starts empty
+ * (0 tokens built). Returns ZHA_ERR_INVALID / ZHA_ERR_CAPACITY / ZHA_ERR_UNSUPPORTED
+ * on bad arguments; *out is set only on success. The learned reference queries
+ * are the only trained parameters of the method [ZHA: 어떻게 쓰나]. */
+zha_status zha_tree_create(const zha_config* cfg, void* d_store, size_t store_bytes,
+                           const float* d_ref_q, zha_tree** out);
+
+/* Release a handle (the store and reference queries stay the caller's). NULL is ignored. */
+void zha_tree_destroy(zha_tree* tree);
+
+/* N_b: tokens covered by complete level-1 chunks so far (a multiple of C). */
+int64_t zha_tree_built_tokens(const zha_tree* tree);
+
+/* Where level `level` (1..L) lives in the store: float offset of node (g=0,i=0),
+ * node capacity per KV head, floats per node. For reading summaries back. */
+zha_status zha_tree_level_layout(const zha_tree* tree, int32_t level, int64_t* offset_floats,
+                                 int64_t* capacity, int32_t* node_floats);
+
+/* Build every level over the complete chunks of the first n_tokens keys of
+ * d_K [n_kv_heads][ld][head_dim] (prefill). Level 1: for chunk i and plane r,
+ * s_j = q_r.k_j/sqrt(d) over the chunk, F = LSE_j s_j, khat = sum_j softmax(s)_j k_j,
+ * bhat = F - q_r.khat/sqrt(d). Level l >= 2 merges each run of C level-(l-1)
+ * nodes: u_c = q_r.khat_{r,c}/sqrt(d) + bhat_{r,c}, F = LSE_c u_c,
+ * khat = sum_c softmax(u)_c khat_{r,c}, bhat = F - q_r.khat/sqrt(d)
+ * [ZHA: 무엇과 다른가: tangent-plane summary; "parents merge the child summaries
+ * in the same way"]. Afterwards N_b = C*floor(n_tokens/C). Requires
+ * 0 <= n_tokens <= min(ld, max_tokens). V is not read. */
+zha_status zha_build(zha_tree* tree, const void* d_K, int64_t ld, int64_t n_tokens, void* stream);
+
+/* Incremental build while decoding: n_tokens is the cache length after the
+ * caller has written the newest keys; the new N_b = C*floor(n_tokens/C) must be
+ * >= the tree's N_b (else ZHA_ERR_STATE). Summarises each newly completed chunk
+ * and merges every upper-level node the new chunks complete (level 1 every C
+ * steps, level 2 every C^2 steps [ZHA: 무엇과 다른가]). One launch when up to
+ * 8 chunks are new; a no-op when none is. */
+zha_status zha_append_chunk(zha_tree* tree, const void* d_K, int64_t ld, int64_t n_tokens,
+                            void* stream);
+
+/* Workspace bytes zha_route needs for `batch` queries at n_tokens (grows with
+ * n_tokens, so sizing for the largest n_tokens covers smaller ones). */
+size_t zha_route_workspace_bytes(const zha_config* cfg, int32_t batch, int64_t n_tokens);
+
+/* uint32 words of the per-level kept bitmaps zha_route can return: level-major
+ * for l = 1..L, each [batch][n_q_heads][ceil(n_l / 32)] with n_l =
+ * floor(N_b / C^l) nodes at n_tokens; bit i of a head's words = node i kept. */
+size_t zha_route_kept_words(const zha_config* cfg, int32_t batch, int64_t n_tokens);
+
+/* Per-level top-p routing of `batch` decode queries d_Q [batch][n_q_heads][d]
+ * against the tree at n_tokens (C*floor(n_tokens/C) must equal the tree's N_b,
+ * else ZHA_ERR_STATE) [ZHA: 전제와 한계]. For each query head and level L..1:
+ * candidates are all level-L nodes at the top, below that the children of the
+ * nodes kept one level up plus the level's orphans (nodes whose parent does not
+ * exist yet); each candidate n scores sigma_n = max_r (q.khat_{r,n}/sqrt(d) +
+ * bhat_{r,n}); pi = softmax(sigma) over the candidates; the kept set is the
+ * shortest prefix of the candidates ordered by sigma descending (ties: lower
+ * node index first) whose pi sums to >= p; p >= 1 keeps all; 0 < p required.
+ * Output: d_chunk_ids [batch][n_q_heads][max_sel] int32, the kept level-1 chunk
+ * ids ascending, and d_n_chunks [batch][n_q_heads] their count (the sink and
+ * the tail [N_b, n_tokens) are implicit and not listed). d_kept_bits (nullable,
+ * zha_route_kept_words words) receives every level's kept bitmap. d_ws:
+ * >= zha_route_workspace_bytes bytes. d_status: ZHA_DEV_SELECTION_TRUNCATED. */
+zha_status zha_route(const zha_tree* tree, const float* d_Q, int32_t batch, int64_t n_tokens,
+                     float p, int32_t* d_chunk_ids, int32_t* d_n_chunks, int32_t max_sel,
+                     uint32_t* d_kept_bits, void* d_ws, size_t ws_bytes, int32_t* d_status,
+                     void* stream);
+
+/* Workspace bytes zha_sparse_attend needs for `batch` queries at n_tokens. */
+size_t zha_attend_workspace_bytes(const zha_config* cfg, int32_t batch, int64_t n_tokens);
+
+/* Exact attention of each query head over S = {0} u tokens(listed chunks) u
+ * [N_b, n_tokens), N_b = C*floor(n_tokens/C): o = sum_{j in S} softmax_j(q.k_j/
+ * sqrt(d)) v_j, normalised over S only [Attention: "Scaled dot-product attention
+ * 의 식"; ZHA: 전제와 한계]. Chunk lists as zha_route writes them (ascending
+ * ids < N_b/C, counts <= max_sel); they may also come from elsewhere. The tree
+ * supplies only its configuration (its summaries are not read). Output d_O
+ * [batch][n_q_heads][d] float32 and, if d_lse is not NULL, d_lse
+ * [batch][n_q_heads] = log sum_{j in S} exp(q.k_j/sqrt(d)). d_ws: >=
+ * zha_attend_workspace_bytes bytes. d_status (nullable): ZHA_DEV_BAD_SELECTION.
+ * Requires 1 <= n_tokens <= ld. */
+zha_status zha_sparse_attend(const zha_tree* tree, const float* d_Q, const void* d_K,
+                             const void* d_V, int64_t ld, int64_t n_tokens, int32_t batch,
+                             const int32_t* d_chunk_ids, const int32_t* d_n_chunks,
+                             int32_t max_sel, float* d_O, float* d_lse, void* d_ws,
+                             size_t ws_bytes, int32_t* d_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZHA_H */

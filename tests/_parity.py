@@ -1,0 +1,135 @@
+"""Helpers that run the CUDA path through the C ABI and compare it with the
+CPU oracle on the same seeded inputs (test infrastructure)."""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+import oracle as O
+from hierarchical_sparse_attention_zha_b200 import workloads as W
+
+# Tolerances. Summaries: norm-wise relative 1e-4 (khat: max abs error over the
+# row / max abs of the row; bhat: abs error / max(1, |bhat|)). Scores: ties are
+# disagreements within 1e-5 of the cut score or of the cut's cumulative mass.
+# Attention output: absolute 2e-2 for bf16 caches and 1e-4 for fp32 caches, and
+# also a tighter bound derived from fp32 accumulation over exactly stored
+# inputs: |do| <= 2e-5 * max|v| + 2e-6 and |d lse| <= 2e-5 * max(1, |lse|),
+# which catches a dropped or duplicated token that 2e-2 would hide.
+SUMMARY_RTOL = 1e-4
+TIE_TOL = 1e-5
+O_ATOL = {"bf16": 2e-2, "f32": 1e-4}
+O_DERIVED_REL = 2e-5
+
+
+def cache_f64(inp: W.Inputs, g: int, n: int | None = None) -> np.ndarray:
+    x = inp.K[g] if n is None else inp.K[g, :n]
+    return O.bf16_bits_to_f64(x) if inp.spec.kv_dtype == "bf16" else x.astype(np.float64)
+
+
+def values_f64(inp: W.Inputs, g: int, n: int | None = None) -> np.ndarray:
+    x = inp.V[g] if n is None else inp.V[g, :n]
+    return O.bf16_bits_to_f64(x) if inp.spec.kv_dtype == "bf16" else x.astype(np.float64)
+
+
+def to_device(inp: W.Inputs, device="cuda"):
+    if inp.spec.kv_dtype == "bf16":
+        K = torch.from_numpy(inp.K.view(np.int16)).to(device).view(torch.bfloat16)
+        V = torch.from_numpy(inp.V.view(np.int16)).to(device).view(torch.bfloat16)
+    else:
+        K = torch.from_numpy(inp.K).to(device)
+        V = torch.from_numpy(inp.V).to(device)
+    return K, V, torch.from_numpy(inp.ref_q).to(device), torch.from_numpy(inp.Q).to(device)
+
+
+def config_for(spec: W.Workload, max_tokens: int | None = None):
+    from hierarchical_sparse_attention_zha_b200 import zha
+    return zha.make_config(spec.n_kv_heads, spec.n_q_heads, spec.head_dim, spec.chunk, spec.levels,
+                           spec.n_ref, torch.bfloat16 if spec.kv_dtype == "bf16" else torch.float32,
+                           max_tokens or spec.capacity)
+
+
+def summary_errors(kh_gpu: np.ndarray, bh_gpu: np.ndarray, kh_ref: np.ndarray, bh_ref: np.ndarray):
+    """Norm-wise relative errors per (node, plane)."""
+    dk = np.max(np.abs(kh_gpu - kh_ref), axis=-1) / np.maximum(np.max(np.abs(kh_ref), axis=-1), 1e-30)
+    db = np.abs(bh_gpu - bh_ref) / np.maximum(1.0, np.abs(bh_ref))
+    return float(np.max(dk)) if dk.size else 0.0, float(np.max(db)) if db.size else 0.0
+
+
+def kept_from_bits(bits: np.ndarray, spec: W.Workload, batch: int, n_tokens: int) -> dict:
+    """Split the route's kept bitmaps into {level: [B][Hq] arrays of node ids}."""
+    nb = spec.chunk * (n_tokens // spec.chunk)
+    out, off = {}, 0
+    for lvl in range(1, spec.levels + 1):
+        n_l = nb // spec.chunk ** lvl
+        w = (n_l + 31) // 32
+        blk = bits[off: off + batch * spec.n_q_heads * w].reshape(batch, spec.n_q_heads, w)
+        off += batch * spec.n_q_heads * w
+        lv = {}
+        for b in range(batch):
+            for h in range(spec.n_q_heads):
+                words = blk[b, h].astype(np.uint32)
+                ids = np.nonzero(np.unpackbits(words.view(np.uint8), bitorder="little"))[0]
+                lv[(b, h)] = ids[ids < n_l]
+        out[lvl] = lv
+    return out
+
+
+@dataclass
+class RouteReport:
+    heads: int = 0
+    levels_compared: int = 0
+    ties: int = 0
+    hard: list = field(default_factory=list)
+    exact_heads: set = field(default_factory=set)
+
+
+def compare_route_head(q, otree, p, gpu_kept_by_level: dict, report: RouteReport, key) -> None:
+    """Compare one head level by level, each level conditioned on the GPU's kept
+    set one level up (the oracle's own selection at that level is compared)."""
+    forced = {lvl: ids for lvl, ids in gpu_kept_by_level.items()}
+    tr = O.route(q, otree, p, forced_kept=forced)
+    exact = True
+    for lvl, lt in tr.levels.items():
+        report.levels_compared += 1
+        own = set(lt.topp.kept.tolist())
+        gpu = set(np.asarray(gpu_kept_by_level[lvl]).tolist())
+        if own == gpu:
+            continue
+        exact = False
+        cand_pos = {int(n): i for i, n in enumerate(lt.candidates)}
+        sel = lt.topp
+        m = sel.m
+        sigma_cut = lt.sigma[sel.order[m - 1]] if m > 0 else math.inf
+        near_mass = (m >= 1 and abs(sel.cum[m - 1] - p) <= TIE_TOL) or \
+                    (m >= 2 and abs(sel.cum[m - 2] - p) <= TIE_TOL)
+        for node in own ^ gpu:
+            if node not in cand_pos:
+                report.hard.append((key, lvl, node, "not a candidate"))
+                continue
+            if abs(lt.sigma[cand_pos[node]] - sigma_cut) <= TIE_TOL or near_mass:
+                report.ties += 1
+            else:
+                report.hard.append((key, lvl, node, float(lt.sigma[cand_pos[node]]), float(sigma_cut)))
+    report.heads += 1
+    if exact:
+        report.exact_heads.add(key)
+
+
+def attend_errors(q, Kf, Vf, tokens, o_gpu, lse_gpu):
+    o_ref, lse_ref = O.attend(q, Kf, Vf, tokens)
+    vmax = float(np.max(np.abs(Vf[tokens]))) if len(tokens) else 1.0
+    do = float(np.max(np.abs(o_gpu - o_ref)))
+    dl = abs(float(lse_gpu) - lse_ref)
+    return do, dl, vmax, lse_ref
+
+
+def derived_o_bound(vmax: float) -> float:
+    return O_DERIVED_REL * vmax + 2e-6
+
+
+def derived_lse_bound(lse_ref: float) -> float:
+    return O_DERIVED_REL * max(1.0, abs(lse_ref))

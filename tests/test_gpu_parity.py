@@ -1,0 +1,299 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Every case draws seeded inputs, runs build -> route -> sparse attend on the GPU
+and checks, against the oracle on the same bytes:
+  * every summary of every level (norm-wise relative 1e-4);
+  * the kept set of every level of every query head, the level conditioned on
+    the GPU's kept set one level up; disagreements are allowed only as ties
+    (score within 1e-5 of the cut, or cumulative mass within 1e-5 of p), which
+    are counted and reported;
+  * the attention output and log-normaliser over the GPU's leaf set (absolute
+    2e-2 bf16 / 1e-4 fp32, and a tighter fp32-accumulation bound).
+Small cases are checked exhaustively; the full-size workloads on sampled nodes
+and heads (the oracle computes those one by one).
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from hierarchical_sparse_attention_zha_b200 import workloads as W
+from _parity import (O_ATOL, SUMMARY_RTOL, RouteReport, attend_errors, cache_f64, compare_route_head,
+                     config_for, derived_lse_bound, derived_o_bound, kept_from_bits, summary_errors,
+                     to_device, values_f64)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def zha():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from hierarchical_sparse_attention_zha_b200 import zha as z
+    return z
+
+
+def run_pipeline(zha, inp, n_tokens, p=None, max_sel=None, batch_index=0, stream=None):
+    spec = inp.spec
+    K, V, refq, Q = to_device(inp)
+    cfg = config_for(spec)
+    tree = zha.Tree(cfg, refq)
+    tree.build(K, n_tokens, stream=stream)
+    q = Q[batch_index].contiguous()
+    B = q.shape[0]
+    p = spec.p if p is None else p
+    max_sel = max_sel or max(1, n_tokens // spec.chunk)
+    bits = torch.zeros(zha.route_kept_words(cfg, B, n_tokens) + 1, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ids, cnt = tree.route(q, n_tokens, p, max_sel, kept_bits=bits, status=status, stream=stream)
+    out, lse = tree.sparse_attend(q, K, V, n_tokens, ids, cnt, status=status, stream=stream)
+    torch.cuda.synchronize()
+    return dict(tree=tree, K=K, V=V, Q=q, ids=ids.cpu().numpy(), cnt=cnt.cpu().numpy(),
+                bits=bits.cpu().numpy().view(np.uint32), out=out.cpu().numpy().astype(np.float64),
+                lse=lse.cpu().numpy().astype(np.float64), status=int(status.item()), p=p)
+
+
+def check_case(zha, inp, n_tokens, p=None, heads=None, all_nodes=True, batch_index=0):
+    """Full comparison; returns the route report."""
+    spec = inp.spec
+    res = run_pipeline(zha, inp, n_tokens, p=p, batch_index=batch_index)
+    p = res["p"]
+    assert res["status"] == 0
+    G = spec.group
+    B = spec.batch
+    kept = kept_from_bits(res["bits"], spec, B, n_tokens)
+    report = RouteReport()
+    for g in range(spec.n_kv_heads):
+        Kf = cache_f64(inp, g, n_tokens)
+        Vf = values_f64(inp, g, n_tokens)
+        otree = O.build_tree(Kf, inp.ref_q[g], spec.chunk, spec.levels, n_tokens)
+        # summaries, every level
+        for lvl in range(1, spec.levels + 1):
+            n_l = otree.n_nodes(lvl)
+            if n_l == 0:
+                continue
+            kh, bh = res["tree"].level(lvl)
+            kh = kh[g, :n_l].cpu().numpy().astype(np.float64)
+            bh = bh[g, :n_l].cpu().numpy().astype(np.float64)
+            ek, eb = summary_errors(kh, bh, *otree.nodes[lvl])
+            assert ek <= SUMMARY_RTOL and eb <= SUMMARY_RTOL, (g, lvl, ek, eb)
+        for b in range(B):
+            for h in range(g * G, (g + 1) * G):
+                if heads is not None and (b, h) not in heads:
+                    continue
+                q = inp.Q[batch_index, b, h].astype(np.float64)
+                gpu_kept = {lvl: kept[lvl][(b, h)] for lvl in kept}
+                compare_route_head(q, otree, p, gpu_kept, report, (b, h))
+                # the chunk list equals the level-1 bitmap, ascending
+                n = int(res["cnt"][b, h])
+                assert list(res["ids"][b, h, :n]) == list(gpu_kept[1])
+                S = O.leaf_token_set(res["ids"][b, h, :n], spec.chunk, n_tokens)
+                do, dl, vmax, lse_ref = attend_errors(q, Kf, Vf, S, res["out"][b, h], res["lse"][b, h])
+                assert do <= O_ATOL[spec.kv_dtype], (b, h, do)
+                assert do <= derived_o_bound(vmax), (b, h, do, vmax)
+                assert dl <= derived_lse_bound(lse_ref), (b, h, dl, lse_ref)
+    assert not report.hard, report.hard[:10]
+    return report
+
+
+# ---------------------------------------------------------------------------
+# Small and mid-size cases, exhaustively compared
+# ---------------------------------------------------------------------------
+
+CASES = {
+    "tiny": (W.WORKLOADS["tiny"], 4096),
+    "tiny_ragged": (W.WORKLOADS["tiny"], 4091),
+    "32k": (W.WORKLOADS["32k"], 32768),
+    "256k_small": (W.scaled("256k", n_kv_heads=2, n_q_heads=8, n_tokens=65536, stream_tokens=64), 65536 + 37),
+    "deep_small": (W.scaled("deep", n_kv_heads=2, n_q_heads=8, n_tokens=16384, stream_tokens=16), 16384 + 9),
+    "1m_small": (W.scaled("1m", n_kv_heads=1, n_q_heads=8, n_tokens=262144, stream_tokens=128,
+                          n_needles=4), 262144 + 100),
+}
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_parity_small_and_mid(zha, name):
+    spec, n_tokens = CASES[name]
+    inp = W.generate(spec)
+    rep = check_case(zha, inp, n_tokens)
+    print(f"{name}: heads {rep.heads} levels {rep.levels_compared} ties {rep.ties} "
+          f"exact heads {len(rep.exact_heads)}")
+    assert rep.heads == spec.batch * spec.n_q_heads
+
+
+@pytest.mark.parametrize("n_tokens", [1, 3, 4, 5, 15, 16, 17, 63, 64, 65, 83, 200, 257])
+def test_edge_token_counts(zha, n_tokens):
+    """C=4, L=3: no chunk, only a tail, exact chunk boundaries, orphans at every level."""
+    spec = W.scaled("tiny", chunk=4, levels=3, n_tokens=260, n_needles=0, batch=3)
+    inp = W.generate(spec)
+    check_case(zha, inp, n_tokens)
+
+
+@pytest.mark.parametrize("p", [1e-6, 0.3, 0.999])
+def test_extreme_p(zha, p):
+    spec = W.scaled("tiny", n_tokens=2048, n_needles=2, batch=4)
+    check_case(zha, W.generate(spec), 2048 - 3, p=p)
+
+
+@pytest.mark.parametrize("name", ["tiny_ragged", "256k_small"])
+def test_p1_routes_everything_and_equals_dense_attention(zha, name):
+    spec, n_tokens = CASES[name]
+    if spec.n_kv_heads > 1:
+        spec = W.scaled(spec, n_kv_heads=1, n_q_heads=spec.group)
+    inp = W.generate(spec)
+    res = run_pipeline(zha, inp, n_tokens, p=1.0)
+    nb = spec.chunk * (n_tokens // spec.chunk)
+    for b in range(spec.batch):
+        for h in range(spec.n_q_heads):
+            assert list(res["ids"][b, h, : res["cnt"][b, h]]) == list(range(nb // spec.chunk))
+            Kf, Vf = cache_f64(inp, 0, n_tokens), values_f64(inp, 0, n_tokens)
+            q = inp.Q[0, b, h].astype(np.float64)
+            _, dense = O.sdpa(q[None], Kf, Vf)
+            assert np.max(np.abs(res["out"][b, h] - dense[0])) <= O_ATOL[spec.kv_dtype]
+            assert np.max(np.abs(res["out"][b, h] - dense[0])) <= derived_o_bound(np.abs(Vf).max())
+
+
+def test_selection_overflow_is_flagged_and_truncated(zha):
+    spec = W.scaled("deep", n_kv_heads=1, n_q_heads=4, n_tokens=4096, batch=2)
+    inp = W.generate(spec)
+    full = run_pipeline(zha, inp, 4096)
+    small = run_pipeline(zha, inp, 4096, max_sel=3)
+    assert small["status"] & zha.ZHA_DEV_SELECTION_TRUNCATED
+    assert np.array_equal(small["cnt"], full["cnt"])
+    assert np.array_equal(small["ids"][..., :3], full["ids"][..., :3])
+
+
+def test_bad_external_selection_is_flagged_not_fatal(zha):
+    spec = W.scaled("tiny", n_tokens=1024, n_needles=0, batch=2)
+    inp = W.generate(spec)
+    K, V, refq, Q = to_device(inp)
+    cfg = config_for(spec)
+    tree = zha.Tree(cfg, refq)
+    tree.build(K, 1024)
+    q = Q[0].contiguous()
+    ids = torch.tensor([[[5, 3, 70, -1]] * 4] * 2, dtype=torch.int32, device="cuda")
+    cnt = torch.full((2, 4), 4, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = tree.sparse_attend(q, K, V, 1024, ids, cnt, status=status)
+    torch.cuda.synchronize()
+    assert status.item() & zha.ZHA_DEV_BAD_SELECTION
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+
+
+def test_external_selection_parity(zha):
+    """sparse_attend on oracle-chosen chunk lists (random sorted subsets)."""
+    spec = W.scaled("32k", n_kv_heads=2, n_q_heads=8, n_tokens=8192 + 64)
+    inp = W.generate(spec)
+    K, V, refq, Q = to_device(inp)
+    tree = zha.Tree(config_for(spec), refq)
+    n_tokens = 8192 + 40
+    rng = np.random.default_rng(11)
+    n_ch = n_tokens // spec.chunk
+    max_sel = 40
+    ids = np.full((spec.batch, spec.n_q_heads, max_sel), -7, np.int32)
+    cnt = np.zeros((spec.batch, spec.n_q_heads), np.int32)
+    for b in range(spec.batch):
+        for h in range(spec.n_q_heads):
+            k = int(rng.integers(0, max_sel + 1))
+            sel = np.sort(rng.choice(n_ch, size=k, replace=False))
+            ids[b, h, :k] = sel
+            cnt[b, h] = k
+    out, lse = tree.sparse_attend(Q[0].contiguous(), K, V, n_tokens,
+                                  torch.from_numpy(ids).cuda(), torch.from_numpy(cnt).cuda())
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    for b in range(spec.batch):
+        for h in range(spec.n_q_heads):
+            g = h // spec.group
+            S = O.leaf_token_set(ids[b, h, : cnt[b, h]], spec.chunk, n_tokens)
+            do, dl, vmax, lse_ref = attend_errors(inp.Q[0, b, h].astype(np.float64),
+                                                  cache_f64(inp, g, n_tokens), values_f64(inp, g, n_tokens),
+                                                  S, out[b, h], lse[b, h])
+            assert do <= derived_o_bound(vmax) and dl <= derived_lse_bound(lse_ref)
+
+
+def test_append_matches_a_fresh_build_and_the_oracle(zha):
+    spec = W.scaled("tiny", chunk=4, levels=3, n_tokens=300, n_needles=0, batch=2, stream_tokens=0)
+    inp = W.generate(spec)
+    K, V, refq, Q = to_device(inp)
+    cfg = config_for(spec)
+    inc = zha.Tree(cfg, refq)
+    inc.build(K, 37)
+    for n in range(38, 300):
+        inc.append_chunk(K, n)            # summarises chunks as they complete
+    assert inc.built_tokens == 296
+    big = zha.Tree(cfg, refq)
+    big.build(K, 40)
+    big.append_chunk(K, 299)              # many chunks at once: the bulk path
+    fresh = zha.Tree(cfg, refq)
+    fresh.build(K, 299)
+    torch.cuda.synchronize()
+    otree = O.build_tree(inp.K[0].astype(np.float64), inp.ref_q[0], 4, 3, 299)
+    for lvl in (1, 2, 3):
+        n_l = 296 // 4 ** lvl
+        for t in (inc, big):
+            assert torch.equal(t.level(lvl)[0][:, :n_l], fresh.level(lvl)[0][:, :n_l])
+            assert torch.equal(t.level(lvl)[1][:, :n_l], fresh.level(lvl)[1][:, :n_l])
+        kh, bh = fresh.level(lvl)
+        ek, eb = summary_errors(kh[0, :n_l].cpu().numpy(), bh[0, :n_l].cpu().numpy(), *otree.nodes[lvl])
+        assert ek <= SUMMARY_RTOL and eb <= SUMMARY_RTOL
+    with pytest.raises(zha.ZhaError) as e:
+        inc.append_chunk(K, 200)
+    assert e.value.status == zha.ZHA_ERR_STATE
+
+
+def test_deterministic_and_stream_ordered(zha):
+    spec = W.scaled("256k", n_kv_heads=1, n_q_heads=4, n_tokens=16384)
+    inp = W.generate(spec)
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        a = run_pipeline(zha, inp, 16384 - 5, stream=s)
+        b = run_pipeline(zha, inp, 16384 - 5, stream=s)
+    for k in ("ids", "cnt", "bits", "out", "lse"):
+        assert np.array_equal(a[k], b[k]), k
+
+
+# ---------------------------------------------------------------------------
+# Full-size workloads: sampled nodes and heads
+# ---------------------------------------------------------------------------
+
+@pytest.mark.slow
+@pytest.mark.parametrize("key", ["32k", "256k", "deep", "1m"])
+def test_parity_full_size_sampled(zha, key):
+    spec = W.WORKLOADS[key]
+    inp = W.generate(spec)
+    n_tokens = spec.n_tokens
+    res = run_pipeline(zha, inp, n_tokens)
+    assert res["status"] == 0
+    rng = np.random.default_rng(5)
+    G, C = spec.group, spec.chunk
+    g = int(rng.integers(spec.n_kv_heads))
+    Kf = cache_f64(inp, g, n_tokens)
+    Vf = values_f64(inp, g, n_tokens)
+    # sampled summaries of every level vs the direct summary of the raw keys under them
+    for lvl in range(1, spec.levels + 1):
+        n_l = n_tokens // C ** lvl
+        kh, bh = res["tree"].level(lvl)
+        for i in rng.choice(n_l, size=min(n_l, 16 if lvl > 1 else 64), replace=False):
+            span = C ** lvl
+            kd, bd = O.summarise_chunk(inp.ref_q[g], Kf[i * span:(i + 1) * span])
+            ek, eb = summary_errors(kh[g, i].cpu().numpy()[None], bh[g, i].cpu().numpy()[None],
+                                    kd[None], bd[None])
+            assert ek <= SUMMARY_RTOL and eb <= SUMMARY_RTOL, (lvl, i, ek, eb)
+    # routing and attention of sampled heads of KV head g
+    otree = O.build_tree(Kf, inp.ref_q[g], C, spec.levels, n_tokens)
+    kept = kept_from_bits(res["bits"], spec, spec.batch, n_tokens)
+    report = RouteReport()
+    for _ in range(4):
+        b, h = int(rng.integers(spec.batch)), g * G + int(rng.integers(G))
+        q = inp.Q[0, b, h].astype(np.float64)
+        compare_route_head(q, otree, spec.p, {l: kept[l][(b, h)] for l in kept}, report, (b, h))
+        n = int(res["cnt"][b, h])
+        S = O.leaf_token_set(res["ids"][b, h, :n], C, n_tokens)
+        do, dl, vmax, lse_ref = attend_errors(q, Kf, Vf, S, res["out"][b, h], res["lse"][b, h])
+        assert do <= O_ATOL[spec.kv_dtype] and do <= derived_o_bound(vmax), (b, h, do)
+        assert dl <= derived_lse_bound(lse_ref), (b, h, dl)
+    assert not report.hard, report.hard[:10]
+    print(f"{key}: sampled heads {report.heads} ties {report.ties}")
