@@ -24,15 +24,6 @@ cudaError_t launch_attend(const Geom& G, const float* Q, const void* K, const vo
                           cudaStream_t s);
 }  // namespace zha
 
-struct zha_tree {
-  zha_config cfg;
-  zha::Geom geom;
-  float* store;
-  size_t store_bytes;
-  const float* ref_q;
-  int64_t nb;  // tokens covered by complete level-1 chunks
-};
-
 static std::atomic<uint64_t> g_launches{0};
 void zha_count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
@@ -47,6 +38,8 @@ static zha_status fail(zha_status s, const char* fmt, ...) {
   g_err = buf;
   return s;
 }
+
+zha_status zha_report_error(zha_status s, const char* msg) { return fail(s, "%s", msg); }
 
 static zha_status cuda_fail(cudaError_t e, const char* where) {
   return fail(ZHA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));

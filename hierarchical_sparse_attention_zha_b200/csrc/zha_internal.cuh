@@ -173,7 +173,23 @@ __device__ __forceinline__ float order_key_float(uint32_t k) {
   return __uint_as_float(u);
 }
 
+cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n_tokens, float p,
+                         int32_t* chunk_ids, int32_t* n_chunks, int32_t max_sel, uint32_t* bits,
+                         float* sigma, int32_t* kp, const RouteLayout& lay, int32_t* status,
+                         const float* store, cudaStream_t s);
+
 }  // namespace zha
 
-// Launch bookkeeping shared by the host wrappers.
+// The host handle behind the opaque zha_tree of the C ABI.
+struct zha_tree {
+  zha_config cfg;
+  zha::Geom geom;
+  float* store;
+  size_t store_bytes;
+  const float* ref_q;
+  int64_t nb;  // tokens covered by complete level-1 chunks
+};
+
+// Launch bookkeeping and error reporting shared by the host wrappers.
 void zha_count_launch();
+zha_status zha_report_error(zha_status s, const char* msg);

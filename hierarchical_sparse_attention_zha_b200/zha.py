@@ -67,6 +67,7 @@ def _load() -> ctypes.CDLL:
         "zha_route_kept_words": (c_size_t, [POINTER(Config), c_int32, c_int64]),
         "zha_route": (c_int32, [P, P, c_int32, c_int64, c_float, P, P, c_int32, P, P, c_size_t,
                                 P, P]),
+        "zha_route_noalloc": (c_int32, [P, P, c_int32, c_int64, c_float, P, P, c_int32, P, P, P]),
         "zha_attend_workspace_bytes": (c_size_t, [POINTER(Config), c_int32, c_int64]),
         "zha_sparse_attend": (c_int32, [P, P, P, P, c_int64, c_int64, c_int32, P, P, c_int32, P,
                                         P, P, c_size_t, P, P]),

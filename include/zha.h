@@ -163,6 +163,37 @@ zha_status zha_route(const zha_tree* tree, const float* d_Q, int32_t batch, int6
                      uint32_t* d_kept_bits, void* d_ws, size_t ws_bytes, int32_t* d_status,
                      void* stream);
 
+/* Size of the routing scratch built into the library for zha_route_noalloc. */
+#define ZHA_ROUTE_NOALLOC_SCRATCH_BYTES (32u << 20) /* 32 MiB per GPU that loads the library */
+
+/* zha_route for callers that cannot allocate device memory. A plugin inside an
+ * inference server that owns all device memory may be forbidden to call
+ * cudaMalloc; a serving loop with a fixed memory plan cannot allocate per
+ * request; a plain C host program may have no device allocator at all. Such
+ * callers still pass Q, the outputs, d_kept_bits (nullable) and d_status, as
+ * for zha_route, and get the same results, but the scratch zha_route would take
+ * as d_ws lives in one fixed device array inside the library
+ * (ZHA_ROUTE_NOALLOC_SCRATCH_BYTES, held by every GPU that loads the library
+ * until the process exits). This entry point calls no cudaMalloc, cudaFree or
+ * other allocating routine.
+ *  - A call that needs more scratch than that (zha_route_workspace_bytes, less
+ *    the kept bitmaps when d_kept_bits is given) returns ZHA_ERR_CAPACITY and
+ *    launches nothing; use zha_route with a workspace then.
+ *  - The first call on each device looks up the array's device address (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents (nothing in it needs to start at zero: every call clears or
+ *    writes what it reads). Calls whose kernels overlap on the GPU -- on
+ *    different streams, or from different threads without ordering -- race on
+ *    it; order them.
+ * The pages have no counterpart of this call: it only changes where the
+ * scratch of zha_route lives. */
+zha_status zha_route_noalloc(const zha_tree* tree, const float* d_Q, int32_t batch,
+                             int64_t n_tokens, float p, int32_t* d_chunk_ids, int32_t* d_n_chunks,
+                             int32_t max_sel, uint32_t* d_kept_bits, int32_t* d_status,
+                             void* stream);
+
 /* Workspace bytes zha_sparse_attend needs for `batch` queries at n_tokens. */
 size_t zha_attend_workspace_bytes(const zha_config* cfg, int32_t batch, int64_t n_tokens);
 
