@@ -16,7 +16,9 @@
 // heads selected inside the range, streams them once through shared memory and
 // updates a per-head online-softmax state for the heads that selected each
 // chunk. One more CTA per (KV head, block) covers the tail [N_b, N) and the
-// sink. combine_kernel merges a head's range states in ascending order.
+// sink. The range states are merged by combine_ranges_kernel (zha_attend_tc.cu).
+// This CUDA-core kernel serves fp32 caches and head_dim 64; bf16 caches with
+// head_dim 128 go to the tensor-core kernel in zha_attend_tc.cu.
 #include "zha_internal.cuh"
 
 namespace zha {
@@ -24,7 +26,15 @@ namespace zha {
 constexpr int kAttThreads = 256;
 constexpr int kAttQ = 32;       // query heads per CTA
 constexpr int kAttT = 64;       // tokens per tile
-constexpr int kCombineWarps = 4;
+
+cudaError_t launch_combine(const Geom& G, int32_t batch, const int32_t* chunk_ids,
+                           const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
+                           const float* partial, const AttendLayout& lay, int32_t* status,
+                           cudaStream_t s);
+cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const void* V, int64_t ld,
+                             int64_t n_tokens, int32_t batch, const int32_t* chunk_ids,
+                             const int32_t* n_chunks, int32_t max_sel, float* partial,
+                             const AttendLayout& lay, int32_t* status, cudaStream_t s);
 
 template <int D>
 __host__ __device__ inline size_t attend_smem_bytes(int range_chunks) {
@@ -286,65 +296,6 @@ attend_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const float* 
   }
 }
 
-// One warp per query head: merge its range states (ascending) and the tail state.
-template <int D>
-__global__ void __launch_bounds__(kCombineWarps * 32)
-combine_kernel(Geom G, int32_t batch, int64_t n_chunk_total, const int32_t* __restrict__ chunk_ids,
-               const int32_t* __restrict__ n_chunks, int32_t max_sel, int32_t range_chunks,
-               int64_t n_ranges, const float* __restrict__ partial, int64_t slots_per_head,
-               float* __restrict__ O, float* __restrict__ lse, int32_t* status) {
-  constexpr int EPL = D / 32;
-  const int lane = threadIdx.x & 31;
-  const int64_t bh = int64_t(blockIdx.x) * kCombineWarps + (threadIdx.x >> 5);
-  if (bh >= int64_t(batch) * G.hq) return;
-  int n = n_chunks[bh];
-  bool bad = n < 0 || n > max_sel;
-  n = max(0, min(n, max_sel));
-  const int32_t* list = chunk_ids + bh * max_sel;
-  float M = -INFINITY, L = 0.f, acc[EPL] = {};
-  auto merge = [&](int64_t rho) {
-    const float* slot = partial + (bh * slots_per_head + rho) * (D + 4);
-    const float ms = slot[0], ls = slot[1];
-    if (!(ls > 0.f)) return;
-    float o[EPL];
-    load_slice<EPL>(slot + 4, EPL * lane, o);
-    const float mn = fmaxf(M, ms);
-    const float a = expf(M - mn), b = expf(ms - mn);
-    L = L * a + ls * b;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e) acc[e] = acc[e] * a + o[e] * b;
-    M = mn;
-  };
-  int64_t prev_id = -1;
-  for (int base = 0; base < n; base += 32) {
-    const int i = base + lane;
-    const int64_t id = i < n ? int64_t(list[i]) : -1;
-    const int64_t before = __shfl_up_sync(0xffffffffu, id, 1);
-    const int64_t pid = lane == 0 ? prev_id : before;
-    const bool valid = i < n && id >= 0 && id < n_chunk_total && id > pid;
-    if (i < n && !valid) bad = true;
-    const bool starts = valid && (pid < 0 || id / range_chunks != pid / range_chunks);
-    unsigned ball = __ballot_sync(0xffffffffu, starts);
-    while (ball) {
-      const int src = __ffs(ball) - 1;
-      ball &= ball - 1u;
-      const int64_t cid = __shfl_sync(0xffffffffu, id, src);
-      merge(cid / range_chunks);
-    }
-    prev_id = __shfl_sync(0xffffffffu, id, 31);
-    if (base + 32 > n) prev_id = -1;
-  }
-  merge(n_ranges);
-  bad = __any_sync(0xffffffffu, bad);
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-#pragma unroll
-  for (int e = 0; e < EPL; ++e) O[bh * D + EPL * lane + e] = acc[e] * inv;
-  if (lane == 0) {
-    if (lse != nullptr) lse[bh] = L > 0.f ? M + logf(L) : -INFINITY;
-    if (bad && status != nullptr) atomicOr(status, ZHA_DEV_BAD_SELECTION);
-  }
-}
-
 template <typename T, int D>
 static cudaError_t launch_attend_t(const Geom& G, const float* Q, const void* K, const void* V,
                                    int64_t ld, int64_t n_tokens, int32_t batch,
@@ -363,12 +314,7 @@ static cudaError_t launch_attend_t(const Geom& G, const float* Q, const void* K,
       n_chunks, max_sel, lay.range_chunks, lay.n_ranges, partial, lay.slots_per_head);
   zha_count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const int64_t heads = int64_t(batch) * G.hq;
-  combine_kernel<D><<<unsigned((heads + kCombineWarps - 1) / kCombineWarps), kCombineWarps * 32, 0,
-                      s>>>(G, batch, lay.n_chunks, chunk_ids, n_chunks, max_sel, lay.range_chunks,
-                           lay.n_ranges, partial, lay.slots_per_head, O, lse, status);
-  zha_count_launch();
-  return cudaGetLastError();
+  return launch_combine(G, batch, chunk_ids, n_chunks, max_sel, O, lse, partial, lay, status, s);
 }
 
 cudaError_t launch_attend(const Geom& G, const float* Q, const void* K, const void* V, int64_t ld,
@@ -376,6 +322,13 @@ cudaError_t launch_attend(const Geom& G, const float* Q, const void* K, const vo
                           const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
                           float* partial, const AttendLayout& lay, int32_t* status,
                           cudaStream_t s) {
+  if (G.kv_bf16 && G.d == 128) {
+    // bf16 caches with d = 128: the tensor-core kernel.
+    cudaError_t e = launch_attend_tc(G, Q, K, V, ld, n_tokens, batch, chunk_ids, n_chunks, max_sel,
+                                     partial, lay, status, s);
+    if (e != cudaSuccess) return e;
+    return launch_combine(G, batch, chunk_ids, n_chunks, max_sel, O, lse, partial, lay, status, s);
+  }
   if (G.kv_bf16)
     return G.d == 128 ? launch_attend_t<__nv_bfloat16, 128>(G, Q, K, V, ld, n_tokens, batch,
                                                             chunk_ids, n_chunks, max_sel, O, lse,

@@ -27,6 +27,7 @@ ZHA_F32 = 0
 ZHA_BF16 = 1
 ZHA_DEV_SELECTION_TRUNCATED = 1
 ZHA_DEV_BAD_SELECTION = 2
+ZHA_DEV_TIMEOUT = 4
 
 
 class ZhaError(RuntimeError):

@@ -59,6 +59,7 @@ typedef enum {
 /* Bits OR-ed into *d_status by device code. */
 #define ZHA_DEV_SELECTION_TRUNCATED 1 /* zha_route: a head kept more than max_sel chunks; its list holds the first max_sel (ascending) and d_n_chunks the true count */
 #define ZHA_DEV_BAD_SELECTION 2       /* zha_sparse_attend: a chunk list had an id out of range, was not strictly ascending, or a count above max_sel; the offending entries were skipped */
+#define ZHA_DEV_TIMEOUT 4             /* a kernel's bounded wait for its tensor-core work ran out; its outputs are not valid (it released its resources and returned) */
 
 typedef enum { ZHA_F32 = 0, ZHA_BF16 = 1 } zha_dtype;
 
@@ -205,7 +206,8 @@ size_t zha_attend_workspace_bytes(const zha_config* cfg, int32_t batch, int64_t 
  * supplies only its configuration (its summaries are not read). Output d_O
  * [batch][n_q_heads][d] float32 and, if d_lse is not NULL, d_lse
  * [batch][n_q_heads] = log sum_{j in S} exp(q.k_j/sqrt(d)). d_ws: >=
- * zha_attend_workspace_bytes bytes. d_status (nullable): ZHA_DEV_BAD_SELECTION.
+ * zha_attend_workspace_bytes bytes. d_status (nullable): ZHA_DEV_BAD_SELECTION,
+ * ZHA_DEV_TIMEOUT.
  * Requires 1 <= n_tokens <= ld. */
 zha_status zha_sparse_attend(const zha_tree* tree, const float* d_Q, const void* d_K,
                              const void* d_V, int64_t ld, int64_t n_tokens, int32_t batch,
