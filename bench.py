@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--impl", default="zha", choices=["zha", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--context", type=int, default=0,
+                    help="override the workload's context length (profiling runs)")
+    ap.add_argument("--flush-mb", type=int, default=512, help="L2 flush buffer between steps")
     return ap.parse_args()
 
 
@@ -303,6 +306,8 @@ def run_zha(args, world, rank, local):
     K_steps, W_steps = args.steps, args.warmup
     n_e2e = 0 if args.no_e2e else min(K_steps, 64)
     total_steps = W_steps + K_steps + n_e2e
+    if args.context:
+        base = W.scaled(base, n_tokens=args.context)
     spec = W.scaled(base, stream_tokens=-(-(total_steps + 2) // base.chunk) * base.chunk)
     t_gen = time.perf_counter()
     inp = W.generate(spec, n_batches=total_steps, rank=rank)
@@ -346,7 +351,7 @@ def run_zha(args, world, rank, local):
     out = torch.empty(B, spec.n_q_heads, spec.head_dim, dtype=torch.float32, device=dev)
     lse = torch.empty(B, spec.n_q_heads, dtype=torch.float32, device=dev)
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    flush = torch.empty(max(1, args.flush_mb) << 20, dtype=torch.uint8, device=dev)
 
     def step(s, n_tok, ev=None):
         if ev is not None:
@@ -476,7 +481,7 @@ def run_zha(args, world, rank, local):
             "data": "synthetic (seeded generators; see DESIGN.md)",
             "config": {"workload": spec.name, **base.describe(), "decode_from": N0,
                        "steps_context": [positions[0], positions[-1]],
-                       "l2": "flushed between timed steps (512 MiB memset outside the events)",
+                       "l2": f"flushed between timed steps ({args.flush_mb} MiB memset outside the events)",
                        "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
                          "frac": ach / peak, "traffic": None, "kernel": dominant,

@@ -49,7 +49,7 @@ struct TcMisc {
   uint32_t any, mask0, nsel, err;
   float m[kTcQ], l[kTcQ], scale[kTcQ], mnew[kTcQ];
   float red[4][kTcQ];
-  uint32_t tmask[kTcTok];
+  uint32_t tmask[2][kTcTok];
   uint32_t scan[33];
 };
 
@@ -83,11 +83,26 @@ __device__ __forceinline__ int lower_bound_ids(const int32_t* a, int n, int64_t 
   return lo;
 }
 
+// Per query head: where each range's entries start in its chunk list, so
+// that the attention CTAs read two offsets instead of searching the list.
+__global__ void __launch_bounds__(128)
+attend_prep_kernel(const int32_t* __restrict__ chunk_ids, const int32_t* __restrict__ n_chunks,
+                   int32_t max_sel, int32_t range_chunks, int64_t n_ranges, int64_t n_chunk_total,
+                   int32_t* __restrict__ ptr, int64_t ptr_stride) {
+  const int64_t bh = blockIdx.x;
+  const int32_t* list = chunk_ids + bh * max_sel;
+  const int n = max(0, min(n_chunks[bh], max_sel));
+  int32_t* out = ptr + bh * ptr_stride;
+  for (int64_t r = threadIdx.x; r <= n_ranges; r += blockDim.x)
+    out[r] = lower_bound_ids(list, n, r < n_ranges ? r * range_chunks : n_chunk_total);
+  if (threadIdx.x == 0) out[n_ranges + 1] = (n > 0 && list[0] == 0) ? 1 : 0;
+}
+
 __global__ void __launch_bounds__(kTcThreads, 2)
 attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const float* __restrict__ Q,
                  const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V, int64_t ld,
-                 const int32_t* __restrict__ chunk_ids, const int32_t* __restrict__ n_chunks,
-                 int32_t max_sel, int32_t range_chunks, int64_t n_ranges,
+                 const int32_t* __restrict__ chunk_ids, const int32_t* __restrict__ ptr,
+                 int64_t ptr_stride, int32_t max_sel, int32_t range_chunks, int64_t n_ranges,
                  float* __restrict__ partial, int64_t slots_per_head, int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -115,10 +130,10 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
   if (tid < nq) {
     const int qi = qb0 + tid;
     const int64_t bh = int64_t(qi / GQ) * G.hq + g * GQ + qi % GQ;
-    const int32_t* list = chunk_ids + bh * max_sel;
-    const int n = min(n_chunks[bh], max_sel);
+    const int32_t* pr = ptr + bh * ptr_stride;
     if (!tail) {
-      const int lo = lower_bound_ids(list, n, c_lo), hi = lower_bound_ids(list, n, c_hi);
+      const int32_t* list = chunk_ids + bh * max_sel;
+      const int lo = pr[rho], hi = pr[rho + 1];
       bool any = false;
       for (int i = lo; i < hi; ++i) {
         const int64_t c = list[i];
@@ -126,8 +141,7 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
       }
       if (any) atomicOr(&ms.any, 1u << tid);
     } else {
-      const bool has0 = n > 0 && list[0] == 0;
-      if (nb > 0 && !has0) atomicOr(&ms.mask0, 1u << tid);
+      if (nb > 0 && pr[n_ranges + 1] == 0) atomicOr(&ms.mask0, 1u << tid);
     }
   }
   __syncthreads();
@@ -164,6 +178,41 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
   } else {
     n_tok = (n_tokens - nb) + (ms.mask0 != 0u ? 1 : 0);
   }
+  const int n_tiles = int((n_tok + kTcTok - 1) / kTcTok);
+
+  // Token of row `row` in tile `tile` (row < tokens of the tile) and its head mask.
+  auto token_of = [&](int tile, int row, int64_t& tok, uint32_t& msk) {
+    const int64_t u = int64_t(tile) * kTcTok + row;
+    tok = 0;
+    msk = 0u;
+    if (u >= n_tok) return;
+    if (!tail) {
+      const uint32_t k = s_sel[u / C];
+      tok = (c_lo + k) * C + u % C;
+      msk = s_mask[k];
+    } else if (u < n_tokens - nb) {
+      tok = nb + u;
+      msk = all_q;
+    } else {
+      msk = ms.mask0;
+    }
+  };
+  // Row `tid` of tile `tile`: 16 x 16-byte pieces into the swizzled K (or V)
+  // staging, zero-filled past the last token; one cp.async group.
+  auto issue_rows = [&](int tile, bool is_v) {
+    int64_t tok;
+    uint32_t msk;
+    token_of(tile, tid, tok, msk);
+    if (!is_v) ms.tmask[tile & 1][tid] = msk;
+    const int64_t u = int64_t(tile) * kTcTok + tid;
+    const uint32_t bytes = u < n_tok ? 16u : 0u;
+    const __nv_bfloat16* row = (is_v ? V : K) + (int64_t(g) * ld + tok) * kTcD;
+    const uint32_t dst = is_v ? sV : sK;
+#pragma unroll
+    for (int j = 0; j < kTcD / 8; ++j)
+      tc::cp_async16(dst + tc::sw128_offset(tid, 8 * j, kTcTok), row + 8 * j, bytes);
+    tc::cp_async_commit();
+  };
 
   // Query block -> three bf16 terms, K-major rows (row = query head).
   for (int v = tid; v < kTcQ * (kTcD / 8); v += blockDim.x) {
@@ -194,6 +243,10 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
   if (tid < kTcQ) { ms.m[tid] = -INFINITY; ms.l[tid] = 0.f; }
   if (tid == 0) tc::mbar_init(&ms.mbar, 1);
   if (warp == 0) tc::tmem_alloc(&ms.tmem_base, 64);
+  if (n_tiles > 0) {        // first tile's K and V in flight during the set-up
+    issue_rows(0, false);
+    issue_rows(0, true);
+  }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -207,39 +260,12 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
   uint32_t phase = 0;
   bool failed = false;
 
-  for (int64_t t0 = 0; t0 < n_tok && !failed; t0 += kTcTok) {
-    const int nt = int(min64(kTcTok, n_tok - t0));
-    // Stage token row `tid` of K and V (16 x 16-byte pieces each), zero past nt.
-    {
-      const int row = tid;
-      int64_t tok = 0;
-      uint32_t msk = 0u;
-      if (row < nt) {
-        const int64_t u = t0 + row;
-        if (!tail) {
-          const uint32_t k = s_sel[u / C];
-          tok = (c_lo + k) * C + u % C;
-          msk = s_mask[k];
-        } else if (u < n_tokens - nb) {
-          tok = nb + u;
-          msk = all_q;
-        } else {
-          tok = 0;
-          msk = ms.mask0;
-        }
-      }
-      ms.tmask[row] = msk;
-      const __nv_bfloat16* krow = K + (int64_t(g) * ld + tok) * kTcD;
-      const __nv_bfloat16* vrow = V + (int64_t(g) * ld + tok) * kTcD;
-      const uint32_t bytes = row < nt ? 16u : 0u;
-#pragma unroll
-      for (int j = 0; j < kTcD / 8; ++j) {
-        const uint32_t off = tc::sw128_offset(row, 8 * j, kTcTok);
-        tc::cp_async16(sK + off, krow + 8 * j, bytes);
-        tc::cp_async16(sV + off, vrow + 8 * j, bytes);
-      }
-      tc::cp_async_wait_all();
-    }
+  // Pipeline: tile i's S MMA runs once its K rows have landed; tile i+1's K
+  // rows are requested as soon as that MMA has consumed the K staging, and
+  // its V rows once the P.V MMA of tile i has consumed the V staging.
+  for (int i = 0; i < n_tiles && !failed; ++i) {
+    const bool has_next = i + 1 < n_tiles;
+    tc::cp_async_wait_pending1();          // K_i done (V_i may still be in flight)
     tc::fence_async_smem();
     __syncthreads();
 
@@ -259,10 +285,11 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
     if (!tc::mbar_wait(&ms.mbar, phase, kTcWaitTries)) atomicOr(&ms.err, 1u);
     phase ^= 1u;
     tc::fence_after_sync();
+    if (has_next) issue_rows(i + 1, false);     // the K staging is free again
 
     float s[kTcQ];
     tc::tmem_ld32(tbase + t_lane, s);
-    const uint32_t tm = ms.tmask[tid];
+    const uint32_t tm = ms.tmask[i & 1][tid];
 #pragma unroll
     for (int q = 0; q < kTcQ; ++q) s[q] = ((tm >> q) & 1u) ? s[q] * G.scale : -INFINITY;
     {
@@ -293,10 +320,9 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
         *reinterpret_cast<__nv_bfloat16*>(smem + kOffP + off) = hi;
         *reinterpret_cast<__nv_bfloat16*>(smem + kOffP + 8192 + off) = lo;
       }
-      const float sum = transpose_reduce32<false>(v);
-      __syncthreads();            // every head's max was read before red[] is reused
-      ms.red[warp][lane] = sum;
+      ms.red[warp][lane] = transpose_reduce32<false>(v);
     }
+    if (has_next) tc::cp_async_wait_pending1(); else tc::cp_async_wait_pending0();   // V_i done
     tc::fence_async_smem();
     tc::fence_before_sync();
     __syncthreads();
@@ -320,6 +346,7 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
     if (!tc::mbar_wait(&ms.mbar, phase, kTcWaitTries)) atomicOr(&ms.err, 1u);
     phase ^= 1u;
     tc::fence_after_sync();
+    if (has_next) issue_rows(i + 1, true);      // the V staging is free again
     {
       float o[kTcQ];
       tc::tmem_ld32(tbase + t_lane + 32, o);
@@ -330,6 +357,7 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
     __syncthreads();
     failed = ms.err != 0u;
   }
+  tc::cp_async_wait_pending0();   // nothing of ours left in flight
 
   if (!failed) {
 #pragma unroll
@@ -494,11 +522,16 @@ cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const
   if (e != cudaSuccess) return e;
   const int64_t nb = int64_t(G.chunk) * (n_tokens / G.chunk);
   const int qn = batch * G.group;
+  int32_t* ptr = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(partial) + lay.ptr_offset_bytes);
+  attend_prep_kernel<<<unsigned(int64_t(batch) * G.hq), 128, 0, s>>>(
+      chunk_ids, n_chunks, max_sel, lay.range_chunks, lay.n_ranges, lay.n_chunks, ptr, lay.ptr_stride);
+  zha_count_launch();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   dim3 grid(unsigned(lay.n_ranges + 1), unsigned(G.hkv), unsigned((qn + kTcQ - 1) / kTcQ));
   attend_tc_kernel<<<grid, kTcThreads, smem, s>>>(
       G, batch, n_tokens, nb, Q, static_cast<const __nv_bfloat16*>(K),
-      static_cast<const __nv_bfloat16*>(V), ld, chunk_ids, n_chunks, max_sel, lay.range_chunks,
-      lay.n_ranges, partial, lay.slots_per_head, status);
+      static_cast<const __nv_bfloat16*>(V), ld, chunk_ids, ptr, lay.ptr_stride, max_sel,
+      lay.range_chunks, lay.n_ranges, partial, lay.slots_per_head, status);
   zha_count_launch();
   return cudaGetLastError();
 }

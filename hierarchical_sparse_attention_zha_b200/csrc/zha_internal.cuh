@@ -93,20 +93,27 @@ inline int32_t attend_range_chunks(int32_t chunk) {
   return w < 1 ? 1 : w;
 }
 
+// After the slots: per query head, the index in its chunk list of the first
+// entry of each range ([n_ranges + 1] int32, the last = end of the in-range
+// entries) plus one flag word (1 if the list starts with chunk 0).
 struct AttendLayout {
   int64_t n_chunks, n_ranges, slots_per_head, slot_floats, bytes;
+  int64_t ptr_offset_bytes, ptr_stride;
   int32_t range_chunks;
 };
 
 inline AttendLayout attend_layout(const Geom& g, int32_t batch, int64_t n_tokens) {
   AttendLayout a{};
   const int64_t nb = int64_t(g.chunk) * (n_tokens / g.chunk);
+  const int64_t heads = int64_t(batch) * g.hq;
   a.n_chunks = nb / g.chunk;
   a.range_chunks = attend_range_chunks(g.chunk);
   a.n_ranges = (a.n_chunks + a.range_chunks - 1) / a.range_chunks;
   a.slots_per_head = a.n_ranges + 1;
   a.slot_floats = g.d + 4;
-  a.bytes = round_up(int64_t(batch) * g.hq * a.slots_per_head * a.slot_floats * 4, 256);
+  a.ptr_offset_bytes = round_up(heads * a.slots_per_head * a.slot_floats * 4, 256);
+  a.ptr_stride = a.n_ranges + 2;
+  a.bytes = a.ptr_offset_bytes + round_up(heads * a.ptr_stride * 4, 256);
   return a;
 }
 

@@ -9,8 +9,9 @@
 //
 // Per level l = L..1 the host launches two kernels:
 //   score_kernel  -- one warp per candidate node (the union over the query heads
-//                    of a KV head), the node's R planes held in registers, one
-//                    score per query head that has the node as candidate;
+//                    of a KV head), the node's R planes held in registers (lane
+//                    = part of one plane's row), one score per query head that
+//                    has the node as candidate;
 //   select_kernel -- one CTA per query head: softmax over its candidates, radix
 //                    select of the cut on the key (score desc, node index asc)
 //                    with fixed-point mass histograms, kept bitmap (and at
@@ -20,7 +21,7 @@
 namespace zha {
 
 constexpr int kScoreThreads = 256;
-constexpr int kScoreTile = 32;       // nodes per score CTA
+constexpr int kScoreTile = 64;       // nodes per score CTA
 constexpr int kScoreQBlock = 64;     // query heads per score CTA (u64 masks)
 constexpr int kSelectThreads = 512;
 constexpr int kSelectCache = 16384;  // candidate scores cached in shared memory
@@ -32,48 +33,45 @@ constexpr double kMassScale = 1099511627776.0;  // 2^40: fixed-point unit of pro
 // n / C is kept by (b, h) at level l+1. sigma = max_r (q . khat_r / sqrt(d) + bhat_r).
 // ---------------------------------------------------------------------------
 
-// v[RP] partial sums per lane -> lane L holds the full sum of value L >> (5 - log2 RP).
-template <int RP>
-__device__ __forceinline__ float transpose_reduce(float (&v)[RP]) {
-  const int lane = threadIdx.x & 31;
-  int count = RP;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    if (count > 1) {
-      const int half = count >> 1;
-      const bool upper = (lane & o) != 0;
-#pragma unroll
-      for (int i = 0; i < RP / 2; ++i) {
-        if (i < half) {
-          const float send = upper ? v[i] : v[i + half];
-          const float keep = upper ? v[i + half] : v[i];
-          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-      }
-      count = half;
-    } else {
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
-    }
-  }
-  return v[0];
-}
+// Lane L of a warp holds part (L % P) of plane r = L / P of a node, P = 32 / RP
+// lanes per plane (RP = R rounded up to a power of two): EP = D / P
+// consecutive elements of khat_r. A query's score is then EP FMAs per lane,
+// log2(P) shuffles to finish each plane's dot product and log2(RP) shuffles for
+// the maximum over planes. Node records reach shared memory by coalesced
+// cp.async into a per-warp buffer whose rows and parts are padded so that the
+// lanes' reads in this mapping fall into distinct banks; each warp requests
+// its next node before it scores the current one.
+template <int D, int RP>
+struct ScoreShape {
+  static constexpr int P = 32 / RP;
+  static constexpr int EP = D / P;
+  static constexpr int QS = EP + 4;          // padded stride of one query part in shared memory
+  static constexpr int QROW = P * QS;        // floats per staged query
+  static constexpr int KROW = P * QS;        // floats per staged plane
+  static constexpr int KBUF = RP * KROW;     // floats per staged node (planes only)
+  static_assert(EP % 4 == 0, "each lane must hold whole float4s of its plane");
+};
 
-template <int RP>
-__device__ __forceinline__ int reduced_index() {
-  constexpr int LOG = RP == 1 ? 0 : RP == 2 ? 1 : RP == 4 ? 2 : RP == 8 ? 3 : RP == 16 ? 4 : 5;
-  return (threadIdx.x & 31) >> (5 - LOG);
+__device__ __forceinline__ void cp_async16_ca(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" : : "r"(dst), "l"(src) : "memory");
 }
 
 template <int D, int RP>
 __global__ void __launch_bounds__(kScoreThreads)
-score_kernel(Geom G, int level, int64_t n_nodes, int64_t n_par, int32_t batch,
+score_kernel(Geom G, int level, int64_t n_nodes, int64_t n_par, int32_t batch, int tile,
              const float* __restrict__ Q, const uint32_t* __restrict__ kept_up, int64_t words_up,
              float* __restrict__ sigma, const float* __restrict__ store) {
-  constexpr int EPL = D / 32;
+  using S = ScoreShape<D, RP>;
+  constexpr int NW = kScoreThreads / 32;
+  extern __shared__ float4 smem_v4[];
+  float* s_kbuf = reinterpret_cast<float*>(smem_v4);       // [NW][KBUF]
+  float* s_q = s_kbuf + NW * S::KBUF;                       // [nq][P][QS]
   __shared__ unsigned long long s_mask[kScoreTile];
-  __shared__ uint32_t s_kw[kScoreQBlock][2];
+  __shared__ uint32_t s_kw[kScoreQBlock][3];
+  __shared__ int64_t s_out[kScoreQBlock];
+  __shared__ unsigned long long s_any;
   const int g = blockIdx.y;
-  const int64_t n0 = int64_t(blockIdx.x) * kScoreTile;
+  const int64_t n0 = int64_t(blockIdx.x) * tile;
   const int GQ = G.group;
   const int qn_total = batch * GQ;
   const int qb0 = blockIdx.z * kScoreQBlock;
@@ -81,71 +79,110 @@ score_kernel(Geom G, int level, int64_t n_nodes, int64_t n_par, int32_t batch,
   const int C = G.chunk, R = G.nref;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t orphan0 = int64_t(C) * n_par;
-  const int64_t p_lo = n0 / C;
-  const int64_t w_lo = p_lo >> 5;
+  const int64_t w_lo = (n0 / C) >> 5;
 
-  if (tid < nq && n0 < orphan0) {
+  if (tid == 0) s_any = 0ull;
+  if (tid < nq) {
     const int qi = qb0 + tid;
-    const int b = qi / GQ, h = g * GQ + qi % GQ;
-    const uint32_t* kw = kept_up + (int64_t(b) * G.hq + h) * words_up;
-    s_kw[tid][0] = kw[w_lo];
-    s_kw[tid][1] = (w_lo + 1 < words_up) ? kw[w_lo + 1] : 0u;
+    const int64_t bh = int64_t(qi / GQ) * G.hq + g * GQ + qi % GQ;
+    s_out[tid] = bh * n_nodes;
+    if (n0 < orphan0) {
+      const uint32_t* kw = kept_up + bh * words_up;
+#pragma unroll
+      for (int k = 0; k < 3; ++k) s_kw[tid][k] = (w_lo + k < words_up) ? kw[w_lo + k] : 0u;
+    }
   }
   __syncthreads();
-  if (tid < kScoreTile) {
+  if (tid < tile) {
     const int64_t n = n0 + tid;
     unsigned long long m = 0ull;
     if (n < n_nodes) {
       if (n >= orphan0) {
         m = nq == 64 ? ~0ull : ((1ull << nq) - 1ull);
       } else {
-        const int64_t p = n / C;
-        const int slot = int((p >> 5) - w_lo);
-        const int bit = int(p & 31);
-        for (int s = 0; s < nq; ++s) m |= (unsigned long long)((s_kw[s][slot] >> bit) & 1u) << s;
+        const int64_t pnode = n / C;
+        const int slot = int((pnode >> 5) - w_lo);
+        const int bit = int(pnode & 31);
+        for (int q = 0; q < nq; ++q) m |= (unsigned long long)((s_kw[q][slot] >> bit) & 1u) << q;
       }
     }
     s_mask[tid] = m;
+    if (m) atomicOr(&s_any, m);
+  }
+  __syncthreads();
+  const unsigned long long any = s_any;
+  if (any == 0ull) return;
+  // Stage the rows of the query heads this tile needs, split in P parts.
+  for (int v = tid; v < nq * (D / 4); v += blockDim.x) {
+    const int q = v / (D / 4), e = (v % (D / 4)) * 4;
+    if (!((any >> q) & 1ull)) continue;
+    const int qi = qb0 + q;
+    const int64_t bh = int64_t(qi / GQ) * G.hq + g * GQ + qi % GQ;
+    const float4 x = *reinterpret_cast<const float4*>(Q + bh * D + e);
+    *reinterpret_cast<float4*>(s_q + q * S::QROW + (e / S::EP) * S::QS + e % S::EP) = x;
   }
   __syncthreads();
 
-  for (int t = warp; t < kScoreTile; t += kScoreThreads / 32) {
-    unsigned long long m = s_mask[t];
-    if (m == 0ull) continue;
+  float* kb = s_kbuf + warp * S::KBUF;
+  const uint32_t kb_s = static_cast<uint32_t>(__cvta_generic_to_shared(kb));
+  const float* level_base = store + G.off[level] + int64_t(g) * G.cap[level] * G.node_floats;
+  // Copy the planes of node n (R * D floats) into this warp's buffer.
+  auto stage = [&](int t) {
+    const float* rec = level_base + (n0 + t) * G.node_floats;
+    for (int c = lane; c < R * (D / 4); c += 32) {
+      const int e = 4 * c, r = e / D, col = e % D;
+      cp_async16_ca(kb_s + 4u * uint32_t(r * S::KROW + (col / S::EP) * S::QS + col % S::EP), rec + e);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  auto next_node = [&](int t) {
+    for (t += NW; t < tile; t += NW)
+      if (s_mask[t] != 0ull) return t;
+    return tile;
+  };
+
+  const int r = lane / S::P, part = lane % S::P;
+  const bool live = r < R;
+  int t = warp < tile && s_mask[warp] != 0ull ? warp : next_node(warp);
+  if (t < tile) stage(t);
+  while (t < tile) {
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncwarp();
+    float kr[S::EP];
+    if (live) {
+#pragma unroll
+      for (int e = 0; e < S::EP; e += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(kb + r * S::KROW + part * S::QS + e);
+        kr[e] = x.x; kr[e + 1] = x.y; kr[e + 2] = x.z; kr[e + 3] = x.w;
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < S::EP; ++e) kr[e] = 0.f;
+    }
     const int64_t n = n0 + t;
-    const float* rec = store + G.off[level] + (int64_t(g) * G.cap[level] + n) * G.node_floats;
-    float kr[RP][EPL];
-#pragma unroll
-    for (int r = 0; r < RP; ++r) {
-      if (r < R) {
-        load_slice<EPL>(rec + r * D, EPL * lane, kr[r]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) kr[r][e] = 0.f;
-      }
-    }
-    const int rl = reduced_index<RP>();
-    const float bl = rl < R ? rec[R * D + rl] : 0.f;
+    const float b = live ? __ldg(level_base + n * G.node_floats + R * D + r) : 0.f;
+    unsigned long long m = s_mask[t];
+    __syncwarp();
+    const int tn = next_node(t);
+    if (tn < tile) stage(tn);          // overlaps the scoring below
     while (m) {
-      const int s = __ffsll(m) - 1;
+      const int q = __ffsll(m) - 1;
       m &= m - 1ull;
-      const int qi = qb0 + s;
-      const int b = qi / GQ, h = g * GQ + qi % GQ;
-      float q[EPL];
-      load_slice<EPL>(Q + (int64_t(b) * G.hq + h) * D, EPL * lane, q);
-      float v[RP];
+      const float* qs = s_q + q * S::QROW + part * S::QS;
+      float dot = 0.f;
 #pragma unroll
-      for (int r = 0; r < RP; ++r) {
-        float a = 0.f;
-#pragma unroll
-        for (int e = 0; e < EPL; ++e) a += q[e] * kr[r][e];
-        v[r] = a;
+      for (int e = 0; e < S::EP; e += 4) {
+        const float4 x = *reinterpret_cast<const float4*>(qs + e);
+        dot += kr[e] * x.x + kr[e + 1] * x.y + kr[e + 2] * x.z + kr[e + 3] * x.w;
       }
-      const float dot = transpose_reduce<RP>(v);
-      const float tr = rl < R ? dot * G.scale + bl : -INFINITY;
-      const float sg = warp_max(tr);
-      if (lane == 0) sigma[(int64_t(b) * G.hq + h) * n_nodes + n] = sg;
+#pragma unroll
+      for (int o = 1; o < S::P; o <<= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      float tr = live ? dot * G.scale + b : -INFINITY;
+#pragma unroll
+      for (int o = S::P; o < 32; o <<= 1) tr = fmaxf(tr, __shfl_xor_sync(0xffffffffu, tr, o));
+      if (lane == 0) sigma[s_out[q] + n] = tr;
     }
+    t = tn;
   }
 }
 
@@ -420,11 +457,20 @@ static cudaError_t launch_score_t(const Geom& G, int level, int64_t n_nodes, int
                                   int32_t batch, const float* Q, const uint32_t* kept_up,
                                   int64_t words_up, float* sigma, const float* store,
                                   cudaStream_t s) {
+  using S = ScoreShape<D, RP>;
   const int qn = batch * G.group;
-  dim3 grid(unsigned((n_nodes + kScoreTile - 1) / kScoreTile), unsigned(G.hkv),
+  // Nodes per CTA: enough CTAs to fill the GPU twice over, at most kScoreTile.
+  int tile = kScoreTile;
+  while (tile > kScoreThreads / 32 && (n_nodes * G.hkv) / tile < 2 * 148) tile >>= 1;
+  dim3 grid(unsigned((n_nodes + tile - 1) / tile), unsigned(G.hkv),
             unsigned((qn + kScoreQBlock - 1) / kScoreQBlock));
-  score_kernel<D, RP><<<grid, kScoreThreads, 0, s>>>(G, level, n_nodes, n_par, batch, Q, kept_up,
-                                                     words_up, sigma, store);
+  const size_t smem = (size_t(kScoreThreads / 32) * S::KBUF +
+                       size_t(qn < kScoreQBlock ? qn : kScoreQBlock) * S::QROW) * 4;
+  cudaError_t e = cudaFuncSetAttribute(score_kernel<D, RP>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  score_kernel<D, RP><<<grid, kScoreThreads, smem, s>>>(G, level, n_nodes, n_par, batch, tile, Q,
+                                                        kept_up, words_up, sigma, store);
   zha_count_launch();
   return cudaGetLastError();
 }
@@ -434,12 +480,14 @@ static cudaError_t launch_score_d(const Geom& G, int level, int64_t n_nodes, int
                                   int32_t batch, const float* Q, const uint32_t* kept_up,
                                   int64_t words_up, float* sigma, const float* store,
                                   cudaStream_t s) {
+  // Planes are padded to a power of two RP >= 128 / D so that each lane holds
+  // at least one float4 of its plane's row.
   const int R = G.nref;
 #define ZHA_SCORE_CASE(RP)                                                                      \
-  if (R <= RP)                                                                                  \
+  if (R <= RP && RP * D >= 128)                                                                 \
     return launch_score_t<D, RP>(G, level, n_nodes, n_par, batch, Q, kept_up, words_up, sigma, \
                                  store, s);
-  ZHA_SCORE_CASE(1)
+  if constexpr (D >= 128) ZHA_SCORE_CASE(1)
   ZHA_SCORE_CASE(2)
   ZHA_SCORE_CASE(4)
   ZHA_SCORE_CASE(8)

@@ -127,8 +127,15 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" : : "r"(dst), "l"(src), "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// Wait until at most 1 (or 0) of this thread's committed groups is pending.
+__device__ __forceinline__ void cp_async_wait_pending1() {
+  asm volatile("cp.async.wait_group 1;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_pending0() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // Byte offset of element (row, col) of a bf16 tile stored as 128-byte-swizzled

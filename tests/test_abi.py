@@ -93,7 +93,9 @@ def test_route_workspace_and_kept_words_arithmetic(zha):
     assert zha.route_workspace_bytes(cfg, 4, 1000) < ws        # grows with n_tokens
     # attend: one slot per (head, range of 1024 tokens) plus the tail, d+4 floats each
     ranges = -(-(nb // 64) // 16)
-    assert zha.attend_workspace_bytes(cfg, 4, n) == -(-(heads * (ranges + 1) * 132 * 4) // 256) * 256
+    slots = -(-(heads * (ranges + 1) * 132 * 4) // 256) * 256
+    ptrs = -(-(heads * (ranges + 2) * 4) // 256) * 256       # per-range list offsets
+    assert zha.attend_workspace_bytes(cfg, 4, n) == slots + ptrs
 
 
 def test_host_checks_reject_before_any_launch(zha):

@@ -301,3 +301,13 @@ def test_parity_full_size_sampled(zha, key):
         assert dl <= derived_lse_bound(lse_ref), (b, h, dl)
     assert not report.hard, report.hard[:10]
     print(f"{key}: sampled heads {report.heads} ties {report.ties}")
+
+
+@pytest.mark.parametrize("n_ref,head_dim,kv", [(1, 64, "f32"), (3, 64, "f32"), (16, 64, "bf16"),
+                                               (32, 128, "bf16"), (1, 128, "bf16"), (7, 128, "f32")])
+def test_reference_query_counts_and_head_dims(zha, n_ref, head_dim, kv):
+    """Every plane-count / head-dim variant of the scoring kernel, and both
+    attention kernels (tensor cores for bf16 d=128, CUDA cores otherwise)."""
+    spec = W.scaled("tiny", n_ref=n_ref, head_dim=head_dim, kv_dtype=kv, n_kv_heads=2, n_q_heads=8,
+                    n_tokens=3000, chunk=8, levels=3, batch=5, n_needles=0)
+    check_case(zha, W.generate(spec), 2990)
