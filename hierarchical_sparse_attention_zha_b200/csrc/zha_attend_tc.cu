@@ -9,9 +9,10 @@
 // (page "ZHA는 KV 캐시를 트리로 요약해 어텐션 비용을 준(sub)이차로 낮춘다") token 0
 // and the in-progress chunk are always attended.
 //
-// One CTA = (range of W chunks, KV head, block of 32 query heads of that KV head),
-// 128 threads. The selected chunks of the range are streamed in tiles of 128
-// tokens. Per tile:
+// Work item = (range of W chunks, KV head, block of 32 query heads of that KV
+// head), built by attend_items_kernel; attend_tc_kernel is persistent (two
+// CTAs of 128 threads per SM take items from a queue). The selected chunks of
+// an item are streamed in tiles of 128 tokens. Per tile:
 //   S^T[tok][q] = K_tile . Q^T          tcgen05.mma, M=128 tokens, N=32 heads, K=d,
 //                                       Q split in three bf16 terms (fp32 accuracy),
 //                                       accumulator in TMEM columns [0, 32)
@@ -84,11 +85,12 @@ __device__ __forceinline__ int lower_bound_ids(const int32_t* a, int n, int64_t 
 }
 
 // Per query head: where each range's entries start in its chunk list, so
-// that the attention CTAs read two offsets instead of searching the list.
+// that the work-item pass reads two offsets instead of searching the list.
+// Block 0 also clears the two work-item counters.
 __global__ void __launch_bounds__(128)
 attend_prep_kernel(const int32_t* __restrict__ chunk_ids, const int32_t* __restrict__ n_chunks,
                    int32_t max_sel, int32_t range_chunks, int64_t n_ranges, int64_t n_chunk_total,
-                   int32_t* __restrict__ ptr, int64_t ptr_stride) {
+                   int32_t* __restrict__ ptr, int64_t ptr_stride, uint32_t* __restrict__ counters) {
   const int64_t bh = blockIdx.x;
   const int32_t* list = chunk_ids + bh * max_sel;
   const int n = max(0, min(n_chunks[bh], max_sel));
@@ -96,14 +98,80 @@ attend_prep_kernel(const int32_t* __restrict__ chunk_ids, const int32_t* __restr
   for (int64_t r = threadIdx.x; r <= n_ranges; r += blockDim.x)
     out[r] = lower_bound_ids(list, n, r < n_ranges ? r * range_chunks : n_chunk_total);
   if (threadIdx.x == 0) out[n_ranges + 1] = (n > 0 && list[0] == 0) ? 1 : 0;
+  if (bh == 0 && threadIdx.x < 2) counters[threadIdx.x] = 0u;
 }
 
+// One warp per (range, KV head, block of 32 query heads): which chunks of the
+// range any head of the block selected, and by which heads; appends a work
+// item when there is something to attend (always for the sink/tail range).
+// Item: [g | qb << 16, range, n_sel | tail << 31, head mask | offsets[W] | masks[W]].
+__global__ void __launch_bounds__(32)
+attend_items_kernel(Geom G, int32_t batch, int64_t nb, const int32_t* __restrict__ chunk_ids,
+                    const int32_t* __restrict__ ptr, int64_t ptr_stride, int32_t max_sel,
+                    int32_t range_chunks, int64_t n_ranges, uint32_t* __restrict__ counters,
+                    uint32_t* __restrict__ items, int64_t item_words) {
+  extern __shared__ uint32_t s_m[];      // [W]
+  const int g = blockIdx.y, qb = blockIdx.z;
+  const int64_t rho = blockIdx.x;
+  const bool tail = rho == n_ranges;
+  const int GQ = G.group, C = G.chunk;
+  const int qb0 = qb * kTcQ;
+  const int nq = min(kTcQ, batch * GQ - qb0);
+  const int lane = threadIdx.x;
+  const int64_t c_lo = rho * range_chunks;
+  const int64_t c_hi = min64(c_lo + range_chunks, nb / C);
+  for (int i = lane; i < range_chunks; i += 32) s_m[i] = 0u;
+  __syncwarp();
+  bool mine = false;
+  if (lane < nq) {
+    const int qi = qb0 + lane;
+    const int64_t bh = int64_t(qi / GQ) * G.hq + g * GQ + qi % GQ;
+    const int32_t* pr = ptr + bh * ptr_stride;
+    if (!tail) {
+      const int32_t* list = chunk_ids + bh * max_sel;
+      const int lo = pr[rho], hi = pr[rho + 1];
+      for (int i = lo; i < hi; ++i) {
+        const int64_t c = list[i];
+        if (c >= c_lo && c < c_hi) { atomicOr(&s_m[c - c_lo], 1u << lane); mine = true; }
+      }
+    } else {
+      mine = nb > 0 && pr[n_ranges + 1] == 0;      // this head needs the sink token
+    }
+  }
+  const uint32_t heads = __ballot_sync(0xffffffffu, mine);
+  __syncwarp();
+  if (!tail && heads == 0u) return;
+  uint32_t slot = 0;
+  if (lane == 0) slot = atomicAdd(&counters[0], 1u);
+  slot = __shfl_sync(0xffffffffu, slot, 0);
+  uint32_t* it = items + int64_t(slot) * item_words;
+  uint32_t n_sel = 0;
+  for (int i0 = 0; i0 < range_chunks; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t m = i < range_chunks ? s_m[i] : 0u;
+    const uint32_t ball = __ballot_sync(0xffffffffu, m != 0u);
+    if (m != 0u) {
+      const uint32_t pos = n_sel + __popc(ball & ((1u << lane) - 1u));
+      it[4 + pos] = uint32_t(i);
+      it[4 + range_chunks + pos] = m;
+    }
+    n_sel += __popc(ball);
+  }
+  if (lane == 0) {
+    it[0] = uint32_t(g) | (uint32_t(qb) << 16);
+    it[1] = uint32_t(rho);
+    it[2] = n_sel | (tail ? 0x80000000u : 0u);
+    it[3] = heads;
+  }
+}
+
+// Persistent: each CTA takes work items from the queue until it is empty.
 __global__ void __launch_bounds__(kTcThreads, 2)
 attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const float* __restrict__ Q,
                  const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V, int64_t ld,
-                 const int32_t* __restrict__ chunk_ids, const int32_t* __restrict__ ptr,
-                 int64_t ptr_stride, int32_t max_sel, int32_t range_chunks, int64_t n_ranges,
-                 float* __restrict__ partial, int64_t slots_per_head, int32_t* status) {
+                 int32_t range_chunks, const uint32_t* __restrict__ items, int64_t item_words,
+                 uint32_t* __restrict__ counters, float* __restrict__ partial, int64_t slots_per_head,
+                 int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -112,141 +180,13 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
   uint32_t* s_sel = s_mask + range_chunks;
   const uint32_t sK = tc::smem_u32(smem + kOffK), sV = tc::smem_u32(smem + kOffV);
   const uint32_t sQ = tc::smem_u32(smem + kOffQ), sP = tc::smem_u32(smem + kOffP);
-
-  const int g = blockIdx.y;
-  const int64_t rho = blockIdx.x;
-  const bool tail = rho == n_ranges;
   const int GQ = G.group;
-  const int qb0 = blockIdx.z * kTcQ;
-  const int nq = min(kTcQ, batch * GQ - qb0);
   const int C = G.chunk;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t c_lo = rho * range_chunks;
-  const int64_t c_hi = min64(c_lo + range_chunks, nb / C);
+  const uint32_t n_items = counters[0];
 
-  if (tid == 0) { ms.any = 0u; ms.mask0 = 0u; ms.err = 0u; }
-  for (int i = tid; i < range_chunks; i += blockDim.x) s_mask[i] = 0u;
-  __syncthreads();
-  if (tid < nq) {
-    const int qi = qb0 + tid;
-    const int64_t bh = int64_t(qi / GQ) * G.hq + g * GQ + qi % GQ;
-    const int32_t* pr = ptr + bh * ptr_stride;
-    if (!tail) {
-      const int32_t* list = chunk_ids + bh * max_sel;
-      const int lo = pr[rho], hi = pr[rho + 1];
-      bool any = false;
-      for (int i = lo; i < hi; ++i) {
-        const int64_t c = list[i];
-        if (c >= c_lo && c < c_hi) { atomicOr(&s_mask[c - c_lo], 1u << tid); any = true; }
-      }
-      if (any) atomicOr(&ms.any, 1u << tid);
-    } else {
-      if (nb > 0 && pr[n_ranges + 1] == 0) atomicOr(&ms.mask0, 1u << tid);
-    }
-  }
-  __syncthreads();
-  const uint32_t all_q = nq == 32 ? 0xffffffffu : ((1u << nq) - 1u);
-  const uint32_t active = tail ? all_q : ms.any;
-  if (active == 0u) return;
-
-  // Ordered list of the range's selected chunks.
-  int64_t n_tok;
-  if (!tail) {
-    uint32_t base = 0;
-    for (int i0 = 0; i0 < range_chunks; i0 += blockDim.x) {
-      const int i = i0 + tid;
-      const uint32_t f = (i < range_chunks && s_mask[i] != 0u) ? 1u : 0u;
-      uint32_t v = f;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t nv = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += nv;
-      }
-      if (lane == 31) ms.scan[warp] = v;
-      __syncthreads();
-      if (tid == 0) {
-        uint32_t run = 0;
-        for (int w = 0; w < kTcThreads / 32; ++w) { const uint32_t x = ms.scan[w]; ms.scan[w] = run; run += x; }
-        ms.scan[32] = run;
-      }
-      __syncthreads();
-      if (f) s_sel[base + ms.scan[warp] + v - f] = uint32_t(i);
-      base += ms.scan[32];
-      __syncthreads();
-    }
-    n_tok = int64_t(base) * C;
-  } else {
-    n_tok = (n_tokens - nb) + (ms.mask0 != 0u ? 1 : 0);
-  }
-  const int n_tiles = int((n_tok + kTcTok - 1) / kTcTok);
-
-  // Token of row `row` in tile `tile` (row < tokens of the tile) and its head mask.
-  auto token_of = [&](int tile, int row, int64_t& tok, uint32_t& msk) {
-    const int64_t u = int64_t(tile) * kTcTok + row;
-    tok = 0;
-    msk = 0u;
-    if (u >= n_tok) return;
-    if (!tail) {
-      const uint32_t k = s_sel[u / C];
-      tok = (c_lo + k) * C + u % C;
-      msk = s_mask[k];
-    } else if (u < n_tokens - nb) {
-      tok = nb + u;
-      msk = all_q;
-    } else {
-      msk = ms.mask0;
-    }
-  };
-  // Row `tid` of tile `tile`: 16 x 16-byte pieces into the swizzled K (or V)
-  // staging, zero-filled past the last token; one cp.async group.
-  auto issue_rows = [&](int tile, bool is_v) {
-    int64_t tok;
-    uint32_t msk;
-    token_of(tile, tid, tok, msk);
-    if (!is_v) ms.tmask[tile & 1][tid] = msk;
-    const int64_t u = int64_t(tile) * kTcTok + tid;
-    const uint32_t bytes = u < n_tok ? 16u : 0u;
-    const __nv_bfloat16* row = (is_v ? V : K) + (int64_t(g) * ld + tok) * kTcD;
-    const uint32_t dst = is_v ? sV : sK;
-#pragma unroll
-    for (int j = 0; j < kTcD / 8; ++j)
-      tc::cp_async16(dst + tc::sw128_offset(tid, 8 * j, kTcTok), row + 8 * j, bytes);
-    tc::cp_async_commit();
-  };
-
-  // Query block -> three bf16 terms, K-major rows (row = query head).
-  for (int v = tid; v < kTcQ * (kTcD / 8); v += blockDim.x) {
-    const int q = v / (kTcD / 8), col = (v % (kTcD / 8)) * 8;
-    float x[8];
-    if (q < nq) {
-      const int qi = qb0 + q;
-      const int64_t bh = int64_t(qi / GQ) * G.hq + g * GQ + qi % GQ;
-      const float4 a = *reinterpret_cast<const float4*>(Q + bh * kTcD + col);
-      const float4 b = *reinterpret_cast<const float4*>(Q + bh * kTcD + col + 4);
-      x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = 0.f;
-    }
-    const uint32_t off = tc::sw128_offset(q, col, kTcQ);
-#pragma unroll
-    for (int term = 0; term < 3; ++term) {
-      __align__(16) __nv_bfloat16 h[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        h[i] = __float2bfloat16_rn(x[i]);
-        x[i] -= __bfloat162float(h[i]);
-      }
-      *reinterpret_cast<uint4*>(smem + kOffQ + term * 8192 + off) = *reinterpret_cast<uint4*>(h);
-    }
-  }
-  if (tid < kTcQ) { ms.m[tid] = -INFINITY; ms.l[tid] = 0.f; }
-  if (tid == 0) tc::mbar_init(&ms.mbar, 1);
+  if (tid == 0) { ms.err = 0u; tc::mbar_init(&ms.mbar, 1); }
   if (warp == 0) tc::tmem_alloc(&ms.tmem_base, 64);
-  if (n_tiles > 0) {        // first tile's K and V in flight during the set-up
-    issue_rows(0, false);
-    issue_rows(0, true);
-  }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -254,112 +194,196 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
   const uint32_t t_lane = uint32_t(warp * 32) << 16;
   constexpr uint32_t idesc_s = tc::idesc_bf16(kTcTok, kTcQ, 0, 0);
   constexpr uint32_t idesc_pv = tc::idesc_bf16(kTcD, kTcQ, 1, 0);
-  float acc[kTcQ];
-#pragma unroll
-  for (int q = 0; q < kTcQ; ++q) acc[q] = 0.f;
   uint32_t phase = 0;
   bool failed = false;
 
-  // Pipeline: tile i's S MMA runs once its K rows have landed; tile i+1's K
-  // rows are requested as soon as that MMA has consumed the K staging, and
-  // its V rows once the P.V MMA of tile i has consumed the V staging.
-  for (int i = 0; i < n_tiles && !failed; ++i) {
-    const bool has_next = i + 1 < n_tiles;
-    tc::cp_async_wait_pending1();          // K_i done (V_i may still be in flight)
-    tc::fence_async_smem();
+  while (!failed) {
+    if (tid == 0) ms.any = atomicAdd(&counters[1], 1u);
+    __syncthreads();
+    const uint32_t item = ms.any;
+    if (item >= n_items) break;
+    const uint32_t* it = items + int64_t(item) * item_words;
+    const uint32_t h0 = it[0], h2 = it[2];
+    const int g = int(h0 & 0xffffu), qb = int(h0 >> 16);
+    const int64_t rho = int64_t(it[1]);
+    const bool tail = (h2 >> 31) != 0u;
+    const int n_sel = int(h2 & 0x7fffffffu);
+    const uint32_t heads = it[3];
+    for (int i = tid; i < n_sel; i += blockDim.x) {
+      s_sel[i] = it[4 + i];
+      s_mask[i] = it[4 + range_chunks + i];
+    }
+    const int qb0 = qb * kTcQ;
+    const int nq = min(kTcQ, batch * GQ - qb0);
+    const uint32_t all_q = nq == 32 ? 0xffffffffu : ((1u << nq) - 1u);
+    const int64_t c_lo = rho * range_chunks;
+    const int64_t n_tok = tail ? (n_tokens - nb) + (heads != 0u ? 1 : 0) : int64_t(n_sel) * C;
+    const int n_tiles = int((n_tok + kTcTok - 1) / kTcTok);
     __syncthreads();
 
-    // S^T = K . Q^T (three Q terms accumulate into one TMEM tile).
-    if (tid == 0) {
-      tc::fence_after_sync();
-#pragma unroll
-      for (int term = 0; term < 3; ++term)
-#pragma unroll
-        for (int ks = 0; ks < kTcD / 16; ++ks) {
-          const uint64_t a = tc::desc_sw128(sK + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-          const uint64_t b = tc::desc_sw128(sQ + term * 8192 + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
-          tc::mma_bf16(tbase, a, b, idesc_s, (term | ks) != 0);
-        }
-      tc::mma_commit(&ms.mbar);
-    }
-    if (!tc::mbar_wait(&ms.mbar, phase, kTcWaitTries)) atomicOr(&ms.err, 1u);
-    phase ^= 1u;
-    tc::fence_after_sync();
-    if (has_next) issue_rows(i + 1, false);     // the K staging is free again
-
-    float s[kTcQ];
-    tc::tmem_ld32(tbase + t_lane, s);
-    const uint32_t tm = ms.tmask[i & 1][tid];
-#pragma unroll
-    for (int q = 0; q < kTcQ; ++q) s[q] = ((tm >> q) & 1u) ? s[q] * G.scale : -INFINITY;
-    {
-      float v[kTcQ];
-#pragma unroll
-      for (int q = 0; q < kTcQ; ++q) v[q] = s[q];
-      ms.red[warp][lane] = transpose_reduce32<true>(v);
-    }
-    __syncthreads();
-    if (tid < kTcQ) {
-      const float mt = fmaxf(fmaxf(ms.red[0][tid], ms.red[1][tid]), fmaxf(ms.red[2][tid], ms.red[3][tid]));
-      const float mo = ms.m[tid];
-      const float mn = fmaxf(mo, mt);
-      ms.mnew[tid] = mn;
-      ms.scale[tid] = mn == -INFINITY ? 1.f : expf(mo - mn);
-    }
-    __syncthreads();
-    {
-      float v[kTcQ];
-#pragma unroll
-      for (int q = 0; q < kTcQ; ++q) {
-        const float mn = ms.mnew[q];
-        const float p = (mn == -INFINITY) ? 0.f : expf(s[q] - mn);
-        v[q] = p;
-        const __nv_bfloat16 hi = __float2bfloat16_rn(p);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(p - __bfloat162float(hi));
-        const uint32_t off = tc::sw128_offset(q, tid, kTcQ);
-        *reinterpret_cast<__nv_bfloat16*>(smem + kOffP + off) = hi;
-        *reinterpret_cast<__nv_bfloat16*>(smem + kOffP + 8192 + off) = lo;
+    auto token_of = [&](int tile, int row, int64_t& tok, uint32_t& msk) {
+      const int64_t u = int64_t(tile) * kTcTok + row;
+      tok = 0;
+      msk = 0u;
+      if (u >= n_tok) return;
+      if (!tail) {
+        const int64_t k = u / C;
+        tok = (c_lo + s_sel[k]) * C + u % C;
+        msk = s_mask[k];
+      } else if (u < n_tokens - nb) {
+        tok = nb + u;
+        msk = all_q;
+      } else {
+        msk = heads;          // the sink, for the heads whose list lacks chunk 0
       }
-      ms.red[warp][lane] = transpose_reduce32<false>(v);
-    }
-    if (has_next) tc::cp_async_wait_pending1(); else tc::cp_async_wait_pending0();   // V_i done
-    tc::fence_async_smem();
-    tc::fence_before_sync();
-    __syncthreads();
-    if (tid < kTcQ) {
-      ms.l[tid] = ms.l[tid] * ms.scale[tid] + (ms.red[0][tid] + ms.red[1][tid] + ms.red[2][tid] + ms.red[3][tid]);
-      ms.m[tid] = ms.mnew[tid];
-    }
-    // O^T tile = V^T . P (two P terms).
-    if (tid == 0) {
-      tc::fence_after_sync();
+    };
+    auto issue_rows = [&](int tile, bool is_v) {
+      int64_t tok;
+      uint32_t msk;
+      token_of(tile, tid, tok, msk);
+      if (!is_v) ms.tmask[tile & 1][tid] = msk;
+      const int64_t u = int64_t(tile) * kTcTok + tid;
+      const uint32_t bytes = u < n_tok ? 16u : 0u;
+      const __nv_bfloat16* row = (is_v ? V : K) + (int64_t(g) * ld + tok) * kTcD;
+      const uint32_t dst = is_v ? sV : sK;
 #pragma unroll
-      for (int term = 0; term < 2; ++term)
-#pragma unroll
-        for (int ks = 0; ks < kTcTok / 16; ++ks) {
-          const uint64_t a = tc::desc_sw128(sV + ks * 2048, 16384, 1024);
-          const uint64_t b = tc::desc_sw128(sP + term * 8192 + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
-          tc::mma_bf16(tbase + 32, a, b, idesc_pv, (term | ks) != 0);
-        }
-      tc::mma_commit(&ms.mbar);
-    }
-    if (!tc::mbar_wait(&ms.mbar, phase, kTcWaitTries)) atomicOr(&ms.err, 1u);
-    phase ^= 1u;
-    tc::fence_after_sync();
-    if (has_next) issue_rows(i + 1, true);      // the V staging is free again
-    {
-      float o[kTcQ];
-      tc::tmem_ld32(tbase + t_lane + 32, o);
-#pragma unroll
-      for (int q = 0; q < kTcQ; ++q) acc[q] = acc[q] * ms.scale[q] + o[q];
-    }
-    tc::fence_before_sync();
-    __syncthreads();
-    failed = ms.err != 0u;
-  }
-  tc::cp_async_wait_pending0();   // nothing of ours left in flight
+      for (int j = 0; j < kTcD / 8; ++j)
+        tc::cp_async16(dst + tc::sw128_offset(tid, 8 * j, kTcTok), row + 8 * j, bytes);
+      tc::cp_async_commit();
+    };
 
-  if (!failed) {
+    if (n_tiles > 0) {
+      issue_rows(0, false);
+      issue_rows(0, true);
+    }
+    // Query block -> three bf16 terms, K-major rows (row = query head).
+    for (int v = tid; v < kTcQ * (kTcD / 8); v += blockDim.x) {
+      const int q = v / (kTcD / 8), col = (v % (kTcD / 8)) * 8;
+      float x[8];
+      if (q < nq) {
+        const int qi = qb0 + q;
+        const int64_t bh = int64_t(qi / GQ) * G.hq + g * GQ + qi % GQ;
+        const float4 a = *reinterpret_cast<const float4*>(Q + bh * kTcD + col);
+        const float4 b = *reinterpret_cast<const float4*>(Q + bh * kTcD + col + 4);
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = 0.f;
+      }
+      const uint32_t off = tc::sw128_offset(q, col, kTcQ);
+#pragma unroll
+      for (int term = 0; term < 3; ++term) {
+        __align__(16) __nv_bfloat16 h[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          h[i] = __float2bfloat16_rn(x[i]);
+          x[i] -= __bfloat162float(h[i]);
+        }
+        *reinterpret_cast<uint4*>(smem + kOffQ + term * 8192 + off) = *reinterpret_cast<uint4*>(h);
+      }
+    }
+    if (tid < kTcQ) { ms.m[tid] = -INFINITY; ms.l[tid] = 0.f; }
+    float acc[kTcQ];
+#pragma unroll
+    for (int q = 0; q < kTcQ; ++q) acc[q] = 0.f;
+
+    // Pipeline: tile i's S MMA runs once its K rows have landed; tile i+1's K
+    // rows are requested as soon as that MMA has consumed the K staging, and
+    // its V rows once the P.V MMA of tile i has consumed the V staging.
+    for (int i = 0; i < n_tiles && !failed; ++i) {
+      const bool has_next = i + 1 < n_tiles;
+      tc::cp_async_wait_pending1();          // K_i done (V_i may still be in flight)
+      tc::fence_async_smem();
+      __syncthreads();
+      if (tid == 0) {
+        tc::fence_after_sync();
+#pragma unroll
+        for (int term = 0; term < 3; ++term)
+#pragma unroll
+          for (int ks = 0; ks < kTcD / 16; ++ks) {
+            const uint64_t a = tc::desc_sw128(sK + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+            const uint64_t b = tc::desc_sw128(sQ + term * 8192 + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
+            tc::mma_bf16(tbase, a, b, idesc_s, (term | ks) != 0);
+          }
+        tc::mma_commit(&ms.mbar);
+      }
+      if (!tc::mbar_wait(&ms.mbar, phase, kTcWaitTries)) atomicOr(&ms.err, 1u);
+      phase ^= 1u;
+      tc::fence_after_sync();
+      if (has_next) issue_rows(i + 1, false);     // the K staging is free again
+
+      float s[kTcQ];
+      tc::tmem_ld32(tbase + t_lane, s);
+      const uint32_t tm = ms.tmask[i & 1][tid];
+#pragma unroll
+      for (int q = 0; q < kTcQ; ++q) s[q] = ((tm >> q) & 1u) ? s[q] * G.scale : -INFINITY;
+      {
+        float v[kTcQ];
+#pragma unroll
+        for (int q = 0; q < kTcQ; ++q) v[q] = s[q];
+        ms.red[warp][lane] = transpose_reduce32<true>(v);
+      }
+      __syncthreads();
+      if (tid < kTcQ) {
+        const float mt = fmaxf(fmaxf(ms.red[0][tid], ms.red[1][tid]), fmaxf(ms.red[2][tid], ms.red[3][tid]));
+        const float mo = ms.m[tid];
+        const float mn = fmaxf(mo, mt);
+        ms.mnew[tid] = mn;
+        ms.scale[tid] = mn == -INFINITY ? 1.f : expf(mo - mn);
+      }
+      __syncthreads();
+      {
+        float v[kTcQ];
+#pragma unroll
+        for (int q = 0; q < kTcQ; ++q) {
+          const float mn = ms.mnew[q];
+          const float p = (mn == -INFINITY) ? 0.f : expf(s[q] - mn);
+          v[q] = p;
+          const __nv_bfloat16 hi = __float2bfloat16_rn(p);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(p - __bfloat162float(hi));
+          const uint32_t off = tc::sw128_offset(q, tid, kTcQ);
+          *reinterpret_cast<__nv_bfloat16*>(smem + kOffP + off) = hi;
+          *reinterpret_cast<__nv_bfloat16*>(smem + kOffP + 8192 + off) = lo;
+        }
+        ms.red[warp][lane] = transpose_reduce32<false>(v);
+      }
+      if (has_next) tc::cp_async_wait_pending1(); else tc::cp_async_wait_pending0();   // V_i done
+      tc::fence_async_smem();
+      tc::fence_before_sync();
+      __syncthreads();
+      if (tid < kTcQ) {
+        ms.l[tid] = ms.l[tid] * ms.scale[tid] + (ms.red[0][tid] + ms.red[1][tid] + ms.red[2][tid] + ms.red[3][tid]);
+        ms.m[tid] = ms.mnew[tid];
+      }
+      if (tid == 0) {
+        tc::fence_after_sync();
+#pragma unroll
+        for (int term = 0; term < 2; ++term)
+#pragma unroll
+          for (int ks = 0; ks < kTcTok / 16; ++ks) {
+            const uint64_t a = tc::desc_sw128(sV + ks * 2048, 16384, 1024);
+            const uint64_t b = tc::desc_sw128(sP + term * 8192 + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
+            tc::mma_bf16(tbase + 32, a, b, idesc_pv, (term | ks) != 0);
+          }
+        tc::mma_commit(&ms.mbar);
+      }
+      if (!tc::mbar_wait(&ms.mbar, phase, kTcWaitTries)) atomicOr(&ms.err, 1u);
+      phase ^= 1u;
+      tc::fence_after_sync();
+      if (has_next) issue_rows(i + 1, true);      // the V staging is free again
+      {
+        float o[kTcQ];
+        tc::tmem_ld32(tbase + t_lane + 32, o);
+#pragma unroll
+        for (int q = 0; q < kTcQ; ++q) acc[q] = acc[q] * ms.scale[q] + o[q];
+      }
+      tc::fence_before_sync();
+      __syncthreads();
+      failed = ms.err != 0u;
+    }
+    tc::cp_async_wait_pending0();
+    if (failed) break;
+    const uint32_t active = tail ? all_q : heads;
 #pragma unroll
     for (int q = 0; q < kTcQ; ++q) {
       if (q < nq && ((active >> q) & 1u)) {
@@ -370,9 +394,9 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
         if (tid == 0) *reinterpret_cast<float4*>(slot) = make_float4(ms.m[q], ms.l[q], 0.f, 0.f);
       }
     }
-  } else if (tid == 0 && status != nullptr) {
-    atomicOr(status, ZHA_DEV_TIMEOUT);
+    __syncthreads();     // ms.m / ms.l and the item's shared data are reused
   }
+  if (failed && tid == 0 && status != nullptr) atomicOr(status, ZHA_DEV_TIMEOUT);
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 0) {
@@ -520,18 +544,31 @@ cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const
   cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(smem));
   if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const int64_t nb = int64_t(G.chunk) * (n_tokens / G.chunk);
-  const int qn = batch * G.group;
-  int32_t* ptr = reinterpret_cast<int32_t*>(reinterpret_cast<char*>(partial) + lay.ptr_offset_bytes);
+  char* base = reinterpret_cast<char*>(partial);
+  int32_t* ptr = reinterpret_cast<int32_t*>(base + lay.ptr_offset_bytes);
+  uint32_t* counters = reinterpret_cast<uint32_t*>(base + lay.counter_offset_bytes);
+  uint32_t* items = reinterpret_cast<uint32_t*>(base + lay.item_offset_bytes);
   attend_prep_kernel<<<unsigned(int64_t(batch) * G.hq), 128, 0, s>>>(
-      chunk_ids, n_chunks, max_sel, lay.range_chunks, lay.n_ranges, lay.n_chunks, ptr, lay.ptr_stride);
+      chunk_ids, n_chunks, max_sel, lay.range_chunks, lay.n_ranges, lay.n_chunks, ptr, lay.ptr_stride,
+      counters);
   zha_count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  dim3 grid(unsigned(lay.n_ranges + 1), unsigned(G.hkv), unsigned((qn + kTcQ - 1) / kTcQ));
-  attend_tc_kernel<<<grid, kTcThreads, smem, s>>>(
+  dim3 grid_items(unsigned(lay.n_ranges + 1), unsigned(G.hkv), unsigned(lay.q_blocks));
+  attend_items_kernel<<<grid_items, 32, size_t(lay.range_chunks) * 4, s>>>(
+      G, batch, nb, chunk_ids, ptr, lay.ptr_stride, max_sel, lay.range_chunks, lay.n_ranges, counters,
+      items, lay.item_words);
+  zha_count_launch();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int64_t want = lay.max_items;
+  const unsigned ctas = unsigned(want < 2 * sms ? want : 2 * sms);
+  attend_tc_kernel<<<ctas, kTcThreads, smem, s>>>(
       G, batch, n_tokens, nb, Q, static_cast<const __nv_bfloat16*>(K),
-      static_cast<const __nv_bfloat16*>(V), ld, chunk_ids, ptr, lay.ptr_stride, max_sel,
-      lay.range_chunks, lay.n_ranges, partial, lay.slots_per_head, status);
+      static_cast<const __nv_bfloat16*>(V), ld, lay.range_chunks, items, lay.item_words, counters,
+      partial, lay.slots_per_head, status);
   zha_count_launch();
   return cudaGetLastError();
 }

@@ -95,7 +95,8 @@ def test_route_workspace_and_kept_words_arithmetic(zha):
     ranges = -(-(nb // 64) // 16)
     slots = -(-(heads * (ranges + 1) * 132 * 4) // 256) * 256
     ptrs = -(-(heads * (ranges + 2) * 4) // 256) * 256       # per-range list offsets
-    assert zha.attend_workspace_bytes(cfg, 4, n) == slots + ptrs
+    items = 4 * 1 * (ranges + 1) * (4 + 2 * 16) * 4           # work items: KV heads x head blocks x ranges
+    assert zha.attend_workspace_bytes(cfg, 4, n) == slots + ptrs + 256 + -(-items // 256) * 256
 
 
 def test_host_checks_reject_before_any_launch(zha):
