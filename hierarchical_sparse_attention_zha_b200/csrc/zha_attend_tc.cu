@@ -19,11 +19,12 @@
 //   masked online softmax per head      thread = token row (tcgen05.ld), per-head
 //                                       max / sum by warp transpose-reductions
 //   O^T[d][q] = V_tile^T . P            tcgen05.mma, M=128 (d), N=32, K=128 tokens,
-//                                       V read MN-major from the same staging, P split
-//                                       in two bf16 terms, TMEM columns [32, 64)
+//                                       V read MN-major from the same staging, P (two
+//                                       bf16 terms) stored MN-major, 64-byte swizzled,
+//                                       TMEM columns [32, 64)
 //   o[q] = o[q] * exp(m_old - m_new) + O^T tile   (thread = d row, registers)
-// K and V rows are staged by cp.async into the canonical 128-byte-swizzled
-// layout; one elected thread issues the MMAs and tcgen05.commit signals an
+// K and V rows are staged by cp.async (16 lanes per 256-byte row) into the
+// canonical 128-byte-swizzled layout; one elected thread issues the MMAs and tcgen05.commit signals an
 // mbarrier whose waits are bounded (a time-out sets ZHA_DEV_TIMEOUT and the CTA
 // releases its TMEM and returns).
 #include "zha_internal.cuh"
@@ -55,7 +56,9 @@ struct TcMisc {
 };
 
 __host__ inline size_t attend_tc_smem_bytes(int range_chunks) {
-  return size_t(kOffMisc) + sizeof(TcMisc) + 8 * size_t(range_chunks) + 1024;
+  // tiles + misc + per-range chunk offsets and masks + the item's token table + alignment
+  return size_t(kOffMisc) + sizeof(TcMisc) + 8 * size_t(range_chunks) +
+         2 * size_t(kAttendRangeTokens) + 1024;
 }
 
 template <bool kMax>
@@ -166,6 +169,9 @@ attend_items_kernel(Geom G, int32_t batch, int64_t nb, const int32_t* __restrict
 }
 
 // Persistent: each CTA takes work items from the queue until it is empty.
+// Scores are kept in base-2 units (s * log2(e) / sqrt(d)) so that the softmax
+// uses exp2; the running maximum is converted back to natural-log units when
+// the item's state is written.
 __global__ void __launch_bounds__(kTcThreads, 2)
 attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const float* __restrict__ Q,
                  const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V, int64_t ld,
@@ -178,12 +184,14 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
   TcMisc& ms = *reinterpret_cast<TcMisc*>(smem + kOffMisc);
   uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem + kOffMisc + sizeof(TcMisc));
   uint32_t* s_sel = s_mask + range_chunks;
+  int16_t* s_tok = reinterpret_cast<int16_t*>(s_sel + range_chunks);   // [kAttendRangeTokens]
   const uint32_t sK = tc::smem_u32(smem + kOffK), sV = tc::smem_u32(smem + kOffV);
   const uint32_t sQ = tc::smem_u32(smem + kOffQ), sP = tc::smem_u32(smem + kOffP);
   const int GQ = G.group;
   const int C = G.chunk;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t n_items = counters[0];
+  const float scale2 = G.scale * 1.4426950408889634f;      // 1/sqrt(d) * log2(e)
 
   if (tid == 0) { ms.err = 0u; tc::mbar_init(&ms.mbar, 1); }
   if (warp == 0) tc::tmem_alloc(&ms.tmem_base, 64);
@@ -193,9 +201,11 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
   const uint32_t tbase = ms.tmem_base;
   const uint32_t t_lane = uint32_t(warp * 32) << 16;
   constexpr uint32_t idesc_s = tc::idesc_bf16(kTcTok, kTcQ, 0, 0);
-  constexpr uint32_t idesc_pv = tc::idesc_bf16(kTcD, kTcQ, 1, 0);
+  constexpr uint32_t idesc_pv = tc::idesc_bf16(kTcD, kTcQ, 1, 1);
   uint32_t phase = 0;
   bool failed = false;
+  // Copy mapping: 16 lanes per 256-byte row, rows r0, r0 + 8, ..., r0 + 120.
+  const int piece = tid & 15, r0 = tid >> 4;
 
   while (!failed) {
     if (tid == 0) ms.any = atomicAdd(&counters[1], 1u);
@@ -216,40 +226,38 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
     const int qb0 = qb * kTcQ;
     const int nq = min(kTcQ, batch * GQ - qb0);
     const uint32_t all_q = nq == 32 ? 0xffffffffu : ((1u << nq) - 1u);
-    const int64_t c_lo = rho * range_chunks;
-    const int64_t n_tok = tail ? (n_tokens - nb) + (heads != 0u ? 1 : 0) : int64_t(n_sel) * C;
-    const int n_tiles = int((n_tok + kTcTok - 1) / kTcTok);
+    const int64_t n_tail = n_tokens - nb;
+    const int n_tok = tail ? int(n_tail) + (heads != 0u ? 1 : 0) : n_sel * C;
+    const int n_tiles = (n_tok + kTcTok - 1) / kTcTok;
+    // Token table of the item: offset from the item's first token (-1 = the sink).
+    const int64_t tok_base = tail ? nb : rho * range_chunks * C;
+    __syncthreads();
+    for (int u = tid; u < n_tok; u += blockDim.x)
+      s_tok[u] = tail ? int16_t(u < n_tail ? u : -1) : int16_t(int(s_sel[u / C]) * C + u % C);
     __syncthreads();
 
-    auto token_of = [&](int tile, int row, int64_t& tok, uint32_t& msk) {
-      const int64_t u = int64_t(tile) * kTcTok + row;
-      tok = 0;
-      msk = 0u;
-      if (u >= n_tok) return;
-      if (!tail) {
-        const int64_t k = u / C;
-        tok = (c_lo + s_sel[k]) * C + u % C;
-        msk = s_mask[k];
-      } else if (u < n_tokens - nb) {
-        tok = nb + u;
-        msk = all_q;
-      } else {
-        msk = heads;          // the sink, for the heads whose list lacks chunk 0
-      }
-    };
+    // Rows of tile `tile` into the K (or V) staging, one cp.async group; the
+    // K call also records the head mask of row `tid` for the softmax.
     auto issue_rows = [&](int tile, bool is_v) {
-      int64_t tok;
-      uint32_t msk;
-      token_of(tile, tid, tok, msk);
-      if (!is_v) ms.tmask[tile & 1][tid] = msk;
-      const int64_t u = int64_t(tile) * kTcTok + tid;
-      const uint32_t bytes = u < n_tok ? 16u : 0u;
-      const __nv_bfloat16* row = (is_v ? V : K) + (int64_t(g) * ld + tok) * kTcD;
+      const __nv_bfloat16* src = (is_v ? V : K) + int64_t(g) * ld * kTcD;
       const uint32_t dst = is_v ? sV : sK;
 #pragma unroll
-      for (int j = 0; j < kTcD / 8; ++j)
-        tc::cp_async16(dst + tc::sw128_offset(tid, 8 * j, kTcTok), row + 8 * j, bytes);
+      for (int k = 0; k < kTcTok / 8; ++k) {
+        const int row = r0 + 8 * k;
+        const int u = tile * kTcTok + row;
+        const bool valid = u < n_tok;
+        const int rel = valid ? int(s_tok[u]) : 0;
+        const int64_t tok = rel < 0 ? 0 : tok_base + rel;
+        tc::cp_async16(dst + tc::sw128_offset(row, 8 * piece, kTcTok), src + tok * kTcD + 8 * piece,
+                       valid ? 16u : 0u);
+      }
       tc::cp_async_commit();
+      if (!is_v) {
+        const int u = tile * kTcTok + tid;
+        uint32_t msk = 0u;
+        if (u < n_tok) msk = tail ? (u < n_tail ? all_q : heads) : s_mask[u / C];
+        ms.tmask[tile & 1][tid] = msk;
+      }
     };
 
     if (n_tiles > 0) {
@@ -310,13 +318,13 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
       if (!tc::mbar_wait(&ms.mbar, phase, kTcWaitTries)) atomicOr(&ms.err, 1u);
       phase ^= 1u;
       tc::fence_after_sync();
+      const uint32_t tm = ms.tmask[i & 1][tid];
       if (has_next) issue_rows(i + 1, false);     // the K staging is free again
 
       float s[kTcQ];
       tc::tmem_ld32(tbase + t_lane, s);
-      const uint32_t tm = ms.tmask[i & 1][tid];
 #pragma unroll
-      for (int q = 0; q < kTcQ; ++q) s[q] = ((tm >> q) & 1u) ? s[q] * G.scale : -INFINITY;
+      for (int q = 0; q < kTcQ; ++q) s[q] = ((tm >> q) & 1u) ? s[q] * scale2 : -INFINITY;
       {
         float v[kTcQ];
 #pragma unroll
@@ -329,21 +337,28 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
         const float mo = ms.m[tid];
         const float mn = fmaxf(mo, mt);
         ms.mnew[tid] = mn;
-        ms.scale[tid] = mn == -INFINITY ? 1.f : expf(mo - mn);
+        ms.scale[tid] = mn == -INFINITY ? 1.f : exp2f(mo - mn);
       }
       __syncthreads();
       {
+        // p = 2^(s - m_new); P stored MN-major (token row, 32 heads = 64 B) in
+        // two bf16 terms, 16 bytes (8 heads) per store.
         float v[kTcQ];
 #pragma unroll
-        for (int q = 0; q < kTcQ; ++q) {
-          const float mn = ms.mnew[q];
-          const float p = (mn == -INFINITY) ? 0.f : expf(s[q] - mn);
-          v[q] = p;
-          const __nv_bfloat16 hi = __float2bfloat16_rn(p);
-          const __nv_bfloat16 lo = __float2bfloat16_rn(p - __bfloat162float(hi));
-          const uint32_t off = tc::sw128_offset(q, tid, kTcQ);
-          *reinterpret_cast<__nv_bfloat16*>(smem + kOffP + off) = hi;
-          *reinterpret_cast<__nv_bfloat16*>(smem + kOffP + 8192 + off) = lo;
+        for (int c = 0; c < kTcQ / 8; ++c) {
+          __align__(16) __nv_bfloat16 hi[8], lo[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int q = 8 * c + j;
+            const float mn = ms.mnew[q];
+            const float p = (mn == -INFINITY) ? 0.f : exp2f(s[q] - mn);
+            v[q] = p;
+            hi[j] = __float2bfloat16_rn(p);
+            lo[j] = __float2bfloat16_rn(p - __bfloat162float(hi[j]));
+          }
+          const uint32_t off = tc::sw64_mn_chunk(tid, c);
+          *reinterpret_cast<uint4*>(smem + kOffP + off) = *reinterpret_cast<uint4*>(hi);
+          *reinterpret_cast<uint4*>(smem + kOffP + 8192 + off) = *reinterpret_cast<uint4*>(lo);
         }
         ms.red[warp][lane] = transpose_reduce32<false>(v);
       }
@@ -362,7 +377,7 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
 #pragma unroll
           for (int ks = 0; ks < kTcTok / 16; ++ks) {
             const uint64_t a = tc::desc_sw128(sV + ks * 2048, 16384, 1024);
-            const uint64_t b = tc::desc_sw128(sP + term * 8192 + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
+            const uint64_t b = tc::desc_sw64(sP + term * 8192 + ks * 1024, 8192, 512);
             tc::mma_bf16(tbase + 32, a, b, idesc_pv, (term | ks) != 0);
           }
         tc::mma_commit(&ms.mbar);
@@ -391,7 +406,8 @@ attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const floa
         const int64_t bh = int64_t(qi / GQ) * G.hq + g * GQ + qi % GQ;
         float* slot = partial + (bh * slots_per_head + rho) * (kTcD + 4);
         slot[4 + tid] = acc[q];
-        if (tid == 0) *reinterpret_cast<float4*>(slot) = make_float4(ms.m[q], ms.l[q], 0.f, 0.f);
+        if (tid == 0)   // maximum back to natural-log units
+          *reinterpret_cast<float4*>(slot) = make_float4(ms.m[q] * 0.6931471805599453f, ms.l[q], 0.f, 0.f);
       }
     }
     __syncthreads();     // ms.m / ms.l and the item's shared data are reused

@@ -26,6 +26,25 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t lbo, uin
   return d;
 }
 
+// The same for a 64-byte-swizzled canonical layout (layout type 4).
+__device__ __forceinline__ uint64_t desc_sw64(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr >> 4) & 0x3FFFu);
+  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(4) << 61;
+  return d;
+}
+
+// Byte offset of the 16-byte chunk `c` (elements 8c..8c+7 along MN) of K-row
+// `k` of a bf16 operand stored MN-major with 64-byte swizzling: rows of 32
+// MN-elements (64 B), 8 rows per 512-byte atom, chunk index XOR-ed with
+// (k % 8) / 2.
+__device__ __forceinline__ uint32_t sw64_mn_chunk(int k, int c) {
+  return uint32_t((k >> 3) * 512 + (k & 7) * 64 + ((c ^ ((k & 7) >> 1)) << 4));
+}
+
 // Instruction descriptor, kind::f16 with bf16 inputs and fp32 accumulation.
 // a_mn / b_mn: operand is MN-major (1) instead of K-major (0).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
