@@ -11,7 +11,8 @@
 //   score_kernel  -- one warp per candidate node (the union over the query heads
 //                    of a KV head), the node's R planes held in registers (lane
 //                    = part of one plane's row), one score per query head that
-//                    has the node as candidate;
+//                    has the node as candidate; head_dim 128 with R <= 16 uses
+//                    the tensor-core scorer in zha_score_tc.cu instead;
 //   select_kernel -- one CTA per query head: softmax over its candidates, radix
 //                    select of the cut on the key (score desc, node index asc)
 //                    with fixed-point mass histograms, kept bitmap (and at
@@ -449,6 +450,10 @@ select_kernel(Geom G, SelectArgs a) {
   }
 }
 
+cudaError_t launch_score_tc(const Geom& G, int level, int64_t n_nodes, int64_t n_par, int32_t batch,
+                            const float* Q, const uint32_t* kept_up, int64_t words_up, float* sigma,
+                            const float* store, int32_t* status, cudaStream_t s);
+
 // ---------------------------------------------------------------------------
 // Host launcher: levels L..1, score then select.
 // ---------------------------------------------------------------------------
@@ -527,10 +532,13 @@ cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n
     const int64_t words_up = level < G.levels ? lay.words[level + 1] : 0;
     float* sg = sigma + lay.sig_off[level];
     if (n_nodes > 0) {
-      e = G.d == 128 ? launch_score_d<128>(G, level, n_nodes, n_par, batch, Q, up, words_up, sg,
-                                           store, s)
-                     : launch_score_d<64>(G, level, n_nodes, n_par, batch, Q, up, words_up, sg,
-                                          store, s);
+      if (G.d == 128 && G.nref <= 16)      // tensor cores (zha_score_tc.cu)
+        e = launch_score_tc(G, level, n_nodes, n_par, batch, Q, up, words_up, sg, store, status, s);
+      else
+        e = G.d == 128 ? launch_score_d<128>(G, level, n_nodes, n_par, batch, Q, up, words_up, sg,
+                                             store, s)
+                       : launch_score_d<64>(G, level, n_nodes, n_par, batch, Q, up, words_up, sg,
+                                            store, s);
       if (e != cudaSuccess) return e;
     }
     a.level = level;
