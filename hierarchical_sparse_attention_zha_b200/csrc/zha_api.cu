@@ -17,6 +17,10 @@ cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n
                          int32_t* chunk_ids, int32_t* n_chunks, int32_t max_sel, uint32_t* bits,
                          float* sigma, int32_t* kp, const RouteLayout& lay, int32_t* status,
                          const float* store, cudaStream_t s);
+cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const void* V, int64_t ld,
+                             int64_t n_tokens, int32_t batch, const int32_t* chunk_ids,
+                             const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
+                             void* ws, const TcAttendLayout& lay, int32_t* status, cudaStream_t s);
 cudaError_t launch_attend(const Geom& G, const float* Q, const void* K, const void* V, int64_t ld,
                           int64_t n_tokens, int32_t batch, const int32_t* chunk_ids,
                           const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
@@ -246,6 +250,7 @@ zha_status zha_route(const zha_tree* tree, const float* d_Q, int32_t batch, int6
 size_t zha_attend_workspace_bytes(const zha_config* cfg, int32_t batch, int64_t n_tokens) {
   zha::Geom G;
   if (make_geom(cfg, &G, nullptr) != ZHA_OK || batch < 1 || n_tokens < 0) return 0;
+  if (zha::use_tc_attend(G)) return size_t(zha::tc_attend_layout(G, batch, n_tokens).bytes);
   return size_t(zha::attend_layout(G, batch, n_tokens).bytes);
 }
 
@@ -266,6 +271,22 @@ zha_status zha_sparse_attend(const zha_tree* tree, const float* d_Q, const void*
     return fail(ZHA_ERR_INVALID, "zha_sparse_attend: need 1 <= n_tokens <= ld");
   if (d_chunk_ids == nullptr || d_n_chunks == nullptr || max_sel < 1)
     return fail(ZHA_ERR_INVALID, "zha_sparse_attend: chunk_ids / n_chunks NULL or max_sel < 1");
+  if (zha::use_tc_attend(G)) {
+    const zha::TcAttendLayout lay = zha::tc_attend_layout(G, batch, n_tokens);
+    if (lay.groups > zha::kTcMaxGroups || n_tokens > 2147483647LL - 256)
+      return fail(ZHA_ERR_UNSUPPORTED,
+                  "zha_sparse_attend: more than %d (KV head, 32-query block) groups or 2^31 tokens",
+                  zha::kTcMaxGroups);
+    if (d_ws == nullptr || !aligned(d_ws, 256) || int64_t(ws_bytes) < lay.bytes)
+      return fail(ZHA_ERR_CAPACITY,
+                  "zha_sparse_attend: workspace must be 256-byte aligned with %lld bytes",
+                  (long long)lay.bytes);
+    cudaError_t e = zha::launch_attend_tc(G, d_Q, d_K, d_V, ld, n_tokens, batch, d_chunk_ids,
+                                          d_n_chunks, max_sel, d_O, d_lse, d_ws, lay, d_status,
+                                          static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "zha_sparse_attend");
+    return ZHA_OK;
+  }
   const zha::AttendLayout lay = zha::attend_layout(G, batch, n_tokens);
   if (lay.n_ranges + 1 > 2147483647LL)
     return fail(ZHA_ERR_UNSUPPORTED, "zha_sparse_attend: too many tokens");

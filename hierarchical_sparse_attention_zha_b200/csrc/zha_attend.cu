@@ -33,8 +33,8 @@ cudaError_t launch_combine(const Geom& G, int32_t batch, const int32_t* chunk_id
                            cudaStream_t s);
 cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const void* V, int64_t ld,
                              int64_t n_tokens, int32_t batch, const int32_t* chunk_ids,
-                             const int32_t* n_chunks, int32_t max_sel, float* partial,
-                             const AttendLayout& lay, int32_t* status, cudaStream_t s);
+                             const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
+                             void* ws, const TcAttendLayout& lay, int32_t* status, cudaStream_t s);
 
 template <int D>
 __host__ __device__ inline size_t attend_smem_bytes(int range_chunks) {
@@ -317,18 +317,142 @@ static cudaError_t launch_attend_t(const Geom& G, const float* Q, const void* K,
   return launch_combine(G, batch, chunk_ids, n_chunks, max_sel, O, lse, partial, lay, status, s);
 }
 
+// ---------------------------------------------------------------------------
+// Combine: one CTA (D threads, thread = output dim) per query head. The head's
+// chunk list is scanned in windows; the range states it touched are merged
+// with one maximum per window, so the state loads are independent.
+// ---------------------------------------------------------------------------
+constexpr int kCombineWindow = 4096;
+
+template <int D>
+__global__ void __launch_bounds__(D)
+combine_ranges_kernel(Geom G, int32_t batch, int64_t n_chunk_total, const int32_t* __restrict__ chunk_ids,
+                      const int32_t* __restrict__ n_chunks, int32_t max_sel, int32_t range_chunks,
+                      int64_t n_ranges, const float* __restrict__ partial, int64_t slots_per_head,
+                      float* __restrict__ O, float* __restrict__ lse, int32_t* status) {
+  __shared__ int32_t s_rng[kCombineWindow + 1];
+  __shared__ float s_w[kCombineWindow + 1];
+  __shared__ float s_red[D / 32 + 1];
+  __shared__ uint32_t s_scan[33];
+  __shared__ int s_bad;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = D / 32;
+  const int64_t bh = blockIdx.x;
+  int n = n_chunks[bh];
+  if (tid == 0) s_bad = (n < 0 || n > max_sel) ? 1 : 0;
+  n = max(0, min(n, max_sel));
+  const int32_t* list = chunk_ids + bh * max_sel;
+  const float* slots = partial + bh * slots_per_head * (D + 4);
+  float M = -INFINITY, L = 0.f, acc = 0.f;
+
+  auto merge_window = [&](int cnt) {
+    // window maximum
+    float mloc = -INFINITY;
+    for (int i = tid; i < cnt; i += D) {
+      const float* sl = slots + int64_t(s_rng[i]) * (D + 4);
+      if (sl[1] > 0.f) mloc = fmaxf(mloc, sl[0]);
+    }
+    mloc = warp_max(mloc);
+    if (lane == 0) s_red[warp] = mloc;
+    __syncthreads();
+    float mw = -INFINITY;
+    for (int w = 0; w < NW; ++w) mw = fmaxf(mw, s_red[w]);
+    __syncthreads();
+    const float mn = fmaxf(M, mw);
+    if (mn == -INFINITY) return;
+    const float r = expf(M - mn);
+    acc *= r;
+    L *= r;
+    float lsum = 0.f;
+    for (int i = tid; i < cnt; i += D) {
+      const float* sl = slots + int64_t(s_rng[i]) * (D + 4);
+      const float w = sl[1] > 0.f ? expf(sl[0] - mn) : 0.f;
+      s_w[i] = w;
+      lsum += w * sl[1];
+    }
+    lsum = warp_sum(lsum);
+    if (lane == 0) s_red[warp] = lsum;
+    __syncthreads();
+    for (int w = 0; w < NW; ++w) L += s_red[w];
+    int i = 0;
+    for (; i + 4 <= cnt; i += 4) {
+      const float o0 = slots[int64_t(s_rng[i]) * (D + 4) + 4 + tid];
+      const float o1 = slots[int64_t(s_rng[i + 1]) * (D + 4) + 4 + tid];
+      const float o2 = slots[int64_t(s_rng[i + 2]) * (D + 4) + 4 + tid];
+      const float o3 = slots[int64_t(s_rng[i + 3]) * (D + 4) + 4 + tid];
+      acc += s_w[i] * o0 + s_w[i + 1] * o1 + s_w[i + 2] * o2 + s_w[i + 3] * o3;
+    }
+    for (; i < cnt; ++i) acc += s_w[i] * slots[int64_t(s_rng[i]) * (D + 4) + 4 + tid];
+    __syncthreads();
+    M = mn;
+  };
+
+  for (int w0 = 0; w0 < n; w0 += kCombineWindow) {
+    const int w1 = min(n, w0 + kCombineWindow);
+    int cnt = 0;
+    for (int b0 = w0; b0 < w1; b0 += D) {
+      const int i = b0 + tid;
+      int64_t id = -1, prev = -1;
+      bool start = false;
+      if (i < w1) {
+        id = list[i];
+        prev = i > 0 ? int64_t(list[i - 1]) : -1;
+        const bool valid = id >= 0 && id < n_chunk_total && id > prev;
+        if (!valid) s_bad = 1;
+        start = valid && (i == 0 || prev < 0 || id / range_chunks != prev / range_chunks);
+      }
+      uint32_t v = start ? 1u : 0u, x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) s_scan[warp] = x;
+      __syncthreads();
+      if (tid == 0) {
+        uint32_t run = 0;
+        for (int w = 0; w < NW; ++w) { const uint32_t t = s_scan[w]; s_scan[w] = run; run += t; }
+        s_scan[32] = run;
+      }
+      __syncthreads();
+      if (start) s_rng[cnt + s_scan[warp] + x - v] = int32_t(id / range_chunks);
+      cnt += int(s_scan[32]);
+      __syncthreads();
+    }
+    merge_window(cnt);
+  }
+  if (tid == 0) s_rng[0] = int32_t(n_ranges);
+  __syncthreads();
+  merge_window(1);
+  O[bh * D + tid] = L > 0.f ? acc / L : 0.f;
+  if (tid == 0) {
+    if (lse != nullptr) lse[bh] = L > 0.f ? M + logf(L) : -INFINITY;
+    if (s_bad && status != nullptr) atomicOr(status, ZHA_DEV_BAD_SELECTION);
+  }
+}
+
+cudaError_t launch_combine(const Geom& G, int32_t batch, const int32_t* chunk_ids,
+                           const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
+                           const float* partial, const AttendLayout& lay, int32_t* status,
+                           cudaStream_t s) {
+  const unsigned heads = unsigned(int64_t(batch) * G.hq);
+  if (G.d == 128)
+    combine_ranges_kernel<128><<<heads, 128, 0, s>>>(G, batch, lay.n_chunks, chunk_ids, n_chunks,
+                                                     max_sel, lay.range_chunks, lay.n_ranges,
+                                                     partial, lay.slots_per_head, O, lse, status);
+  else
+    combine_ranges_kernel<64><<<heads, 64, 0, s>>>(G, batch, lay.n_chunks, chunk_ids, n_chunks,
+                                                   max_sel, lay.range_chunks, lay.n_ranges, partial,
+                                                   lay.slots_per_head, O, lse, status);
+  zha_count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_attend(const Geom& G, const float* Q, const void* K, const void* V, int64_t ld,
                           int64_t n_tokens, int32_t batch, const int32_t* chunk_ids,
                           const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
                           float* partial, const AttendLayout& lay, int32_t* status,
                           cudaStream_t s) {
-  if (G.kv_bf16 && G.d == 128) {
-    // bf16 caches with d = 128: the tensor-core kernel.
-    cudaError_t e = launch_attend_tc(G, Q, K, V, ld, n_tokens, batch, chunk_ids, n_chunks, max_sel,
-                                     partial, lay, status, s);
-    if (e != cudaSuccess) return e;
-    return launch_combine(G, batch, chunk_ids, n_chunks, max_sel, O, lse, partial, lay, status, s);
-  }
   if (G.kv_bf16)
     return G.d == 128 ? launch_attend_t<__nv_bfloat16, 128>(G, Q, K, V, ld, n_tokens, batch,
                                                             chunk_ids, n_chunks, max_sel, O, lse,

@@ -1,6 +1,5 @@
 // zha_attend_tc.cu -- sparse attention over the routed leaf tokens on the
-// sm_100a tensor cores (bf16 caches, head_dim 128), and the combine of the
-// per-range states used by both attention kernels.
+// sm_100a tensor cores (bf16 caches, head_dim 128).
 //
 // Citations: [Attention: "Scaled dot-product attention 의 식"] o = softmax(q K^T /
 // sqrt(d)) V; [Attention: "FlashAttention 계열"] online softmax (running max m,
@@ -9,57 +8,86 @@
 // (page "ZHA는 KV 캐시를 트리로 요약해 어텐션 비용을 준(sub)이차로 낮춘다") token 0
 // and the in-progress chunk are always attended.
 //
-// Work item = (range of W chunks, KV head, block of 32 query heads of that KV
-// head), built by attend_items_kernel; attend_tc_kernel is persistent (two
-// CTAs of 128 threads per SM take items from a queue). The selected chunks of
-// an item are streamed in tiles of 128 tokens. Per tile:
-//   S^T[tok][q] = K_tile . Q^T          tcgen05.mma, M=128 tokens, N=32 heads, K=d,
-//                                       Q split in three bf16 terms (fp32 accuracy),
-//                                       accumulator in TMEM columns [0, 32)
-//   masked online softmax per head      thread = token row (tcgen05.ld), per-head
-//                                       max / sum by warp transpose-reductions
-//   O^T[d][q] = V_tile^T . P            tcgen05.mma, M=128 (d), N=32, K=128 tokens,
-//                                       V read MN-major from the same staging, P (two
-//                                       bf16 terms) stored MN-major, 64-byte swizzled,
-//                                       TMEM columns [32, 64)
-//   o[q] = o[q] * exp(m_old - m_new) + O^T tile   (thread = d row, registers)
-// K and V rows are staged by cp.async (16 lanes per 256-byte row) into the
-// canonical 128-byte-swizzled layout; one elected thread issues the MMAs and tcgen05.commit signals an
-// mbarrier whose waits are bounded (a time-out sets ZHA_DEV_TIMEOUT and the CTA
-// releases its TMEM and returns).
+// Three launches:
+//  1. union_prep_kernel, one CTA per unit (group = KV head g with a block of up
+//     to 32 of its query heads; unit = the group inside one block of chunks):
+//     folds the heads' ascending chunk lists into one ascending union list with
+//     a 32-bit head mask per chunk (chunk 0 always present, for the sink), and
+//     validates the lists. Warp q marks head q's chunks in its own bitmap row;
+//     a 32 x 32 bit transpose by shuffles turns rows into per-chunk masks.
+//  2. attend_split_kernel, one CTA per SM: each unit's list is cut into tiles of
+//     128 rows (floor(128 / C) chunks; a group's last unit also carries the tail
+//     [N_b, N)); the tiles of all units form one sequence that is split evenly
+//     over the CTAs. Each CTA streams its span with warp-specialised roles:
+//       producers (2 warps)  cp.async of K and V rows into a 3-stage ring of
+//                            128-byte-swizzled tiles, per-tile row metadata
+//                            (prefetched one tile ahead)
+//       MMA issuer (1 lane)  S^T = K_tile . Q^T (M = 128 rows, N = 32 heads,
+//                            Q in two bf16 terms) into one of two TMEM buffers;
+//                            O^T += V_tile^T . P (M = d, N = 32, P in two bf16
+//                            terms) into a TMEM accumulator kept across tiles;
+//                            it polls both "tile landed" and "P ready" so that
+//                            neither kind of MMA waits behind the other
+//       softmax (4 warps)    thread = tile row: masked scores in log2 units, a
+//                            running maximum per head that is raised only when
+//                            a score exceeds it by more than 2^8 (then O and the
+//                            row sums are rescaled), P written into the K half of
+//                            the stage (K is consumed once S is done)
+//     When its span leaves a group the CTA writes one state [m, l, o] per head.
+//  3. combine_split_kernel, one warp per query head: merges the states of the
+//     CTAs whose span met the head's group.
+// Every wait on an mbarrier is bounded; a time-out sets ZHA_DEV_TIMEOUT and the
+// roles leave their loops, release TMEM and return.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "zha_internal.cuh"
 #include "zha_tc.cuh"
 
 namespace zha {
 
-constexpr int kTcTok = 128;
-constexpr int kTcQ = 32;
-constexpr int kTcD = 128;
-constexpr int kTcThreads = 128;
-constexpr uint32_t kTcWaitTries = 1u << 22;
+namespace {
 
-// Shared-memory plan (bytes from a 1024-byte aligned base).
-constexpr int kOffK = 0;                      // [2 column blocks][128 rows][128 B]
-constexpr int kOffV = 32768;
-constexpr int kOffQ = 65536;                  // 3 terms x [2][32][128 B]
-constexpr int kOffP = kOffQ + 3 * 8192;       // 2 terms x [2 token blocks][32][128 B]
-constexpr int kOffMisc = kOffP + 2 * 8192;    // 106496
+constexpr int kTok = 128;                 // rows per tile
+constexpr int kQ = 32;                    // query heads per group
+constexpr int kD = 128;
+constexpr int kStages = 3;
+constexpr int kStageBytes = 65536;        // K [2][128][128 B] then V [2][128][128 B]
+constexpr int kOffQ = kStages * kStageBytes;          // [2 halves][64 rows: 32 hi, 32 lo][128 B]
+constexpr int kOffMisc = kOffQ + 16384;
+constexpr uint32_t kTmemCols = 256;      // S: 2 x 64 columns, O: 64 columns at 128
+constexpr uint32_t kTmemO = 128;
+constexpr int kThreads = 256;             // warps 0-1 producers, 2 MMA, 3 idle, 4-7 softmax
+constexpr int kProducers = 64;
+constexpr int kMaxEntries = 64;           // chunks per tile (C >= 2)
+constexpr uint32_t kWaitTries = 1u << 22;
+constexpr uint32_t kPollLimit = 1u << 27; // polls of the MMA issuer without progress
+constexpr float kRescaleSlack = 8.f;      // log2 units: p may reach 2^8 before a rescale
+constexpr int kWinChunks = 16384;         // chunks per pass of the union fold
+constexpr int kWinWords = kWinChunks / 32;
+constexpr int kRowWords = kWinWords + 1;  // padded bitmap row (bank-conflict-free columns)
 
-struct TcMisc {
-  uint64_t mbar;
-  uint32_t tmem_base;
-  uint32_t any, mask0, nsel, err;
-  float m[kTcQ], l[kTcQ], scale[kTcQ], mnew[kTcQ];
-  float red[4][kTcQ];
-  uint32_t tmask[2][kTcTok];
-  uint32_t scan[33];
+struct Misc {
+  uint64_t full[kStages], empty[kStages], s_full[2], p_full[2], o_done, q_ready, drain;
+  uint32_t tmem_base, err;
+  uint32_t flags[2][4];
+  float red[2][4][kQ];
+  float mrun[2][kQ];                      // running maxima per head, by group parity
+  float scl[kQ];                          // rescale factors of the current tile
+  int32_t tok0[kStages][kMaxEntries];
+  int32_t nvalid[kStages][kMaxEntries];
+  uint32_t emask[kStages][kMaxEntries];
+  uint16_t rowj[kTok];                    // (entry << 8) | row in chunk, 0xffff = unused row
 };
 
-__host__ inline size_t attend_tc_smem_bytes(int range_chunks) {
-  // tiles + misc + per-range chunk offsets and masks + the item's token table + alignment
-  return size_t(kOffMisc) + sizeof(TcMisc) + 8 * size_t(range_chunks) +
-         2 * size_t(kAttendRangeTokens) + 1024;
+__host__ inline size_t split_smem_bytes(int64_t units) {
+  return size_t(kOffMisc) + sizeof(Misc) + 4 * size_t(units + 1) + 1024;
 }
+
+// Chunks per tile for chunk size C.
+__host__ __device__ inline int chunks_per_tile(int C) { return C >= kTok ? 1 : kTok / C; }
 
 template <bool kMax>
 __device__ __forceinline__ float transpose_reduce32(float (&v)[32]) {
@@ -78,513 +106,866 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[32]) {
   return v[0];   // lane L holds the reduction of value L
 }
 
-__device__ __forceinline__ int lower_bound_ids(const int32_t* a, int n, int64_t x) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (int64_t(a[mid]) < x) lo = mid + 1; else hi = mid;
+// 32 x 32 bit transpose across a warp: lane i holds row i (bit j = column j);
+// afterwards lane j holds column j (bit i = row i). Five block swaps.
+__device__ __forceinline__ uint32_t transpose_bits32(uint32_t x) {
+  const int lane = threadIdx.x & 31;
+  constexpr uint32_t kMask[5] = {0x0000FFFFu, 0x00FF00FFu, 0x0F0F0F0Fu, 0x33333333u, 0x55555555u};
+#pragma unroll
+  for (int i = 0, s = 16; i < 5; ++i, s >>= 1) {
+    const uint32_t y = __shfl_xor_sync(0xffffffffu, x, s);
+    const uint32_t m = kMask[i];
+    x = (lane & s) == 0 ? ((x & m) | ((y & m) << s)) : ((x & ~m) | ((y & ~m) >> s));
   }
-  return lo;
+  return x;
 }
 
-// Per query head: where each range's entries start in its chunk list, so
-// that the work-item pass reads two offsets instead of searching the list.
-// Block 0 also clears the two work-item counters.
-__global__ void __launch_bounds__(128)
-attend_prep_kernel(const int32_t* __restrict__ chunk_ids, const int32_t* __restrict__ n_chunks,
-                   int32_t max_sel, int32_t range_chunks, int64_t n_ranges, int64_t n_chunk_total,
-                   int32_t* __restrict__ ptr, int64_t ptr_stride, uint32_t* __restrict__ counters) {
-  const int64_t bh = blockIdx.x;
-  const int32_t* list = chunk_ids + bh * max_sel;
-  const int n = max(0, min(n_chunks[bh], max_sel));
-  int32_t* out = ptr + bh * ptr_stride;
-  for (int64_t r = threadIdx.x; r <= n_ranges; r += blockDim.x)
-    out[r] = lower_bound_ids(list, n, r < n_ranges ? r * range_chunks : n_chunk_total);
-  if (threadIdx.x == 0) out[n_ranges + 1] = (n > 0 && list[0] == 0) ? 1 : 0;
-  if (bh == 0 && threadIdx.x < 2) counters[threadIdx.x] = 0u;
+// Query head (flattened b * hq + h) of query q of group v.
+__device__ __forceinline__ int64_t head_of(const Geom& G, int q_blocks, int v, int q) {
+  const int g = v / q_blocks, qi = (v % q_blocks) * kQ + q;
+  return int64_t(qi / G.group) * G.hq + g * G.group + qi % G.group;
 }
 
-// One warp per (range, KV head, block of 32 query heads): which chunks of the
-// range any head of the block selected, and by which heads; appends a work
-// item when there is something to attend (always for the sink/tail range).
-// Item: [g | qb << 16, range, n_sel | tail << 31, head mask | offsets[W] | masks[W]].
-__global__ void __launch_bounds__(32)
-attend_items_kernel(Geom G, int32_t batch, int64_t nb, const int32_t* __restrict__ chunk_ids,
-                    const int32_t* __restrict__ ptr, int64_t ptr_stride, int32_t max_sel,
-                    int32_t range_chunks, int64_t n_ranges, uint32_t* __restrict__ counters,
-                    uint32_t* __restrict__ items, int64_t item_words) {
-  extern __shared__ uint32_t s_m[];      // [W]
-  const int g = blockIdx.y, qb = blockIdx.z;
-  const int64_t rho = blockIdx.x;
-  const bool tail = rho == n_ranges;
-  const int GQ = G.group, C = G.chunk;
-  const int qb0 = qb * kTcQ;
-  const int nq = min(kTcQ, batch * GQ - qb0);
-  const int lane = threadIdx.x;
-  const int64_t c_lo = rho * range_chunks;
-  const int64_t c_hi = min64(c_lo + range_chunks, nb / C);
-  for (int i = lane; i < range_chunks; i += 32) s_m[i] = 0u;
-  __syncwarp();
-  bool mine = false;
-  if (lane < nq) {
-    const int qi = qb0 + lane;
-    const int64_t bh = int64_t(qi / GQ) * G.hq + g * GQ + qi % GQ;
-    const int32_t* pr = ptr + bh * ptr_stride;
-    if (!tail) {
-      const int32_t* list = chunk_ids + bh * max_sel;
-      const int lo = pr[rho], hi = pr[rho + 1];
-      for (int i = lo; i < hi; ++i) {
-        const int64_t c = list[i];
-        if (c >= c_lo && c < c_hi) { atomicOr(&s_m[c - c_lo], 1u << lane); mine = true; }
+__device__ __forceinline__ int group_width(const Geom& G, int batch, int q_blocks, int v) {
+  return min(kQ, batch * G.group - (v % q_blocks) * kQ);
+}
+
+// First index of the ascending list a[0..n) with a[i] >= x (warp-cooperative:
+// each round probes 32 evenly spaced entries of the remaining range).
+__device__ __forceinline__ int warp_lower_bound(const int32_t* a, int n, int64_t x) {
+  const int lane = threadIdx.x & 31;
+  int lo = 0, hi = n;                      // answer in [lo, hi]
+  while (hi - lo > 32) {
+    const int step = (hi - lo + 31) / 32;
+    const int idx = lo + lane * step;
+    const bool below = idx < hi && int64_t(a[idx]) < x;
+    const uint32_t ball = __ballot_sync(0xffffffffu, below);
+    const int k = __popc(ball);            // probes below x (a prefix when ascending)
+    const int nlo = k == 0 ? lo : lo + (k - 1) * step + 1;
+    const int nhi = min(hi, lo + k * step);
+    lo = nlo;
+    hi = max(nlo, nhi);
+  }
+  const int idx = lo + lane;
+  const bool below = idx < hi && int64_t(a[idx]) < x;
+  return lo + __popc(__ballot_sync(0xffffffffu, below));
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// 1. Union of a group's chunk lists inside one block of chunks. A list entry is
+// valid when it lies in [0, N_b / C) and is above the entry before it; anything
+// else (and a count outside [0, max_sel]) sets ZHA_DEV_BAD_SELECTION, and which
+// in-range entries of such a list are attended is then unspecified. Each unit
+// validates its share of every list's indices, so each entry is checked once.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024)
+union_prep_kernel(Geom G, int32_t batch, int32_t q_blocks, int32_t n_blocks, int64_t block_chunks,
+                  int64_t nb, int64_t n_chunks, const int32_t* __restrict__ chunk_ids,
+                  const int32_t* __restrict__ n_sel, int32_t max_sel, int32_t* __restrict__ ids,
+                  uint32_t* __restrict__ masks, int64_t cap, int32_t* __restrict__ counts,
+                  int32_t* status) {
+  extern __shared__ uint32_t s_bits[];                 // [32][kRowWords]
+  __shared__ uint32_t s_scan[33];
+  const int u = blockIdx.x, v = u / n_blocks, blk = u % n_blocks;
+  const int tid = threadIdx.x, lane = tid & 31, q = tid >> 5;
+  const int nq = group_width(G, batch, q_blocks, v);
+  const int64_t c_lo = int64_t(blk) * block_chunks;
+  const int64_t c_hi = min64(n_chunks, c_lo + block_chunks);
+  const int32_t* list = nullptr;
+  int n = 0, cursor = 0;
+  bool bad = false;
+  if (q < nq) {
+    const int64_t bh = head_of(G, q_blocks, v, q);
+    list = chunk_ids + bh * max_sel;
+    const int raw = n_sel[bh];
+    bad = raw < 0 || raw > max_sel;
+    n = max(0, min(raw, max_sel));
+    const int i0 = int(int64_t(n) * blk / n_blocks), i1 = int(int64_t(n) * (blk + 1) / n_blocks);
+    for (int i = i0 + lane; i < i1; i += 32) {
+      const int32_t id = list[i], prev = i > 0 ? list[i - 1] : -1;
+      if (!(id >= 0 && int64_t(id) < n_chunks && id > prev)) bad = true;
+    }
+    if (n > 0 && c_lo < c_hi) cursor = warp_lower_bound(list, n, c_lo);
+  }
+  uint32_t* row = s_bits + q * kRowWords;
+  int64_t total = 0;
+  int32_t* out_ids = ids + int64_t(v) * cap + c_lo;
+  uint32_t* out_masks = masks + int64_t(v) * cap + c_lo;
+
+  for (int64_t win0 = c_lo; win0 < c_hi; win0 += kWinChunks) {
+    const int wlen = int(min64(kWinChunks, c_hi - win0));
+    const int words = (wlen + 31) / 32;
+    const int64_t win_end = win0 + wlen;
+    for (int w = lane; w < words; w += 32) row[w] = 0u;
+    __syncwarp();
+    while (cursor < n) {
+      int stop = 0x7fffffff;
+      int32_t id[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int idx = cursor + 32 * k + lane;
+        id[k] = idx < n ? list[idx] : 0x7fffffff;
       }
-    } else {
-      mine = nb > 0 && pr[n_ranges + 1] == 0;      // this head needs the sink token
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int idx = cursor + 32 * k + lane;
+        if (idx >= n) break;
+        if (int64_t(id[k]) >= win_end) stop = min(stop, idx);
+        else if (int64_t(id[k]) >= win0) {
+          const int off = int(id[k] - win0);
+          atomicOr(&row[off >> 5], 1u << (off & 31));
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) stop = min(stop, __shfl_xor_sync(0xffffffffu, stop, o));
+      if (stop != 0x7fffffff) { cursor = stop; break; }
+      cursor += 256;
     }
-  }
-  const uint32_t heads = __ballot_sync(0xffffffffu, mine);
-  __syncwarp();
-  if (!tail && heads == 0u) return;
-  uint32_t slot = 0;
-  if (lane == 0) slot = atomicAdd(&counters[0], 1u);
-  slot = __shfl_sync(0xffffffffu, slot, 0);
-  uint32_t* it = items + int64_t(slot) * item_words;
-  uint32_t n_sel = 0;
-  for (int i0 = 0; i0 < range_chunks; i0 += 32) {
-    const int i = i0 + lane;
-    const uint32_t m = i < range_chunks ? s_m[i] : 0u;
-    const uint32_t ball = __ballot_sync(0xffffffffu, m != 0u);
-    if (m != 0u) {
-      const uint32_t pos = n_sel + __popc(ball & ((1u << lane) - 1u));
-      it[4 + pos] = uint32_t(i);
-      it[4 + range_chunks + pos] = m;
+    __syncthreads();
+    // Warp wq owns words [wq * per, wq * per + per): transpose each word's 32
+    // rows into per-chunk masks, then compact in chunk order.
+    const int per = (words + 31) / 32;            // <= 16
+    uint32_t msk[16], ball[16];
+    uint32_t warp_cnt = 0;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      msk[k] = 0u;
+      ball[k] = 0u;
+      const int w = q * per + k;
+      if (k < per && w < words) {                  // uniform over the warp
+        const uint32_t x = s_bits[lane * kRowWords + w];
+        const uint32_t m = transpose_bits32(x);
+        const int off = 32 * w + lane;
+        const bool present = off < wlen && (m != 0u || (win0 + off == 0 && nb > 0));
+        msk[k] = m;
+        ball[k] = __ballot_sync(0xffffffffu, present);
+        warp_cnt += __popc(ball[k]);
+      }
     }
-    n_sel += __popc(ball);
+    if (lane == 0) s_scan[q] = warp_cnt;
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t run = 0;
+      for (int w = 0; w < 32; ++w) { const uint32_t t = s_scan[w]; s_scan[w] = run; run += t; }
+      s_scan[32] = run;
+    }
+    __syncthreads();
+    int64_t pos = total + s_scan[q];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      if ((ball[k] >> lane) & 1u) {
+        const int64_t at = pos + __popc(ball[k] & ((1u << lane) - 1u));
+        const int off = 32 * (q * per + k) + lane;
+        out_ids[at] = int32_t(win0 + off);
+        out_masks[at] = msk[k];
+      }
+      pos += __popc(ball[k]);
+    }
+    total += s_scan[32];
+    __syncthreads();                                   // s_bits and s_scan are reused
   }
-  if (lane == 0) {
-    it[0] = uint32_t(g) | (uint32_t(qb) << 16);
-    it[1] = uint32_t(rho);
-    it[2] = n_sel | (tail ? 0x80000000u : 0u);
-    it[3] = heads;
+  const int any_bad = __syncthreads_or(bad ? 1 : 0);
+  if (tid == 0) {
+    counts[u] = int32_t(total);
+    if (any_bad && status != nullptr) atomicOr(status, ZHA_DEV_BAD_SELECTION);
   }
 }
 
-// Persistent: each CTA takes work items from the queue until it is empty.
-// Scores are kept in base-2 units (s * log2(e) / sqrt(d)) so that the softmax
-// uses exp2; the running maximum is converted back to natural-log units when
-// the item's state is written.
-__global__ void __launch_bounds__(kTcThreads, 2)
-attend_tc_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const float* __restrict__ Q,
-                 const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V, int64_t ld,
-                 int32_t range_chunks, const uint32_t* __restrict__ items, int64_t item_words,
-                 uint32_t* __restrict__ counters, float* __restrict__ partial, int64_t slots_per_head,
-                 int32_t* status) {
+// ---------------------------------------------------------------------------
+// 2. Split attention over the units' tiles. Each role walks the CTA's span
+// [t0, t1) of the tile sequence the same way; li is the CTA-local tile index
+// that drives every barrier's phase.
+// ---------------------------------------------------------------------------
+struct SpanWalk {
+  const int32_t* toff;       // tile offsets of the units (shared memory)
+  int n_blocks;
+  int u;                     // current unit
+  // Advance to the unit holding tile t (t is non-decreasing between calls).
+  __device__ __forceinline__ void seek(int64_t t) {
+    while (t >= toff[u + 1]) ++u;
+  }
+  __device__ __forceinline__ int group() const { return u / n_blocks; }
+  __device__ __forceinline__ bool group_start(int64_t t, int64_t t0) const {
+    return t == t0 || t == toff[(u / n_blocks) * n_blocks];
+  }
+  __device__ __forceinline__ bool group_end(int64_t t, int64_t t1) const {
+    return t + 1 == t1 || t + 1 == toff[(u / n_blocks + 1) * n_blocks];
+  }
+};
+
+// kTma: K and V rows arrive by tiled tensor copies (one box of C rows per chunk
+// and 64-column half, issued by one thread); needs C % 8 == 0 so that every box
+// starts on a 1024-byte swizzle atom. Otherwise two warps stage rows with
+// cp.async (zero-filling rows without a token).
+template <bool kTma>
+__global__ void __launch_bounds__(kThreads, 1)
+attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    Geom G, int32_t batch, int32_t q_blocks, int32_t n_blocks, int64_t block_chunks,
+                    int32_t units, int64_t n_tokens, int64_t nb, const float* __restrict__ Q,
+                    const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
+                    int64_t ld, const int32_t* __restrict__ ids, const uint32_t* __restrict__ masks,
+                    int64_t cap, const int32_t* __restrict__ counts, int32_t* __restrict__ split,
+                    float* __restrict__ slots, int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  TcMisc& ms = *reinterpret_cast<TcMisc*>(smem + kOffMisc);
-  uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem + kOffMisc + sizeof(TcMisc));
-  uint32_t* s_sel = s_mask + range_chunks;
-  int16_t* s_tok = reinterpret_cast<int16_t*>(s_sel + range_chunks);   // [kAttendRangeTokens]
-  const uint32_t sK = tc::smem_u32(smem + kOffK), sV = tc::smem_u32(smem + kOffV);
-  const uint32_t sQ = tc::smem_u32(smem + kOffQ), sP = tc::smem_u32(smem + kOffP);
-  const int GQ = G.group;
-  const int C = G.chunk;
+  Misc& ms = *reinterpret_cast<Misc*>(smem + kOffMisc);
+  int32_t* s_toff = reinterpret_cast<int32_t*>(smem + kOffMisc + sizeof(Misc));   // [units + 1]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t n_items = counters[0];
-  const float scale2 = G.scale * 1.4426950408889634f;      // 1/sqrt(d) * log2(e)
+  const int C = G.chunk;
+  const int cpt = chunks_per_tile(C);
+  const int64_t n_tail = n_tokens - nb;
+  const int has_tail = n_tail > 0 ? 1 : 0;
+  // Tiles of unit u: its entries, plus the tail in a group's last block.
+  auto unit_tiles = [&](int uu) -> int {
+    const int e = counts[uu] + ((uu % n_blocks == n_blocks - 1) ? has_tail : 0);
+    return (e + cpt - 1) / cpt;
+  };
 
-  if (tid == 0) { ms.err = 0u; tc::mbar_init(&ms.mbar, 1); }
-  if (warp == 0) tc::tmem_alloc(&ms.tmem_base, 64);
+  // Tile offsets of the units: warp 0, a blocked scan.
+  if (warp == 0) {
+    const int per = (units + 31) / 32;
+    const int b0 = min(units, lane * per), b1 = min(units, b0 + per);
+    int sum = 0;
+    for (int uu = b0; uu < b1; ++uu) sum += unit_tiles(uu);
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - sum;
+    for (int uu = b0; uu < b1; ++uu) {
+      s_toff[uu] = run;
+      run += unit_tiles(uu);
+    }
+    if (lane == 31) s_toff[units] = incl;
+  }
+  if (tid < kTok) {
+    const int j = C >= kTok ? 0 : tid / C, rr = C >= kTok ? tid : tid % C;
+    ms.rowj[tid] = (j < cpt && rr < C) ? uint16_t((j << 8) | rr) : uint16_t(0xffff);
+  }
+  if (tid < kQ) ms.mrun[0][tid] = -INFINITY;
+  if (tid == 0) {
+    ms.err = 0u;
+    for (int st = 0; st < kStages; ++st) {
+      tc::mbar_init(&ms.full[st], kTma ? 1 : kProducers + 1);
+      tc::mbar_init(&ms.empty[st], 1);
+    }
+    for (int bb = 0; bb < 2; ++bb) {
+      tc::mbar_init(&ms.s_full[bb], 1);
+      tc::mbar_init(&ms.p_full[bb], 128);
+    }
+    tc::mbar_init(&ms.o_done, 1);
+    tc::mbar_init(&ms.q_ready, 128);
+    tc::mbar_init(&ms.drain, 1);
+  }
+  if (kTma) {
+    // Rows of a tile that no chunk fills keep what the stage held before; the
+    // V rows must at least be finite (P is 0 there), so clear them once.
+    for (int i = tid; i < kStages * 2048; i += kThreads) {
+      const int st = i / 2048, k = i % 2048;
+      *reinterpret_cast<uint4*>(smem + st * kStageBytes + 32768 + k * 16) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    tc::fence_async_smem();
+  }
+  if (warp == 2) tc::tmem_alloc(&ms.tmem_base, kTmemCols);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tbase = ms.tmem_base;
-  const uint32_t t_lane = uint32_t(warp * 32) << 16;
-  constexpr uint32_t idesc_s = tc::idesc_bf16(kTcTok, kTcQ, 0, 0);
-  constexpr uint32_t idesc_pv = tc::idesc_bf16(kTcD, kTcQ, 1, 1);
-  uint32_t phase = 0;
-  bool failed = false;
-  // Copy mapping: 16 lanes per 256-byte row, rows r0, r0 + 8, ..., r0 + 120.
-  const int piece = tid & 15, r0 = tid >> 4;
 
-  while (!failed) {
-    if (tid == 0) ms.any = atomicAdd(&counters[1], 1u);
-    __syncthreads();
-    const uint32_t item = ms.any;
-    if (item >= n_items) break;
-    const uint32_t* it = items + int64_t(item) * item_words;
-    const uint32_t h0 = it[0], h2 = it[2];
-    const int g = int(h0 & 0xffffu), qb = int(h0 >> 16);
-    const int64_t rho = int64_t(it[1]);
-    const bool tail = (h2 >> 31) != 0u;
-    const int n_sel = int(h2 & 0x7fffffffu);
-    const uint32_t heads = it[3];
-    for (int i = tid; i < n_sel; i += blockDim.x) {
-      s_sel[i] = it[4 + i];
-      s_mask[i] = it[4 + range_chunks + i];
+  const int64_t T = s_toff[units];
+  const int nct = int(gridDim.x), cta = int(blockIdx.x);
+  const int64_t t0 = int64_t(cta) * T / nct, t1 = int64_t(cta + 1) * T / nct;
+  if (cta == 0) {
+    for (int uu = tid; uu <= units; uu += blockDim.x) split[uu] = s_toff[uu];
+    if (tid == 0) split[units + 1] = nct;
+  }
+  int u0 = 0;
+  if (t0 < t1) {            // last unit whose first tile is <= t0 (it holds t0)
+    int lo = 0, hi = units - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (int64_t(s_toff[mid]) <= t0) lo = mid; else hi = mid - 1;
     }
-    const int qb0 = qb * kTcQ;
-    const int nq = min(kTcQ, batch * GQ - qb0);
-    const uint32_t all_q = nq == 32 ? 0xffffffffu : ((1u << nq) - 1u);
-    const int64_t n_tail = n_tokens - nb;
-    const int n_tok = tail ? int(n_tail) + (heads != 0u ? 1 : 0) : n_sel * C;
-    const int n_tiles = (n_tok + kTcTok - 1) / kTcTok;
-    // Token table of the item: offset from the item's first token (-1 = the sink).
-    const int64_t tok_base = tail ? nb : rho * range_chunks * C;
-    __syncthreads();
-    for (int u = tid; u < n_tok; u += blockDim.x)
-      s_tok[u] = tail ? int16_t(u < n_tail ? u : -1) : int16_t(int(s_sel[u / C]) * C + u % C);
-    __syncthreads();
+    u0 = lo;
+  }
 
-    // Rows of tile `tile` into the K (or V) staging, one cp.async group; the
-    // K call also records the head mask of row `tid` for the softmax.
-    auto issue_rows = [&](int tile, bool is_v) {
-      const __nv_bfloat16* src = (is_v ? V : K) + int64_t(g) * ld * kTcD;
-      const uint32_t dst = is_v ? sV : sK;
+  if (warp < 2) {
+    // ---------------- producers: K and V rows of each tile ----------------
+    // Warp 0 lanes read the entries of the next tile into registers while the
+    // current tile's copies are issued; they land in shared memory once the
+    // stage is free.
+    const int ptid = tid, piece = ptid & 15, rs = ptid >> 4;
+    SpanWalk wk{s_toff, n_blocks, u0};
+    int32_t pf_tok0[2] = {-1, -1}, pf_nv[2] = {0, 0};
+    uint32_t pf_m[2] = {0u, 0u};
+    auto prefetch = [&](int64_t t) {
+      wk.seek(t);
+      const int uu = wk.u, v = uu / n_blocks, blk = uu % n_blocks;
+      const int E = counts[uu];
+      const bool tail_here = has_tail && blk == n_blocks - 1;
+      const int nq = group_width(G, batch, q_blocks, v);
+      const uint32_t allq = nq == 32 ? 0xffffffffu : ((1u << nq) - 1u);
+      const int64_t tu = t - s_toff[uu];
+      const int64_t base = int64_t(v) * cap + int64_t(blk) * block_chunks;
 #pragma unroll
-      for (int k = 0; k < kTcTok / 8; ++k) {
-        const int row = r0 + 8 * k;
-        const int u = tile * kTcTok + row;
-        const bool valid = u < n_tok;
-        const int rel = valid ? int(s_tok[u]) : 0;
-        const int64_t tok = rel < 0 ? 0 : tok_base + rel;
-        tc::cp_async16(dst + tc::sw128_offset(row, 8 * piece, kTcTok), src + tok * kTcD + 8 * piece,
-                       valid ? 16u : 0u);
-      }
-      tc::cp_async_commit();
-      if (!is_v) {
-        const int u = tile * kTcTok + tid;
-        uint32_t msk = 0u;
-        if (u < n_tok) msk = tail ? (u < n_tail ? all_q : heads) : s_mask[u / C];
-        ms.tmask[tile & 1][tid] = msk;
+      for (int h = 0; h < 2; ++h) {
+        const int j = lane + 32 * h;
+        const int64_t e = tu * cpt + j;
+        pf_tok0[h] = -1; pf_nv[h] = 0; pf_m[h] = 0u;
+        if (j < cpt) {
+          if (e < E) {
+            pf_tok0[h] = ids[base + e] * C;
+            pf_nv[h] = C;
+            pf_m[h] = masks[base + e];
+          } else if (e == E && tail_here) {
+            pf_tok0[h] = int32_t(nb);
+            pf_nv[h] = int32_t(n_tail);
+            pf_m[h] = allq;
+          }
+        }
       }
     };
-
-    if (n_tiles > 0) {
-      issue_rows(0, false);
-      issue_rows(0, true);
-    }
-    // Query block -> three bf16 terms, K-major rows (row = query head).
-    for (int v = tid; v < kTcQ * (kTcD / 8); v += blockDim.x) {
-      const int q = v / (kTcD / 8), col = (v % (kTcD / 8)) * 8;
-      float x[8];
-      if (q < nq) {
-        const int qi = qb0 + q;
-        const int64_t bh = int64_t(qi / GQ) * G.hq + g * GQ + qi % GQ;
-        const float4 a = *reinterpret_cast<const float4*>(Q + bh * kTcD + col);
-        const float4 b = *reinterpret_cast<const float4*>(Q + bh * kTcD + col + 4);
-        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-      } else {
+    bool failed = false;
+    if (warp == 0 && t0 < t1) prefetch(t0);
+    SpanWalk wc{s_toff, n_blocks, u0};
+    int64_t li = 0;
+    if (kTma) {
+      if (warp == 0) {
+        for (int64_t t = t0; t < t1; ++t, ++li) {
+          wc.seek(t);
+          const int32_t g = wc.group() / q_blocks;
+          const int st = int(li % kStages);
+          const int64_t use = li / kStages;
+          bool bad = false;
+          if (use > 0) bad = !tc::mbar_wait(&ms.empty[st], uint32_t((use - 1) & 1), kWaitTries);
+          if (__any_sync(0xffffffffu, bad)) { failed = true; break; }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) x[i] = 0.f;
-      }
-      const uint32_t off = tc::sw128_offset(q, col, kTcQ);
-#pragma unroll
-      for (int term = 0; term < 3; ++term) {
-        __align__(16) __nv_bfloat16 h[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          h[i] = __float2bfloat16_rn(x[i]);
-          x[i] -= __bfloat162float(h[i]);
+          for (int h = 0; h < 2; ++h) {
+            const int j = lane + 32 * h;
+            if (j < cpt) {
+              ms.tok0[st][j] = pf_tok0[h];
+              ms.nvalid[st][j] = pf_nv[h];
+              ms.emask[st][j] = pf_m[h];
+            }
+          }
+          const uint32_t n_ok = __popc(__ballot_sync(0xffffffffu, pf_tok0[0] >= 0 && lane < cpt)) +
+                                __popc(__ballot_sync(0xffffffffu, pf_tok0[1] >= 0 && lane + 32 < cpt));
+          __syncwarp();
+          if (lane == 0) {
+            const uint32_t sK = tc::smem_u32(smem + st * kStageBytes), sV = sK + 32768;
+            tc::mbar_arrive_expect_tx(&ms.full[st], n_ok * 512u * uint32_t(C));
+            for (int j = 0; j < cpt; ++j) {
+              const int32_t tok0 = ms.tok0[st][j];
+              if (tok0 < 0) continue;
+              const uint32_t roff = uint32_t(j * C * 128);
+              tc::tma_load_3d(sK + roff, &tmK, 0, tok0, g, &ms.full[st]);
+              tc::tma_load_3d(sK + 16384 + roff, &tmK, 64, tok0, g, &ms.full[st]);
+              tc::tma_load_3d(sV + roff, &tmV, 0, tok0, g, &ms.full[st]);
+              tc::tma_load_3d(sV + 16384 + roff, &tmV, 64, tok0, g, &ms.full[st]);
+            }
+          }
+          __syncwarp();
+          if (t + 1 < t1) prefetch(t + 1);
         }
-        *reinterpret_cast<uint4*>(smem + kOffQ + term * 8192 + off) = *reinterpret_cast<uint4*>(h);
+        if (failed && lane == 0) atomicOr(&ms.err, 1u);
       }
-    }
-    if (tid < kTcQ) { ms.m[tid] = -INFINITY; ms.l[tid] = 0.f; }
-    float acc[kTcQ];
+    } else {
+    for (int64_t t = t0; t < t1; ++t, ++li) {
+      wc.seek(t);
+      const int64_t g = wc.group() / q_blocks;
+      const int st = int(li % kStages);
+      const int64_t use = li / kStages;
+      bool bad = false;
+      if (use > 0) bad = !tc::mbar_wait(&ms.empty[st], uint32_t((use - 1) & 1), kWaitTries);
+      if (warp == 0 && !bad) {
 #pragma unroll
-    for (int q = 0; q < kTcQ; ++q) acc[q] = 0.f;
-
-    // Pipeline: tile i's S MMA runs once its K rows have landed; tile i+1's K
-    // rows are requested as soon as that MMA has consumed the K staging, and
-    // its V rows once the P.V MMA of tile i has consumed the V staging.
-    for (int i = 0; i < n_tiles && !failed; ++i) {
-      const bool has_next = i + 1 < n_tiles;
-      tc::cp_async_wait_pending1();          // K_i done (V_i may still be in flight)
-      tc::fence_async_smem();
-      __syncthreads();
-      if (tid == 0) {
-        tc::fence_after_sync();
-#pragma unroll
-        for (int term = 0; term < 3; ++term)
-#pragma unroll
-          for (int ks = 0; ks < kTcD / 16; ++ks) {
-            const uint64_t a = tc::desc_sw128(sK + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-            const uint64_t b = tc::desc_sw128(sQ + term * 8192 + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
-            tc::mma_bf16(tbase, a, b, idesc_s, (term | ks) != 0);
+        for (int h = 0; h < 2; ++h) {
+          const int j = lane + 32 * h;
+          if (j < cpt) {
+            ms.tok0[st][j] = pf_tok0[h];
+            ms.nvalid[st][j] = pf_nv[h];
+            ms.emask[st][j] = pf_m[h];
           }
-        tc::mma_commit(&ms.mbar);
-      }
-      if (!tc::mbar_wait(&ms.mbar, phase, kTcWaitTries)) atomicOr(&ms.err, 1u);
-      phase ^= 1u;
-      tc::fence_after_sync();
-      const uint32_t tm = ms.tmask[i & 1][tid];
-      if (has_next) issue_rows(i + 1, false);     // the K staging is free again
-
-      float s[kTcQ];
-      tc::tmem_ld32(tbase + t_lane, s);
-#pragma unroll
-      for (int q = 0; q < kTcQ; ++q) s[q] = ((tm >> q) & 1u) ? s[q] * scale2 : -INFINITY;
-      {
-        float v[kTcQ];
-#pragma unroll
-        for (int q = 0; q < kTcQ; ++q) v[q] = s[q];
-        ms.red[warp][lane] = transpose_reduce32<true>(v);
-      }
-      __syncthreads();
-      if (tid < kTcQ) {
-        const float mt = fmaxf(fmaxf(ms.red[0][tid], ms.red[1][tid]), fmaxf(ms.red[2][tid], ms.red[3][tid]));
-        const float mo = ms.m[tid];
-        const float mn = fmaxf(mo, mt);
-        ms.mnew[tid] = mn;
-        ms.scale[tid] = mn == -INFINITY ? 1.f : exp2f(mo - mn);
-      }
-      __syncthreads();
-      {
-        // p = 2^(s - m_new); P stored MN-major (token row, 32 heads = 64 B) in
-        // two bf16 terms, 16 bytes (8 heads) per store.
-        float v[kTcQ];
-#pragma unroll
-        for (int c = 0; c < kTcQ / 8; ++c) {
-          __align__(16) __nv_bfloat16 hi[8], lo[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int q = 8 * c + j;
-            const float mn = ms.mnew[q];
-            const float p = (mn == -INFINITY) ? 0.f : exp2f(s[q] - mn);
-            v[q] = p;
-            hi[j] = __float2bfloat16_rn(p);
-            lo[j] = __float2bfloat16_rn(p - __bfloat162float(hi[j]));
-          }
-          const uint32_t off = tc::sw64_mn_chunk(tid, c);
-          *reinterpret_cast<uint4*>(smem + kOffP + off) = *reinterpret_cast<uint4*>(hi);
-          *reinterpret_cast<uint4*>(smem + kOffP + 8192 + off) = *reinterpret_cast<uint4*>(lo);
         }
-        ms.red[warp][lane] = transpose_reduce32<false>(v);
       }
-      if (has_next) tc::cp_async_wait_pending1(); else tc::cp_async_wait_pending0();   // V_i done
-      tc::fence_async_smem();
-      tc::fence_before_sync();
-      __syncthreads();
-      if (tid < kTcQ) {
-        ms.l[tid] = ms.l[tid] * ms.scale[tid] + (ms.red[0][tid] + ms.red[1][tid] + ms.red[2][tid] + ms.red[3][tid]);
-        ms.m[tid] = ms.mnew[tid];
+      if (tc::named_sync_or(2, kProducers, bad)) { failed = true; break; }
+      if (warp == 0 && t + 1 < t1) prefetch(t + 1);
+      const __nv_bfloat16* kb = K + g * ld * kD;
+      const __nv_bfloat16* vb = V + g * ld * kD;
+      const uint32_t sK = tc::smem_u32(smem + st * kStageBytes), sV = sK + 32768;
+#pragma unroll 4
+      for (int k = 0; k < kTok / 4; ++k) {
+        const int r = rs + 4 * k;
+        const uint32_t jr = ms.rowj[r];
+        bool valid = false;
+        int64_t tok = 0;
+        if (jr != 0xffffu) {
+          const int j = int(jr >> 8), rr = int(jr & 255u);
+          const int32_t tok0 = ms.tok0[st][j];
+          if (tok0 >= 0 && rr < ms.nvalid[st][j]) { valid = true; tok = int64_t(tok0) + rr; }
+        }
+        const uint32_t off = tc::sw128_offset(r, 8 * piece, kTok);
+        tc::cp_async16(sK + off, kb + tok * kD + 8 * piece, valid ? 16u : 0u);
+        tc::cp_async16(sV + off, vb + tok * kD + 8 * piece, valid ? 16u : 0u);
       }
-      if (tid == 0) {
-        tc::fence_after_sync();
-#pragma unroll
-        for (int term = 0; term < 2; ++term)
-#pragma unroll
-          for (int ks = 0; ks < kTcTok / 16; ++ks) {
-            const uint64_t a = tc::desc_sw128(sV + ks * 2048, 16384, 1024);
-            const uint64_t b = tc::desc_sw64(sP + term * 8192 + ks * 1024, 8192, 512);
-            tc::mma_bf16(tbase + 32, a, b, idesc_pv, (term | ks) != 0);
-          }
-        tc::mma_commit(&ms.mbar);
-      }
-      if (!tc::mbar_wait(&ms.mbar, phase, kTcWaitTries)) atomicOr(&ms.err, 1u);
-      phase ^= 1u;
-      tc::fence_after_sync();
-      if (has_next) issue_rows(i + 1, true);      // the V staging is free again
-      {
-        float o[kTcQ];
-        tc::tmem_ld32(tbase + t_lane + 32, o);
-#pragma unroll
-        for (int q = 0; q < kTcQ; ++q) acc[q] = acc[q] * ms.scale[q] + o[q];
-      }
-      tc::fence_before_sync();
-      __syncthreads();
-      failed = ms.err != 0u;
+      tc::cp_async_arrive_noinc(&ms.full[st]);
+      if (ptid == 0) tc::mbar_arrive(&ms.full[st]);
     }
     tc::cp_async_wait_pending0();
-    if (failed) break;
-    const uint32_t active = tail ? all_q : heads;
+    if (failed && ptid == 0) atomicOr(&ms.err, 1u);
+    }
+  } else if (warp == 2) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      // The two bf16 terms of Q (and of P) are stacked along N: one MMA gives
+      // both partial products, summed when TMEM is read.
+      constexpr uint32_t idesc_s = tc::idesc_bf16(kTok, 2 * kQ, 0, 0);
+      constexpr uint32_t idesc_pv = tc::idesc_bf16(kD, 2 * kQ, 1, 1);
+      const uint32_t sQ = tc::smem_u32(smem + kOffQ);
+      const int64_t n = t1 - t0;
+      SpanWalk ws_{s_toff, n_blocks, u0}, wp_{s_toff, n_blocks, u0};
+      int64_t ns = 0, np = 0;        // next tile to score (S), next tile to apply (PV)
+      int seg = 0;                   // groups whose Q has been taken
+      uint32_t idle = 0;
+      bool failed = false;
+      while (np < n) {
+        bool progress = false;
+        // PV first: it frees a stage for the producers.
+        if (np < ns && tc::mbar_test(&ms.p_full[np & 1], uint32_t((np >> 1) & 1))) {
+          const int64_t t = t0 + np;
+          wp_.seek(t);
+          const bool first = wp_.group_start(t, t0);
+          tc::fence_after_sync();
+          const uint32_t sP = tc::smem_u32(smem + (np % kStages) * kStageBytes), sV = sP + 32768;
 #pragma unroll
-    for (int q = 0; q < kTcQ; ++q) {
-      if (q < nq && ((active >> q) & 1u)) {
-        const int qi = qb0 + q;
-        const int64_t bh = int64_t(qi / GQ) * G.hq + g * GQ + qi % GQ;
-        float* slot = partial + (bh * slots_per_head + rho) * (kTcD + 4);
-        slot[4 + tid] = acc[q];
-        if (tid == 0)   // maximum back to natural-log units
-          *reinterpret_cast<float4*>(slot) = make_float4(ms.m[q] * 0.6931471805599453f, ms.l[q], 0.f, 0.f);
+          for (int ks = 0; ks < kTok / 16; ++ks) {
+            const uint64_t a = tc::desc_sw128(sV + ks * 2048, 16384, 1024);
+            const uint64_t b = tc::desc_sw128(sP + ks * 2048, 8192, 1024);
+            tc::mma_bf16(tbase + kTmemO, a, b, idesc_pv, (first && ks == 0) ? 0u : 1u);
+          }
+          tc::mma_commit(&ms.o_done);
+          tc::mma_commit(&ms.empty[np % kStages]);
+          ++np;
+          progress = true;
+        }
+        // S of the next tile once it has landed, its S buffer is free (the
+        // softmax has taken S of tile ns - 2, i.e. PV of it was issued) and,
+        // at a group start, the group's Q is in place.
+        if (ns < n && ns <= np + 1 &&
+            tc::mbar_test(&ms.full[ns % kStages], uint32_t((ns / kStages) & 1))) {
+          const int64_t t = t0 + ns;
+          ws_.seek(t);
+          const bool start = ws_.group_start(t, t0);
+          if (!start || tc::mbar_test(&ms.q_ready, uint32_t(seg & 1))) {
+            if (start) ++seg;
+            tc::fence_after_sync();
+            const uint32_t sK = tc::smem_u32(smem + (ns % kStages) * kStageBytes);
+            const uint32_t d_s = tbase + uint32_t(ns & 1) * 64;
+#pragma unroll
+            for (int ks = 0; ks < kD / 16; ++ks) {
+              const uint64_t a = tc::desc_sw128(sK + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+              const uint64_t b = tc::desc_sw128(sQ + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024);
+              tc::mma_bf16(d_s, a, b, idesc_s, ks != 0 ? 1u : 0u);
+            }
+            tc::mma_commit(&ms.s_full[ns & 1]);
+            ++ns;
+            progress = true;
+          }
+        }
+        if (progress) {
+          idle = 0;
+        } else if (++idle > kPollLimit) {
+          failed = true;
+          break;
+        }
+      }
+      tc::mma_commit(&ms.drain);
+      if (!tc::mbar_wait(&ms.drain, 0u, kWaitTries)) failed = true;
+      if (failed) atomicOr(&ms.err, 1u);
+    }
+  } else if (warp >= 4) {
+    // ---------------- softmax: thread = tile row / TMEM lane / output dim ----------------
+    const int sw = warp - 4;                       // TMEM lane quadrant sw
+    const int stid = tid - 128;
+    const int r = stid;
+    const uint32_t t_lane = uint32_t(sw * 32) << 16;
+    const float scale2 = G.scale * 1.4426950408889634f;     // 1/sqrt(d) * log2(e)
+    // Running maxima live in ms.mrun[gp] (gp = parity of the group count of
+    // this span; the other buffer is reset for the next group); row sums of p
+    // in registers.
+    float lrow[kQ];
+#pragma unroll
+    for (int q = 0; q < kQ; ++q) lrow[q] = 0.f;
+    int gp = 0;
+
+    // Q of group vq -> two bf16 terms, K-major 128-byte-swizzled rows: row q the
+    // high term of head q, row 32 + q its low term.
+    auto write_q = [&](int vq) {
+      const int nq = group_width(G, batch, q_blocks, vq);
+      const int q = stid >> 2, quarter = stid & 3;
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        const int col = quarter * 32 + c8 * 8;
+        float x[8];
+        if (q < nq) {
+          const float* src = Q + head_of(G, q_blocks, vq, q) * kD + col;
+          const float4 a = *reinterpret_cast<const float4*>(src);
+          const float4 b = *reinterpret_cast<const float4*>(src + 4);
+          x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) x[i] = 0.f;
+        }
+        __align__(16) __nv_bfloat16 hi[8], lo[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          hi[i] = __float2bfloat16_rn(x[i]);
+          lo[i] = __float2bfloat16_rn(x[i] - __bfloat162float(hi[i]));
+        }
+        *reinterpret_cast<uint4*>(smem + kOffQ + tc::sw128_offset(q, col, 2 * kQ)) =
+            *reinterpret_cast<const uint4*>(hi);
+        *reinterpret_cast<uint4*>(smem + kOffQ + tc::sw128_offset(kQ + q, col, 2 * kQ)) =
+            *reinterpret_cast<const uint4*>(lo);
+      }
+      tc::fence_async_smem();
+      tc::mbar_arrive(&ms.q_ready);
+    };
+
+    SpanWalk wk{s_toff, n_blocks, u0};
+    int od = 0;                    // PV completions (o_done phases) consumed
+    bool failed = false, pending_bad = false;
+    // Wait for the PV of tile k. Called only before this thread arrives on
+    // p_full of tile k + 1, so at most one completion is ahead of `od`.
+    auto wait_pv = [&](int64_t k) -> bool {
+      bool ok = true;
+      while (od <= k) {
+        ok &= tc::mbar_wait(&ms.o_done, uint32_t(od & 1), kWaitTries);
+        ++od;
+      }
+      return ok;
+    };
+    uint32_t allq = 0u;
+    if (t0 < t1) write_q(u0 / n_blocks);
+    int64_t li = 0;
+    for (int64_t t = t0; t < t1; ++t, ++li) {
+      wk.seek(t);
+      const int v = wk.group();
+      const bool start = wk.group_start(t, t0);
+      const bool end = wk.group_end(t, t1);
+      if (start) {
+        const int nq = group_width(G, batch, q_blocks, v);
+        allq = nq == 32 ? 0xffffffffu : ((1u << nq) - 1u);
+      }
+      const int st = int(li % kStages);
+      bool bad = !tc::mbar_wait(&ms.full[st], uint32_t((li / kStages) & 1), kWaitTries);
+      bad |= !tc::mbar_wait(&ms.s_full[li & 1], uint32_t((li >> 1) & 1), kWaitTries);
+      bad |= pending_bad;
+      pending_bad = false;
+      tc::fence_after_sync();
+      float s[kQ];
+      tc::tmem_ld32(tbase + t_lane + uint32_t(li & 1) * 64, s);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {      // + the low-term products, 16 columns at a time
+        float s_lo[16];
+        tc::tmem_ld16(tbase + t_lane + uint32_t(li & 1) * 64 + 32 + 16 * h, s_lo);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) s[16 * h + i] += s_lo[i];
+      }
+      uint32_t rmask = 0u;
+      {
+        const uint32_t jr = ms.rowj[r];
+        if (jr != 0xffffu) {
+          const int j = int(jr >> 8), rr = int(jr & 255u);
+          const int32_t tok0 = ms.tok0[st][j];
+          if (tok0 >= 0 && rr < ms.nvalid[st][j]) rmask = (tok0 + rr == 0) ? allq : ms.emask[st][j];
+        }
+      }
+      bool fire = false;
+      const float* mrun = ms.mrun[gp];
+#pragma unroll
+      for (int q = 0; q < kQ; ++q) {
+        s[q] = ((rmask >> q) & 1u) ? s[q] * scale2 : -INFINITY;
+        fire |= s[q] > mrun[q] + kRescaleSlack;
+      }
+      const uint32_t word = (__any_sync(0xffffffffu, fire) ? 1u : 0u) |
+                            (__any_sync(0xffffffffu, bad) ? 2u : 0u);
+      if (lane == 0) ms.flags[li & 1][sw] = word;
+      tc::named_sync(1, 128);
+      const uint32_t all = ms.flags[li & 1][0] | ms.flags[li & 1][1] | ms.flags[li & 1][2] |
+                           ms.flags[li & 1][3];
+      if (all & 2u) { failed = true; break; }
+      // S of this tile is complete, so Q may be replaced for the next group now.
+      if (end && t + 1 < t1) write_q(v + 1);
+      if (all & 1u) {
+        // Raise the running maxima to this tile's (per head), rescale l and O.
+        float tmp[kQ];
+#pragma unroll
+        for (int q = 0; q < kQ; ++q) tmp[q] = s[q];
+        ms.red[0][sw][lane] = transpose_reduce32<true>(tmp);
+        tc::named_sync(1, 128);
+        if (sw == 0) {                   // lane = head
+          const float mt = fmaxf(fmaxf(ms.red[0][0][lane], ms.red[0][1][lane]),
+                                 fmaxf(ms.red[0][2][lane], ms.red[0][3][lane]));
+          const float mo = ms.mrun[gp][lane];
+          const float mn = fmaxf(mo, mt);
+          ms.scl[lane] = mn == -INFINITY ? 1.f : exp2f(mo - mn);
+          ms.mrun[gp][lane] = mn;
+        }
+        tc::named_sync(1, 128);
+        const float* scl = ms.scl;
+#pragma unroll
+        for (int q = 0; q < kQ; ++q) lrow[q] *= scl[q];
+        if (!start) {                    // O holds earlier tiles of this group
+          pending_bad |= !wait_pv(li - 1);
+          tc::fence_after_sync();
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            float o[kQ];
+            tc::tmem_ld32(tbase + t_lane + kTmemO + 32 * h, o);
+#pragma unroll
+            for (int q = 0; q < kQ; ++q) o[q] *= scl[q];
+            tc::tmem_st32(tbase + t_lane + kTmemO + 32 * h, o);
+          }
+        }
+      }
+      // p = 2^(s - m), stored MN-major over the stage's consumed K rows: row =
+      // token, 64 bf16 (the high terms of the 32 heads, then the low terms),
+      // 128-byte swizzled.
+      uint8_t* sP = smem + st * kStageBytes;
+#pragma unroll
+      for (int c = 0; c < kQ / 8; ++c) {
+        __align__(16) __nv_bfloat16 hi[8], lo[8];
+#pragma unroll
+        for (int jq = 0; jq < 8; ++jq) {
+          const int q = 8 * c + jq;
+          const float p = mrun[q] == -INFINITY ? 0.f : exp2f(s[q] - mrun[q]);
+          lrow[q] += p;
+          hi[jq] = __float2bfloat16_rn(p);
+          lo[jq] = __float2bfloat16_rn(p - __bfloat162float(hi[jq]));
+        }
+        *reinterpret_cast<uint4*>(sP + tc::sw128_offset(r, 8 * c, kTok)) =
+            *reinterpret_cast<const uint4*>(hi);
+        *reinterpret_cast<uint4*>(sP + tc::sw128_offset(r, 32 + 8 * c, kTok)) =
+            *reinterpret_cast<const uint4*>(lo);
+      }
+      // PV of the previous tile must be complete before p_full of this one
+      // (it usually is by now); a time-out is reported at the next barrier.
+      if (li > 0) pending_bad |= !wait_pv(li - 1);
+      tc::fence_async_smem();
+      tc::fence_before_sync();
+      tc::mbar_arrive(&ms.p_full[li & 1]);
+      if (end) {
+        // The group's piece of this span is done: write one state per head.
+        const bool bad2 = !wait_pv(li) || pending_bad;
+        pending_bad = false;
+        tc::fence_after_sync();
+        float o[kQ];
+        tc::tmem_ld32(tbase + t_lane + kTmemO, o);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          float o_lo[16];
+          tc::tmem_ld16(tbase + t_lane + kTmemO + 32 + 16 * h, o_lo);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o[16 * h + i] += o_lo[i];
+        }
+        float tmp[kQ];
+#pragma unroll
+        for (int q = 0; q < kQ; ++q) tmp[q] = lrow[q];
+        ms.red[1][sw][lane] = transpose_reduce32<false>(tmp);
+        if (sw == 0) ms.mrun[gp ^ 1][lane] = -INFINITY;   // the next group starts afresh
+        if (tc::named_sync_or(1, 128, bad2)) { failed = true; break; }
+        const int nq = group_width(G, batch, q_blocks, v);
+        float* base = slots + int64_t(cta + v) * kQ * (kD + 4);
+#pragma unroll
+        for (int q = 0; q < kQ; ++q)
+          if (q < nq) base[q * (kD + 4) + 4 + r] = o[q];
+        if (sw == 0 && lane < nq) {
+          const float mq = ms.mrun[gp][lane];
+          const float L = ms.red[1][0][lane] + ms.red[1][1][lane] + ms.red[1][2][lane] + ms.red[1][3][lane];
+          // maximum back to natural-log units
+          *reinterpret_cast<float4*>(base + lane * (kD + 4)) =
+              make_float4(mq * 0.6931471805599453f, L, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int q = 0; q < kQ; ++q) lrow[q] = 0.f;
+        gp ^= 1;
       }
     }
-    __syncthreads();     // ms.m / ms.l and the item's shared data are reused
+    if (failed && stid == 0) atomicOr(&ms.err, 1u);
   }
-  if (failed && tid == 0 && status != nullptr) atomicOr(status, ZHA_DEV_TIMEOUT);
+
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == 2) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tbase, 64);
+    tc::tmem_dealloc(tbase, kTmemCols);
   }
+  if (tid == 0 && ms.err != 0u && status != nullptr) atomicOr(status, ZHA_DEV_TIMEOUT);
 }
 
 // ---------------------------------------------------------------------------
-// Combine: one CTA (D threads, thread = output dim) per query head. The head's
-// chunk list is scanned in windows; the range states it touched are merged
-// with one maximum per window, so the state loads are independent.
+// 3. Combine: one warp per query head over the states of the CTAs whose span
+// met the head's group. CTA c covers tiles [c T / n, (c + 1) T / n), so the
+// CTA holding tile t is ((t + 1) n - 1) / T. Lane = 4 output dims.
 // ---------------------------------------------------------------------------
-constexpr int kCombineWindow = 4096;
-
-template <int D>
-__global__ void __launch_bounds__(D)
-combine_ranges_kernel(Geom G, int32_t batch, int64_t n_chunk_total, const int32_t* __restrict__ chunk_ids,
-                      const int32_t* __restrict__ n_chunks, int32_t max_sel, int32_t range_chunks,
-                      int64_t n_ranges, const float* __restrict__ partial, int64_t slots_per_head,
-                      float* __restrict__ O, float* __restrict__ lse, int32_t* status) {
-  __shared__ int32_t s_rng[kCombineWindow + 1];
-  __shared__ float s_w[kCombineWindow + 1];
-  __shared__ float s_red[D / 32 + 1];
-  __shared__ uint32_t s_scan[33];
-  __shared__ int s_bad;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int NW = D / 32;
-  const int64_t bh = blockIdx.x;
-  int n = n_chunks[bh];
-  if (tid == 0) s_bad = (n < 0 || n > max_sel) ? 1 : 0;
-  n = max(0, min(n, max_sel));
-  const int32_t* list = chunk_ids + bh * max_sel;
-  const float* slots = partial + bh * slots_per_head * (D + 4);
-  float M = -INFINITY, L = 0.f, acc = 0.f;
-
-  auto merge_window = [&](int cnt) {
-    // window maximum
-    float mloc = -INFINITY;
-    for (int i = tid; i < cnt; i += D) {
-      const float* sl = slots + int64_t(s_rng[i]) * (D + 4);
-      if (sl[1] > 0.f) mloc = fmaxf(mloc, sl[0]);
-    }
-    mloc = warp_max(mloc);
-    if (lane == 0) s_red[warp] = mloc;
-    __syncthreads();
-    float mw = -INFINITY;
-    for (int w = 0; w < NW; ++w) mw = fmaxf(mw, s_red[w]);
-    __syncthreads();
-    const float mn = fmaxf(M, mw);
-    if (mn == -INFINITY) return;
-    const float r = expf(M - mn);
-    acc *= r;
-    L *= r;
-    float lsum = 0.f;
-    for (int i = tid; i < cnt; i += D) {
-      const float* sl = slots + int64_t(s_rng[i]) * (D + 4);
-      const float w = sl[1] > 0.f ? expf(sl[0] - mn) : 0.f;
-      s_w[i] = w;
-      lsum += w * sl[1];
-    }
-    lsum = warp_sum(lsum);
-    if (lane == 0) s_red[warp] = lsum;
-    __syncthreads();
-    for (int w = 0; w < NW; ++w) L += s_red[w];
-    int i = 0;
-    for (; i + 4 <= cnt; i += 4) {
-      const float o0 = slots[int64_t(s_rng[i]) * (D + 4) + 4 + tid];
-      const float o1 = slots[int64_t(s_rng[i + 1]) * (D + 4) + 4 + tid];
-      const float o2 = slots[int64_t(s_rng[i + 2]) * (D + 4) + 4 + tid];
-      const float o3 = slots[int64_t(s_rng[i + 3]) * (D + 4) + 4 + tid];
-      acc += s_w[i] * o0 + s_w[i + 1] * o1 + s_w[i + 2] * o2 + s_w[i + 3] * o3;
-    }
-    for (; i < cnt; ++i) acc += s_w[i] * slots[int64_t(s_rng[i]) * (D + 4) + 4 + tid];
-    __syncthreads();
-    M = mn;
+__global__ void __launch_bounds__(256)
+combine_split_kernel(Geom G, int32_t batch, int32_t q_blocks, int32_t n_blocks, int32_t units,
+                     const int32_t* __restrict__ split, const float* __restrict__ slots,
+                     float* __restrict__ O, float* __restrict__ lse) {
+  const int lane = threadIdx.x & 31;
+  const int64_t bh = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (bh >= int64_t(batch) * G.hq) return;
+  const int b = int(bh / G.hq), h = int(bh % G.hq);
+  const int qi = b * G.group + h % G.group;
+  const int v = (h / G.group) * q_blocks + qi / kQ, q = qi % kQ;
+  const int64_t lo = split[v * n_blocks], hi = split[(v + 1) * n_blocks], T = split[units];
+  const int64_t nct = split[units + 1];
+  const int c_lo = int(((lo + 1) * nct - 1) / T), c_hi = int((hi * nct - 1) / T);
+  const int n_st = c_hi - c_lo + 1;
+  // A CTA between c_lo and c_hi meets the group unless its span is empty (more
+  // CTAs than tiles); only states that were written are read.
+  auto written = [&](int i) -> bool {
+    const int64_t c = c_lo + i;
+    return (c + 1) * T / nct > c * T / nct;
   };
-
-  for (int w0 = 0; w0 < n; w0 += kCombineWindow) {
-    const int w1 = min(n, w0 + kCombineWindow);
-    int cnt = 0;
-    for (int b0 = w0; b0 < w1; b0 += D) {
-      const int i = b0 + tid;
-      int64_t id = -1, prev = -1;
-      bool start = false;
-      if (i < w1) {
-        id = list[i];
-        prev = i > 0 ? int64_t(list[i - 1]) : -1;
-        const bool valid = id >= 0 && id < n_chunk_total && id > prev;
-        if (!valid) s_bad = 1;
-        start = valid && (i == 0 || prev < 0 || id / range_chunks != prev / range_chunks);
-      }
-      uint32_t v = start ? 1u : 0u, x = v;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-      }
-      if (lane == 31) s_scan[warp] = x;
-      __syncthreads();
-      if (tid == 0) {
-        uint32_t run = 0;
-        for (int w = 0; w < NW; ++w) { const uint32_t t = s_scan[w]; s_scan[w] = run; run += t; }
-        s_scan[32] = run;
-      }
-      __syncthreads();
-      if (start) s_rng[cnt + s_scan[warp] + x - v] = int32_t(id / range_chunks);
-      cnt += int(s_scan[32]);
-      __syncthreads();
+  auto state = [&](int i) -> const float* {
+    return slots + (int64_t(c_lo + i + v) * kQ + q) * (kD + 4);
+  };
+  float M = -INFINITY;
+  for (int i = lane; i < n_st; i += 32)
+    if (written(i)) {
+      const float2 ml = *reinterpret_cast<const float2*>(state(i));
+      if (ml.y > 0.f) M = fmaxf(M, ml.x);
     }
-    merge_window(cnt);
+  M = warp_max(M);
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i0 = 0; i0 < n_st; i0 += 32) {
+    float w = 0.f;
+    if (i0 + lane < n_st && written(i0 + lane)) {
+      const float2 ml = *reinterpret_cast<const float2*>(state(i0 + lane));
+      if (ml.y > 0.f) {
+        w = expf(ml.x - M);
+        L += w * ml.y;
+      }
+    }
+    uint32_t ball = __ballot_sync(0xffffffffu, w > 0.f);
+    while (ball) {                 // up to four states per round, loads in flight together
+      int src[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        src[k] = ball ? __ffs(ball) - 1 : -1;
+        if (ball) ball &= ball - 1u;
+      }
+      float4 o[4];
+      float wk[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        wk[k] = __shfl_sync(0xffffffffu, w, src[k] < 0 ? 0 : src[k]);
+        o[k] = src[k] < 0 ? make_float4(0.f, 0.f, 0.f, 0.f)
+                          : *reinterpret_cast<const float4*>(state(i0 + src[k]) + 4 + 4 * lane);
+        if (src[k] < 0) wk[k] = 0.f;
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc.x += wk[k] * o[k].x; acc.y += wk[k] * o[k].y;
+        acc.z += wk[k] * o[k].z; acc.w += wk[k] * o[k].w;
+      }
+    }
   }
-  if (tid == 0) s_rng[0] = int32_t(n_ranges);
-  __syncthreads();
-  merge_window(1);
-  O[bh * D + tid] = L > 0.f ? acc / L : 0.f;
-  if (tid == 0) {
-    if (lse != nullptr) lse[bh] = L > 0.f ? M + logf(L) : -INFINITY;
-    if (s_bad && status != nullptr) atomicOr(status, ZHA_DEV_BAD_SELECTION);
-  }
+  L = warp_sum(L);
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  *reinterpret_cast<float4*>(O + bh * kD + 4 * lane) =
+      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (lse != nullptr && lane == 0) lse[bh] = L > 0.f ? M + logf(L) : -INFINITY;
 }
 
-cudaError_t launch_combine(const Geom& G, int32_t batch, const int32_t* chunk_ids,
-                           const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
-                           const float* partial, const AttendLayout& lay, int32_t* status,
-                           cudaStream_t s) {
-  const unsigned heads = unsigned(int64_t(batch) * G.hq);
-  if (G.d == 128)
-    combine_ranges_kernel<128><<<heads, 128, 0, s>>>(G, batch, lay.n_chunks, chunk_ids, n_chunks,
-                                                     max_sel, lay.range_chunks, lay.n_ranges,
-                                                     partial, lay.slots_per_head, O, lse, status);
-  else
-    combine_ranges_kernel<64><<<heads, 64, 0, s>>>(G, batch, lay.n_chunks, chunk_ids, n_chunks,
-                                                   max_sel, lay.range_chunks, lay.n_ranges, partial,
-                                                   lay.slots_per_head, O, lse, status);
-  zha_count_launch();
-  return cudaGetLastError();
+namespace {
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (the library
+// links only the CUDA runtime).
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
 }
+
+// [Hkv][ld][d] bf16 cache as a 3-D tensor {d, n_tokens, Hkv}: rows at or past
+// n_tokens read as zeros. Box = 64 columns (128 B, the swizzle span) x box_rows.
+bool kv_tensor_map(CUtensorMap* m, const void* base, int64_t n_tokens, int64_t ld, int hkv,
+                   int box_rows) {
+  const PFN_cuTensorMapEncodeTiled_v12000 fn = encode_tiled();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {cuuint64_t(kD), cuuint64_t(n_tokens), cuuint64_t(hkv)};
+  const cuuint64_t strides[2] = {cuuint64_t(kD) * 2, cuuint64_t(ld) * kD * 2};
+  const cuuint32_t box[3] = {64u, cuuint32_t(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
 
 cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const void* V, int64_t ld,
                              int64_t n_tokens, int32_t batch, const int32_t* chunk_ids,
-                             const int32_t* n_chunks, int32_t max_sel, float* partial,
-                             const AttendLayout& lay, int32_t* status, cudaStream_t s) {
-  const size_t smem = attend_tc_smem_bytes(lay.range_chunks);
-  cudaError_t e = cudaFuncSetAttribute(attend_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(smem));
+                             const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
+                             void* ws, const TcAttendLayout& lay, int32_t* status, cudaStream_t s) {
+  char* base = static_cast<char*>(ws);
+  int32_t* ids = reinterpret_cast<int32_t*>(base + lay.ids_off);
+  uint32_t* masks = reinterpret_cast<uint32_t*>(base + lay.masks_off);
+  int32_t* counts = reinterpret_cast<int32_t*>(base + lay.counts_off);
+  int32_t* split = reinterpret_cast<int32_t*>(base + lay.split_off);
+  float* slots = reinterpret_cast<float*>(base + lay.slots_off);
+  const int64_t nb = int64_t(G.chunk) * (n_tokens / G.chunk);
+  const int units = int(lay.units);
+
+  const size_t prep_smem = sizeof(uint32_t) * 32 * kRowWords;
+  cudaError_t e = cudaFuncSetAttribute(union_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(prep_smem));
   if (e != cudaSuccess) return e;
+  union_prep_kernel<<<unsigned(units), 1024, prep_smem, s>>>(
+      G, batch, lay.q_blocks, lay.n_blocks, lay.block_chunks, nb, lay.n_chunks, chunk_ids, n_chunks,
+      max_sel, ids, masks, lay.cap, counts, status);
+  zha_count_launch();
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  // Tensor copies when every chunk box starts on a swizzle atom (C % 8 == 0).
+  CUtensorMap mk{}, mv{};
+  const bool tma = G.chunk % 8 == 0 && kv_tensor_map(&mk, K, n_tokens, ld, G.hkv, G.chunk) &&
+                   kv_tensor_map(&mv, V, n_tokens, ld, G.hkv, G.chunk);
+  auto kern = tma ? attend_split_kernel<true> : attend_split_kernel<false>;
+  const size_t smem = split_smem_bytes(units);
+  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem))) !=
+      cudaSuccess)
+    return e;
   int dev = 0, sms = 148;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  const int64_t nb = int64_t(G.chunk) * (n_tokens / G.chunk);
-  char* base = reinterpret_cast<char*>(partial);
-  int32_t* ptr = reinterpret_cast<int32_t*>(base + lay.ptr_offset_bytes);
-  uint32_t* counters = reinterpret_cast<uint32_t*>(base + lay.counter_offset_bytes);
-  uint32_t* items = reinterpret_cast<uint32_t*>(base + lay.item_offset_bytes);
-  attend_prep_kernel<<<unsigned(int64_t(batch) * G.hq), 128, 0, s>>>(
-      chunk_ids, n_chunks, max_sel, lay.range_chunks, lay.n_ranges, lay.n_chunks, ptr, lay.ptr_stride,
-      counters);
+  const unsigned ctas = unsigned(sms < kTcMaxCtas ? sms : kTcMaxCtas);
+  kern<<<ctas, kThreads, smem, s>>>(
+      mk, mv, G, batch, lay.q_blocks, lay.n_blocks, lay.block_chunks, units, n_tokens, nb, Q,
+      static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V), ld, ids, masks,
+      lay.cap, counts, split, slots, status);
   zha_count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  dim3 grid_items(unsigned(lay.n_ranges + 1), unsigned(G.hkv), unsigned(lay.q_blocks));
-  attend_items_kernel<<<grid_items, 32, size_t(lay.range_chunks) * 4, s>>>(
-      G, batch, nb, chunk_ids, ptr, lay.ptr_stride, max_sel, lay.range_chunks, lay.n_ranges, counters,
-      items, lay.item_words);
-  zha_count_launch();
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const int64_t want = lay.max_items;
-  const unsigned ctas = unsigned(want < 2 * sms ? want : 2 * sms);
-  attend_tc_kernel<<<ctas, kTcThreads, smem, s>>>(
-      G, batch, n_tokens, nb, Q, static_cast<const __nv_bfloat16*>(K),
-      static_cast<const __nv_bfloat16*>(V), ld, lay.range_chunks, items, lay.item_words, counters,
-      partial, lay.slots_per_head, status);
+
+  const int64_t heads = int64_t(batch) * G.hq;
+  combine_split_kernel<<<unsigned((heads * 32 + 255) / 256), 256, 0, s>>>(
+      G, batch, lay.q_blocks, lay.n_blocks, units, split, slots, O, lse);
   zha_count_launch();
   return cudaGetLastError();
 }

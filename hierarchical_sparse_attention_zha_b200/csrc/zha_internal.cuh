@@ -129,6 +129,59 @@ inline AttendLayout attend_layout(const Geom& g, int32_t batch, int64_t n_tokens
 }
 
 // ---------------------------------------------------------------------------
+// Tensor-core attend workspace (bf16 caches, d = 128). A "group" v is a KV head
+// g and a block of up to 32 of its query heads (v = g * q_blocks + qb). The
+// chunk range [0, N_b / C) is cut into n_blocks blocks of block_chunks chunks;
+// a "unit" u = v * n_blocks + b is one group's union inside one block.
+//   ids   [groups][cap] int32   per unit, at offset b * block_chunks: the
+//                               ascending union of the chunks the group's heads
+//                               listed in block b (chunk 0 always present when
+//                               N_b > 0); cap = n_blocks * block_chunks
+//   masks [groups][cap] uint32  bit q = query q of the group listed that chunk
+//   counts[units] int32         union entries per unit
+//   split [units + 1 + 2] int32 tile offsets of the units, then the CTA count
+//                               (written by the attend kernel for the combine)
+//   slots [(kTcMaxCtas + groups) * 32][d + 4] float  per (CTA span piece, query)
+//                               state [m, l, 0, 0, o[d]]; the piece of CTA c
+//                               inside group v has index c + v
+// ---------------------------------------------------------------------------
+constexpr int kTcMaxCtas = 296;
+constexpr int kTcMaxGroups = 1024;
+constexpr int kTcMaxUnits = 1024;
+constexpr int64_t kTcBlockChunks = 2048;
+
+struct TcAttendLayout {
+  int64_t n_chunks, block_chunks, cap, groups, units;
+  int64_t ids_off, masks_off, counts_off, split_off, slots_off, bytes;
+  int32_t q_blocks, n_blocks;
+};
+
+inline TcAttendLayout tc_attend_layout(const Geom& g, int32_t batch, int64_t n_tokens) {
+  TcAttendLayout a{};
+  a.n_chunks = n_tokens / g.chunk;
+  a.q_blocks = int32_t((int64_t(batch) * g.group + kAttendHeadsPerBlock - 1) / kAttendHeadsPerBlock);
+  a.groups = int64_t(g.hkv) * a.q_blocks;
+  int64_t nblk = (a.n_chunks + kTcBlockChunks - 1) / kTcBlockChunks;
+  const int64_t lim = kTcMaxUnits / a.groups;
+  if (nblk > lim) nblk = lim;
+  if (nblk < 1) nblk = 1;
+  a.n_blocks = int32_t(nblk);
+  int64_t per = (a.n_chunks + nblk - 1) / nblk;
+  a.block_chunks = round_up(per < 1 ? 1 : per, 32);
+  a.cap = nblk * a.block_chunks;
+  a.units = a.groups * nblk;
+  a.ids_off = 0;
+  a.masks_off = round_up(a.groups * a.cap * 4, 256);
+  a.counts_off = a.masks_off + round_up(a.groups * a.cap * 4, 256);
+  a.split_off = a.counts_off + round_up(a.units * 4, 256);
+  a.slots_off = a.split_off + round_up((a.units + 3) * 4, 256);
+  a.bytes = a.slots_off + round_up((kTcMaxCtas + a.groups) * 32 * int64_t(g.d + 4) * 4, 256);
+  return a;
+}
+
+inline bool use_tc_attend(const Geom& g) { return g.kv_bf16 && g.d == 128; }
+
+// ---------------------------------------------------------------------------
 // Device helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float warp_sum(float v) {

@@ -91,12 +91,17 @@ def test_route_workspace_and_kept_words_arithmetic(zha):
     sig = sum(-(-heads * (nb // 64 ** l) // 64) * 64 for l in (1, 2, 3))
     assert ws >= sig * 4 + words * 4
     assert zha.route_workspace_bytes(cfg, 4, 1000) < ws        # grows with n_tokens
-    # attend: one slot per (head, range of 1024 tokens) plus the tail, d+4 floats each
-    ranges = -(-(nb // 64) // 16)
-    slots = -(-(heads * (ranges + 1) * 132 * 4) // 256) * 256
-    ptrs = -(-(heads * (ranges + 2) * 4) // 256) * 256       # per-range list offsets
-    items = 4 * 1 * (ranges + 1) * (4 + 2 * 16) * 4           # work items: KV heads x head blocks x ranges
-    assert zha.attend_workspace_bytes(cfg, 4, n) == slots + ptrs + 256 + -(-items // 256) * 256
+    # attend (bf16, d = 128: tensor-core path): union lists per (KV head, block of
+    # 32 query heads) laid out in blocks of <= 2048 chunks (a multiple of 32),
+    # a count per (group, block), the tile split, and one state per (CTA piece, head)
+    r256 = lambda x: -(-x // 256) * 256
+    groups, n_ch = 4 * 1, n // 64
+    n_blocks = -(-n_ch // 2048)
+    block = -(-(-(-n_ch // n_blocks)) // 32) * 32
+    cap, units = n_blocks * block, groups * n_blocks
+    lists = 2 * r256(groups * cap * 4)
+    slots = r256((296 + groups) * 32 * 132 * 4)
+    assert zha.attend_workspace_bytes(cfg, 4, n) == lists + r256(units * 4) + r256((units + 3) * 4) + slots
 
 
 def test_host_checks_reject_before_any_launch(zha):
