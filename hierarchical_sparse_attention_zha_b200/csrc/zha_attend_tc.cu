@@ -59,7 +59,8 @@ constexpr int kOffQ = kStages * kStageBytes;          // [2 halves][64 rows: 32 
 constexpr int kOffMisc = kOffQ + 16384;
 constexpr uint32_t kTmemCols = 256;      // S: 2 x 64 columns, O: 64 columns at 128
 constexpr uint32_t kTmemO = 128;
-constexpr int kThreads = 256;             // warps 0-1 producers, 2 MMA, 3 idle, 4-7 softmax
+constexpr int kThreads = 384;             // warps 0-1 producers, 2 MMA, 3 idle, 4-11 softmax
+constexpr int kHalfQ = 16;                // heads per softmax warpgroup
 constexpr int kProducers = 64;
 constexpr int kMaxEntries = 64;           // chunks per tile (C >= 2)
 constexpr uint32_t kWaitTries = 1u << 22;
@@ -72,8 +73,8 @@ constexpr int kRowWords = kWinWords + 1;  // padded bitmap row (bank-conflict-fr
 struct Misc {
   uint64_t full[kStages], empty[kStages], s_full[2], p_full[2], o_done, q_ready, drain;
   uint32_t tmem_base, err;
-  uint32_t flags[2][4];
-  float red[2][4][kQ];
+  uint32_t flags[2][2][4];
+  float red[2][2][4][16];
   float mrun[2][kQ];                      // running maxima per head, by group parity
   float scl[kQ];                          // rescale factors of the current tile
   int32_t tok0[kStages][kMaxEntries];
@@ -104,6 +105,26 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[32]) {
     }
   }
   return v[0];   // lane L holds the reduction of value L
+}
+
+// Reduction of 16 values over the 32 lanes of a warp: lane L ends with the
+// reduction of value L % 16.
+template <bool kMax>
+__device__ __forceinline__ float transpose_reduce16(float (&v)[16]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 8, half = 8; o > 0; o >>= 1, half >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < half; ++i) {
+      const float send = upper ? v[i] : v[i + half];
+      const float keep = upper ? v[i + half] : v[i];
+      const float got = __shfl_xor_sync(0xffffffffu, send, o);
+      v[i] = kMax ? fmaxf(keep, got) : keep + got;
+    }
+  }
+  const float other = __shfl_xor_sync(0xffffffffu, v[0], 16);
+  return kMax ? fmaxf(v[0], other) : v[0] + other;
 }
 
 // 32 x 32 bit transpose across a warp: lane i holds row i (bit j = column j);
@@ -356,10 +377,10 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     }
     for (int bb = 0; bb < 2; ++bb) {
       tc::mbar_init(&ms.s_full[bb], 1);
-      tc::mbar_init(&ms.p_full[bb], 128);
+      tc::mbar_init(&ms.p_full[bb], 256);
     }
     tc::mbar_init(&ms.o_done, 1);
-    tc::mbar_init(&ms.q_ready, 128);
+    tc::mbar_init(&ms.q_ready, 256);
     tc::mbar_init(&ms.drain, 1);
   }
   if (kTma) {
@@ -589,28 +610,30 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       if (failed) atomicOr(&ms.err, 1u);
     }
   } else if (warp >= 4) {
-    // ---------------- softmax: thread = tile row / TMEM lane / output dim ----------------
-    const int sw = warp - 4;                       // TMEM lane quadrant sw
-    const int stid = tid - 128;
-    const int r = stid;
+    // ---------------- softmax: two warpgroups, thread = tile row / TMEM lane ----------------
+    // Warpgroup wg (warps 4 + 4 wg .. 7 + 4 wg) owns heads [16 wg, 16 wg + 16):
+    // its S and O columns, its part of P, its running maxima and row sums.
+    const int wg = (warp - 4) >> 2;
+    const int sw = warp & 3;                       // TMEM lane quadrant
+    const int stid = tid - 128;                    // 0..255 over both warpgroups
+    const int r = sw * 32 + lane;                  // tile row / output dim
+    const int q0 = kHalfQ * wg;
+    const int bar_id = 1 + 2 * wg;                 // named barrier of the warpgroup
     const uint32_t t_lane = uint32_t(sw * 32) << 16;
     const float scale2 = G.scale * 1.4426950408889634f;     // 1/sqrt(d) * log2(e)
-    // Running maxima live in ms.mrun[gp] (gp = parity of the group count of
-    // this span; the other buffer is reset for the next group); row sums of p
-    // in registers.
-    float lrow[kQ];
+    float lrow[kHalfQ];
 #pragma unroll
-    for (int q = 0; q < kQ; ++q) lrow[q] = 0.f;
-    int gp = 0;
+    for (int i = 0; i < kHalfQ; ++i) lrow[i] = 0.f;
+    int gp = 0;                                    // group parity: ms.mrun[gp] is live
 
     // Q of group vq -> two bf16 terms, K-major 128-byte-swizzled rows: row q the
-    // high term of head q, row 32 + q its low term.
+    // high term of head q, row 32 + q its low term (both warpgroups share it).
     auto write_q = [&](int vq) {
       const int nq = group_width(G, batch, q_blocks, vq);
-      const int q = stid >> 2, quarter = stid & 3;
+      const int q = stid >> 3, part = stid & 7;
 #pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8) {
-        const int col = quarter * 32 + c8 * 8;
+      for (int c8 = 0; c8 < 2; ++c8) {
+        const int col = part * 16 + c8 * 8;
         float x[8];
         if (q < nq) {
           const float* src = Q + head_of(G, q_blocks, vq, q) * kD + col;
@@ -667,14 +690,14 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       bad |= pending_bad;
       pending_bad = false;
       tc::fence_after_sync();
-      float s[kQ];
-      tc::tmem_ld32(tbase + t_lane + uint32_t(li & 1) * 64, s);
+      float s[kHalfQ];
+      {
+        const uint32_t col = tbase + t_lane + uint32_t(li & 1) * 64 + q0;
+        float s_lo[kHalfQ];
+        tc::tmem_ld16(col, s);
+        tc::tmem_ld16(col + 32, s_lo);
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {      // + the low-term products, 16 columns at a time
-        float s_lo[16];
-        tc::tmem_ld16(tbase + t_lane + uint32_t(li & 1) * 64 + 32 + 16 * h, s_lo);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) s[16 * h + i] += s_lo[i];
+        for (int i = 0; i < kHalfQ; ++i) s[i] += s_lo[i];
       }
       uint32_t rmask = 0u;
       {
@@ -684,73 +707,75 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           const int32_t tok0 = ms.tok0[st][j];
           if (tok0 >= 0 && rr < ms.nvalid[st][j]) rmask = (tok0 + rr == 0) ? allq : ms.emask[st][j];
         }
+        rmask >>= q0;
       }
+      const float* mrun = ms.mrun[gp] + q0;
       bool fire = false;
-      const float* mrun = ms.mrun[gp];
 #pragma unroll
-      for (int q = 0; q < kQ; ++q) {
-        s[q] = ((rmask >> q) & 1u) ? s[q] * scale2 : -INFINITY;
-        fire |= s[q] > mrun[q] + kRescaleSlack;
+      for (int i = 0; i < kHalfQ; ++i) {
+        s[i] = ((rmask >> i) & 1u) ? s[i] * scale2 : -INFINITY;
+        fire |= s[i] > mrun[i] + kRescaleSlack;
       }
       const uint32_t word = (__any_sync(0xffffffffu, fire) ? 1u : 0u) |
                             (__any_sync(0xffffffffu, bad) ? 2u : 0u);
-      if (lane == 0) ms.flags[li & 1][sw] = word;
-      tc::named_sync(1, 128);
-      const uint32_t all = ms.flags[li & 1][0] | ms.flags[li & 1][1] | ms.flags[li & 1][2] |
-                           ms.flags[li & 1][3];
+      if (lane == 0) ms.flags[li & 1][wg][sw] = word;
+      tc::named_sync(bar_id, 128);
+      const uint32_t all = ms.flags[li & 1][wg][0] | ms.flags[li & 1][wg][1] |
+                           ms.flags[li & 1][wg][2] | ms.flags[li & 1][wg][3];
       if (all & 2u) { failed = true; break; }
       // S of this tile is complete, so Q may be replaced for the next group now.
       if (end && t + 1 < t1) write_q(v + 1);
       if (all & 1u) {
-        // Raise the running maxima to this tile's (per head), rescale l and O.
-        float tmp[kQ];
+        // Raise this warpgroup's running maxima to the tile's, rescale l and O.
+        float tmp[kHalfQ];
 #pragma unroll
-        for (int q = 0; q < kQ; ++q) tmp[q] = s[q];
-        ms.red[0][sw][lane] = transpose_reduce32<true>(tmp);
-        tc::named_sync(1, 128);
-        if (sw == 0) {                   // lane = head
-          const float mt = fmaxf(fmaxf(ms.red[0][0][lane], ms.red[0][1][lane]),
-                                 fmaxf(ms.red[0][2][lane], ms.red[0][3][lane]));
-          const float mo = ms.mrun[gp][lane];
+        for (int i = 0; i < kHalfQ; ++i) tmp[i] = s[i];
+        const float wmax = transpose_reduce16<true>(tmp);
+        if (lane < kHalfQ) ms.red[0][wg][sw][lane] = wmax;
+        tc::named_sync(bar_id, 128);
+        if (sw == 0 && lane < kHalfQ) {  // lane = head q0 + lane
+          const float mt = fmaxf(fmaxf(ms.red[0][wg][0][lane], ms.red[0][wg][1][lane]),
+                                 fmaxf(ms.red[0][wg][2][lane], ms.red[0][wg][3][lane]));
+          const float mo = ms.mrun[gp][q0 + lane];
           const float mn = fmaxf(mo, mt);
-          ms.scl[lane] = mn == -INFINITY ? 1.f : exp2f(mo - mn);
-          ms.mrun[gp][lane] = mn;
+          ms.scl[q0 + lane] = mn == -INFINITY ? 1.f : exp2f(mo - mn);
+          ms.mrun[gp][q0 + lane] = mn;
         }
-        tc::named_sync(1, 128);
-        const float* scl = ms.scl;
+        tc::named_sync(bar_id, 128);
+        const float* scl = ms.scl + q0;
 #pragma unroll
-        for (int q = 0; q < kQ; ++q) lrow[q] *= scl[q];
+        for (int i = 0; i < kHalfQ; ++i) lrow[i] *= scl[i];
         if (!start) {                    // O holds earlier tiles of this group
           pending_bad |= !wait_pv(li - 1);
           tc::fence_after_sync();
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            float o[kQ];
-            tc::tmem_ld32(tbase + t_lane + kTmemO + 32 * h, o);
+            float o[kHalfQ];
+            tc::tmem_ld16(tbase + t_lane + kTmemO + 32 * h + q0, o);
 #pragma unroll
-            for (int q = 0; q < kQ; ++q) o[q] *= scl[q];
-            tc::tmem_st32(tbase + t_lane + kTmemO + 32 * h, o);
+            for (int i = 0; i < kHalfQ; ++i) o[i] *= scl[i];
+            tc::tmem_st16(tbase + t_lane + kTmemO + 32 * h + q0, o);
           }
         }
       }
       // p = 2^(s - m), stored MN-major over the stage's consumed K rows: row =
       // token, 64 bf16 (the high terms of the 32 heads, then the low terms),
-      // 128-byte swizzled.
+      // 128-byte swizzled; this warpgroup writes its 16 heads of each half.
       uint8_t* sP = smem + st * kStageBytes;
 #pragma unroll
-      for (int c = 0; c < kQ / 8; ++c) {
+      for (int c = 0; c < kHalfQ / 8; ++c) {
         __align__(16) __nv_bfloat16 hi[8], lo[8];
 #pragma unroll
         for (int jq = 0; jq < 8; ++jq) {
-          const int q = 8 * c + jq;
-          const float p = mrun[q] == -INFINITY ? 0.f : exp2f(s[q] - mrun[q]);
-          lrow[q] += p;
+          const int i = 8 * c + jq;
+          const float p = mrun[i] == -INFINITY ? 0.f : exp2f(s[i] - mrun[i]);
+          lrow[i] += p;
           hi[jq] = __float2bfloat16_rn(p);
           lo[jq] = __float2bfloat16_rn(p - __bfloat162float(hi[jq]));
         }
-        *reinterpret_cast<uint4*>(sP + tc::sw128_offset(r, 8 * c, kTok)) =
+        *reinterpret_cast<uint4*>(sP + tc::sw128_offset(r, q0 + 8 * c, kTok)) =
             *reinterpret_cast<const uint4*>(hi);
-        *reinterpret_cast<uint4*>(sP + tc::sw128_offset(r, 32 + 8 * c, kTok)) =
+        *reinterpret_cast<uint4*>(sP + tc::sw128_offset(r, kQ + q0 + 8 * c, kTok)) =
             *reinterpret_cast<const uint4*>(lo);
       }
       // PV of the previous tile must be complete before p_full of this one
@@ -764,39 +789,40 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         const bool bad2 = !wait_pv(li) || pending_bad;
         pending_bad = false;
         tc::fence_after_sync();
-        float o[kQ];
-        tc::tmem_ld32(tbase + t_lane + kTmemO, o);
+        float o[kHalfQ];
+        {
+          float o_lo[kHalfQ];
+          tc::tmem_ld16(tbase + t_lane + kTmemO + q0, o);
+          tc::tmem_ld16(tbase + t_lane + kTmemO + 32 + q0, o_lo);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          float o_lo[16];
-          tc::tmem_ld16(tbase + t_lane + kTmemO + 32 + 16 * h, o_lo);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) o[16 * h + i] += o_lo[i];
+          for (int i = 0; i < kHalfQ; ++i) o[i] += o_lo[i];
         }
-        float tmp[kQ];
+        float tmp[kHalfQ];
 #pragma unroll
-        for (int q = 0; q < kQ; ++q) tmp[q] = lrow[q];
-        ms.red[1][sw][lane] = transpose_reduce32<false>(tmp);
-        if (sw == 0) ms.mrun[gp ^ 1][lane] = -INFINITY;   // the next group starts afresh
-        if (tc::named_sync_or(1, 128, bad2)) { failed = true; break; }
+        for (int i = 0; i < kHalfQ; ++i) tmp[i] = lrow[i];
+        const float wsum = transpose_reduce16<false>(tmp);
+        if (lane < kHalfQ) ms.red[1][wg][sw][lane] = wsum;
+        if (sw == 0 && lane < kHalfQ) ms.mrun[gp ^ 1][q0 + lane] = -INFINITY;   // next group
+        if (tc::named_sync_or(bar_id, 128, bad2)) { failed = true; break; }
         const int nq = group_width(G, batch, q_blocks, v);
         float* base = slots + int64_t(cta + v) * kQ * (kD + 4);
 #pragma unroll
-        for (int q = 0; q < kQ; ++q)
-          if (q < nq) base[q * (kD + 4) + 4 + r] = o[q];
-        if (sw == 0 && lane < nq) {
-          const float mq = ms.mrun[gp][lane];
-          const float L = ms.red[1][0][lane] + ms.red[1][1][lane] + ms.red[1][2][lane] + ms.red[1][3][lane];
+        for (int i = 0; i < kHalfQ; ++i)
+          if (q0 + i < nq) base[(q0 + i) * (kD + 4) + 4 + r] = o[i];
+        if (sw == 0 && lane < kHalfQ && q0 + lane < nq) {
+          const float mq = ms.mrun[gp][q0 + lane];
+          const float L = ms.red[1][wg][0][lane] + ms.red[1][wg][1][lane] + ms.red[1][wg][2][lane] +
+                          ms.red[1][wg][3][lane];
           // maximum back to natural-log units
-          *reinterpret_cast<float4*>(base + lane * (kD + 4)) =
+          *reinterpret_cast<float4*>(base + (q0 + lane) * (kD + 4)) =
               make_float4(mq * 0.6931471805599453f, L, 0.f, 0.f);
         }
 #pragma unroll
-        for (int q = 0; q < kQ; ++q) lrow[q] = 0.f;
+        for (int i = 0; i < kHalfQ; ++i) lrow[i] = 0.f;
         gp ^= 1;
       }
     }
-    if (failed && stid == 0) atomicOr(&ms.err, 1u);
+    if (failed && (stid & 127) == 0) atomicOr(&ms.err, 1u);
   }
 
   tc::fence_before_sync();
