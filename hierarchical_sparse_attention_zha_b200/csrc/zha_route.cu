@@ -453,6 +453,10 @@ select_kernel(Geom G, SelectArgs a) {
 cudaError_t launch_score_tc(const Geom& G, int level, int64_t n_nodes, int64_t n_par, int32_t batch,
                             const float* Q, const uint32_t* kept_up, int64_t words_up, float* sigma,
                             const float* store, int32_t* status, cudaStream_t s);
+bool score_tma_supported(const Geom& G);
+cudaError_t launch_score_tma(const Geom& G, int level, int64_t n_nodes, int64_t n_par, int32_t batch,
+                             const float* Q, const uint32_t* kept_up, int64_t words_up, float* sigma,
+                             const float* store, int32_t* status, cudaStream_t s, bool* used);
 
 // ---------------------------------------------------------------------------
 // Host launcher: levels L..1, score then select.
@@ -532,7 +536,15 @@ cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n
     const int64_t words_up = level < G.levels ? lay.words[level + 1] : 0;
     float* sg = sigma + lay.sig_off[level];
     if (n_nodes > 0) {
-      if (G.d == 128 && G.nref <= 16)      // tensor cores (zha_score_tc.cu)
+      bool done = false;
+      if (score_tma_supported(G)) {      // tensor copies + tensor cores (zha_score_tma.cu)
+        e = launch_score_tma(G, level, n_nodes, n_par, batch, Q, up, words_up, sg, store, status, s,
+                             &done);
+        if (e != cudaSuccess) return e;
+      }
+      if (done)
+        ;
+      else if (G.d == 128 && G.nref <= 16)      // tensor cores (zha_score_tc.cu)
         e = launch_score_tc(G, level, n_nodes, n_par, batch, Q, up, words_up, sg, store, status, s);
       else
         e = G.d == 128 ? launch_score_d<128>(G, level, n_nodes, n_par, batch, Q, up, words_up, sg,
