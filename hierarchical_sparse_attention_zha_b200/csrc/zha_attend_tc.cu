@@ -63,7 +63,7 @@ constexpr int kThreads = 384;             // warps 0-1 producers, 2 MMA, 3 idle,
 constexpr int kHalfQ = 16;                // heads per softmax warpgroup
 constexpr int kProducers = 64;
 constexpr int kMaxEntries = 64;           // chunks per tile (C >= 2)
-constexpr uint32_t kWaitTries = 1u << 22;
+constexpr uint32_t kWaitTries = tc::kWaitPolls;
 constexpr uint32_t kPollLimit = 1u << 27; // polls of the MMA issuer without progress
 constexpr float kRescaleSlack = 8.f;      // log2 units: p may reach 2^8 before a rescale
 constexpr int kWinChunks = 16384;         // chunks per pass of the union fold

@@ -32,7 +32,7 @@ constexpr int kStNodes = 8;                // nodes per MMA tile (8 x 16 planes 
 constexpr int kStQ = 32;                   // query heads per CTA (MMA N)
 constexpr int kStD = 128;
 constexpr int kStTile = 64;                // nodes per CTA at most
-constexpr uint32_t kStWaitTries = 1u << 22;
+constexpr uint32_t kStWaitTries = tc::kWaitPolls;
 constexpr int kStOffA = 0;                 // 3 terms x [128 rows][64 cols] bf16 = 3 x 16 KB
 constexpr int kStOffQ = 3 * 16384;         // 3 terms x [2 col blocks][32 rows][128 B] = 3 x 8 KB
 constexpr int kStOffMisc = kStOffQ + 3 * 8192;

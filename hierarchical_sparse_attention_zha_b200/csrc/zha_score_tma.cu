@@ -20,7 +20,8 @@
 //                           128-byte swizzled, rows (node, plane) = MMA rows.
 //   converters (warps 4-11) thread = (row, 32-column box): each fp32 value ->
 //                           three bf16 terms (x = t0 + t1 + t2 to fp32's 24 bits),
-//                           stored from registers straight into tensor memory, where
+//                           stored from registers straight into tensor memory (three
+//                           half-buffers), where
 //                           the MMA reads its A operand (shared memory only carries
 //                           the raw tiles and Q)
 //   MMA issuer (warp 1)     S^T[(node, plane)][head] over the half's 4 K-steps:
@@ -53,11 +54,13 @@ constexpr int kRawBytes = 32768;          // [2 boxes][128 rows][128 B]
 constexpr int kOffRaw = 0;
 constexpr int kOffQ = kRawSlots * kRawBytes;          // 2 halves x [96 rows][128 B]
 constexpr int kOffMisc = kOffQ + 2 * 12288;
-constexpr int kThreads = 512;
+constexpr int kThreads = 512;             // warps: 0 producer, 1 MMA, 2-3 idle, 4-11 convert, 12-15 epilogue
 constexpr int kConv = 256;                // converter threads (warps 4-11)
-constexpr uint32_t kWaitTries = 1u << 22;
+constexpr int kEpiWarp0 = 12;
+constexpr uint32_t kWaitTries = tc::kWaitPolls;
 constexpr uint32_t kTmemCols = 512;       // D buffers (96 columns) at 0 and 128; A half-buffers
-constexpr uint32_t kTmemA = 256;          // (3 terms x 32 columns) at 256 and 384
+constexpr uint32_t kTmemA = 224;          // (3 terms x 32 columns) at 224, 320 and 416
+constexpr int kABufs = 3;
 
 struct Meta {                             // one half-tile, producer -> converters
   int32_t node0, group, half, flags;      // flags: 1 = first tile of a group, 2 = end
@@ -74,11 +77,11 @@ struct EMeta {                            // converters -> epilogue, per tile
 
 struct Misc {
   uint64_t raw_full[kRawSlots], raw_empty[kRawSlots];
-  uint64_t conv_done[2], a_free[2], d_full[2], d_free[2], q_ready;
+  uint64_t conv_done[kABufs], a_free[kABufs], d_full[2], d_free[2], q_ready;
   uint32_t tmem_base, err;
   Meta meta[kRawSlots];
   alignas(128) float bhat_raw[kRawSlots][kNodes * kR];  // tensor-copied with the first half of a tile
-  CMeta cmeta[2];
+  CMeta cmeta[kABufs];
   EMeta emeta[2];
 };
 
@@ -139,9 +142,11 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
       tc::mbar_init(&ms.raw_full[s], 1);
       tc::mbar_init(&ms.raw_empty[s], kConv);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kABufs; ++b) {
       tc::mbar_init(&ms.conv_done[b], kConv);
       tc::mbar_init(&ms.a_free[b], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&ms.d_full[b], 1);
       tc::mbar_init(&ms.d_free[b], 128);
       tc::mbar_init(&emeta_full[b], 1);
@@ -247,8 +252,8 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
       int seg = 0;
       bool failed = false;
       while (true) {
-        const int ab = int(k & 1);
-        if (!tc::mbar_wait(&ms.conv_done[ab], uint32_t((k >> 1) & 1), kWaitTries)) { failed = true; break; }
+        const int ab = int(k % kABufs);
+        if (!tc::mbar_wait(&ms.conv_done[ab], uint32_t((k / kABufs) & 1), kWaitTries)) { failed = true; break; }
         const CMeta cm = ms.cmeta[ab];
         if (cm.half == 0 || (cm.flags & 2)) {
           // The D buffer of this tile must have been read by the epilogue.
@@ -268,7 +273,7 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
         }
         tc::fence_after_sync();
         const uint32_t d = tbase + uint32_t(tile_i & 1) * 128;
-        const uint32_t tA = tbase + kTmemA + uint32_t(ab) * 128;     // term t at + 32 t
+        const uint32_t tA = tbase + kTmemA + uint32_t(ab) * 96;      // term t at + 32 t
         const uint32_t sQ = tc::smem_u32(smem + kOffQ) + uint32_t(cm.half) * 12288;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {           // K-step = 16 bf16 = 8 TMEM columns
@@ -286,7 +291,7 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
       }
       if (failed) atomicOr(&ms.err, 1u);
     }
-  } else if (warp >= 4 && warp < 12) {
+  } else if (warp >= 4 && warp < kEpiWarp0) {
     // ---------------- converters ----------------
     const int ctid = tid - 128;                     // 0..255
     const int cq = warp & 3;                        // TMEM lane quadrant
@@ -297,22 +302,23 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
     while (true) {
       const int slot = int(k % kRawSlots);
       const int64_t use = k / kRawSlots;
-      const int ab = int(k & 1);
+      const int ab = int(k % kABufs);
       bool bad = !tc::mbar_wait(&ms.raw_full[slot], uint32_t(use & 1), kWaitTries);
       if (tc::named_sync_or(1, kConv, bad)) { failed = true; break; }
       const Meta mt = ms.meta[slot];
       const bool end = (mt.flags & 2) != 0;
       // A half-buffer ab was last read by the MMAs of half k - 2; the tile's
       // metadata slot by the epilogue of tile_i - 2.
-      // (also before the end marker: the MMA issuer reads cmeta[ab] of half k - 2 first)
-      if (k >= 2) bad |= !tc::mbar_wait(&ms.a_free[ab], uint32_t(((k >> 1) - 1) & 1), kWaitTries);
+      // (also before the end marker: the MMA issuer reads cmeta[ab] of half k - 3 first)
+      if (k >= kABufs)
+        bad |= !tc::mbar_wait(&ms.a_free[ab], uint32_t(((k / kABufs) - 1) & 1), kWaitTries);
       if ((end || mt.half == 0) && tile_i >= 2)
         bad |= !tc::mbar_wait(&ms.d_free[tile_i & 1], uint32_t(((tile_i >> 1) - 1) & 1), kWaitTries);
       // A new group's Q replaces the old one once every MMA that reads it (the
       // previous half's) is complete.
       const bool new_q = !end && mt.half == 0 && (mt.flags & 1);
       if (new_q && k >= 1)
-        bad |= !tc::mbar_wait(&ms.a_free[(k - 1) & 1], uint32_t(((k - 1) >> 1) & 1), kWaitTries);
+        bad |= !tc::mbar_wait(&ms.a_free[(k - 1) % kABufs], uint32_t(((k - 1) / kABufs) & 1), kWaitTries);
       if (tc::named_sync_or(1, kConv, bad)) { failed = true; break; }
       if (end) {
         if (ctid == 0) {
@@ -381,7 +387,7 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
           split3_x2(x.x, x.y, t0[2 * c], t1[2 * c], t2[2 * c]);
           split3_x2(x.z, x.w, t0[2 * c + 1], t1[2 * c + 1], t2[2 * c + 1]);
         }
-        const uint32_t tA = tbase + (uint32_t(cq * 32) << 16) + kTmemA + uint32_t(ab) * 128 + cb * 16;
+        const uint32_t tA = tbase + (uint32_t(cq * 32) << 16) + kTmemA + uint32_t(ab) * 96 + cb * 16;
         tc::tmem_st16u(tA, t0);
         tc::tmem_st16u(tA + 32, t1);
         tc::tmem_st16u(tA + 64, t2);
@@ -398,7 +404,7 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
       ++k;
     }
     if (failed && ctid == 0) atomicOr(&ms.err, 1u);
-  } else if (warp >= 12) {
+  } else if (warp >= kEpiWarp0) {
     // ---------------- epilogue: thread = TMEM lane = (node, plane) row ----------------
     const int eq = warp & 3;
     const int r = eq * 32 + lane, nj = r >> 4, plane = r & 15;
@@ -417,15 +423,13 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
       const float bhat_r = ms.emeta[b].bhat[r];
       if (em_flags & 2) break;
       float v[kQn];
-      {
-        float w[kQn];
-        tc::tmem_ld32(tbase + t_lane + uint32_t(b) * 128, v);
-        tc::tmem_ld32(tbase + t_lane + uint32_t(b) * 128 + 32, w);
+      tc::tmem_ld32(tbase + t_lane + uint32_t(b) * 128, v);
 #pragma unroll
-        for (int q = 0; q < kQn; ++q) v[q] += w[q];
-        tc::tmem_ld32(tbase + t_lane + uint32_t(b) * 128 + 64, w);
+      for (int g4 = 0; g4 < 4; ++g4) {            // + column groups 32..63 and 64..95, 16 at a time
+        float w[16];
+        tc::tmem_ld16(tbase + t_lane + uint32_t(b) * 128 + 32 + 16 * g4, w);
 #pragma unroll
-        for (int q = 0; q < kQn; ++q) v[q] += w[q];
+        for (int i = 0; i < 16; ++i) v[16 * (g4 & 1) + i] += w[i];
       }
       tc::fence_before_sync();
       tc::mbar_arrive(&ms.d_free[b]);

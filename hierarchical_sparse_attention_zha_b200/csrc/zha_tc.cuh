@@ -194,6 +194,14 @@ __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[1
         "r"(v[15])
       : "memory");
 }
+// Warp-wide: store 8 consecutive 32-bit columns of raw bits (no wait).
+__device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+               :
+               : "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]),
+                 "r"(v[6]), "r"(v[7])
+               : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -235,18 +243,22 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 }
 
 // Wait for phase `parity` of the barrier to complete; gives up after
-// `max_tries` polls (each poll may suspend the thread for a short while) and
-// returns false then.
+// `max_tries` polls and returns false then. Each poll asks the hardware to
+// suspend the thread until the phase completes or kSuspendNs elapse, so a
+// waiting warp takes no issue slots from the warps doing the work; the whole
+// wait is bounded by about max_tries * kSuspendNs.
+constexpr uint32_t kSuspendNs = 65536;
+constexpr uint32_t kWaitPolls = 1u << 15;      // ~2 s with kSuspendNs
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t max_tries) {
   const uint32_t a = smem_u32(bar);
   for (uint32_t i = 0; i < max_tries; ++i) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok)
-        : "r"(a), "r"(parity)
+        : "r"(a), "r"(parity), "r"(kSuspendNs)
         : "memory");
     if (ok) return true;
   }
