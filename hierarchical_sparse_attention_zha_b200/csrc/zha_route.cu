@@ -316,8 +316,16 @@ select_kernel(Geom G, SelectArgs a) {
   const int64_t orphan0 = int64_t(C) * a.n_par;
   const int64_t n_child = int64_t(n_kp) * C;
   const int64_t n_c = n_child + (a.n_nodes - orphan0);
+  // Candidate i -> node: child (i % C) of kept parent i / C, or an orphan.
+  // Candidate and node indices fit 32 bits; the division is 32-bit.
+  const uint32_t uC = uint32_t(C), u_nchild = uint32_t(n_child);
   auto node_of = [&](int64_t i) -> int64_t {
-    return i < n_child ? int64_t(kp[i / C]) * C + i % C : orphan0 + (i - n_child);
+    const uint32_t ui = uint32_t(i);
+    if (ui < u_nchild) {
+      const uint32_t par = ui / uC;
+      return int64_t(kp[par]) * C + (ui - par * uC);
+    }
+    return orphan0 + (ui - u_nchild);
   };
   const float* sig = a.sigma + int64_t(bh) * a.n_nodes;
   const bool cached = n_c <= kSelectCache;
@@ -356,11 +364,27 @@ select_kernel(Geom G, SelectArgs a) {
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int k = lane; k < 256; k += 32) wh[k] = 0ull;
       __syncthreads();
+      // Runs of equal buckets are summed in a register and flushed once: the
+      // leading digits of nearby scores coincide, and per-element atomics on
+      // one bucket would serialise the whole warp.
+      uint32_t cb = 0xffffffffu;
+      unsigned long long cs = 0ull;
       for (int64_t i = tid; i < n_c; i += blockDim.x) {
         const float s = sigma_of(i);
         const uint32_t key = ~float_order_key(s);
-        if ((key & pmask) == prefix) atomicAdd(&wh[(key >> shift) & 255u], mass_of(s));
+        if ((key & pmask) == prefix) {
+          const uint32_t b = (key >> shift) & 255u;
+          const unsigned long long mm = mass_of(s);
+          if (b == cb) {
+            cs += mm;
+          } else {
+            if (cs != 0ull) atomicAdd(&wh[cb], cs);
+            cb = b;
+            cs = mm;
+          }
+        }
       }
+      if (cs != 0ull) atomicAdd(&wh[cb], cs);
       __syncthreads();
       // bucket totals into warp 0's histogram
       for (int k = tid; k < 256; k += blockDim.x) {
