@@ -835,24 +835,29 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 }
 
 // ---------------------------------------------------------------------------
-// 3. Combine: one warp per query head over the states of the CTAs whose span
-// met the head's group. CTA c covers tiles [c T / n, (c + 1) T / n), so the
-// CTA holding tile t is ((t + 1) n - 1) / T. Lane = 4 output dims.
+// 3. Combine: one CTA of 4 warps per query head over the states of the CTAs
+// whose span met the head's group. CTA c covers tiles [c T / n, (c + 1) T / n),
+// so the CTA holding tile t is ((t + 1) n - 1) / T. Warp w merges states
+// i = w, w + 4, ... (lane = 4 output dims); the four partial merges are then
+// combined through shared memory.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256)
+constexpr int kCombineWarps = 4;
+
+__global__ void __launch_bounds__(32 * kCombineWarps)
 combine_split_kernel(Geom G, int32_t batch, int32_t q_blocks, int32_t n_blocks, int32_t units,
                      const int32_t* __restrict__ split, const float* __restrict__ slots,
                      float* __restrict__ O, float* __restrict__ lse) {
-  const int lane = threadIdx.x & 31;
-  const int64_t bh = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (bh >= int64_t(batch) * G.hq) return;
+  __shared__ float4 s_acc[kCombineWarps][32];
+  __shared__ float s_m[kCombineWarps], s_l[kCombineWarps];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t bh = blockIdx.x;
   const int b = int(bh / G.hq), h = int(bh % G.hq);
   const int qi = b * G.group + h % G.group;
   const int v = (h / G.group) * q_blocks + qi / kQ, q = qi % kQ;
   const int64_t lo = split[v * n_blocks], hi = split[(v + 1) * n_blocks], T = split[units];
   const int64_t nct = split[units + 1];
   const int c_lo = int(((lo + 1) * nct - 1) / T), c_hi = int((hi * nct - 1) / T);
-  const int n_st = c_hi - c_lo + 1;
+  const int n_st = c_hi - c_lo + 1;                     // >= 1: every group has a tile
   // A CTA between c_lo and c_hi meets the group unless its span is empty (more
   // CTAs than tiles); only states that were written are read.
   auto written = [&](int i) -> bool {
@@ -862,26 +867,28 @@ combine_split_kernel(Geom G, int32_t batch, int32_t q_blocks, int32_t n_blocks, 
   auto state = [&](int i) -> const float* {
     return slots + (int64_t(c_lo + i + v) * kQ + q) * (kD + 4);
   };
-  float M = -INFINITY;
-  for (int i = lane; i < n_st; i += 32)
-    if (written(i)) {
-      const float2 ml = *reinterpret_cast<const float2*>(state(i));
-      if (ml.y > 0.f) M = fmaxf(M, ml.x);
-    }
-  M = warp_max(M);
-  float L = 0.f;
+  // This warp's states: i = warp + 4 (32 r + j); in round r lane j holds
+  // state (r, j)'s (m, l). Rounds are merged with the usual rescaling.
+  float M = -INFINITY, L = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i0 = 0; i0 < n_st; i0 += 32) {
-    float w = 0.f;
-    if (i0 + lane < n_st && written(i0 + lane)) {
-      const float2 ml = *reinterpret_cast<const float2*>(state(i0 + lane));
-      if (ml.y > 0.f) {
-        w = expf(ml.x - M);
-        L += w * ml.y;
-      }
+  for (int r0 = 0; warp + kCombineWarps * r0 < n_st; r0 += 32) {
+    float m_j = -INFINITY, l_j = 0.f;
+    const int i_lane = warp + kCombineWarps * (r0 + lane);
+    if (i_lane < n_st && written(i_lane)) {
+      const float2 ml = *reinterpret_cast<const float2*>(state(i_lane));
+      if (ml.y > 0.f) { m_j = ml.x; l_j = ml.y; }
     }
-    uint32_t ball = __ballot_sync(0xffffffffu, w > 0.f);
-    while (ball) {                 // up to four states per round, loads in flight together
+    const float Mr = warp_max(m_j);
+    if (Mr == -INFINITY) continue;
+    const float Mn = fmaxf(M, Mr);
+    const float sc = M == -INFINITY ? 0.f : expf(M - Mn);
+    L *= sc;
+    acc.x *= sc; acc.y *= sc; acc.z *= sc; acc.w *= sc;
+    M = Mn;
+    const float w_j = l_j > 0.f ? expf(m_j - M) : 0.f;
+    L += warp_sum(w_j * l_j);
+    uint32_t ball = __ballot_sync(0xffffffffu, w_j > 0.f);
+    while (ball) {                 // up to four states per step, loads in flight together
       int src[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
@@ -892,9 +899,10 @@ combine_split_kernel(Geom G, int32_t batch, int32_t q_blocks, int32_t n_blocks, 
       float wk[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        wk[k] = __shfl_sync(0xffffffffu, w, src[k] < 0 ? 0 : src[k]);
+        wk[k] = __shfl_sync(0xffffffffu, w_j, src[k] < 0 ? 0 : src[k]);
         o[k] = src[k] < 0 ? make_float4(0.f, 0.f, 0.f, 0.f)
-                          : *reinterpret_cast<const float4*>(state(i0 + src[k]) + 4 + 4 * lane);
+                          : *reinterpret_cast<const float4*>(
+                                state(warp + kCombineWarps * (r0 + src[k])) + 4 + 4 * lane);
         if (src[k] < 0) wk[k] = 0.f;
       }
 #pragma unroll
@@ -904,11 +912,28 @@ combine_split_kernel(Geom G, int32_t batch, int32_t q_blocks, int32_t n_blocks, 
       }
     }
   }
-  L = warp_sum(L);
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  *reinterpret_cast<float4*>(O + bh * kD + 4 * lane) =
-      make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-  if (lse != nullptr && lane == 0) lse[bh] = L > 0.f ? M + logf(L) : -INFINITY;
+  s_acc[warp][lane] = acc;
+  if (lane == 0) { s_m[warp] = M; s_l[warp] = L; }
+  __syncthreads();
+  if (warp == 0) {
+    float Mt = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w)
+      if (s_l[w] > 0.f) Mt = fmaxf(Mt, s_m[w]);
+    float Lt = 0.f;
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int w = 0; w < kCombineWarps; ++w) {
+      if (!(s_l[w] > 0.f)) continue;
+      const float r = expf(s_m[w] - Mt);
+      Lt += r * s_l[w];
+      const float4 a = s_acc[w][lane];
+      o.x += r * a.x; o.y += r * a.y; o.z += r * a.z; o.w += r * a.w;
+    }
+    const float inv = Lt > 0.f ? 1.f / Lt : 0.f;
+    *reinterpret_cast<float4*>(O + bh * kD + 4 * lane) = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+    if (lse != nullptr && lane == 0) lse[bh] = Lt > 0.f ? Mt + logf(Lt) : -INFINITY;
+  }
 }
 
 namespace {
@@ -990,7 +1015,7 @@ cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   const int64_t heads = int64_t(batch) * G.hq;
-  combine_split_kernel<<<unsigned((heads * 32 + 255) / 256), 256, 0, s>>>(
+  combine_split_kernel<<<unsigned(heads), 32 * kCombineWarps, 0, s>>>(
       G, batch, lay.q_blocks, lay.n_blocks, units, split, slots, O, lse);
   zha_count_launch();
   return cudaGetLastError();

@@ -26,6 +26,7 @@ constexpr int kScoreTile = 64;       // nodes per score CTA
 constexpr int kScoreQBlock = 64;     // query heads per score CTA (u64 masks)
 constexpr int kSelectThreads = 512;
 constexpr int kSelectCache = 16384;  // candidate scores cached in shared memory
+constexpr int kSelectKpCache = 4096;  // kept parents held in shared memory
 constexpr double kMassScale = 1099511627776.0;  // 2^40: fixed-point unit of probability
 
 // ---------------------------------------------------------------------------
@@ -280,6 +281,7 @@ select_kernel(Geom G, SelectArgs a) {
   extern __shared__ float4 smem_v4[];
   unsigned long long* hist = reinterpret_cast<unsigned long long*>(smem_v4);  // [nwarps][256]
   float* s_sig = reinterpret_cast<float*>(hist + (kSelectThreads / 32) * 256);
+  int32_t* s_kp = reinterpret_cast<int32_t*>(s_sig + kSelectCache);           // [kSelectKpCache]
   __shared__ float s_f[33];
   __shared__ unsigned long long s_u[33];
   __shared__ uint32_t s_w[33];
@@ -293,7 +295,9 @@ select_kernel(Geom G, SelectArgs a) {
   for (int64_t w = tid; w < a.words_here; w += blockDim.x) bits[w] = 0u;
 
   // Kept parents of this head, ascending (compaction of the level-(l+1) bitmap).
-  int32_t* kp = a.kp + int64_t(bh) * a.kp_stride;
+  // Parents fit in shared memory unless the level above is very wide.
+  const bool kp_in_smem = a.words_up <= kSelectKpCache / 32;
+  int32_t* kp = kp_in_smem ? s_kp : a.kp + int64_t(bh) * a.kp_stride;
   uint32_t n_kp = 0;
   if (a.kept_up != nullptr && a.words_up > 0) {
     const uint32_t* up = a.kept_up + int64_t(bh) * a.words_up;
@@ -311,7 +315,7 @@ select_kernel(Geom G, SelectArgs a) {
       n_kp += tot;
     }
   }
-  __syncthreads();   // kp visible to the block (global memory, same CTA)
+  __syncthreads();   // kp visible to the block
 
   const int64_t orphan0 = int64_t(C) * a.n_par;
   const int64_t n_child = int64_t(n_kp) * C;
@@ -329,8 +333,22 @@ select_kernel(Geom G, SelectArgs a) {
   };
   const float* sig = a.sigma + int64_t(bh) * a.n_nodes;
   const bool cached = n_c <= kSelectCache;
-  if (cached)
-    for (int64_t i = tid; i < n_c; i += blockDim.x) s_sig[i] = sig[node_of(i)];
+  if (cached) {
+    // Eight independent loads in flight per thread.
+    for (int64_t i0 = tid; i0 < n_c; i0 += 8 * int64_t(blockDim.x)) {
+      float v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t i = i0 + int64_t(u) * blockDim.x;
+        v[u] = i < n_c ? sig[node_of(i)] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t i = i0 + int64_t(u) * blockDim.x;
+        if (i < n_c) s_sig[i] = v[u];
+      }
+    }
+  }
   __syncthreads();
   auto sigma_of = [&](int64_t i) -> float { return cached ? s_sig[i] : sig[node_of(i)]; };
 
@@ -532,7 +550,7 @@ static cudaError_t launch_score_d(const Geom& G, int level, int64_t n_nodes, int
 
 size_t select_smem_bytes() {
   return size_t(kSelectThreads / 32) * 256 * sizeof(unsigned long long) +
-         size_t(kSelectCache) * sizeof(float);
+         size_t(kSelectCache) * sizeof(float) + size_t(kSelectKpCache) * sizeof(int32_t);
 }
 
 cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n_tokens, float p,

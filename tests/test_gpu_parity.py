@@ -311,3 +311,26 @@ def test_reference_query_counts_and_head_dims(zha, n_ref, head_dim, kv):
     spec = W.scaled("tiny", n_ref=n_ref, head_dim=head_dim, kv_dtype=kv, n_kv_heads=2, n_q_heads=8,
                     n_tokens=3000, chunk=8, levels=3, batch=5, n_needles=0)
     check_case(zha, W.generate(spec), 2990)
+
+
+@pytest.mark.gpu
+def test_one_group_spread_over_every_cta_matches_dense(zha):
+    """One KV head with <= 32 query heads is one attention group; with every
+    chunk listed its tiles outnumber the CTAs, so every CTA's span meets the
+    group and the combine merges more states than one pass of its warps holds."""
+    spec = W.scaled("32k", n_kv_heads=1, n_q_heads=4, n_tokens=40000 + 64, batch=2)
+    inp = W.generate(spec)
+    K, V, refq, Q = to_device(inp)
+    tree = zha.Tree(config_for(spec), refq)
+    n_tokens = 40000 + 17
+    n_ch = n_tokens // spec.chunk
+    ids = torch.arange(n_ch, dtype=torch.int32, device="cuda").repeat(spec.batch, spec.n_q_heads, 1)
+    cnt = torch.full((spec.batch, spec.n_q_heads), n_ch, dtype=torch.int32, device="cuda")
+    out, lse = tree.sparse_attend(Q[0].contiguous(), K, V, n_tokens, ids.contiguous(), cnt)
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    Kf, Vf = cache_f64(inp, 0, n_tokens), values_f64(inp, 0, n_tokens)
+    for b in range(spec.batch):
+        for h in range(spec.n_q_heads):
+            q = inp.Q[0, b, h].astype(np.float64)
+            _, dense = O.sdpa(q[None], Kf, Vf)
+            assert np.max(np.abs(out[b, h] - dense[0])) <= derived_o_bound(np.abs(Vf).max())
