@@ -189,6 +189,8 @@ union_prep_kernel(Geom G, int32_t batch, int32_t q_blocks, int32_t n_blocks, int
                   int32_t* status) {
   extern __shared__ uint32_t s_bits[];                 // [32][kRowWords]
   __shared__ uint32_t s_scan[33];
+  pdl_trigger();
+  pdl_wait();
   const int u = blockIdx.x, v = u / n_blocks, blk = u % n_blocks;
   const int tid = threadIdx.x, lane = tid & 31, q = tid >> 5;
   const int nq = group_width(G, batch, q_blocks, v);
@@ -334,6 +336,8 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
                                              ~uintptr_t(1023));
   Misc& ms = *reinterpret_cast<Misc*>(smem + kOffMisc);
   int32_t* s_toff = reinterpret_cast<int32_t*>(smem + kOffMisc + sizeof(Misc));   // [units + 1]
+  pdl_trigger();
+  pdl_wait();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int C = G.chunk;
   const int cpt = chunks_per_tile(C);
@@ -849,6 +853,8 @@ combine_split_kernel(Geom G, int32_t batch, int32_t q_blocks, int32_t n_blocks, 
                      float* __restrict__ O, float* __restrict__ lse) {
   __shared__ float4 s_acc[kCombineWarps][32];
   __shared__ float s_m[kCombineWarps], s_l[kCombineWarps];
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t bh = blockIdx.x;
   const int b = int(bh / G.hq), h = int(bh % G.hq);
@@ -988,11 +994,11 @@ cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const
   cudaError_t e = cudaFuncSetAttribute(union_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        int(prep_smem));
   if (e != cudaSuccess) return e;
-  union_prep_kernel<<<unsigned(units), 1024, prep_smem, s>>>(
-      G, batch, lay.q_blocks, lay.n_blocks, lay.block_chunks, nb, lay.n_chunks, chunk_ids, n_chunks,
-      max_sel, ids, masks, lay.cap, counts, status);
+  if ((e = launch_pdl(union_prep_kernel, dim3(unsigned(units)), dim3(1024), prep_smem, s, G, batch,
+                      lay.q_blocks, lay.n_blocks, lay.block_chunks, nb, lay.n_chunks, chunk_ids,
+                      n_chunks, max_sel, ids, masks, lay.cap, counts, status)) != cudaSuccess)
+    return e;
   zha_count_launch();
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   // Tensor copies when every chunk box starts on a swizzle atom (C % 8 == 0).
   CUtensorMap mk{}, mv{};
@@ -1007,18 +1013,18 @@ cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   const unsigned ctas = unsigned(sms < kTcMaxCtas ? sms : kTcMaxCtas);
-  kern<<<ctas, kThreads, smem, s>>>(
-      mk, mv, G, batch, lay.q_blocks, lay.n_blocks, lay.block_chunks, units, n_tokens, nb, Q,
-      static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V), ld, ids, masks,
-      lay.cap, counts, split, slots, status);
+  if ((e = launch_pdl(kern, dim3(ctas), dim3(kThreads), smem, s, mk, mv, G, batch, lay.q_blocks,
+                      lay.n_blocks, lay.block_chunks, units, n_tokens, nb, Q,
+                      static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V), ld,
+                      ids, masks, lay.cap, counts, split, slots, status)) != cudaSuccess)
+    return e;
   zha_count_launch();
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   const int64_t heads = int64_t(batch) * G.hq;
-  combine_split_kernel<<<unsigned(heads), 32 * kCombineWarps, 0, s>>>(
-      G, batch, lay.q_blocks, lay.n_blocks, units, split, slots, O, lse);
+  e = launch_pdl(combine_split_kernel, dim3(unsigned(heads)), dim3(32 * kCombineWarps), 0, s, G, batch,
+                 lay.q_blocks, lay.n_blocks, units, split, slots, O, lse);
   zha_count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace zha

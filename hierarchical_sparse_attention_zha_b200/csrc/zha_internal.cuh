@@ -182,6 +182,35 @@ inline TcAttendLayout tc_attend_layout(const Geom& g, int32_t batch, int64_t n_t
 inline bool use_tc_attend(const Geom& g) { return g.kv_bf16 && g.d == 128; }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch: a kernel launched with launch_pdl may be
+// scheduled while the previous kernel on the stream is finishing. It calls
+// pdl_trigger() on entry (its own dependents may then be scheduled once all of
+// its CTAs are resident) and pdl_wait() before it touches anything the previous
+// kernel wrote (pdl_wait returns once that kernel has completed and its memory
+// is visible). Both are no-ops for a kernel launched the ordinary way.
+// ---------------------------------------------------------------------------
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // Device helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float warp_sum(float v) {

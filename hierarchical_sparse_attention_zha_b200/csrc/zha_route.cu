@@ -67,6 +67,8 @@ score_kernel(Geom G, int level, int64_t n_nodes, int64_t n_par, int32_t batch, i
   constexpr int NW = kScoreThreads / 32;
   extern __shared__ float4 smem_v4[];
   float* s_kbuf = reinterpret_cast<float*>(smem_v4);       // [NW][KBUF]
+  pdl_trigger();
+  pdl_wait();
   float* s_q = s_kbuf + NW * S::KBUF;                       // [nq][P][QS]
   __shared__ unsigned long long s_mask[kScoreTile];
   __shared__ uint32_t s_kw[kScoreQBlock][3];
@@ -287,6 +289,8 @@ select_kernel(Geom G, SelectArgs a) {
   __shared__ uint32_t s_w[33];
   __shared__ uint32_t s_bucket;
   __shared__ unsigned long long s_before;
+  pdl_trigger();
+  pdl_wait();
 
   const int bh = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
@@ -520,10 +524,10 @@ static cudaError_t launch_score_t(const Geom& G, int level, int64_t n_nodes, int
   cudaError_t e = cudaFuncSetAttribute(score_kernel<D, RP>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  score_kernel<D, RP><<<grid, kScoreThreads, smem, s>>>(G, level, n_nodes, n_par, batch, tile, Q,
-                                                        kept_up, words_up, sigma, store);
+  e = launch_pdl(score_kernel<D, RP>, grid, dim3(kScoreThreads), smem, s, G, level, n_nodes, n_par,
+                 batch, tile, Q, kept_up, words_up, sigma, store);
   zha_count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 template <int D>
@@ -605,7 +609,8 @@ cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n
     a.sigma = sg;
     a.chunk_ids = level == 1 ? chunk_ids : nullptr;
     a.n_chunks = level == 1 ? n_chunks : nullptr;
-    select_kernel<<<heads, kSelectThreads, smem, s>>>(G, a);
+    if ((e = launch_pdl(select_kernel, dim3(heads), dim3(kSelectThreads), smem, s, G, a)) != cudaSuccess)
+      return e;
     zha_count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

@@ -75,6 +75,8 @@ score_tc_kernel(Geom G, int level, int64_t n_nodes, int64_t n_par, int32_t batch
                 const float* __restrict__ Q, const uint32_t* __restrict__ kept_up, int64_t words_up,
                 float* __restrict__ sigma, const float* __restrict__ store, int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
+  pdl_trigger();
+  pdl_wait();
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   StMisc& ms = *reinterpret_cast<StMisc*>(smem + kStOffMisc);
@@ -284,10 +286,10 @@ cudaError_t launch_score_tc(const Geom& G, int level, int64_t n_nodes, int64_t n
   int tile = kStTile;
   while (tile > kStNodes && (n_nodes * G.hkv) / tile < 2 * 148) tile >>= 1;
   dim3 grid(unsigned((n_nodes + tile - 1) / tile), unsigned(G.hkv), unsigned((qn + kStQ - 1) / kStQ));
-  score_tc_kernel<<<grid, kStThreads, smem, s>>>(G, level, n_nodes, n_par, batch, tile, Q, kept_up,
-                                                  words_up, sigma, store, status);
+  e = launch_pdl(score_tc_kernel, grid, dim3(kStThreads), smem, s, G, level, n_nodes, n_par, batch,
+                 tile, Q, kept_up, words_up, sigma, store, status);
   zha_count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace zha

@@ -153,11 +153,13 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
     }
     tc::mbar_init(&ms.q_ready, kConv);
   }
+  pdl_trigger();
   if (warp == 1) tc::tmem_alloc(&ms.tmem_base, kTmemCols);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tbase = ms.tmem_base;
+  pdl_wait();                                      // inputs of the previous kernel from here on
 
   if (warp == 0) {
     // ---------------- producer ----------------
@@ -530,11 +532,11 @@ cudaError_t launch_score_tma(const Geom& G, int level, int64_t n_nodes, int64_t 
   const int32_t groups = G.hkv * q_blocks;
   const int64_t tiles = groups * ((n_nodes + kNodes - 1) / kNodes);
   const unsigned ctas = unsigned(tiles < sms ? tiles : sms);
-  score_tma_kernel<<<ctas, kThreads, smem, s>>>(map, bmap, G, level, n_nodes, n_par, batch, q_blocks, groups,
-                                                 Q, kept_up, words_up, sigma, level_base, status);
+  e = launch_pdl(score_tma_kernel, dim3(ctas), dim3(kThreads), smem, s, map, bmap, G, level, n_nodes,
+                 n_par, batch, q_blocks, groups, Q, kept_up, words_up, sigma, level_base, status);
   zha_count_launch();
   *used = true;
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace zha
