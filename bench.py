@@ -48,7 +48,19 @@ def parse():
     ap.add_argument("--context", type=int, default=0,
                     help="override the workload's context length (profiling runs)")
     ap.add_argument("--flush-mb", type=int, default=512, help="L2 flush buffer between steps")
+    ap.add_argument("--dump-bytes", default="",
+                    help="write the algorithmic bytes of every timed step (JSON) to this path")
     return ap.parse_args()
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes per call measured by ncu on this workload (profiles/), if any."""
+    path = os.path.join(ROOT, "profiles", "traffic_1m_context.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    return d if d.get("workload") == workload else None
 
 
 def measured_peaks():
@@ -423,6 +435,16 @@ def run_zha(args, world, rank, local):
     dominant = "zha_route" if route_ms.sum() >= att_ms.sum() else "zha_sparse_attend"
     ach = route_gbs if dominant == "zha_route" else att_gbs
     per_launch = (route_b.mean() if dominant == "zha_route" else att_b.mean())
+    if args.dump_bytes and rank == 0:
+        with open(args.dump_bytes, "w") as f:
+            json.dump({"first_timed_step": W_steps, "route_bytes": route_b.tolist(),
+                       "attend_bytes": att_b.tolist()}, f)
+    traffic, traffic_note = None, None
+    mt = measured_traffic(spec.name)
+    if mt is not None and dominant in mt:
+        traffic = float(mt[dominant]["dram_bytes"])
+        traffic_note = (f"ncu dram bytes of one {dominant} call (step {mt['step']}, whose algorithmic "
+                        f"bytes were {mt[dominant]['algorithmic_bytes']:.0f}); see profiles/")
     non_app = ~np.array(appended)
     append_frac = float(app_ms[np.array(appended)].sum() / step_ms.sum()) if any(appended) else 0.0
 
@@ -484,7 +506,8 @@ def run_zha(args, world, rank, local):
                        "l2": f"flushed between timed steps ({args.flush_mb} MiB memset outside the events)",
                        "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
-                         "frac": ach / peak, "traffic": None, "kernel": dominant,
+                         "frac": ach / peak, "traffic": traffic, "traffic_note": traffic_note,
+                         "kernel": dominant,
                          "bytes_per_launch": float(per_launch), "peak_source": peak_kind},
             "step_roofline": {"achieved": step_gbs, "frac": step_gbs / peak,
                               "route_gbs": route_gbs, "attend_gbs": att_gbs,
