@@ -270,7 +270,8 @@ struct SelectArgs {
   const float* sigma;        // [B*Hq][n_nodes]
   int32_t* kp;               // scratch [B*Hq][kp_stride]
   int64_t kp_stride;
-  unsigned long long p_fixed;
+  unsigned long long p_fixed;    // p in units of 2^-40 (select_kernel)
+  unsigned long long p_fixed32;  // p in units of 2^-32 (select_fast_kernel)
   int keep_all;
   int32_t* chunk_ids;        // level 1 only
   int32_t* n_chunks;
@@ -496,6 +497,274 @@ select_kernel(Geom G, SelectArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Selection for one query head at one level, all candidates in shared memory
+// (n_nodes <= kFastMax). Each candidate's order key (score descending, then
+// index ascending) and its softmax mass in 2^-32 fixed point are computed once.
+//  * up to kFastSmallN candidates: thread i counts the mass of every candidate
+//    ordered before it; i is kept iff that mass is below p (the minimal prefix
+//    holding mass p). No radix passes, a handful of barriers.
+//  * more: the cut key by a radix select over 8-bit digits with per-warp
+//    histograms of mass, starting at the first byte in which the candidates'
+//    keys differ; runs of equal buckets are summed in registers before the
+//    atomic add.
+// The rounding of the fixed-point masses adds at most n 2^-33 to any
+// cumulative mass (< 2e-6 at n = 16384).
+// ---------------------------------------------------------------------------
+constexpr int kFastMax = 16384;
+constexpr int kFastSmallN = kSelectThreads;
+constexpr int kHistBins = (kSelectThreads / 32) * 256;   // per-warp 256-bin histograms
+
+__global__ void __launch_bounds__(kSelectThreads)
+select_fast_kernel(Geom G, SelectArgs a) {
+  extern __shared__ float4 smem_v4[];
+  uint32_t* s_key = reinterpret_cast<uint32_t*>(smem_v4);                    // scores, then keys
+  uint32_t* s_m = s_key + kFastMax;                                           // masses
+  unsigned long long* hist = reinterpret_cast<unsigned long long*>(s_m + kFastMax);   // [kHistBins]
+  int32_t* s_kp = reinterpret_cast<int32_t*>(hist + kHistBins);               // [kSelectKpCache]
+  float* s_sig = reinterpret_cast<float*>(s_key);
+  __shared__ float s_f[33];
+  __shared__ unsigned long long s_u[33];
+  __shared__ uint32_t s_w[33];
+  __shared__ uint32_t s_bucket;
+  __shared__ unsigned long long s_before;
+  pdl_trigger();
+  pdl_wait();
+
+  const int bh = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int C = G.chunk;
+  uint32_t* bits = a.kept_here + int64_t(bh) * a.words_here;
+  for (int64_t w = tid; w < a.words_here; w += blockDim.x) bits[w] = 0u;
+
+  // Kept parents of this head, ascending.
+  const bool kp_in_smem = a.words_up <= kSelectKpCache / 32;
+  int32_t* kp = kp_in_smem ? s_kp : a.kp + int64_t(bh) * a.kp_stride;
+  uint32_t n_kp = 0;
+  if (a.kept_up != nullptr && a.words_up > 0) {
+    const uint32_t* up = a.kept_up + int64_t(bh) * a.words_up;
+    for (int64_t w0 = 0; w0 < a.words_up; w0 += blockDim.x) {
+      const int64_t w = w0 + tid;
+      const uint32_t word = w < a.words_up ? up[w] : 0u;
+      uint32_t tot;
+      uint32_t pos = n_kp + block_excl_scan<uint32_t>(__popc(word), s_w, &tot);
+      uint32_t x = word;
+      while (x) {
+        const int bit = __ffs(x) - 1;
+        x &= x - 1u;
+        kp[pos++] = int32_t(w * 32 + bit);
+      }
+      n_kp += tot;
+    }
+  }
+  __syncthreads();
+
+  const int64_t orphan0 = int64_t(C) * a.n_par;
+  const uint32_t uC = uint32_t(C), n_child = n_kp * uC;
+  const int n_c = int(n_child + uint32_t(a.n_nodes - orphan0));
+  auto node_of = [&](int i) -> int64_t {
+    const uint32_t ui = uint32_t(i);
+    if (ui < n_child) {
+      const uint32_t par = ui / uC;
+      return int64_t(kp[par]) * C + (ui - par * uC);
+    }
+    return orphan0 + (ui - n_child);
+  };
+  const float* sig = a.sigma + int64_t(bh) * a.n_nodes;
+  for (int i0 = tid; i0 < n_c; i0 += 8 * kSelectThreads) {      // eight loads in flight
+    float v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * kSelectThreads;
+      v[u] = i < n_c ? sig[node_of(i)] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * kSelectThreads;
+      if (i < n_c) s_sig[i] = v[u];
+    }
+  }
+  __syncthreads();
+
+  // Softmax statistics, then keys and fixed-point masses (same arithmetic for
+  // every use of a candidate's mass).
+  float mx = -INFINITY;
+  for (int i = tid; i < n_c; i += kSelectThreads) mx = fmaxf(mx, s_sig[i]);
+  mx = block_max(mx, s_f);
+  float z = 0.f;
+  for (int i = tid; i < n_c; i += kSelectThreads) z += expf(s_sig[i] - mx);
+  z = block_sum(z, s_f);
+  const float scale32 = 4294967296.f / z;
+  auto mass_of = [&](float s) -> uint32_t { return __float2uint_rn(expf(s - mx) * scale32); };
+  unsigned long long tm = 0;
+  for (int i = tid; i < n_c; i += kSelectThreads) {
+    const float s = s_sig[i];
+    const uint32_t m = mass_of(s);
+    s_m[i] = m;
+    s_key[i] = ~float_order_key(s);
+    tm += m;
+  }
+  unsigned long long total;
+  block_excl_scan<unsigned long long>(tm, s_u, &total);      // its barriers publish s_key / s_m
+  const unsigned long long p32 = a.p_fixed32;
+  const bool keep_all = a.keep_all != 0 || n_c == 0 || total < p32;
+
+  uint32_t kept_total = 0;
+  auto emit = [&](int i, uint32_t pos) {
+    const int64_t node = node_of(i);
+    atomicOr(&bits[node >> 5], 1u << (node & 31));
+    if (a.chunk_ids != nullptr && pos < uint32_t(a.max_sel))
+      a.chunk_ids[int64_t(bh) * a.max_sel + pos] = int32_t(node);
+  };
+  if (keep_all || n_c <= kFastSmallN) {
+    // Thread i = candidate i (candidate order = ascending node index).
+    bool k = false;
+    if (tid < n_c) {
+      if (keep_all) {
+        k = true;
+      } else {
+        const uint32_t ki = s_key[tid];
+        unsigned long long cb = 0ull;
+        for (int j = 0; j < n_c; ++j) {
+          const uint32_t kj = s_key[j];
+          if (kj < ki || (kj == ki && j < tid)) cb += s_m[j];
+        }
+        k = cb < p32;
+      }
+    }
+    if (keep_all && n_c > kSelectThreads) {
+      // keep everything: thread-contiguous ranges, positions by a scan
+      const int per = (n_c + kSelectThreads - 1) / kSelectThreads;
+      const int i_lo = min(n_c, per * tid), i_hi = min(n_c, i_lo + per);
+      uint32_t pos = block_excl_scan<uint32_t>(uint32_t(i_hi - i_lo), s_w, &kept_total);
+      for (int i = i_lo; i < i_hi; ++i) emit(i, pos++);
+    } else {
+      const uint32_t pos = block_excl_scan<uint32_t>(k ? 1u : 0u, s_w, &kept_total);
+      if (k) emit(tid, pos);
+    }
+  } else {
+    // Leading bytes shared by every candidate's key are fixed up front.
+    uint32_t k_and = 0xffffffffu, k_or = 0u;
+    for (int i = tid; i < n_c; i += kSelectThreads) { k_and &= s_key[i]; k_or |= s_key[i]; }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      k_and &= __shfl_xor_sync(0xffffffffu, k_and, o);
+      k_or |= __shfl_xor_sync(0xffffffffu, k_or, o);
+    }
+    if (lane == 0) { s_w[warp] = k_and; s_w[16 + warp] = k_or; }
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t x = 0xffffffffu, y = 0u;
+      for (int w = 0; w < kSelectThreads / 32; ++w) { x &= s_w[w]; y |= s_w[16 + w]; }
+      s_w[32] = x;
+      s_bucket = y;
+    }
+    __syncthreads();
+    k_and = s_w[32];
+    k_or = s_bucket;
+    const int lead = (k_and ^ k_or) == 0u ? 32 : __clz(k_and ^ k_or);   // common leading bits
+    const int first_byte = min(lead / 8, 3);
+    uint32_t pmask = first_byte == 0 ? 0u : ~0u << (32 - 8 * first_byte);
+    uint32_t prefix = k_and & pmask;
+    unsigned long long before = 0ull;
+    unsigned long long* wh = hist + warp * 256;
+#pragma unroll 1
+    for (int shift = 24 - 8 * first_byte; shift >= 0; shift -= 8) {
+      for (int k = lane; k < 256; k += 32) wh[k] = 0ull;
+      __syncthreads();
+      uint32_t cb = 0xffffffffu;
+      unsigned long long cs = 0ull;
+      for (int i = tid; i < n_c; i += kSelectThreads) {
+        const uint32_t key = s_key[i];
+        if ((key & pmask) == prefix) {
+          const uint32_t bkt = (key >> shift) & 255u;
+          if (bkt == cb) {
+            cs += s_m[i];
+          } else {
+            if (cs != 0ull) atomicAdd(&wh[cb], cs);
+            cb = bkt;
+            cs = s_m[i];
+          }
+        }
+      }
+      if (cs != 0ull) atomicAdd(&wh[cb], cs);
+      __syncthreads();
+      for (int k = tid; k < 256; k += kSelectThreads) {     // bucket totals into warp 0's histogram
+        unsigned long long v = 0ull;
+        for (int w = 0; w < kSelectThreads / 32; ++w) v += hist[w * 256 + k];
+        hist[k] = v;
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane owns buckets [8 lane, 8 lane + 8): first bucket whose cumulative
+        // mass (with `before`) reaches p
+        unsigned long long loc[8], run = 0ull;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) { loc[k] = hist[8 * lane + k]; run += loc[k]; }
+        const unsigned long long incl = warp_incl_scan<unsigned long long>(run);
+        unsigned long long acc = before + incl - run, acc_before = 0ull;
+        int found = -1;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (found < 0 && acc + loc[k] >= p32) { found = 8 * lane + k; acc_before = acc; }
+          acc += loc[k];
+        }
+        const unsigned ball = __ballot_sync(0xffffffffu, found >= 0);
+        const int src = ball ? __ffs(ball) - 1 : 31;
+        const int fb = __shfl_sync(0xffffffffu, found, src);
+        const unsigned long long ab = __shfl_sync(0xffffffffu, acc_before, src);
+        if (lane == 0) {
+          s_bucket = fb < 0 ? 255u : uint32_t(fb);
+          s_before = fb < 0 ? before : ab;
+        }
+      }
+      __syncthreads();
+      prefix |= s_bucket << shift;
+      pmask |= 255u << shift;
+      before = s_before;
+      __syncthreads();                                      // s_bucket / s_before are reused
+    }
+    const uint32_t key_cut = prefix;
+    const uint32_t m_cut = mass_of(order_key_float(~key_cut));
+    const unsigned long long need = p32 > before ? p32 - before : 0ull;
+    const unsigned long long t_keep = m_cut > 0u ? (need + m_cut - 1ull) / m_cut : 0ull;
+    // Kept flags in candidate order: thread-contiguous ranges so that ties at
+    // the cut are taken lowest index first.
+    const int per = (n_c + kSelectThreads - 1) / kSelectThreads;
+    const int i_lo = min(n_c, per * tid), i_hi = min(n_c, i_lo + per);
+    uint32_t my_ties = 0;
+    for (int i = i_lo; i < i_hi; ++i) my_ties += (s_key[i] == key_cut);
+    uint32_t tie_total;
+    const uint32_t tie_rank = block_excl_scan<uint32_t>(my_ties, s_w, &tie_total);
+    uint32_t my_kept = 0;
+    {
+      uint32_t tr = tie_rank;
+      for (int i = i_lo; i < i_hi; ++i) {
+        const uint32_t key = s_key[i];
+        my_kept += (key < key_cut || (key == key_cut && tr++ < t_keep)) ? 1u : 0u;
+      }
+    }
+    uint32_t pos = block_excl_scan<uint32_t>(my_kept, s_w, &kept_total);
+    {
+      uint32_t tr = tie_rank;
+      for (int i = i_lo; i < i_hi; ++i) {
+        const uint32_t key = s_key[i];
+        if (key < key_cut || (key == key_cut && tr++ < t_keep)) emit(i, pos++);
+      }
+    }
+  }
+  if (a.chunk_ids != nullptr && tid == 0) {
+    a.n_chunks[bh] = int32_t(kept_total);
+    if (kept_total > uint32_t(a.max_sel) && a.status != nullptr)
+      atomicOr(a.status, ZHA_DEV_SELECTION_TRUNCATED);
+  }
+}
+
+size_t select_fast_smem_bytes() {
+  return size_t(2 * kFastMax) * sizeof(uint32_t) + size_t(kHistBins) * sizeof(unsigned long long) +
+         size_t(kSelectKpCache) * sizeof(int32_t);
+}
+
 cudaError_t launch_score_tc(const Geom& G, int level, int64_t n_nodes, int64_t n_par, int32_t batch,
                             const float* Q, const uint32_t* kept_up, int64_t words_up, float* sigma,
                             const float* store, int32_t* status, cudaStream_t s);
@@ -569,6 +838,12 @@ cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n
   SelectArgs a{};
   a.p_fixed = (unsigned long long)ceil(double(p) * kMassScale);
   if (a.p_fixed == 0) a.p_fixed = 1;
+  a.p_fixed32 = (unsigned long long)ceil(double(p) * 4294967296.0);
+  if (a.p_fixed32 == 0) a.p_fixed32 = 1;
+  const size_t smem_fast = select_fast_smem_bytes();
+  if ((e = cudaFuncSetAttribute(select_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(smem_fast))) != cudaSuccess)
+    return e;
   a.keep_all = p >= 1.0f;
   a.kp = kp;
   int64_t kp_stride = lay.kp_ints / (heads > 0 ? heads : 1);
@@ -609,8 +884,11 @@ cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n
     a.sigma = sg;
     a.chunk_ids = level == 1 ? chunk_ids : nullptr;
     a.n_chunks = level == 1 ? n_chunks : nullptr;
-    if ((e = launch_pdl(select_kernel, dim3(heads), dim3(kSelectThreads), smem, s, G, a)) != cudaSuccess)
-      return e;
+    if (n_nodes <= kFastMax)
+      e = launch_pdl(select_fast_kernel, dim3(heads), dim3(kSelectThreads), smem_fast, s, G, a);
+    else
+      e = launch_pdl(select_kernel, dim3(heads), dim3(kSelectThreads), smem, s, G, a);
+    if (e != cudaSuccess) return e;
     zha_count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
