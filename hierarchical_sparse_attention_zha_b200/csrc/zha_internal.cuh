@@ -93,18 +93,10 @@ inline int32_t attend_range_chunks(int32_t chunk) {
   return w < 1 ? 1 : w;
 }
 
-// After the slots: per query head, the index in its chunk list of the first
-// entry of each range ([n_ranges + 1] int32, the last = end of the in-range
-// entries) plus one flag word (1 if the list starts with chunk 0); then two
-// counters (work items written, work items taken) and the work-item table of
-// the tensor-core path: per (KV head, block of 32 query heads, range) with
-// work, [header(4) | chunk offsets in the range (W) | head masks (W)] uint32.
-constexpr int kAttendHeadsPerBlock = 32;
+constexpr int kAttendHeadsPerBlock = 32;   // query heads per attention group
 
 struct AttendLayout {
   int64_t n_chunks, n_ranges, slots_per_head, slot_floats, bytes;
-  int64_t ptr_offset_bytes, ptr_stride;
-  int64_t counter_offset_bytes, item_offset_bytes, item_words, max_items;
   int32_t range_chunks, q_blocks;
 };
 
@@ -118,13 +110,7 @@ inline AttendLayout attend_layout(const Geom& g, int32_t batch, int64_t n_tokens
   a.slots_per_head = a.n_ranges + 1;
   a.slot_floats = g.d + 4;
   a.q_blocks = int32_t((int64_t(batch) * g.group + kAttendHeadsPerBlock - 1) / kAttendHeadsPerBlock);
-  a.ptr_offset_bytes = round_up(heads * a.slots_per_head * a.slot_floats * 4, 256);
-  a.ptr_stride = a.n_ranges + 2;
-  a.counter_offset_bytes = a.ptr_offset_bytes + round_up(heads * a.ptr_stride * 4, 256);
-  a.item_offset_bytes = a.counter_offset_bytes + 256;
-  a.item_words = 4 + 2 * int64_t(a.range_chunks);
-  a.max_items = int64_t(g.hkv) * a.q_blocks * (a.n_ranges + 1);
-  a.bytes = a.item_offset_bytes + round_up(a.max_items * a.item_words * 4, 256);
+  a.bytes = round_up(heads * a.slots_per_head * a.slot_floats * 4, 256);
   return a;
 }
 
