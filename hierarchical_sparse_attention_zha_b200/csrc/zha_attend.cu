@@ -16,9 +16,9 @@
 // heads selected inside the range, streams them once through shared memory and
 // updates a per-head online-softmax state for the heads that selected each
 // chunk. One more CTA per (KV head, block) covers the tail [N_b, N) and the
-// sink. The range states are merged by combine_ranges_kernel (zha_attend_tc.cu).
+// sink. The range states are merged by combine_ranges_kernel (below).
 // This CUDA-core kernel serves fp32 caches and head_dim 64; bf16 caches with
-// head_dim 128 go to the tensor-core kernel in zha_attend_tc.cu.
+// head_dim 128 go to the tensor-core kernels in zha_attend_tc.cu.
 #include "zha_internal.cuh"
 
 namespace zha {

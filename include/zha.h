@@ -58,7 +58,7 @@ typedef enum {
 
 /* Bits OR-ed into *d_status by device code. */
 #define ZHA_DEV_SELECTION_TRUNCATED 1 /* zha_route: a head kept more than max_sel chunks; its list holds the first max_sel (ascending) and d_n_chunks the true count */
-#define ZHA_DEV_BAD_SELECTION 2       /* zha_sparse_attend: a chunk list had an id out of range, was not strictly ascending, or a count above max_sel; the offending entries were skipped */
+#define ZHA_DEV_BAD_SELECTION 2       /* zha_sparse_attend: a chunk list had an id out of range, was not strictly ascending, or a count outside [0, max_sel]; out-of-range ids are never read, and which in-range entries of such a list are attended is unspecified */
 #define ZHA_DEV_TIMEOUT 4             /* a kernel's bounded wait for its tensor-core work ran out; its outputs are not valid (it released its resources and returned) */
 
 typedef enum { ZHA_F32 = 0, ZHA_BF16 = 1 } zha_dtype;

@@ -155,3 +155,25 @@ def test_no_cpu_fallback_exists():
     src = open(os.path.join(os.path.dirname(pkg.__file__), "zha.py")).read()
     assert "import oracle" not in src and "from oracle" not in src
     assert "numpy" not in src
+
+
+def test_split_arithmetic_of_the_tensor_core_attention():
+    """The combine finds the CTAs whose span met a group from the tile offsets
+    alone: CTA c covers tiles [c T / n, (c + 1) T / n), so tile t belongs to CTA
+    ((t + 1) n - 1) / T, and a CTA between two such CTAs wrote a state iff its
+    span is non-empty. Checked exhaustively for small T and the launch sizes."""
+    for n in (1, 2, 7, 148, 296):
+        for T in range(1, 700):
+            start = [c * T // n for c in range(n + 1)]
+            for t in range(T):
+                c = ((t + 1) * n - 1) // T
+                assert start[c] <= t < start[c + 1]
+            # a group occupying tiles [lo, hi): the CTAs the combine visits are
+            # exactly those whose span intersects it
+            for lo, hi in ((0, T), (T // 3, T // 3 + 1), (T // 2, T)):
+                if lo >= hi:
+                    continue
+                c_lo, c_hi = ((lo + 1) * n - 1) // T, (hi * n - 1) // T
+                visited = {c for c in range(c_lo, c_hi + 1) if (c + 1) * T // n > c * T // n}
+                meets = {c for c in range(n) if max(start[c], lo) < min(start[c + 1], hi)}
+                assert visited == meets
