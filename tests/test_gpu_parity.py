@@ -334,3 +334,12 @@ def test_one_group_spread_over_every_cta_matches_dense(zha):
             q = inp.Q[0, b, h].astype(np.float64)
             _, dense = O.sdpa(q[None], Kf, Vf)
             assert np.max(np.abs(out[b, h] - dense[0])) <= derived_o_bound(np.abs(Vf).max())
+
+
+@pytest.mark.gpu
+def test_more_than_32_queries_per_kv_head(zha):
+    """64 query heads per KV head (batch 8 x GQA 8): each KV head's queries
+    form two attention groups and two scoring groups."""
+    spec = W.scaled("1m", n_kv_heads=2, n_q_heads=16, n_tokens=8192, stream_tokens=128, batch=8,
+                    n_needles=2)
+    check_case(zha, W.generate(spec), 8192 + 77)
