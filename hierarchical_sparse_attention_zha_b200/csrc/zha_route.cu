@@ -8,15 +8,18 @@
 // parentless chunks down (전제와 한계).
 //
 // Per level l = L..1 the host launches two kernels:
-//   score_kernel  -- one warp per candidate node (the union over the query heads
-//                    of a KV head), the node's R planes held in registers (lane
-//                    = part of one plane's row), one score per query head that
-//                    has the node as candidate; head_dim 128 with R <= 16 uses
-//                    the tensor-core scorer in zha_score_tc.cu instead;
-//   select_kernel -- one CTA per query head: softmax over its candidates, radix
-//                    select of the cut on the key (score desc, node index asc)
-//                    with fixed-point mass histograms, kept bitmap (and at
-//                    level 1 the ascending chunk list).
+//   scoring -- head_dim 128 with R = 16: score_tma_kernel (zha_score_tma.cu,
+//              tensor copies + tcgen05); head_dim 128 with R < 16:
+//              score_tc_kernel (zha_score_tc.cu); otherwise score_kernel here
+//              (one warp per candidate node -- the union over the query heads of
+//              a KV head -- its R planes in registers, one score per query head
+//              that has the node as candidate);
+//   selection -- one CTA per query head: softmax over its candidates, the cut
+//              on the key (score desc, node index asc) by fixed-point mass, kept
+//              bitmap (and at level 1 the ascending chunk list).
+//              select_fast_kernel when the level fits in shared memory
+//              (<= 16384 nodes), select_kernel otherwise.
+// Both kinds are launched with programmatic dependent launch.
 #include "zha_internal.cuh"
 
 namespace zha {

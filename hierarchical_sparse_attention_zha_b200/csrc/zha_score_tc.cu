@@ -1,5 +1,6 @@
-// zha_score_tc.cu -- node scoring on the sm_100a tensor cores (head_dim 128,
-// up to 16 reference queries per tree).
+// zha_score_tc.cu -- node scoring on the sm_100a tensor cores for head_dim 128
+// and fewer than 16 reference queries per tree (R = 16 goes to the tensor-copy
+// kernel in zha_score_tma.cu).
 //
 // Citations: [ZHA: 무엇과 다른가 / 전제와 한계] = page "ZHA는 KV 캐시를 트리로 요약해
 // 어텐션 비용을 준(sub)이차로 낮춘다" (onedev.kr/papers/1556): a node's estimated log

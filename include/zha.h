@@ -158,7 +158,7 @@ size_t zha_route_kept_words(const zha_config* cfg, int32_t batch, int64_t n_toke
  * ids ascending, and d_n_chunks [batch][n_q_heads] their count (the sink and
  * the tail [N_b, n_tokens) are implicit and not listed). d_kept_bits (nullable,
  * zha_route_kept_words words) receives every level's kept bitmap. d_ws:
- * >= zha_route_workspace_bytes bytes. d_status: ZHA_DEV_SELECTION_TRUNCATED. */
+ * >= zha_route_workspace_bytes bytes. d_status: ZHA_DEV_SELECTION_TRUNCATED, ZHA_DEV_TIMEOUT (tensor-core scoring). */
 zha_status zha_route(const zha_tree* tree, const float* d_Q, int32_t batch, int64_t n_tokens,
                      float p, int32_t* d_chunk_ids, int32_t* d_n_chunks, int32_t max_sel,
                      uint32_t* d_kept_bits, void* d_ws, size_t ws_bytes, int32_t* d_status,
