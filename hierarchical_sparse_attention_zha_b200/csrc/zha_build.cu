@@ -10,6 +10,9 @@
 #include "zha_internal.cuh"
 
 namespace zha {
+cudaError_t launch_build_level1_tc(const Geom& G, const void* K, int64_t ld, int64_t c_begin,
+                                   int64_t c_end, const float* refq, float* store, int32_t* status,
+                                   cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // Level 1. One CTA summarises a tile of `nch` consecutive chunks (nch*C <= 128
@@ -270,7 +273,10 @@ static cudaError_t launch_build_t(const Geom& G, const void* K, int64_t ld, int6
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   const int64_t c_begin = nb_old / G.chunk, c_end = nb_new / G.chunk;
-  if (c_end > c_begin) {
+  // bf16, d = 128, R = 16, C = 64: the tensor-core level 1 (zha_build_tc.cu).
+  const cudaError_t etc = launch_build_level1_tc(G, K, ld, c_begin, c_end, refq, store, nullptr, s);
+  if (etc != cudaSuccess && etc != cudaErrorNotSupported) return etc;
+  if (etc != cudaSuccess && c_end > c_begin) {
     const int cpt = l1_chunks_per_tile(G.chunk);
     dim3 grid(unsigned((c_end - c_begin + cpt - 1) / cpt), unsigned(G.hkv));
     build_level1_kernel<T, D><<<grid, kBuildThreads, smem, s>>>(
