@@ -21,6 +21,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <mutex>
+
 #include "zha_internal.cuh"
 #include "zha_tc.cuh"
 
@@ -298,13 +300,14 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
 namespace {
 PFN_cuTensorMapEncodeTiled_v12000 build_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
+  static std::once_flag once;
+  std::call_once(once, [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q{};
     if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
             cudaSuccess && q == cudaDriverEntryPointSuccess)
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+  });
   return fn;
 }
 }  // namespace
