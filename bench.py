@@ -6,6 +6,13 @@ zha_route and zha_sparse_attend process the step's batch of queries at the
 current context length. Inputs are resident in HBM; L2 is flushed (a 512 MiB
 memset) between timed steps, outside the timed events.
 
+The timed window starts 2C - 5 tokens past the workload's context, so that level
+1 holds one node more than at the context itself (16385 at 1M tokens: the
+wide-level selection) and a chunk completes at the window's fifth step (the
+append is timed with the step). Before it, a traced pass (CUDA events around
+every library kernel) gives each kernel's share of the step; inside it, events
+around the dominant kernel's launches give the roofline figure.
+
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 1m|256k|32k|deep|tiny]
                     [--impl zha|reference]
 
@@ -34,6 +41,7 @@ from hierarchical_sparse_attention_zha_b200 import workloads as W  # noqa: E402
 
 METRIC = "routed decode queries/sec/GPU at context N; achieved HBM GB/s vs roofline"
 UNIT = "queries/s"
+L2_NOTE = "GPU arm: L2 flushed between timed steps; CPU arm: not applicable"
 
 
 def parse():
@@ -50,17 +58,32 @@ def parse():
     ap.add_argument("--flush-mb", type=int, default=512, help="L2 flush buffer between steps")
     ap.add_argument("--dump-bytes", default="",
                     help="write the algorithmic bytes of every timed step (JSON) to this path")
+    ap.add_argument("--trace-steps", type=int, default=32,
+                    help="steps of the traced pass before the timed region (0: none)")
+    ap.add_argument("--cpu-budget", type=float, default=12.0,
+                    help="seconds of oracle work per leg of the CPU baseline")
     return ap.parse_args()
 
 
-def measured_traffic(workload: str):
-    """DRAM bytes per call measured by ncu on this workload (profiles/), if any."""
-    path = os.path.join(ROOT, "profiles", "traffic_1m_context.json")
+def measured_traffic(workload: str, kernel_key: str):
+    """DRAM bytes per launch of `kernel_key` measured by ncu on this workload
+    (profiles/traffic_<workload>.json), or None. The record names the kernel's
+    source file and its SHA-256 when captured; a changed source voids it."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", f"traffic_{workload.lower().replace(' ', '_')}.json")
     if not os.path.exists(path):
-        return None
+        return None, None
     with open(path) as f:
         d = json.load(f)
-    return d if d.get("workload") == workload else None
+    rec = d.get("kernels", {}).get(kernel_key)
+    if d.get("workload") != workload or rec is None:
+        return None, None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["source_sha256"]:
+        return None, f"ncu traffic of {kernel_key} predates the current {rec['source']}"
+    return float(rec["dram_bytes_per_launch"]), (
+        f"ncu dram__bytes_read.sum + dram__bytes_write.sum of one {kernel_key} launch "
+        f"({rec.get('note', 'see profiles/')})")
 
 
 def measured_peaks():
@@ -80,7 +103,7 @@ def step_bytes(spec: W.Workload, bits: np.ndarray, ids: np.ndarray, cnt: np.ndar
                n_tokens: int, batch: int) -> dict:
     """Bytes the step must move: unique summaries visited per KV head and level,
     unique selected K/V rows per KV head (sink and tail included), Q in, O and
-    lse out."""
+    lse out; per level also the (query head, candidate) pairs scored."""
     C, L, R, d, G = spec.chunk, spec.levels, spec.n_ref, spec.head_dim, spec.group
     nb = C * (n_tokens // C)
     node_bytes = R * (d + 1) * 4
@@ -95,8 +118,7 @@ def step_bytes(spec: W.Workload, bits: np.ndarray, ids: np.ndarray, cnt: np.ndar
     for l in range(1, L + 1):
         blk = bits[offs[l]: offs[l] + batch * spec.n_q_heads * words[l]].reshape(batch, spec.n_q_heads, words[l])
         kept[l] = np.unpackbits(blk.view(np.uint8), axis=-1, bitorder="little")[..., : n_l[l]].astype(bool)
-    summ_nodes = 0
-    pairs = 0
+    levels = {l: {"nodes": 0, "pairs": 0} for l in range(1, L + 1)}
     for g in range(spec.n_kv_heads):
         hs = slice(g * G, (g + 1) * G)
         for l in range(1, L + 1):
@@ -107,8 +129,9 @@ def step_bytes(spec: W.Workload, bits: np.ndarray, ids: np.ndarray, cnt: np.ndar
             cand[..., orphan0:] = True
             if l < L and orphan0 > 0:
                 cand[..., :orphan0] = np.repeat(kept[l + 1][:, hs, : n_l[l + 1]], C, axis=-1)
-            summ_nodes += int(cand.any(axis=(0, 1)).sum())
-            pairs += int(cand.sum())
+            levels[l]["nodes"] += int(cand.any(axis=(0, 1)).sum())
+            levels[l]["pairs"] += int(cand.sum())
+    summ_nodes = sum(v["nodes"] for v in levels.values())
     kv_tokens = 0
     tail = n_tokens - nb
     for g in range(spec.n_kv_heads):
@@ -126,12 +149,31 @@ def step_bytes(spec: W.Workload, bits: np.ndarray, ids: np.ndarray, cnt: np.ndar
     return {
         "summary_bytes": summ_nodes * node_bytes,
         "summary_nodes": summ_nodes,
-        "score_pairs": pairs,
+        "score_pairs": sum(v["pairs"] for v in levels.values()),
+        "levels": levels,
+        "node_bytes": node_bytes,
+        "q_bytes": q_bytes,
         "kv_bytes": kv_tokens * 2 * d * elt,
         "kv_tokens": kv_tokens,
         "route_bytes": summ_nodes * node_bytes + q_bytes,
         "attend_bytes": kv_tokens * 2 * d * elt + q_bytes + q_bytes + batch * spec.n_q_heads * 4,
     }
+
+
+def kernel_bytes(name: str, tag: int, by: dict) -> float | None:
+    """Algorithmic bytes of one launch of a library kernel in a step whose
+    step_bytes() are `by` (None for kernels without a byte model): a scoring
+    launch reads its level's visited node records and the queries and writes one
+    score per (query head, candidate) pair; a selection launch reads those scores;
+    the attention kernels read the selected K/V rows and the queries."""
+    if name.startswith("score") and tag in by["levels"]:
+        lv = by["levels"][tag]
+        return lv["nodes"] * by["node_bytes"] + lv["pairs"] * 4 + by["q_bytes"]
+    if name.startswith("select") and tag in by["levels"]:
+        return by["levels"][tag]["pairs"] * 4
+    if name in ("attend_split_kernel", "attend_kernel"):
+        return by["kv_bytes"] + by["q_bytes"]
+    return None
 
 
 # ---------------------------------------------------------------------------
@@ -213,24 +255,64 @@ def blas_threads() -> int:
         return os.cpu_count() or 1
 
 
-def cpu_baseline(inp: W.Inputs, n_tokens: int, budget_s: float = 20.0) -> dict:
+def cpu_baseline(inp: W.Inputs, n_tokens: int, q_index: int, budget_s: float,
+                 gpu_kept: dict | None = None) -> dict:
+    """The oracle on this host, on a bounded sample of the workload at context
+    n_tokens (the first timed step's context and queries): route + attend of the
+    query heads of KV head 0 on all cores and on one thread, the oracle's build
+    of KV head 0's tree, and dense fp64 attention of one head over the whole
+    context. With `gpu_kept` ({(b, h): {level: ids}} of the same step) the
+    sampled heads' routes are also compared with the GPU's (ties counted)."""
+    from threadpoolctl import threadpool_limits
+
+    from oracle.parity import RouteReport, compare_route_head
     spec = inp.spec
-    O, Kf, Vf, tree = oracle_setup(inp, n_tokens, 0)
+    import oracle as O
     t0 = time.perf_counter()
-    done = 0
-    for b in range(spec.batch):
-        for h in range(spec.group):
-            oracle_head(O, Kf, Vf, tree, inp.Q[0, b, h].astype(np.float64), spec.p)
+    O, Kf, Vf, tree = oracle_setup(inp, n_tokens, 0)
+    build_s = time.perf_counter() - t0
+    heads = [(b, h) for b in range(spec.batch) for h in range(spec.group)]
+    report = RouteReport()
+
+    def run(limit_s, max_heads):
+        t = time.perf_counter()
+        done = 0
+        for (b, h) in heads[:max_heads]:
+            q = inp.Q[q_index, b, h].astype(np.float64)
+            tr = O.route(q, tree, spec.p)
+            O.attend(q, Kf, Vf, tr.tokens)
+            if gpu_kept is not None and (b, h) in gpu_kept and done >= report.heads:
+                compare_route_head(q, tree, spec.p, gpu_kept[(b, h)], report, (b, h))
             done += 1
-            if time.perf_counter() - t0 > budget_s:
+            if time.perf_counter() - t > limit_s:
                 break
-        if time.perf_counter() - t0 > budget_s:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": done / spec.n_q_heads / dt, "unit": UNIT, "cores": blas_threads(),
-            "kind": "oracle",
-            "sample": (f"fp64 numpy oracle: route + attend of {done} query heads of KV head 0 at "
-                       f"context {n_tokens} (tree prebuilt, untimed); a query = {spec.n_q_heads} heads")}
+        return done, time.perf_counter() - t
+
+    n_all, t_all = run(budget_s, len(heads))
+    with threadpool_limits(limits=1):
+        n_one, t_one = run(budget_s / 2, len(heads))
+        t = time.perf_counter()
+        O.sdpa(inp.Q[q_index, 0, 0].astype(np.float64)[None], Kf, Vf)
+        dense_1t = time.perf_counter() - t
+    t = time.perf_counter()
+    O.sdpa(inp.Q[q_index, 0, 0].astype(np.float64)[None], Kf, Vf)
+    dense_all = time.perf_counter() - t
+    out = {"value": n_all / spec.n_q_heads / t_all, "unit": UNIT, "cores": blas_threads(),
+           "kind": "oracle",
+           "sample": (f"fp64 numpy oracle: route + attend of {n_all} query heads of KV head 0 at "
+                      f"context {n_tokens} (queries of the first timed step; tree prebuilt, "
+                      f"untimed); a query = {spec.n_q_heads} heads"),
+           "single_thread": {"value": n_one / spec.n_q_heads / t_one, "unit": UNIT, "cores": 1,
+                             "heads": n_one},
+           "os_cpu_count": os.cpu_count(),
+           "oracle_build_s": {"kv_heads": 1, "tokens": n_tokens, "seconds": build_s,
+                              "whole_tree_estimate_s": build_s * spec.n_kv_heads},
+           "dense_attention_ms_per_head": {"all_cores": dense_all * 1e3, "one_thread": dense_1t * 1e3,
+                                           "tokens": n_tokens}}
+    if gpu_kept is not None:
+        out["route_parity_sample"] = report.summary()
+        out["route_parity_sample"]["hard_examples"] = [str(x) for x in report.hard[:3]]
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -299,7 +381,8 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": spec.name, **spec.describe(), "l2": "n/a (CPU)"},
+            "data": "synthetic (seeded generators in hierarchical_sparse_attention_zha_b200/workloads.py)",
+            "config": {"workload": spec.name, **spec.describe(), "l2": L2_NOTE},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -310,21 +393,35 @@ def run_reference(args, world, rank):
 # The CUDA path
 # ---------------------------------------------------------------------------
 
+def _kernel_key(name: str, tag: int) -> str:
+    return f"{name}/L{tag}" if name.startswith(("score", "select")) else name
+
+
 def run_zha(args, world, rank, local):
     from hierarchical_sparse_attention_zha_b200 import zha
 
     dev = torch.device("cuda", local)
     base = W.WORKLOADS[args.workload]
-    K_steps, W_steps = args.steps, args.warmup
-    n_e2e = 0 if args.no_e2e else min(K_steps, 64)
-    total_steps = W_steps + K_steps + n_e2e
     if args.context:
         base = W.scaled(base, n_tokens=args.context)
-    spec = W.scaled(base, stream_tokens=-(-(total_steps + 2) // base.chunk) * base.chunk)
+    C = base.chunk
+    K_steps, W_steps = args.steps, args.warmup
+    T_steps = max(0, args.trace_steps)
+    n_e2e = 0 if args.no_e2e else min(K_steps, 64)
+    e2e_warm = 4 if n_e2e else 0
+    # First timed context: 2C - 5 tokens past the workload's context (level 1
+    # then holds one node more; a chunk completes at the fifth timed step).
+    p_first = base.n_tokens + 2 * C - min(5, C)
+    N0 = p_first - 1 - W_steps - T_steps
+    if N0 < 1:
+        raise SystemExit("bench: the warm-up and traced steps do not fit before the timed window")
+    n_batches = W_steps + T_steps + K_steps + e2e_warm + n_e2e
+    last = p_first + K_steps + e2e_warm + n_e2e + 1
+    spec = W.scaled(base, stream_tokens=-(-(last - base.n_tokens) // C) * C)
     t_gen = time.perf_counter()
-    inp = W.generate(spec, n_batches=total_steps, rank=rank)
+    inp = W.generate(spec, n_batches=n_batches, rank=rank)
     t_gen = time.perf_counter() - t_gen
-    N0, C, B = spec.n_tokens, spec.chunk, spec.batch
+    B = spec.batch
     kv_t = torch.bfloat16 if spec.kv_dtype == "bf16" else torch.float32
     if spec.kv_dtype == "bf16":
         K = torch.from_numpy(inp.K.view(np.int16)).to(dev).view(torch.bfloat16)
@@ -338,9 +435,8 @@ def run_zha(args, world, rank, local):
     cfg = zha.make_config(spec.n_kv_heads, spec.n_q_heads, spec.head_dim, C, spec.levels, spec.n_ref,
                           kv_t, cap)
     tree = zha.Tree(cfg, refq)
-    stream = torch.cuda.current_stream(dev)
 
-    # prefill build, timed on its own
+    # prefill build, timed on its own (after one untimed build)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     tree.build(K, N0)
     torch.cuda.synchronize()
@@ -355,7 +451,7 @@ def run_zha(args, world, rank, local):
     ids = torch.empty(B, spec.n_q_heads, max_sel, dtype=torch.int32, device=dev)
     cnt = torch.empty(B, spec.n_q_heads, dtype=torch.int32, device=dev)
     words = zha.route_kept_words(cfg, B, cap)
-    bits = torch.zeros(total_steps, words + 1, dtype=torch.int32, device=dev)
+    bits = torch.zeros(n_batches, words + 1, dtype=torch.int32, device=dev)
     ids_keep = torch.empty(K_steps, B, spec.n_q_heads, max_sel, dtype=torch.int32, device=dev)
     cnt_keep = torch.empty(K_steps, B, spec.n_q_heads, dtype=torch.int32, device=dev)
     ws_r = torch.empty(zha.route_workspace_bytes(cfg, B, cap) // 4 + 64, dtype=torch.float32, device=dev)
@@ -384,14 +480,46 @@ def run_zha(args, world, rank, local):
         return appended
 
     pos = N0
-    for s in range(W_steps):
+    s = 0
+    for _ in range(W_steps):
         pos += 1
         step(s, pos)
+        s += 1
         flush.zero_()
     torch.cuda.synchronize()
 
+    # traced pass: CUDA events around every library kernel (shares of the step)
+    kernels, dominant = {}, ("score_tma_kernel", 1)
+    if T_steps:
+        zha.trace_enable(64 * T_steps)
+        trace_bytes = []
+        for _ in range(T_steps):
+            pos += 1
+            step(s, pos)
+            trace_bytes.append((s, pos))
+            s += 1
+            flush.zero_()
+        torch.cuda.synchronize()
+        recs = zha.trace_records()
+        zha.trace_enable(0)
+        tot = sum(ms for _, _, ms in recs)
+        for name, tag, ms in recs:
+            k = kernels.setdefault(_kernel_key(name, tag), {"name": name, "tag": tag, "launches": 0,
+                                                           "total_us": 0.0})
+            k["launches"] += 1
+            k["total_us"] += ms * 1e3
+        for k in kernels.values():
+            k["mean_us"] = k["total_us"] / k["launches"]
+            k["share"] = k["total_us"] / (tot * 1e3) if tot > 0 else 0.0
+        if kernels:
+            top = max(kernels.values(), key=lambda k: k["total_us"])
+            dominant = (top["name"], top["tag"])
+    torch.cuda.synchronize()
+
+    # timed region; events also bracket the dominant kernel's launches
+    zha.trace_enable(4 * K_steps + 16, dominant[0], dominant[1])
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_steps)]
-    positions, appended = [], []
+    positions, appended, s_timed = [], [], []
     clocks = Clocks(torch.cuda.current_device()) if rank == 0 else None
     launches0 = zha.launch_count()
     barrier(world)
@@ -400,10 +528,11 @@ def run_zha(args, world, rank, local):
         clocks.start()
     t_wall = time.perf_counter()
     for k in range(K_steps):
-        s = W_steps + k
         pos += 1
         positions.append(pos)
+        s_timed.append(s)
         appended.append(step(s, pos, evs[k]))
+        s += 1
         ids_keep[k].copy_(ids)
         cnt_keep[k].copy_(cnt)
         flush.zero_()
@@ -412,6 +541,8 @@ def run_zha(args, world, rank, local):
     t_wall = time.perf_counter() - t_wall
     clk = clocks.stop() if clocks else None
     launches = zha.launch_count() - launches0
+    dom_recs = zha.trace_records()
+    zha.trace_enable(0)
     st = int(status.item())
 
     step_ms = np.array([e[0].elapsed_time(e[3]) for e in evs])
@@ -423,29 +554,48 @@ def run_zha(args, world, rank, local):
     ms_per_step = total_ms_max / K_steps
 
     # algorithmic bytes, per step, from the recorded selections
-    bits_h = bits[W_steps: W_steps + K_steps].cpu().numpy().view(np.uint32)
+    bits_h = bits.cpu().numpy().view(np.uint32)
     ids_h, cnt_h = ids_keep.cpu().numpy(), cnt_keep.cpu().numpy()
-    by = [step_bytes(spec, bits_h[k], ids_h[k], cnt_h[k], positions[k], B) for k in range(K_steps)]
+    by = [step_bytes(spec, bits_h[s_timed[k]], ids_h[k], cnt_h[k], positions[k], B)
+          for k in range(K_steps)]
     route_b = np.array([x["route_bytes"] for x in by], float)
     att_b = np.array([x["attend_bytes"] for x in by], float)
     peak, peak_kind = measured_peaks()
     route_gbs = route_b.sum() / (route_ms.sum() * 1e-3) / 1e9
     att_gbs = att_b.sum() / (att_ms.sum() * 1e-3) / 1e9
     step_gbs = (route_b.sum() + att_b.sum()) / (total_ms * 1e-3) / 1e9
-    dominant = "zha_route" if route_ms.sum() >= att_ms.sum() else "zha_sparse_attend"
-    ach = route_gbs if dominant == "zha_route" else att_gbs
-    per_launch = (route_b.mean() if dominant == "zha_route" else att_b.mean())
+
+    # the dominant kernel: one launch per step, bytes from that step's selection
+    dom_key = _kernel_key(*dominant)
+    dom_ms = [ms for _, _, ms in dom_recs]
+    dom_b = [kernel_bytes(dominant[0], dominant[1], by[k]) for k in range(K_steps)]
+    roofline = None
+    if len(dom_ms) == K_steps and all(b is not None for b in dom_b) and sum(dom_ms) > 0:
+        ach = sum(dom_b) / (sum(dom_ms) * 1e-3) / 1e9
+        traffic, traffic_note = measured_traffic(spec.name, dom_key)
+        roofline = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                    "traffic": traffic, "traffic_note": traffic_note, "kernel": dom_key,
+                    "bytes_per_launch": float(np.mean(dom_b)), "mean_us": float(np.mean(dom_ms)) * 1e3,
+                    "launches": len(dom_ms), "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                    if peak_kind == "measured" else "fallback 6650 GB/s"}
     if args.dump_bytes and rank == 0:
         with open(args.dump_bytes, "w") as f:
-            json.dump({"first_timed_step": W_steps, "route_bytes": route_b.tolist(),
-                       "attend_bytes": att_b.tolist()}, f)
-    traffic, traffic_note = None, None
-    mt = measured_traffic(spec.name)
-    if mt is not None and dominant in mt:
-        traffic = float(mt[dominant]["dram_bytes"])
-        traffic_note = (f"ncu dram bytes of one {dominant} call (step {mt['step']}, whose algorithmic "
-                        f"bytes were {mt[dominant]['algorithmic_bytes']:.0f}); see profiles/")
-    non_app = ~np.array(appended)
+            json.dump({"first_timed_step": W_steps + T_steps, "route_bytes": route_b.tolist(),
+                       "attend_bytes": att_b.tolist(),
+                       "levels": [{str(l): v for l, v in x["levels"].items()} for x in by]}, f)
+    # per-kernel achieved bandwidth of the traced pass (scoring and selection
+    # kernels run once per step and level; their bytes follow from the bitmaps)
+    if T_steps and kernels:
+        no_ids = np.zeros((B, spec.n_q_heads, 1), np.int32)
+        no_cnt = np.zeros((B, spec.n_q_heads), np.int32)
+        by_t = [step_bytes(spec, bits_h[st_], no_ids, no_cnt, p_, B) for st_, p_ in trace_bytes]
+        for k in kernels.values():
+            name, tag = k.pop("name"), k["tag"]
+            bt = [kernel_bytes(name, tag, x) for x in by_t]
+            if name.startswith(("score", "select")) and all(b is not None for b in bt) and \
+                    k["launches"] == len(by_t):
+                k["gbs"] = sum(bt) / (k["total_us"] * 1e-6) / 1e9
+                k["frac"] = k["gbs"] / peak
     append_frac = float(app_ms[np.array(appended)].sum() / step_ms.sum()) if any(appended) else 0.0
 
     # end to end through the API with host buffers
@@ -462,37 +612,70 @@ def run_zha(args, world, rank, local):
         src_k = torch.from_numpy(inp.K.view(np.int16)).view(torch.bfloat16) if spec.kv_dtype == "bf16" else torch.from_numpy(inp.K)
         src_v = torch.from_numpy(inp.V.view(np.int16)).view(torch.bfloat16) if spec.kv_dtype == "bf16" else torch.from_numpy(inp.V)
         ee = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_e2e)]
+        host_s, host_calls = 0.0, 0
         barrier(world)
         torch.cuda.synchronize()
-        for k in range(n_e2e):
-            s = W_steps + K_steps + k
+        for k in range(e2e_warm + n_e2e):
+            timed = k >= e2e_warm
             t_new = pos           # index of the token written this step
             pos += 1
             kv_new_k.copy_(src_k[:, t_new: t_new + 1])
             kv_new_v.copy_(src_v[:, t_new: t_new + 1])
-            ee[k][0].record()
+            if timed:
+                ee[k - e2e_warm][0].record()
             K[:, t_new: t_new + 1].copy_(kv_new_k, non_blocking=True)
             V[:, t_new: t_new + 1].copy_(kv_new_v, non_blocking=True)
             q_dev.copy_(Qh[s], non_blocking=True)
+            th = time.perf_counter()
+            n_calls = 2
             if pos % C == 0:
                 tree.append_chunk(K, pos)
+                n_calls += 1
             tree.route(q_dev, pos, spec.p, max_sel, chunk_ids=ids, n_chunks=cnt, ws=ws_r,
                        kept_bits=bits[s], status=status)
             tree.sparse_attend(q_dev, K, V, pos, ids, cnt, out=out, lse=lse, ws=ws_a, status=status)
+            if timed:
+                host_s += time.perf_counter() - th
+                host_calls += n_calls
             out_h.copy_(out, non_blocking=True)
             lse_h.copy_(lse, non_blocking=True)
-            ee[k][1].record()
-            ee[k][1].synchronize()
+            if timed:
+                ee[k - e2e_warm][1].record()
+                ee[k - e2e_warm][1].synchronize()
+            else:
+                torch.cuda.synchronize()
+            s += 1
             flush.zero_()
         torch.cuda.synchronize()
         e2e_ms = float(np.sum([a.elapsed_time(b) for a, b in ee]))
         e2e_ms = allreduce_max(e2e_ms, world) / n_e2e
         e2e = {"value": world * B / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms, "steps": n_e2e}
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms, "steps": n_e2e,
+               "warmup": e2e_warm, "host_us_per_call": host_s * 1e6 / max(1, host_calls),
+               "note": "timed region: H2D of the step's queries and new K/V row from pinned memory, "
+                       "the library calls (Python binding -> C ABI), D2H of O and lse, then a host "
+                       "synchronisation"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(inp, positions[0])
+        kept0 = {}           # the GPU's kept sets of KV head 0's heads at the first timed step
+        nb0 = C * (positions[0] // C)
+        offs, o = {}, 0
+        for l in range(1, spec.levels + 1):
+            offs[l] = o
+            o += B * spec.n_q_heads * ((nb0 // C ** l + 31) // 32)
+        for b in range(B):
+            for h in range(spec.group):
+                per = {}
+                for l in range(1, spec.levels + 1):
+                    n_l = nb0 // C ** l
+                    w = (n_l + 31) // 32
+                    blk = bits_h[s_timed[0]][offs[l] + (b * spec.n_q_heads + h) * w:
+                                             offs[l] + (b * spec.n_q_heads + h + 1) * w]
+                    nz = np.nonzero(np.unpackbits(blk.view(np.uint8), bitorder="little"))[0]
+                    per[l] = nz[nz < n_l]
+                kept0[(b, h)] = per
+        cpu = cpu_baseline(inp, positions[0], s_timed[0], args.cpu_budget, gpu_kept=kept0)
 
     value = world * K_steps * B / (total_ms_max * 1e-3)
     if rank == 0:
@@ -500,25 +683,28 @@ def run_zha(args, world, rank, local):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K_steps,
             "warmup": W_steps, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic (seeded generators; see DESIGN.md)",
-            "config": {"workload": spec.name, **base.describe(), "decode_from": N0,
-                       "steps_context": [positions[0], positions[-1]],
-                       "l2": f"flushed between timed steps ({args.flush_mb} MiB memset outside the events)",
-                       "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
-            "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
-                         "frac": ach / peak, "traffic": traffic, "traffic_note": traffic_note,
-                         "kernel": dominant,
-                         "bytes_per_launch": float(per_launch), "peak_source": peak_kind},
+            "data": "synthetic (seeded generators in hierarchical_sparse_attention_zha_b200/workloads.py)",
+            "config": {"workload": spec.name, **base.describe(), "l2": L2_NOTE},
+            "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+            "window": {"decode_from": N0, "steps_context": [positions[0], positions[-1]],
+                       "level1_nodes": [positions[0] // C, positions[-1] // C],
+                       "appends": int(sum(appended)),
+                       "l2_flush": f"{args.flush_mb} MiB memset between timed steps, outside the events"},
+            "roofline": roofline,
             "step_roofline": {"achieved": step_gbs, "frac": step_gbs / peak,
                               "route_gbs": route_gbs, "attend_gbs": att_gbs,
                               "route_ms": float(route_ms.mean()), "attend_ms": float(att_ms.mean()),
                               "append_share": append_frac,
+                              "append_ms_when_appending": float(app_ms[np.array(appended)].mean())
+                              if any(appended) else None,
                               "bytes_per_step": float((route_b + att_b).mean()),
                               "summary_mb": float(np.mean([x["summary_bytes"] for x in by]) / 1e6),
                               "kv_mb": float(np.mean([x["kv_bytes"] for x in by]) / 1e6),
                               "kv_tokens": float(np.mean([x["kv_tokens"] for x in by])),
                               "score_pairs": float(np.mean([x["score_pairs"] for x in by]))},
-            "build_ms": build_ms, "gen_s": t_gen, "wall_s_timed_region": t_wall,
+            "kernels": {"source": f"traced pass of {T_steps} steps before the timed region "
+                                  "(CUDA events around each library launch)", "by_kernel": kernels},
+            "build_ms": build_ms, "build_tokens": N0, "gen_s": t_gen, "wall_s_timed_region": t_wall,
             "gpu_launches": int(launches), "device_status": st,
             "clocks": clk, "e2e": e2e, "cpu_baseline": cpu,
         }

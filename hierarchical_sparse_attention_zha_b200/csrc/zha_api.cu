@@ -88,8 +88,9 @@ static zha_status make_geom(const zha_config* c, zha::Geom* g, size_t* bytes) {
     G.off[l] = off;
     off += int64_t(G.hkv) * G.cap[l] * G.node_floats;
   }
+  G.status_off = zha::round_up(off, 64);           // 256-byte aligned, one 256-byte block
   *g = G;
-  if (bytes) *bytes = size_t(zha::round_up(off * 4, 256));
+  if (bytes) *bytes = size_t(G.status_off * 4 + 256);
   return ZHA_OK;
 }
 
@@ -173,8 +174,12 @@ zha_status zha_build(zha_tree* tree, const void* d_K, int64_t ld, int64_t n_toke
   zha_status st = check_cache(tree, d_K, ld, n_tokens, "zha_build");
   if (st != ZHA_OK) return st;
   const int64_t nb = int64_t(tree->geom.chunk) * (n_tokens / tree->geom.chunk);
-  cudaError_t e = zha::launch_build(tree->geom, d_K, ld, 0, nb, tree->ref_q, tree->store,
-                                    static_cast<cudaStream_t>(stream));
+  // A full build starts the tree's status afresh.
+  cudaError_t e = cudaMemsetAsync(zha::tree_status_word(tree->geom, tree->store), 0, sizeof(int32_t),
+                                  static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "zha_build");
+  e = zha::launch_build(tree->geom, d_K, ld, 0, nb, tree->ref_q, tree->store,
+                        static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "zha_build");
   tree->nb = nb;
   return ZHA_OK;
@@ -212,25 +217,40 @@ size_t zha_route_kept_words(const zha_config* cfg, int32_t batch, int64_t n_toke
   return size_t(zha::route_layout(G, batch, n_tokens).bits_words);
 }
 
+}  // extern "C"
+
+// Argument checks of a routing call (zha_route and zha_route_noalloc share them).
+zha_status zha_check_route_args(const zha_tree* tree, const float* d_Q, int32_t batch,
+                                int64_t n_tokens, float p, const int32_t* d_chunk_ids,
+                                const int32_t* d_n_chunks, int32_t max_sel, const char* who) {
+  if (tree == nullptr) return fail(ZHA_ERR_INVALID, "%s: tree is NULL", who);
+  const zha::Geom& G = tree->geom;
+  if (d_Q == nullptr || !aligned(d_Q, 16))
+    return fail(ZHA_ERR_INVALID, "%s: Q must be a non-NULL 16-byte aligned device pointer", who);
+  if (batch < 1 || batch > 65535) return fail(ZHA_ERR_INVALID, "%s: batch must be 1..65535", who);
+  if (n_tokens < 1 || n_tokens > G.max_tokens)
+    return fail(ZHA_ERR_INVALID, "%s: n_tokens %lld outside [1, max_tokens]", who,
+                (long long)n_tokens);
+  if (!(p > 0.f) || !std::isfinite(p)) return fail(ZHA_ERR_INVALID, "%s: p must be > 0", who);
+  const int64_t nb = int64_t(G.chunk) * (n_tokens / G.chunk);
+  if (nb != tree->nb)
+    return fail(ZHA_ERR_STATE, "%s: tree covers %lld tokens, n_tokens %lld needs %lld", who,
+                (long long)tree->nb, (long long)n_tokens, (long long)nb);
+  if (d_chunk_ids == nullptr || d_n_chunks == nullptr || max_sel < 1)
+    return fail(ZHA_ERR_INVALID, "%s: chunk_ids / n_chunks NULL or max_sel < 1", who);
+  return ZHA_OK;
+}
+
+extern "C" {
+
 zha_status zha_route(const zha_tree* tree, const float* d_Q, int32_t batch, int64_t n_tokens,
                      float p, int32_t* d_chunk_ids, int32_t* d_n_chunks, int32_t max_sel,
                      uint32_t* d_kept_bits, void* d_ws, size_t ws_bytes, int32_t* d_status,
                      void* stream) {
-  if (tree == nullptr) return fail(ZHA_ERR_INVALID, "zha_route: tree is NULL");
+  const zha_status st = zha_check_route_args(tree, d_Q, batch, n_tokens, p, d_chunk_ids, d_n_chunks,
+                                             max_sel, "zha_route");
+  if (st != ZHA_OK) return st;
   const zha::Geom& G = tree->geom;
-  if (d_Q == nullptr || !aligned(d_Q, 16))
-    return fail(ZHA_ERR_INVALID, "zha_route: Q must be a non-NULL 16-byte aligned device pointer");
-  if (batch < 1 || batch > 65535) return fail(ZHA_ERR_INVALID, "zha_route: batch must be 1..65535");
-  if (n_tokens < 1 || n_tokens > G.max_tokens)
-    return fail(ZHA_ERR_INVALID, "zha_route: n_tokens %lld outside [1, max_tokens]",
-                (long long)n_tokens);
-  if (!(p > 0.f) || !std::isfinite(p)) return fail(ZHA_ERR_INVALID, "zha_route: p must be > 0");
-  const int64_t nb = int64_t(G.chunk) * (n_tokens / G.chunk);
-  if (nb != tree->nb)
-    return fail(ZHA_ERR_STATE, "zha_route: tree covers %lld tokens, n_tokens %lld needs %lld",
-                (long long)tree->nb, (long long)n_tokens, (long long)nb);
-  if (d_chunk_ids == nullptr || d_n_chunks == nullptr || max_sel < 1)
-    return fail(ZHA_ERR_INVALID, "zha_route: chunk_ids / n_chunks NULL or max_sel < 1");
   const zha::RouteLayout lay = zha::route_layout(G, batch, n_tokens);
   const int64_t need = d_kept_bits ? lay.bytes_no_bits : lay.bytes;
   if (d_ws == nullptr || !aligned(d_ws, 256) || int64_t(ws_bytes) < need)

@@ -19,6 +19,7 @@
 // sink. The range states are merged by combine_ranges_kernel (below).
 // This CUDA-core kernel serves fp32 caches and head_dim 64; bf16 caches with
 // head_dim 128 go to the tensor-core kernels in zha_attend_tc.cu.
+#include "zha_host.cuh"
 #include "zha_internal.cuh"
 
 namespace zha {
@@ -303,15 +304,17 @@ static cudaError_t launch_attend_t(const Geom& G, const float* Q, const void* K,
                                    int32_t max_sel, float* O, float* lse, float* partial,
                                    const AttendLayout& lay, int32_t* status, cudaStream_t s) {
   const size_t smem = attend_smem_bytes<D>(lay.range_chunks);
-  cudaError_t e = cudaFuncSetAttribute(attend_kernel<T, D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  cudaError_t e = ensure_dynamic_smem(attend_kernel<T, D>, smem);
   if (e != cudaSuccess) return e;
   const int64_t nb = int64_t(G.chunk) * (n_tokens / G.chunk);
   const int qn = batch * G.group;
   dim3 grid(unsigned(lay.n_ranges + 1), unsigned(G.hkv), unsigned((qn + kAttQ - 1) / kAttQ));
-  attend_kernel<T, D><<<grid, kAttThreads, smem, s>>>(
-      G, batch, n_tokens, nb, Q, static_cast<const T*>(K), static_cast<const T*>(V), ld, chunk_ids,
-      n_chunks, max_sel, lay.range_chunks, lay.n_ranges, partial, lay.slots_per_head);
+  {
+    TraceScope ts("attend_kernel", 0, s);
+    attend_kernel<T, D><<<grid, kAttThreads, smem, s>>>(
+        G, batch, n_tokens, nb, Q, static_cast<const T*>(K), static_cast<const T*>(V), ld, chunk_ids,
+        n_chunks, max_sel, lay.range_chunks, lay.n_ranges, partial, lay.slots_per_head);
+  }
   zha_count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   return launch_combine(G, batch, chunk_ids, n_chunks, max_sel, O, lse, partial, lay, status, s);
@@ -436,6 +439,7 @@ cudaError_t launch_combine(const Geom& G, int32_t batch, const int32_t* chunk_id
                            const float* partial, const AttendLayout& lay, int32_t* status,
                            cudaStream_t s) {
   const unsigned heads = unsigned(int64_t(batch) * G.hq);
+  TraceScope ts("combine_ranges_kernel", 0, s);
   if (G.d == 128)
     combine_ranges_kernel<128><<<heads, 128, 0, s>>>(G, batch, lay.n_chunks, chunk_ids, n_chunks,
                                                      max_sel, lay.range_chunks, lay.n_ranges,

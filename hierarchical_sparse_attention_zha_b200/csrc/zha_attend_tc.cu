@@ -41,8 +41,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include <mutex>
-
+#include "zha_host.cuh"
 #include "zha_internal.cuh"
 #include "zha_tc.cuh"
 
@@ -944,27 +943,11 @@ combine_split_kernel(Geom G, int32_t batch, int32_t q_blocks, int32_t n_blocks, 
 
 namespace {
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (the library
-// links only the CUDA runtime).
-PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q{};
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 // [Hkv][ld][d] bf16 cache as a 3-D tensor {d, n_tokens, Hkv}: rows at or past
 // n_tokens read as zeros. Box = 64 columns (128 B, the swizzle span) x box_rows.
 bool kv_tensor_map(CUtensorMap* m, const void* base, int64_t n_tokens, int64_t ld, int hkv,
                    int box_rows) {
-  const PFN_cuTensorMapEncodeTiled_v12000 fn = encode_tiled();
+  const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
   if (fn == nullptr) return false;
   const cuuint64_t dims[3] = {cuuint64_t(kD), cuuint64_t(n_tokens), cuuint64_t(hkv)};
   const cuuint64_t strides[2] = {cuuint64_t(kD) * 2, cuuint64_t(ld) * kD * 2};
@@ -991,13 +974,15 @@ cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const
   const int units = int(lay.units);
 
   const size_t prep_smem = sizeof(uint32_t) * 32 * kRowWords;
-  cudaError_t e = cudaFuncSetAttribute(union_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(prep_smem));
+  cudaError_t e = ensure_dynamic_smem(union_prep_kernel, prep_smem);
   if (e != cudaSuccess) return e;
-  if ((e = launch_pdl(union_prep_kernel, dim3(unsigned(units)), dim3(1024), prep_smem, s, G, batch,
-                      lay.q_blocks, lay.n_blocks, lay.block_chunks, nb, lay.n_chunks, chunk_ids,
-                      n_chunks, max_sel, ids, masks, lay.cap, counts, status)) != cudaSuccess)
-    return e;
+  {
+    TraceScope ts("union_prep_kernel", 0, s);
+    e = launch_pdl(union_prep_kernel, dim3(unsigned(units)), dim3(1024), prep_smem, s, G, batch,
+                   lay.q_blocks, lay.n_blocks, lay.block_chunks, nb, lay.n_chunks, chunk_ids, n_chunks,
+                   max_sel, ids, masks, lay.cap, counts, status);
+  }
+  if (e != cudaSuccess) return e;
   zha_count_launch();
 
   // Tensor copies when every chunk box starts on a swizzle atom (C % 8 == 0).
@@ -1006,21 +991,22 @@ cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const
                    kv_tensor_map(&mv, V, n_tokens, ld, G.hkv, G.chunk);
   auto kern = tma ? attend_split_kernel<true> : attend_split_kernel<false>;
   const size_t smem = split_smem_bytes(units);
-  if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem))) !=
-      cudaSuccess)
-    return e;
-  int dev = 0, sms = 148;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  if ((e = ensure_dynamic_smem(kern, smem)) != cudaSuccess) return e;
+  int sms = 148;
+  if ((e = device_sm_count(&sms)) != cudaSuccess) return e;
   const unsigned ctas = unsigned(sms < kTcMaxCtas ? sms : kTcMaxCtas);
-  if ((e = launch_pdl(kern, dim3(ctas), dim3(kThreads), smem, s, mk, mv, G, batch, lay.q_blocks,
-                      lay.n_blocks, lay.block_chunks, units, n_tokens, nb, Q,
-                      static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V), ld,
-                      ids, masks, lay.cap, counts, split, slots, status)) != cudaSuccess)
-    return e;
+  {
+    TraceScope ts("attend_split_kernel", 0, s);
+    e = launch_pdl(kern, dim3(ctas), dim3(kThreads), smem, s, mk, mv, G, batch, lay.q_blocks,
+                   lay.n_blocks, lay.block_chunks, units, n_tokens, nb, Q,
+                   static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V), ld, ids,
+                   masks, lay.cap, counts, split, slots, status);
+  }
+  if (e != cudaSuccess) return e;
   zha_count_launch();
 
   const int64_t heads = int64_t(batch) * G.hq;
+  TraceScope ts("combine_split_kernel", 0, s);
   e = launch_pdl(combine_split_kernel, dim3(unsigned(heads)), dim3(32 * kCombineWarps), 0, s, G, batch,
                  lay.q_blocks, lay.n_blocks, units, split, slots, O, lse);
   zha_count_launch();

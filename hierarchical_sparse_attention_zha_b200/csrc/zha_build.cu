@@ -7,6 +7,7 @@
 // q_r with khat_r = Attn(q_r, K_C, K_C) and bhat_r = F_C(q_r) - q_r.khat_r/sqrt(d),
 // parents merging child summaries "in the same way", level 1 every C steps and
 // level 2 every C^2 steps.
+#include "zha_host.cuh"
 #include "zha_internal.cuh"
 
 namespace zha {
@@ -269,18 +270,21 @@ static cudaError_t launch_build_t(const Geom& G, const void* K, int64_t ld, int6
                                   int64_t nb_new, const float* refq, float* store,
                                   cudaStream_t s) {
   const size_t smem = l1_smem_bytes<D>(G.nref);
-  cudaError_t e = cudaFuncSetAttribute(build_level1_kernel<T, D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  cudaError_t e = ensure_dynamic_smem(build_level1_kernel<T, D>, smem);
   if (e != cudaSuccess) return e;
   const int64_t c_begin = nb_old / G.chunk, c_end = nb_new / G.chunk;
   // bf16, d = 128, R = 16, C = 64: the tensor-core level 1 (zha_build_tc.cu).
-  const cudaError_t etc = launch_build_level1_tc(G, K, ld, c_begin, c_end, refq, store, nullptr, s);
+  const cudaError_t etc =
+      launch_build_level1_tc(G, K, ld, c_begin, c_end, refq, store, tree_status_word(G, store), s);
   if (etc != cudaSuccess && etc != cudaErrorNotSupported) return etc;
   if (etc != cudaSuccess && c_end > c_begin) {
     const int cpt = l1_chunks_per_tile(G.chunk);
     dim3 grid(unsigned((c_end - c_begin + cpt - 1) / cpt), unsigned(G.hkv));
-    build_level1_kernel<T, D><<<grid, kBuildThreads, smem, s>>>(
-        G, static_cast<const T*>(K), ld, c_begin, c_end, refq, store);
+    {
+      TraceScope ts("build_level1_kernel", 1, s);
+      build_level1_kernel<T, D><<<grid, kBuildThreads, smem, s>>>(
+          G, static_cast<const T*>(K), ld, c_begin, c_end, refq, store);
+    }
     zha_count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -291,8 +295,11 @@ static cudaError_t launch_build_t(const Geom& G, const void* K, int64_t ld, int6
     const int64_t items = (p_end - p_begin) * G.nref;
     const int per = kBuildThreads / 32;
     dim3 grid(unsigned((items + per - 1) / per), unsigned(G.hkv));
-    merge_level_kernel<D><<<grid, kBuildThreads, 0, s>>>(G, level, p_begin, p_end - p_begin,
-                                                          refq, store);
+    {
+      TraceScope ts("merge_level_kernel", level, s);
+      merge_level_kernel<D><<<grid, kBuildThreads, 0, s>>>(G, level, p_begin, p_end - p_begin,
+                                                            refq, store);
+    }
     zha_count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
@@ -304,9 +311,9 @@ static cudaError_t launch_append_t(const Geom& G, const void* K, int64_t ld, int
                                    int64_t nb_new, const float* refq, float* store,
                                    cudaStream_t s) {
   const size_t smem = l1_smem_bytes<D>(G.nref);
-  cudaError_t e = cudaFuncSetAttribute(append_kernel<T, D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  cudaError_t e = ensure_dynamic_smem(append_kernel<T, D>, smem);
   if (e != cudaSuccess) return e;
+  TraceScope ts("append_kernel", 0, s);
   append_kernel<T, D><<<G.hkv, kBuildThreads, smem, s>>>(G, static_cast<const T*>(K), ld, nb_old,
                                                           nb_new, refq, store);
   zha_count_launch();

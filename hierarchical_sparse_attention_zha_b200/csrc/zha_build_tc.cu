@@ -21,8 +21,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include <mutex>
-
+#include "zha_host.cuh"
 #include "zha_internal.cuh"
 #include "zha_tc.cuh"
 
@@ -297,21 +296,6 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
   if (tid == 0 && ms.err != 0u && status != nullptr) atomicOr(status, ZHA_DEV_TIMEOUT);
 }
 
-namespace {
-PFN_cuTensorMapEncodeTiled_v12000 build_encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q{};
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess && q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-}  // namespace
-
 // Level-1 summaries of chunks [c_begin, c_end) with the tensor cores; returns
 // cudaErrorNotSupported when the configuration is not covered (the caller then
 // uses the CUDA-core build).
@@ -321,7 +305,7 @@ cudaError_t launch_build_level1_tc(const Geom& G, const void* K, int64_t ld, int
   if (!(G.kv_bf16 && G.d == bD && G.nref == bR && G.chunk == 64))
     return cudaErrorNotSupported;
   if (c_end <= c_begin) return cudaSuccess;
-  const PFN_cuTensorMapEncodeTiled_v12000 fn = build_encode_fn();
+  const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
   if (fn == nullptr) return cudaErrorNotSupported;
   CUtensorMap map{};
   const cuuint64_t dims[3] = {cuuint64_t(bD), cuuint64_t(c_end * G.chunk), cuuint64_t(G.hkv)};
@@ -333,16 +317,15 @@ cudaError_t launch_build_level1_tc(const Geom& G, const void* K, int64_t ld, int
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorNotSupported;
   const size_t smem = size_t(bOffMisc) + sizeof(BMisc) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(build_l1_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(smem));
+  cudaError_t e = ensure_dynamic_smem(build_l1_tc_kernel, smem);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  int sms = 148;
+  if ((e = device_sm_count(&sms)) != cudaSuccess) return e;
   const int cpt = bTok / G.chunk;
   const int64_t tiles = (c_end - c_begin + cpt - 1) / cpt;
   int64_t per_head = (2 * int64_t(sms) + G.hkv - 1) / G.hkv;
   if (per_head > tiles) per_head = tiles;
+  TraceScope ts("build_l1_tc_kernel", 1, s);
   build_l1_tc_kernel<<<dim3(unsigned(per_head), unsigned(G.hkv)), bThreads, smem, s>>>(
       map, G, c_begin, c_end, refq, store, status);
   zha_count_launch();

@@ -24,7 +24,14 @@ struct Geom {
   int64_t max_tokens;
   int64_t cap[ZHA_MAX_LEVELS + 2];       // node capacity per KV head, index by level
   int64_t off[ZHA_MAX_LEVELS + 2];       // float offset of level l's [hkv][cap][node] block
+  int64_t status_off;                    // float offset of the tree's device status word
 };
+
+// The tree's device status word (ZHA_DEV_* bits of the build kernels), in the
+// 256-byte block that follows the summary levels in the store.
+__host__ __device__ inline int32_t* tree_status_word(const Geom& g, float* store) {
+  return reinterpret_cast<int32_t*>(store + g.status_off);
+}
 
 // C^l, saturating at a value above any token count.
 __host__ __device__ inline int64_t span_of(int32_t chunk, int32_t level) {
@@ -168,6 +175,24 @@ inline TcAttendLayout tc_attend_layout(const Geom& g, int32_t batch, int64_t n_t
 inline bool use_tc_attend(const Geom& g) { return g.kv_bf16 && g.d == 128; }
 
 // ---------------------------------------------------------------------------
+// Optional kernel timing (zha_trace.cu): a TraceScope around a launch records
+// CUDA events before and after it on the stream while tracing is enabled.
+// `tag` distinguishes launches of one kernel (the tree level for routing).
+// ---------------------------------------------------------------------------
+int trace_begin(const char* name, int32_t tag, cudaStream_t s);
+void trace_end(int idx, cudaStream_t s);
+
+struct TraceScope {
+  int idx;
+  cudaStream_t s;
+  TraceScope(const char* name, int32_t tag, cudaStream_t stream)
+      : idx(trace_begin(name, tag, stream)), s(stream) {}
+  ~TraceScope() { trace_end(idx, s); }
+  TraceScope(const TraceScope&) = delete;
+  TraceScope& operator=(const TraceScope&) = delete;
+};
+
+// ---------------------------------------------------------------------------
 // Programmatic dependent launch: a kernel launched with launch_pdl may be
 // scheduled while the previous kernel on the stream is finishing. It calls
 // pdl_trigger() on entry (its own dependents may then be scheduled once all of
@@ -279,3 +304,6 @@ struct zha_tree {
 // Launch bookkeeping and error reporting shared by the host wrappers.
 void zha_count_launch();
 zha_status zha_report_error(zha_status s, const char* msg);
+zha_status zha_check_route_args(const zha_tree* tree, const float* d_Q, int32_t batch,
+                                int64_t n_tokens, float p, const int32_t* d_chunk_ids,
+                                const int32_t* d_n_chunks, int32_t max_sel, const char* who);

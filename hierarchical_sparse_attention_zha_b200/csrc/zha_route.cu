@@ -20,6 +20,7 @@
 //              select_fast_kernel when the level fits in shared memory
 //              (<= 16384 nodes), select_kernel otherwise.
 // Both kinds are launched with programmatic dependent launch.
+#include "zha_host.cuh"
 #include "zha_internal.cuh"
 
 namespace zha {
@@ -280,7 +281,17 @@ struct SelectArgs {
   int32_t* n_chunks;
   int32_t max_sel;
   int32_t* status;
+  const int32_t* tree_status;  // top level only: the tree's build status, OR-ed into *status
 };
+
+// The first selection of a route passes the tree's build status on to the
+// caller's status word (a build whose bounded wait ran out left the tree invalid).
+__device__ __forceinline__ void forward_tree_status(const SelectArgs& a) {
+  if (a.tree_status != nullptr && a.status != nullptr && blockIdx.x == 0 && threadIdx.x == 0) {
+    const int32_t v = *a.tree_status;
+    if (v != 0) atomicOr(a.status, v);
+  }
+}
 
 __global__ void __launch_bounds__(kSelectThreads)
 select_kernel(Geom G, SelectArgs a) {
@@ -295,6 +306,7 @@ select_kernel(Geom G, SelectArgs a) {
   __shared__ unsigned long long s_before;
   pdl_trigger();
   pdl_wait();
+  forward_tree_status(a);
 
   const int bh = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
@@ -533,6 +545,7 @@ select_fast_kernel(Geom G, SelectArgs a) {
   __shared__ unsigned long long s_before;
   pdl_trigger();
   pdl_wait();
+  forward_tree_status(a);
 
   const int bh = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -793,9 +806,9 @@ static cudaError_t launch_score_t(const Geom& G, int level, int64_t n_nodes, int
             unsigned((qn + kScoreQBlock - 1) / kScoreQBlock));
   const size_t smem = (size_t(kScoreThreads / 32) * S::KBUF +
                        size_t(qn < kScoreQBlock ? qn : kScoreQBlock) * S::QROW) * 4;
-  cudaError_t e = cudaFuncSetAttribute(score_kernel<D, RP>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  cudaError_t e = ensure_dynamic_smem(score_kernel<D, RP>, smem);
   if (e != cudaSuccess) return e;
+  TraceScope ts("score_kernel", level, s);
   e = launch_pdl(score_kernel<D, RP>, grid, dim3(kScoreThreads), smem, s, G, level, n_nodes, n_par,
                  batch, tile, Q, kept_up, words_up, sigma, store);
   zha_count_launch();
@@ -834,8 +847,7 @@ cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n
                          float* sigma, int32_t* kp, const RouteLayout& lay, int32_t* status,
                          const float* store, cudaStream_t s) {
   const size_t smem = select_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(smem));
+  cudaError_t e = ensure_dynamic_smem(select_kernel, smem);
   if (e != cudaSuccess) return e;
   const int heads = batch * G.hq;
   SelectArgs a{};
@@ -844,8 +856,7 @@ cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n
   a.p_fixed32 = (unsigned long long)ceil(double(p) * 4294967296.0);
   if (a.p_fixed32 == 0) a.p_fixed32 = 1;
   const size_t smem_fast = select_fast_smem_bytes();
-  if ((e = cudaFuncSetAttribute(select_fast_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                int(smem_fast))) != cudaSuccess)
+  if ((e = ensure_dynamic_smem(select_fast_kernel, smem_fast)) != cudaSuccess)
     return e;
   a.keep_all = p >= 1.0f;
   a.kp = kp;
@@ -887,10 +898,14 @@ cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n
     a.sigma = sg;
     a.chunk_ids = level == 1 ? chunk_ids : nullptr;
     a.n_chunks = level == 1 ? n_chunks : nullptr;
-    if (n_nodes <= kFastMax)
+    a.tree_status = level == G.levels ? tree_status_word(G, const_cast<float*>(store)) : nullptr;
+    if (n_nodes <= kFastMax) {
+      TraceScope ts("select_fast_kernel", level, s);
       e = launch_pdl(select_fast_kernel, dim3(heads), dim3(kSelectThreads), smem_fast, s, G, a);
-    else
+    } else {
+      TraceScope ts("select_kernel", level, s);
       e = launch_pdl(select_kernel, dim3(heads), dim3(kSelectThreads), smem, s, G, a);
+    }
     if (e != cudaSuccess) return e;
     zha_count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;

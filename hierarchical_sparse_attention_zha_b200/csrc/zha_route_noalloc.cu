@@ -59,12 +59,10 @@ extern "C" zha_status zha_route_noalloc(const zha_tree* tree, const float* d_Q, 
                                         int64_t n_tokens, float p, int32_t* d_chunk_ids,
                                         int32_t* d_n_chunks, int32_t max_sel,
                                         uint32_t* d_kept_bits, int32_t* d_status, void* stream) {
-  if (tree == nullptr) return zha_report_error(ZHA_ERR_INVALID, "zha_route_noalloc: tree is NULL");
+  zha_status st = zha_check_route_args(tree, d_Q, batch, n_tokens, p, d_chunk_ids, d_n_chunks,
+                                       max_sel, "zha_route_noalloc");
+  if (st != ZHA_OK) return st;
   const zha::Geom& G = tree->geom;
-  if (batch < 1 || batch > 65535)
-    return zha_report_error(ZHA_ERR_INVALID, "zha_route_noalloc: batch must be 1..65535");
-  if (n_tokens < 1 || n_tokens > G.max_tokens)
-    return zha_report_error(ZHA_ERR_INVALID, "zha_route_noalloc: n_tokens outside [1, max_tokens]");
   const zha::RouteLayout lay = zha::route_layout(G, batch, n_tokens);
   const int64_t need = d_kept_bits ? lay.bytes_no_bits : lay.bytes;
   if (need > int64_t(ZHA_ROUTE_NOALLOC_SCRATCH_BYTES)) {
@@ -75,22 +73,8 @@ extern "C" zha_status zha_route_noalloc(const zha_tree* tree, const float* d_Q, 
              (long long)need, (long long)ZHA_ROUTE_NOALLOC_SCRATCH_BYTES);
     return zha_report_error(ZHA_ERR_CAPACITY, msg);
   }
-  // The remaining argument checks are zha_route's; it rejects a workspace of
-  // zero bytes only after them, so check them here by the same rules.
-  if (d_Q == nullptr || (reinterpret_cast<uintptr_t>(d_Q) & 15) != 0)
-    return zha_report_error(ZHA_ERR_INVALID,
-                            "zha_route_noalloc: Q must be a non-NULL 16-byte aligned device pointer");
-  if (!(p > 0.f) || !std::isfinite(p))
-    return zha_report_error(ZHA_ERR_INVALID, "zha_route_noalloc: p must be > 0");
-  const int64_t nb = int64_t(G.chunk) * (n_tokens / G.chunk);
-  if (nb != tree->nb)
-    return zha_report_error(ZHA_ERR_STATE,
-                            "zha_route_noalloc: the tree's built prefix does not match n_tokens");
-  if (d_chunk_ids == nullptr || d_n_chunks == nullptr || max_sel < 1)
-    return zha_report_error(ZHA_ERR_INVALID,
-                            "zha_route_noalloc: chunk_ids / n_chunks NULL or max_sel < 1");
   void* base = nullptr;
-  zha_status st = scratch_address(&base);
+  st = scratch_address(&base);
   if (st != ZHA_OK) return st;
   // Nothing in the scratch has to start at zero: the select kernel clears each
   // level's bitmap before it sets bits, and scores and kept parents are written

@@ -23,6 +23,7 @@
 // the maximum over its node's 16 lanes (a transpose-reduction leaves lane p
 // of the node with heads 2p and 2p+1), then writes the scores of the
 // (node, head) pairs that are candidates.
+#include "zha_host.cuh"
 #include "zha_internal.cuh"
 #include "zha_tc.cuh"
 
@@ -279,14 +280,14 @@ cudaError_t launch_score_tc(const Geom& G, int level, int64_t n_nodes, int64_t n
                             const float* Q, const uint32_t* kept_up, int64_t words_up, float* sigma,
                             const float* store, int32_t* status, cudaStream_t s) {
   const size_t smem = score_tc_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(smem));
+  cudaError_t e = ensure_dynamic_smem(score_tc_kernel, smem);
   if (e != cudaSuccess) return e;
   const int qn = batch * G.group;
   // Nodes per CTA: enough CTAs to fill the GPU twice over, at most kStTile.
   int tile = kStTile;
   while (tile > kStNodes && (n_nodes * G.hkv) / tile < 2 * 148) tile >>= 1;
   dim3 grid(unsigned((n_nodes + tile - 1) / tile), unsigned(G.hkv), unsigned((qn + kStQ - 1) / kStQ));
+  TraceScope ts("score_tc_kernel", level, s);
   e = launch_pdl(score_tc_kernel, grid, dim3(kStThreads), smem, s, G, level, n_nodes, n_par, batch,
                  tile, Q, kept_up, words_up, sigma, store, status);
   zha_count_launch();

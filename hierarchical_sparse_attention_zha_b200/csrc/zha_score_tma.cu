@@ -36,8 +36,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include <mutex>
-
+#include "zha_host.cuh"
 #include "zha_internal.cuh"
 #include "zha_tc.cuh"
 
@@ -473,24 +472,6 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
   if (tid == 0 && ms.err != 0u && status != nullptr) atomicOr(status, ZHA_DEV_TIMEOUT);
 }
 
-namespace {
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_tiled_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q{};
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-}  // namespace
-
 // Level `level` of the summary store as a 3-D fp32 tensor {d, R, Hkv * cap}:
 // box 32 columns (128 B) x 16 planes x 8 nodes, 128-byte swizzled.
 bool score_tma_supported(const Geom& G) { return G.d == kD && G.nref == kR; }
@@ -499,7 +480,7 @@ cudaError_t launch_score_tma(const Geom& G, int level, int64_t n_nodes, int64_t 
                              const float* Q, const uint32_t* kept_up, int64_t words_up, float* sigma,
                              const float* store, int32_t* status, cudaStream_t s, bool* used) {
   *used = false;
-  const PFN_cuTensorMapEncodeTiled_v12000 fn = encode_tiled_fn();
+  const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
   if (fn == nullptr || n_nodes <= 0) return cudaSuccess;
   const float* level_base = store + G.off[level];
   CUtensorMap map{};
@@ -522,16 +503,15 @@ cudaError_t launch_score_tma(const Geom& G, int level, int64_t n_nodes, int64_t 
          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaSuccess;
   const size_t smem = score_tma_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(score_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(smem));
+  cudaError_t e = ensure_dynamic_smem(score_tma_kernel, smem);
   if (e != cudaSuccess) return e;
-  int dev = 0, sms = 148;
-  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  int sms = 148;
+  if ((e = device_sm_count(&sms)) != cudaSuccess) return e;
   const int32_t q_blocks = int32_t((int64_t(batch) * G.group + kQn - 1) / kQn);
   const int32_t groups = G.hkv * q_blocks;
   const int64_t tiles = groups * ((n_nodes + kNodes - 1) / kNodes);
   const unsigned ctas = unsigned(tiles < sms ? tiles : sms);
+  TraceScope ts("score_tma_kernel", level, s);
   e = launch_pdl(score_tma_kernel, dim3(ctas), dim3(kThreads), smem, s, map, bmap, G, level, n_nodes,
                  n_par, batch, q_blocks, groups, Q, kept_up, words_up, sigma, level_base, status);
   zha_count_launch();

@@ -72,6 +72,11 @@ def _load() -> ctypes.CDLL:
         "zha_attend_workspace_bytes": (c_size_t, [POINTER(Config), c_int32, c_int64]),
         "zha_sparse_attend": (c_int32, [P, P, P, P, c_int64, c_int64, c_int32, P, P, c_int32, P,
                                         P, P, c_size_t, P, P]),
+        "zha_trace_enable": (c_int32, [c_int32, c_char_p, c_int32]),
+        "zha_trace_count": (c_int32, []),
+        "zha_trace_dropped": (c_int32, []),
+        "zha_trace_read": (c_int32, [c_int32, POINTER(c_char_p), POINTER(c_int32), POINTER(c_float)]),
+        "zha_trace_clear": (None, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -107,6 +112,30 @@ def ptr(t: torch.Tensor | None):
 def stream_ptr(stream: torch.cuda.Stream | None = None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return c_void_p(s.cuda_stream)
+
+
+def trace_enable(max_records: int, name_filter: str | None = None, tag_filter: int = -1) -> None:
+    """Record CUDA events around the library's kernel launches (see zha.h)."""
+    check(lib.zha_trace_enable(max_records, name_filter.encode() if name_filter else None, tag_filter),
+          "zha_trace_enable")
+
+
+def trace_records() -> list[tuple[str, int, float]]:
+    """(kernel name, tag, device ms) of every recorded launch; synchronise first."""
+    out = []
+    for i in range(int(lib.zha_trace_count())):
+        name, tag, ms = c_char_p(), c_int32(), c_float()
+        check(lib.zha_trace_read(i, byref(name), byref(tag), byref(ms)), "zha_trace_read")
+        out.append((name.value.decode(), int(tag.value), float(ms.value)))
+    return out
+
+
+def trace_dropped() -> int:
+    return int(lib.zha_trace_dropped())
+
+
+def trace_clear() -> None:
+    lib.zha_trace_clear()
 
 
 def make_config(n_kv_heads: int, n_q_heads: int, head_dim: int, chunk: int, levels: int,

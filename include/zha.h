@@ -93,7 +93,10 @@ uint64_t zha_launch_count(void);
  * invalid). Layout, level-major: for l = 1..L, float32
  * [n_kv_heads][floor(max_tokens / C^l)][node_floats], each node holding
  * khat [n_ref][head_dim] then bhat [n_ref], padded to node_floats =
- * n_ref*head_dim + round_up(n_ref, 4). [ZHA: 무엇과 다른가] */
+ * n_ref*head_dim + round_up(n_ref, 4) [ZHA: 무엇과 다른가]; then, at the next
+ * 256-byte boundary, one 256-byte block whose first int32 is the tree's
+ * device status word (ZHA_DEV_TIMEOUT set by a build kernel whose bounded wait
+ * ran out; zha_build clears it, zha_route passes it on to its d_status). */
 size_t zha_tree_bytes(const zha_config* cfg);
 
 /* Create a host handle over a caller-owned store (>= zha_tree_bytes bytes,
@@ -124,7 +127,10 @@ zha_status zha_tree_level_layout(const zha_tree* tree, int32_t level, int64_t* o
  * khat = sum_c softmax(u)_c khat_{r,c}, bhat = F - q_r.khat/sqrt(d)
  * [ZHA: 무엇과 다른가: tangent-plane summary; "parents merge the child summaries
  * in the same way"]. Afterwards N_b = C*floor(n_tokens/C). Requires
- * 0 <= n_tokens <= min(ld, max_tokens). V is not read. */
+ * 0 <= n_tokens <= min(ld, max_tokens). V is not read. The tree's device status
+ * word is cleared first; a build kernel whose bounded wait runs out sets
+ * ZHA_DEV_TIMEOUT there (its summaries are then not valid), and the next
+ * zha_route reports it in its own d_status. */
 zha_status zha_build(zha_tree* tree, const void* d_K, int64_t ld, int64_t n_tokens, void* stream);
 
 /* Incremental build while decoding: n_tokens is the cache length after the
@@ -132,7 +138,8 @@ zha_status zha_build(zha_tree* tree, const void* d_K, int64_t ld, int64_t n_toke
  * >= the tree's N_b (else ZHA_ERR_STATE). Summarises each newly completed chunk
  * and merges every upper-level node the new chunks complete (level 1 every C
  * steps, level 2 every C^2 steps [ZHA: 무엇과 다른가]). One launch when up to
- * 8 chunks are new; a no-op when none is. */
+ * 8 chunks are new; a no-op when none is. A time-out of a build kernel is
+ * recorded in the tree's device status word as for zha_build. */
 zha_status zha_append_chunk(zha_tree* tree, const void* d_K, int64_t ld, int64_t n_tokens,
                             void* stream);
 
@@ -158,7 +165,10 @@ size_t zha_route_kept_words(const zha_config* cfg, int32_t batch, int64_t n_toke
  * ids ascending, and d_n_chunks [batch][n_q_heads] their count (the sink and
  * the tail [N_b, n_tokens) are implicit and not listed). d_kept_bits (nullable,
  * zha_route_kept_words words) receives every level's kept bitmap. d_ws:
- * >= zha_route_workspace_bytes bytes. d_status: ZHA_DEV_SELECTION_TRUNCATED, ZHA_DEV_TIMEOUT (tensor-core scoring). */
+ * >= zha_route_workspace_bytes bytes. d_status (nullable):
+ * ZHA_DEV_SELECTION_TRUNCATED, ZHA_DEV_TIMEOUT (tensor-core scoring, or a
+ * build of this tree whose bounded wait ran out, passed on from the tree's
+ * status word). */
 zha_status zha_route(const zha_tree* tree, const float* d_Q, int32_t batch, int64_t n_tokens,
                      float p, int32_t* d_chunk_ids, int32_t* d_n_chunks, int32_t max_sel,
                      uint32_t* d_kept_bits, void* d_ws, size_t ws_bytes, int32_t* d_status,
@@ -182,7 +192,12 @@ zha_status zha_route(const zha_tree* tree, const float* d_Q, int32_t batch, int6
  *    launches nothing; use zha_route with a workspace then.
  *  - The first call on each device looks up the array's device address (with
  *    that device current) and caches it; make that first call before any
- *    stream capture.
+ *    stream capture. With lazy module loading (the CUDA default) that first
+ *    lookup is also when the driver loads the library's module on the device
+ *    and reserves the array, so a caller whose device memory plan is already
+ *    full can see ZHA_ERR_CUDA (out of memory) there: make the first call at
+ *    initialisation, before committing the memory plan, or run with eager
+ *    module loading (CUDA_MODULE_LOADING=EAGER).
  *  - All calls on a device share the one array and it keeps the last call's
  *    contents (nothing in it needs to start at zero: every call clears or
  *    writes what it reads). Calls whose kernels overlap on the GPU -- on
@@ -214,6 +229,32 @@ zha_status zha_sparse_attend(const zha_tree* tree, const float* d_Q, const void*
                              const int32_t* d_chunk_ids, const int32_t* d_n_chunks,
                              int32_t max_sel, float* d_O, float* d_lse, void* d_ws,
                              size_t ws_bytes, int32_t* d_status, void* stream);
+
+/* ---- Kernel timing (profiling; the pages have no counterpart) ------------
+ * While enabled, every kernel the library launches whose name contains
+ * `name_filter` (NULL or "" = all) and whose tag equals `tag_filter` (-1 = all;
+ * the tag is the tree level for the routing kernels, 0 otherwise) is bracketed
+ * by two CUDA events recorded on its stream. Up to `max_records` launches are
+ * recorded (later ones are counted as dropped); max_records <= 0 disables
+ * tracing. The events are created here (host-side driver objects, no device
+ * memory); each enable discards the previous records. Recording events between
+ * kernels removes their programmatic overlap, so traced calls run a little
+ * slower than untraced ones. Not thread-safe against concurrent launches from
+ * other threads while enabled. */
+zha_status zha_trace_enable(int32_t max_records, const char* name_filter, int32_t tag_filter);
+
+/* Launches recorded since the last enable or clear, and launches dropped
+ * because the records were full. */
+int32_t zha_trace_count(void);
+int32_t zha_trace_dropped(void);
+
+/* Record i (0 <= i < zha_trace_count()): kernel name (static string), tag and
+ * device time in milliseconds. The caller must have synchronised the streams
+ * the kernels ran on. */
+zha_status zha_trace_read(int32_t i, const char** name, int32_t* tag, float* ms);
+
+/* Forget the records (the events are kept for reuse). */
+void zha_trace_clear(void);
 
 #ifdef __cplusplus
 }

@@ -24,7 +24,7 @@ Citations
                   attention states, used only as a second statement of the identity
                   behind ``combine_log_masses``.
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   * Level l of the tree covers C**l tokens; level 0 is the tokens. Node (l, i)
     exists iff (i+1)*C**l <= N_b with N_b = C*floor(N/C).
   * Merge rule: child c's log mass at reference query q_r is its own plane r

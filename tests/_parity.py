@@ -3,14 +3,12 @@ CPU oracle on the same seeded inputs (test infrastructure)."""
 
 from __future__ import annotations
 
-import math
-from dataclasses import dataclass, field
-
 import numpy as np
 import torch
 
 import oracle as O
 from hierarchical_sparse_attention_zha_b200 import workloads as W
+from oracle.parity import TIE_TOL, RouteReport, compare_route_head  # noqa: F401
 
 # Tolerances. Summaries: norm-wise relative 1e-4 (khat: max abs error over the
 # row / max abs of the row; bhat: abs error / max(1, |bhat|)). Scores: ties are
@@ -20,7 +18,6 @@ from hierarchical_sparse_attention_zha_b200 import workloads as W
 # inputs: |do| <= 2e-5 * max|v| + 2e-6 and |d lse| <= 2e-5 * max(1, |lse|),
 # which catches a dropped or duplicated token that 2e-2 would hide.
 SUMMARY_RTOL = 1e-4
-TIE_TOL = 1e-5
 O_ATOL = {"bf16": 2e-2, "f32": 1e-4}
 O_DERIVED_REL = 2e-5
 
@@ -76,47 +73,6 @@ def kept_from_bits(bits: np.ndarray, spec: W.Workload, batch: int, n_tokens: int
                 lv[(b, h)] = ids[ids < n_l]
         out[lvl] = lv
     return out
-
-
-@dataclass
-class RouteReport:
-    heads: int = 0
-    levels_compared: int = 0
-    ties: int = 0
-    hard: list = field(default_factory=list)
-    exact_heads: set = field(default_factory=set)
-
-
-def compare_route_head(q, otree, p, gpu_kept_by_level: dict, report: RouteReport, key) -> None:
-    """Compare one head level by level, each level conditioned on the GPU's kept
-    set one level up (the oracle's own selection at that level is compared)."""
-    forced = {lvl: ids for lvl, ids in gpu_kept_by_level.items()}
-    tr = O.route(q, otree, p, forced_kept=forced)
-    exact = True
-    for lvl, lt in tr.levels.items():
-        report.levels_compared += 1
-        own = set(lt.topp.kept.tolist())
-        gpu = set(np.asarray(gpu_kept_by_level[lvl]).tolist())
-        if own == gpu:
-            continue
-        exact = False
-        cand_pos = {int(n): i for i, n in enumerate(lt.candidates)}
-        sel = lt.topp
-        m = sel.m
-        sigma_cut = lt.sigma[sel.order[m - 1]] if m > 0 else math.inf
-        near_mass = (m >= 1 and abs(sel.cum[m - 1] - p) <= TIE_TOL) or \
-                    (m >= 2 and abs(sel.cum[m - 2] - p) <= TIE_TOL)
-        for node in own ^ gpu:
-            if node not in cand_pos:
-                report.hard.append((key, lvl, node, "not a candidate"))
-                continue
-            if abs(lt.sigma[cand_pos[node]] - sigma_cut) <= TIE_TOL or near_mass:
-                report.ties += 1
-            else:
-                report.hard.append((key, lvl, node, float(lt.sigma[cand_pos[node]]), float(sigma_cut)))
-    report.heads += 1
-    if exact:
-        report.exact_heads.add(key)
 
 
 def attend_errors(q, Kf, Vf, tokens, o_gpu, lse_gpu):

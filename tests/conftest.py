@@ -30,3 +30,31 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
+
+
+# Tie report: every parity case that compares kept sets with the oracle records
+# its RouteReport here; the counts are printed at the end of the session (also
+# under -q), so a run's log says how many disagreements were ties.
+_PARITY_ROWS: list = []
+
+
+@pytest.fixture(scope="session")
+def parity_log():
+    def record(case: str, report) -> None:
+        _PARITY_ROWS.append((case, report.summary()))
+    return record
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    if not _PARITY_ROWS:
+        return
+    tr = terminalreporter
+    tr.section("route parity vs oracle (ties within 1e-5 are counted, not failed)")
+    tot = {"heads": 0, "levels_compared": 0, "ties": 0, "hard": 0}
+    for case, s in _PARITY_ROWS:
+        tr.write_line(f"{case}: heads {s['heads']} levels {s['levels_compared']} ties {s['ties']} "
+                      f"hard {s['hard']} exact-heads {s['exact_heads']}")
+        for k in tot:
+            tot[k] += s[k]
+    tr.write_line(f"TOTAL: heads {tot['heads']} levels {tot['levels_compared']} ties {tot['ties']} "
+                  f"hard {tot['hard']}")

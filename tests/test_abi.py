@@ -67,7 +67,9 @@ def test_tree_bytes_matches_the_documented_layout(zha):
                    max_tokens=T)
         node = R * d + (R + 3) // 4 * 4
         floats = sum(H * (T // C ** l) * node for l in range(1, L + 1))
-        assert zha.tree_bytes(cfg) == (floats * 4 + 255) // 256 * 256
+        # the levels, then a 256-byte block (the tree's device status word) at
+        # the next 256-byte boundary
+        assert zha.tree_bytes(cfg) == (floats * 4 + 255) // 256 * 256 + 256
 
 
 @pytest.mark.parametrize("field,value", [("head_dim", 96), ("chunk", 1), ("chunk", 129),

@@ -36,12 +36,17 @@ def zha():
     return z
 
 
-def run_pipeline(zha, inp, n_tokens, p=None, max_sel=None, batch_index=0, stream=None):
+def run_pipeline(zha, inp, n_tokens, p=None, max_sel=None, batch_index=0, stream=None, tree=None,
+                 dev=None):
+    """Build (unless ``tree`` is given: a tree already built to ``n_tokens``),
+    route and attend on the GPU; ``dev`` = (K, V, ref_q, Q) device tensors."""
     spec = inp.spec
-    K, V, refq, Q = to_device(inp)
-    cfg = config_for(spec)
-    tree = zha.Tree(cfg, refq)
-    tree.build(K, n_tokens, stream=stream)
+    K, V, refq, Q = dev if dev is not None else to_device(inp)
+    if tree is None:
+        cfg = config_for(spec)
+        tree = zha.Tree(cfg, refq)
+        tree.build(K, n_tokens, stream=stream)
+    cfg = tree.cfg
     q = Q[batch_index].contiguous()
     B = q.shape[0]
     p = spec.p if p is None else p
@@ -56,10 +61,11 @@ def run_pipeline(zha, inp, n_tokens, p=None, max_sel=None, batch_index=0, stream
                 lse=lse.cpu().numpy().astype(np.float64), status=int(status.item()), p=p)
 
 
-def check_case(zha, inp, n_tokens, p=None, heads=None, all_nodes=True, batch_index=0):
+def check_case(zha, inp, n_tokens, p=None, heads=None, all_nodes=True, batch_index=0, tree=None,
+               dev=None):
     """Full comparison; returns the route report."""
     spec = inp.spec
-    res = run_pipeline(zha, inp, n_tokens, p=p, batch_index=batch_index)
+    res = run_pipeline(zha, inp, n_tokens, p=p, batch_index=batch_index, tree=tree, dev=dev)
     p = res["p"]
     assert res["status"] == 0
     G = spec.group
@@ -115,27 +121,28 @@ CASES = {
 
 
 @pytest.mark.parametrize("name", list(CASES))
-def test_parity_small_and_mid(zha, name):
+def test_parity_small_and_mid(zha, parity_log, name):
     spec, n_tokens = CASES[name]
     inp = W.generate(spec)
     rep = check_case(zha, inp, n_tokens)
+    parity_log(name, rep)
     print(f"{name}: heads {rep.heads} levels {rep.levels_compared} ties {rep.ties} "
           f"exact heads {len(rep.exact_heads)}")
     assert rep.heads == spec.batch * spec.n_q_heads
 
 
 @pytest.mark.parametrize("n_tokens", [1, 3, 4, 5, 15, 16, 17, 63, 64, 65, 83, 200, 257])
-def test_edge_token_counts(zha, n_tokens):
+def test_edge_token_counts(zha, parity_log, n_tokens):
     """C=4, L=3: no chunk, only a tail, exact chunk boundaries, orphans at every level."""
     spec = W.scaled("tiny", chunk=4, levels=3, n_tokens=260, n_needles=0, batch=3)
     inp = W.generate(spec)
-    check_case(zha, inp, n_tokens)
+    parity_log(f"edge_{n_tokens}", check_case(zha, inp, n_tokens))
 
 
 @pytest.mark.parametrize("p", [1e-6, 0.3, 0.999])
-def test_extreme_p(zha, p):
+def test_extreme_p(zha, parity_log, p):
     spec = W.scaled("tiny", n_tokens=2048, n_needles=2, batch=4)
-    check_case(zha, W.generate(spec), 2048 - 3, p=p)
+    parity_log(f"p_{p}", check_case(zha, W.generate(spec), 2048 - 3, p=p))
 
 
 @pytest.mark.parametrize("name", ["tiny_ragged", "256k_small"])
@@ -263,19 +270,53 @@ def test_deterministic_and_stream_ordered(zha):
 # Full-size workloads: sampled nodes and heads
 # ---------------------------------------------------------------------------
 
+def _sampled_heads(spec, inp, g, rng, n_random=4):
+    """Random heads of KV head g plus every needle head of g (the needles are
+    planted for batch 0's queries; they give the narrowest selections)."""
+    G = spec.group
+    heads = {(b, h) for (b, h, _) in inp.meta.get("needles", []) if h // G == g}
+    target = min(spec.batch * G, len(heads) + n_random)
+    while len(heads) < target:
+        heads.add((int(rng.integers(spec.batch)), g * G + int(rng.integers(G))))
+    return sorted(heads)
+
+
+def _check_sampled(zha, inp, res, g, otree, Kf, Vf, n_tokens, heads, report):
+    spec = inp.spec
+    kept = kept_from_bits(res["bits"], spec, spec.batch, n_tokens)
+    for (b, h) in heads:
+        q = inp.Q[0, b, h].astype(np.float64)
+        compare_route_head(q, otree, spec.p, {l: kept[l][(b, h)] for l in kept}, report, (b, h))
+        n = int(res["cnt"][b, h])
+        assert list(res["ids"][b, h, :n]) == list(kept[1][(b, h)])
+        S = O.leaf_token_set(res["ids"][b, h, :n], spec.chunk, n_tokens)
+        do, dl, vmax, lse_ref = attend_errors(q, Kf, Vf, S, res["out"][b, h], res["lse"][b, h])
+        assert do <= O_ATOL[spec.kv_dtype] and do <= derived_o_bound(vmax), (b, h, do)
+        assert dl <= derived_lse_bound(lse_ref), (b, h, dl)
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("key", ["32k", "256k", "deep", "1m"])
-def test_parity_full_size_sampled(zha, key):
+def test_parity_full_size_sampled(zha, parity_log, key):
+    """The full-size workloads: sampled summaries of every level against the
+    direct summary of the raw keys under them, and routing + attention of
+    sampled heads (random ones and the needle heads) of one KV head. For the
+    1M-context workload the stream then goes on: 101 more tokens through
+    zha_append_chunk one token per call (one new chunk: 16385 level-1 nodes,
+    so level 1 is routed by the wide-level selection), and the appended node
+    and the sampled heads are checked again at the new length."""
     spec = W.WORKLOADS[key]
     inp = W.generate(spec)
     n_tokens = spec.n_tokens
-    res = run_pipeline(zha, inp, n_tokens)
+    dev = to_device(inp)
+    res = run_pipeline(zha, inp, n_tokens, dev=dev)
     assert res["status"] == 0
     rng = np.random.default_rng(5)
-    G, C = spec.group, spec.chunk
+    C = spec.chunk
     g = int(rng.integers(spec.n_kv_heads))
-    Kf = cache_f64(inp, g, n_tokens)
-    Vf = values_f64(inp, g, n_tokens)
+    n_end = n_tokens + (101 if key == "1m" else 0)
+    Kf = cache_f64(inp, g, n_end)
+    Vf = values_f64(inp, g, n_end)
     # sampled summaries of every level vs the direct summary of the raw keys under them
     for lvl in range(1, spec.levels + 1):
         n_l = n_tokens // C ** lvl
@@ -286,21 +327,37 @@ def test_parity_full_size_sampled(zha, key):
             ek, eb = summary_errors(kh[g, i].cpu().numpy()[None], bh[g, i].cpu().numpy()[None],
                                     kd[None], bd[None])
             assert ek <= SUMMARY_RTOL and eb <= SUMMARY_RTOL, (lvl, i, ek, eb)
-    # routing and attention of sampled heads of KV head g
-    otree = O.build_tree(Kf, inp.ref_q[g], C, spec.levels, n_tokens)
-    kept = kept_from_bits(res["bits"], spec, spec.batch, n_tokens)
+    otree = O.build_tree(Kf[:n_tokens], inp.ref_q[g], C, spec.levels, n_tokens)
+    heads = _sampled_heads(spec, inp, g, rng)
     report = RouteReport()
-    for _ in range(4):
-        b, h = int(rng.integers(spec.batch)), g * G + int(rng.integers(G))
-        q = inp.Q[0, b, h].astype(np.float64)
-        compare_route_head(q, otree, spec.p, {l: kept[l][(b, h)] for l in kept}, report, (b, h))
-        n = int(res["cnt"][b, h])
-        S = O.leaf_token_set(res["ids"][b, h, :n], C, n_tokens)
-        do, dl, vmax, lse_ref = attend_errors(q, Kf, Vf, S, res["out"][b, h], res["lse"][b, h])
-        assert do <= O_ATOL[spec.kv_dtype] and do <= derived_o_bound(vmax), (b, h, do)
-        assert dl <= derived_lse_bound(lse_ref), (b, h, dl)
+    _check_sampled(zha, inp, res, g, otree, Kf[:n_tokens], Vf[:n_tokens], n_tokens, heads, report)
     assert not report.hard, report.hard[:10]
-    print(f"{key}: sampled heads {report.heads} ties {report.ties}")
+    parity_log(f"full_{key}", report)
+    if key != "1m":
+        return
+    tree = res["tree"]
+    for n in range(n_tokens + 1, n_end + 1):
+        tree.append_chunk(dev[0], n)
+    assert tree.built_tokens == n_tokens + C
+    res2 = run_pipeline(zha, inp, n_end, tree=tree, dev=dev)
+    assert res2["status"] == 0
+    # the appended level-1 node against the direct summary of its keys; levels
+    # 2 and 3 gain no node (their next parents are incomplete)
+    i_new = n_tokens // C
+    kd, bd = O.summarise_chunk(inp.ref_q[g], Kf[i_new * C:(i_new + 1) * C])
+    kh, bh = tree.level(1)
+    ek, eb = summary_errors(kh[g, i_new].cpu().numpy()[None], bh[g, i_new].cpu().numpy()[None],
+                            kd[None], bd[None])
+    assert ek <= SUMMARY_RTOL and eb <= SUMMARY_RTOL, (ek, eb)
+    otree2 = O.OracleTree(chunk=C, levels=spec.levels, n_tokens=n_end, qhat=otree.qhat,
+                          nodes=dict(otree.nodes))
+    otree2.nodes[1] = (np.concatenate([otree.nodes[1][0], kd[None]]),
+                       np.concatenate([otree.nodes[1][1], bd[None]]))
+    assert otree2.n_nodes(1) == i_new + 1 > 16384
+    report2 = RouteReport()
+    _check_sampled(zha, inp, res2, g, otree2, Kf, Vf, n_end, heads, report2)
+    assert not report2.hard, report2.hard[:10]
+    parity_log("full_1m_stream_16385_nodes", report2)
 
 
 @pytest.mark.parametrize("n_ref,head_dim,kv", [(1, 64, "f32"), (3, 64, "f32"), (16, 64, "bf16"),
@@ -343,3 +400,75 @@ def test_more_than_32_queries_per_kv_head(zha):
     spec = W.scaled("1m", n_kv_heads=2, n_q_heads=16, n_tokens=8192, stream_tokens=128, batch=8,
                     n_needles=2)
     check_case(zha, W.generate(spec), 8192 + 77)
+
+
+# ---------------------------------------------------------------------------
+# Levels wider than 16384 nodes (the wide-level selection) and the incremental
+# path of the 1M-context configuration
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("levels,p", [(1, 0.9), (2, 0.9), (2, 0.999)])
+def test_levels_wider_than_16384_nodes(zha, parity_log, levels, p):
+    """17499 level-1 nodes (C = 4, 69999 tokens). L = 1: every node is a
+    candidate (17499 > 16384: scores read from the route workspace). L = 2,
+    p = 0.9: ~14.6K candidates (cached in shared memory). L = 2, p = 0.999:
+    ~17.4K candidates (not cached)."""
+    spec = W.scaled("deep", n_kv_heads=1, n_q_heads=4, n_tokens=70000, levels=levels, batch=2,
+                    stream_tokens=0)
+    rep = check_case(zha, W.generate(spec), 70000 - 1, p=p)
+    parity_log(f"wide_L{levels}_p{p}", rep)
+
+
+def test_append_bf16_d128_c64_r16_matches_the_oracle(zha, parity_log):
+    """The incremental build of the 1M-context configuration (bf16 keys,
+    head_dim 128, R = 16, C = 64): a tensor-core prefill to an odd chunk count,
+    then one chunk per call across a level-2 boundary (fused append kernel),
+    6 chunks in one call (the same kernel), and 13 chunks from an odd chunk
+    index in one call (the tensor-core level-1 build with c_begin > 0 and a
+    tile whose second chunk lies past the new prefix). Every node of every
+    level is compared with the oracle and with a fresh build (norm-wise
+    relative 1e-4 each); then routing and attention at the final length."""
+    C = 64
+    spec = W.scaled("1m", n_kv_heads=2, n_q_heads=16, n_tokens=C * 90, stream_tokens=0, levels=2,
+                    batch=2, n_needles=2)
+    inp = W.generate(spec)
+    dev = to_device(inp)
+    K, V, refq, Q = dev
+    cfg = config_for(spec)
+    inc = zha.Tree(cfg, refq)
+    inc.build(K, C * 37 + 5)
+    for n in range(C * 37 + 6, C * 65 + 4):
+        inc.append_chunk(K, n)                   # one chunk at each boundary
+    assert inc.built_tokens == C * 65
+    inc.append_chunk(K, C * 71 + 2)              # 6 chunks in one call
+    assert inc.built_tokens == C * 71
+    inc.append_chunk(K, C * 84 + 9)              # 13 chunks from chunk 71 (odd)
+    assert inc.built_tokens == C * 84
+    n_final = C * 84 + 9
+    fresh = zha.Tree(cfg, refq)
+    fresh.build(K, n_final)
+    torch.cuda.synchronize()
+    for g in range(spec.n_kv_heads):
+        otree = O.build_tree(cache_f64(inp, g, n_final), inp.ref_q[g], C, spec.levels, n_final)
+        for lvl in (1, 2):
+            n_l = otree.n_nodes(lvl)
+            for t in (inc, fresh):
+                kh, bh = t.level(lvl)
+                ek, eb = summary_errors(kh[g, :n_l].cpu().numpy().astype(np.float64),
+                                        bh[g, :n_l].cpu().numpy().astype(np.float64), *otree.nodes[lvl])
+                assert ek <= SUMMARY_RTOL and eb <= SUMMARY_RTOL, (g, lvl, ek, eb)
+    rep = check_case(zha, inp, n_final, tree=inc, dev=dev)
+    parity_log("append_bf16_c64", rep)
+
+
+def test_build_status_is_clean_and_reaches_the_route(zha):
+    """The tree's device status word (build time-outs) starts at zero after a
+    build and a route over it reports no bit."""
+    spec = W.scaled("1m", n_kv_heads=1, n_q_heads=8, n_tokens=4096, stream_tokens=64, batch=2,
+                    n_needles=0)
+    inp = W.generate(spec)
+    res = run_pipeline(zha, inp, 4096 + 3)
+    assert res["status"] == 0
+    st = res["tree"].store.view(torch.int32)
+    off = (zha.tree_bytes(res["tree"].cfg) - 256) // 4
+    assert int(st[off].item()) == 0

@@ -93,3 +93,41 @@ def test_noalloc_route_refuses_calls_beyond_its_fixed_scratch(zha):
     assert rc == zha.ZHA_ERR_CAPACITY
     assert "scratch" in zha.last_error() and "zha_route" in zha.last_error()
     assert zha.launch_count() == before
+
+
+def test_noalloc_route_allocates_nothing(zha):
+    """The property the entry point exists for: after a first call (which may
+    load the library's module on the device and reserve its fixed scratch), a
+    further call changes neither the device's free memory nor torch's caching
+    allocator (no cudaMalloc, no torch allocation)."""
+    spec = W.scaled("32k", n_kv_heads=1, n_q_heads=4, n_tokens=8192, stream_tokens=64)
+    inp, K, refq, Q = _inputs(spec, n_batches=1)
+    n_tokens = 8192 + 5
+    cfg = zha.make_config(spec.n_kv_heads, spec.n_q_heads, spec.head_dim, spec.chunk, spec.levels,
+                          spec.n_ref, torch.bfloat16, spec.capacity)
+    tree = zha.Tree(cfg, refq)
+    tree.build(K, n_tokens)
+    B, Hq = spec.batch, spec.n_q_heads
+    max_sel = n_tokens // spec.chunk
+    q = Q[0].contiguous()
+    ids = torch.empty((B, Hq, max_sel), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((B, Hq), dtype=torch.int32, device="cuda")
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = zha.stream_ptr()
+
+    def call():
+        rc = zha.lib.zha_route_noalloc(tree.handle, zha.ptr(q), B, n_tokens, spec.p, zha.ptr(ids),
+                                       zha.ptr(cnt), max_sel, None, zha.ptr(st), stream)
+        assert rc == zha.ZHA_OK, zha.last_error()
+        torch.cuda.synchronize()
+
+    call()                                     # first call on the device: set-up
+    free0, _ = torch.cuda.mem_get_info()
+    stats0 = torch.cuda.memory_stats()
+    call()
+    free1, _ = torch.cuda.mem_get_info()
+    stats1 = torch.cuda.memory_stats()
+    assert free1 == free0
+    for key in ("allocation.all.allocated", "segment.all.allocated", "allocated_bytes.all.allocated"):
+        assert stats1.get(key, 0) == stats0.get(key, 0), key
+    assert int(st.item()) == 0
