@@ -166,6 +166,8 @@ def kernel_bytes(name: str, tag: int, by: dict) -> float | None:
     launch reads its level's visited node records and the queries and writes one
     score per (query head, candidate) pair; a selection launch reads those scores;
     the attention kernels read the selected K/V rows and the queries."""
+    if name in ("score_dense_kernel", "select_top_kernel"):
+        return None                    # several levels in one launch (latency-bound)
     if name.startswith("score") and tag in by["levels"]:
         lv = by["levels"][tag]
         return lv["nodes"] * by["node_bytes"] + lv["pairs"] * 4 + by["q_bytes"]

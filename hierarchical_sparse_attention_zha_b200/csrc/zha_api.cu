@@ -13,10 +13,6 @@ cudaError_t launch_build(const Geom& G, const void* K, int64_t ld, int64_t nb_ol
                          const float* refq, float* store, cudaStream_t s);
 cudaError_t launch_append(const Geom& G, const void* K, int64_t ld, int64_t nb_old, int64_t nb_new,
                           const float* refq, float* store, cudaStream_t s);
-cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n_tokens, float p,
-                         int32_t* chunk_ids, int32_t* n_chunks, int32_t max_sel, uint32_t* bits,
-                         float* sigma, int32_t* kp, const RouteLayout& lay, int32_t* status,
-                         const float* store, cudaStream_t s);
 cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const void* V, int64_t ld,
                              int64_t n_tokens, int32_t batch, const int32_t* chunk_ids,
                              const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
@@ -220,8 +216,13 @@ size_t zha_route_kept_words(const zha_config* cfg, int32_t batch, int64_t n_toke
 }  // extern "C"
 
 // Argument checks of a routing call (zha_route and zha_route_noalloc share them).
+zha_status zha_check_p(float p, const char* who) {
+  if (!(p > 0.f) || !std::isfinite(p)) return fail(ZHA_ERR_INVALID, "%s: p must be > 0", who);
+  return ZHA_OK;
+}
+
 zha_status zha_check_route_args(const zha_tree* tree, const float* d_Q, int32_t batch,
-                                int64_t n_tokens, float p, const int32_t* d_chunk_ids,
+                                int64_t n_tokens, const int32_t* d_chunk_ids,
                                 const int32_t* d_n_chunks, int32_t max_sel, const char* who) {
   if (tree == nullptr) return fail(ZHA_ERR_INVALID, "%s: tree is NULL", who);
   const zha::Geom& G = tree->geom;
@@ -231,7 +232,6 @@ zha_status zha_check_route_args(const zha_tree* tree, const float* d_Q, int32_t 
   if (n_tokens < 1 || n_tokens > G.max_tokens)
     return fail(ZHA_ERR_INVALID, "%s: n_tokens %lld outside [1, max_tokens]", who,
                 (long long)n_tokens);
-  if (!(p > 0.f) || !std::isfinite(p)) return fail(ZHA_ERR_INVALID, "%s: p must be > 0", who);
   const int64_t nb = int64_t(G.chunk) * (n_tokens / G.chunk);
   if (nb != tree->nb)
     return fail(ZHA_ERR_STATE, "%s: tree covers %lld tokens, n_tokens %lld needs %lld", who,
@@ -243,28 +243,67 @@ zha_status zha_check_route_args(const zha_tree* tree, const float* d_Q, int32_t 
 
 extern "C" {
 
-zha_status zha_route(const zha_tree* tree, const float* d_Q, int32_t batch, int64_t n_tokens,
-                     float p, int32_t* d_chunk_ids, int32_t* d_n_chunks, int32_t max_sel,
-                     uint32_t* d_kept_bits, void* d_ws, size_t ws_bytes, int32_t* d_status,
-                     void* stream) {
-  const zha_status st = zha_check_route_args(tree, d_Q, batch, n_tokens, p, d_chunk_ids, d_n_chunks,
-                                             max_sel, "zha_route");
-  if (st != ZHA_OK) return st;
+// zha_route and zha_route_ex after their own argument checks.
+static zha_status route_impl(const zha_tree* tree, const float* d_Q, int32_t batch, int64_t n_tokens,
+                             const zha::RoutePolicy& pol, int32_t* d_chunk_ids, int32_t* d_n_chunks,
+                             int32_t max_sel, uint32_t* d_kept_bits, void* d_ws, size_t ws_bytes,
+                             int32_t* d_status, void* stream, const char* who) {
   const zha::Geom& G = tree->geom;
   const zha::RouteLayout lay = zha::route_layout(G, batch, n_tokens);
   const int64_t need = d_kept_bits ? lay.bytes_no_bits : lay.bytes;
   if (d_ws == nullptr || !aligned(d_ws, 256) || int64_t(ws_bytes) < need)
-    return fail(ZHA_ERR_CAPACITY, "zha_route: workspace must be 256-byte aligned with %lld bytes",
+    return fail(ZHA_ERR_CAPACITY, "%s: workspace must be 256-byte aligned with %lld bytes", who,
                 (long long)need);
   char* ws = static_cast<char*>(d_ws);
   float* sigma = reinterpret_cast<float*>(ws);
   int32_t* kp = reinterpret_cast<int32_t*>(ws + zha::round_up(lay.sig_floats * 4, 256));
   uint32_t* bits = d_kept_bits ? d_kept_bits : reinterpret_cast<uint32_t*>(ws + lay.bytes_no_bits);
-  cudaError_t e = zha::launch_route(G, d_Q, batch, n_tokens, p, d_chunk_ids, d_n_chunks, max_sel,
+  cudaError_t e = zha::launch_route(G, d_Q, batch, n_tokens, pol, d_chunk_ids, d_n_chunks, max_sel,
                                     bits, sigma, kp, lay, d_status, tree->store,
                                     static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "zha_route");
+  if (e != cudaSuccess) return cuda_fail(e, who);
   return ZHA_OK;
+}
+
+zha_status zha_route(const zha_tree* tree, const float* d_Q, int32_t batch, int64_t n_tokens,
+                     float p, int32_t* d_chunk_ids, int32_t* d_n_chunks, int32_t max_sel,
+                     uint32_t* d_kept_bits, void* d_ws, size_t ws_bytes, int32_t* d_status,
+                     void* stream) {
+  zha_status st = zha_check_route_args(tree, d_Q, batch, n_tokens, d_chunk_ids, d_n_chunks, max_sel,
+                                       "zha_route");
+  if (st != ZHA_OK) return st;
+  if ((st = zha_check_p(p, "zha_route")) != ZHA_OK) return st;
+  return route_impl(tree, d_Q, batch, n_tokens, zha::uniform_top_p(p), d_chunk_ids, d_n_chunks,
+                    max_sel, d_kept_bits, d_ws, ws_bytes, d_status, stream, "zha_route");
+}
+
+zha_status zha_route_ex(const zha_tree* tree, const float* d_Q, int32_t batch, int64_t n_tokens,
+                        const zha_route_policy* policy, int32_t* d_chunk_ids, int32_t* d_n_chunks,
+                        int32_t max_sel, uint32_t* d_kept_bits, void* d_ws, size_t ws_bytes,
+                        int32_t* d_status, void* stream) {
+  zha_status st = zha_check_route_args(tree, d_Q, batch, n_tokens, d_chunk_ids, d_n_chunks, max_sel,
+                                       "zha_route_ex");
+  if (st != ZHA_OK) return st;
+  if (policy == nullptr) return fail(ZHA_ERR_INVALID, "zha_route_ex: policy is NULL");
+  if (policy->reserved != 0) return fail(ZHA_ERR_INVALID, "zha_route_ex: policy.reserved must be 0");
+  zha::RoutePolicy pol{};
+  if (policy->mode == ZHA_SELECT_TOP_P) {
+    for (int l = 1; l <= tree->geom.levels; ++l) {
+      if ((st = zha_check_p(policy->p[l - 1], "zha_route_ex")) != ZHA_OK) return st;
+      pol.p[l] = policy->p[l - 1];
+    }
+  } else if (policy->mode == ZHA_SELECT_TOP_K) {
+    pol.topk = 1;
+    for (int l = 1; l <= tree->geom.levels; ++l) {
+      if (policy->k[l - 1] < 1)
+        return fail(ZHA_ERR_INVALID, "zha_route_ex: k of level %d must be >= 1", l);
+      pol.k[l] = policy->k[l - 1];
+    }
+  } else {
+    return fail(ZHA_ERR_INVALID, "zha_route_ex: unknown policy mode %d", policy->mode);
+  }
+  return route_impl(tree, d_Q, batch, n_tokens, pol, d_chunk_ids, d_n_chunks, max_sel, d_kept_bits,
+                    d_ws, ws_bytes, d_status, stream, "zha_route_ex");
 }
 
 size_t zha_attend_workspace_bytes(const zha_config* cfg, int32_t batch, int64_t n_tokens) {

@@ -439,6 +439,9 @@ cudaError_t launch_combine(const Geom& G, int32_t batch, const int32_t* chunk_id
                            const float* partial, const AttendLayout& lay, int32_t* status,
                            cudaStream_t s) {
   const unsigned heads = unsigned(int64_t(batch) * G.hq);
+  cudaError_t e = G.d == 128 ? ensure_dynamic_smem(combine_ranges_kernel<128>, 0)
+                             : ensure_dynamic_smem(combine_ranges_kernel<64>, 0);
+  if (e != cudaSuccess) return e;
   TraceScope ts("combine_ranges_kernel", 0, s);
   if (G.d == 128)
     combine_ranges_kernel<128><<<heads, 128, 0, s>>>(G, batch, lay.n_chunks, chunk_ids, n_chunks,

@@ -1006,6 +1006,7 @@ cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const
   zha_count_launch();
 
   const int64_t heads = int64_t(batch) * G.hq;
+  if ((e = ensure_dynamic_smem(combine_split_kernel, 0)) != cudaSuccess) return e;
   TraceScope ts("combine_split_kernel", 0, s);
   e = launch_pdl(combine_split_kernel, dim3(unsigned(heads)), dim3(32 * kCombineWarps), 0, s, G, batch,
                  lay.q_blocks, lay.n_blocks, units, split, slots, O, lse);

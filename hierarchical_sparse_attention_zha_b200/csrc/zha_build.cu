@@ -295,6 +295,7 @@ static cudaError_t launch_build_t(const Geom& G, const void* K, int64_t ld, int6
     const int64_t items = (p_end - p_begin) * G.nref;
     const int per = kBuildThreads / 32;
     dim3 grid(unsigned((items + per - 1) / per), unsigned(G.hkv));
+    if ((e = ensure_dynamic_smem(merge_level_kernel<D>, 0)) != cudaSuccess) return e;
     {
       TraceScope ts("merge_level_kernel", level, s);
       merge_level_kernel<D><<<grid, kBuildThreads, 0, s>>>(G, level, p_begin, p_end - p_begin,

@@ -62,6 +62,12 @@ cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes) {
   if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(bytes))) !=
       cudaSuccess)
     return e;
+  // Every kernel asks for the largest shared-memory carveout, so that
+  // back-to-back launches of different kernels need no L1 / shared-memory
+  // reconfiguration of the SMs between them.
+  if ((e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                int(cudaSharedmemCarveoutMaxShared))) != cudaSuccess)
+    return e;
   g_smem[dev][kernel] = bytes;
   return cudaSuccess;
 }

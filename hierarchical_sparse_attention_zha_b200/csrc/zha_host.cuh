@@ -17,9 +17,10 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 // Multiprocessors of the current device (queried once per device).
 cudaError_t device_sm_count(int* sms);
 
-// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) for `kernel` on the current
-// device, skipped when an earlier call on this device already set at least
-// `bytes`.
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) and the largest preferred
+// shared-memory carveout for `kernel` on the current device, skipped when an
+// earlier call on this device already set at least `bytes`. Kernels without
+// dynamic shared memory call it with 0 for the carveout alone.
 cudaError_t ensure_dynamic_smem(const void* kernel, size_t bytes);
 
 template <typename... Args>

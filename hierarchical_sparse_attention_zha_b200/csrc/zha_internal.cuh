@@ -284,10 +284,25 @@ __device__ __forceinline__ float order_key_float(uint32_t k) {
   return __uint_as_float(u);
 }
 
-cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n_tokens, float p,
-                         int32_t* chunk_ids, int32_t* n_chunks, int32_t max_sel, uint32_t* bits,
-                         float* sigma, int32_t* kp, const RouteLayout& lay, int32_t* status,
-                         const float* store, cudaStream_t s);
+// Per-level selection rule of a route: top-p with mass p[l], or top-k keeping
+// k[l] nodes, for levels l = 1..L (index l).
+struct RoutePolicy {
+  int32_t topk;
+  float p[ZHA_MAX_LEVELS + 1];
+  int32_t k[ZHA_MAX_LEVELS + 1];
+};
+
+inline RoutePolicy uniform_top_p(float p) {
+  RoutePolicy r{};
+  for (int l = 0; l <= ZHA_MAX_LEVELS; ++l) r.p[l] = p;
+  return r;
+}
+
+cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n_tokens,
+                         const RoutePolicy& pol, int32_t* chunk_ids, int32_t* n_chunks,
+                         int32_t max_sel, uint32_t* bits, float* sigma, int32_t* kp,
+                         const RouteLayout& lay, int32_t* status, const float* store,
+                         cudaStream_t s);
 
 }  // namespace zha
 
@@ -305,5 +320,6 @@ struct zha_tree {
 void zha_count_launch();
 zha_status zha_report_error(zha_status s, const char* msg);
 zha_status zha_check_route_args(const zha_tree* tree, const float* d_Q, int32_t batch,
-                                int64_t n_tokens, float p, const int32_t* d_chunk_ids,
+                                int64_t n_tokens, const int32_t* d_chunk_ids,
                                 const int32_t* d_n_chunks, int32_t max_sel, const char* who);
+zha_status zha_check_p(float p, const char* who);

@@ -62,27 +62,27 @@ __device__ __forceinline__ void cp_async16_ca(uint32_t dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" : : "r"(dst), "l"(src) : "memory");
 }
 
+// One CTA: nodes [tile_i * tile, + tile) of level `level` of KV head g, query
+// heads [qblock * kScoreQBlock, + kScoreQBlock) of g's group.
 template <int D, int RP>
-__global__ void __launch_bounds__(kScoreThreads)
-score_kernel(Geom G, int level, int64_t n_nodes, int64_t n_par, int32_t batch, int tile,
-             const float* __restrict__ Q, const uint32_t* __restrict__ kept_up, int64_t words_up,
-             float* __restrict__ sigma, const float* __restrict__ store) {
+__device__ __forceinline__ void score_tile(const Geom& G, int level, int64_t n_nodes, int64_t n_par,
+                                           int32_t batch, int tile, int64_t tile_i, int g, int qblock,
+                                           const float* __restrict__ Q,
+                                           const uint32_t* __restrict__ kept_up, int64_t words_up,
+                                           float* __restrict__ sigma, const float* __restrict__ store) {
   using S = ScoreShape<D, RP>;
   constexpr int NW = kScoreThreads / 32;
   extern __shared__ float4 smem_v4[];
   float* s_kbuf = reinterpret_cast<float*>(smem_v4);       // [NW][KBUF]
-  pdl_trigger();
-  pdl_wait();
   float* s_q = s_kbuf + NW * S::KBUF;                       // [nq][P][QS]
   __shared__ unsigned long long s_mask[kScoreTile];
   __shared__ uint32_t s_kw[kScoreQBlock][3];
   __shared__ int64_t s_out[kScoreQBlock];
   __shared__ unsigned long long s_any;
-  const int g = blockIdx.y;
-  const int64_t n0 = int64_t(blockIdx.x) * tile;
+  const int64_t n0 = tile_i * tile;
   const int GQ = G.group;
   const int qn_total = batch * GQ;
-  const int qb0 = blockIdx.z * kScoreQBlock;
+  const int qb0 = qblock * kScoreQBlock;
   const int nq = min(kScoreQBlock, qn_total - qb0);
   const int C = G.chunk, R = G.nref;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -194,6 +194,134 @@ score_kernel(Geom G, int level, int64_t n_nodes, int64_t n_par, int32_t batch, i
   }
 }
 
+template <int D, int RP>
+__global__ void __launch_bounds__(kScoreThreads)
+score_kernel(Geom G, int level, int64_t n_nodes, int64_t n_par, int32_t batch, int tile,
+             const float* __restrict__ Q, const uint32_t* __restrict__ kept_up, int64_t words_up,
+             float* __restrict__ sigma, const float* __restrict__ store) {
+  pdl_trigger();
+  pdl_wait();
+  score_tile<D, RP>(G, level, n_nodes, n_par, batch, tile, blockIdx.x, blockIdx.y, blockIdx.z, Q,
+                    kept_up, words_up, sigma, store);
+}
+
+// The small top levels scored densely in one launch: every node of each level
+// for every query head (a superset of the candidates; selection reads only the
+// candidates' scores). A CTA computes one tile of kDenseRows (node, plane) rows
+// -- 64 / R consecutive nodes of one level of KV head g -- against a block of
+// up to kDenseQ query heads of g's group, as a small fp32 matrix product:
+// operands staged in shared memory K-block-major ([k / 4][row][4]), each thread
+// a 4-row x 2-query register tile (rows ty + 16 i, queries tx and tx + 16), so
+// that the 16-byte loads of a warp are broadcast (rows) or contiguous (queries).
+// Then sigma = max over the node's planes of (dot / sqrt(d) + bhat).
+// blockIdx.x runs over the levels' tiles in turn.
+constexpr int kDenseRows = 64;
+constexpr int kDenseQ = 32;
+constexpr int kDenseThreads = 256;
+
+struct DenseLevels {
+  int32_t count;
+  int32_t level[ZHA_MAX_LEVELS];
+  int64_t n_nodes[ZHA_MAX_LEVELS];
+  int64_t tile0[ZHA_MAX_LEVELS + 1];       // first blockIdx.x of each level
+  float* sigma[ZHA_MAX_LEVELS];
+};
+
+template <int D>
+__host__ __device__ constexpr size_t dense_smem_bytes() {
+  return size_t(kDenseRows + kDenseQ) * D * sizeof(float);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kDenseThreads)
+score_dense_kernel(Geom G, DenseLevels dl, int32_t batch, const float* __restrict__ Q,
+                   const float* __restrict__ store) {
+  extern __shared__ float4 smem_v4[];
+  float4* As = smem_v4;                          // [D / 4][kDenseRows]
+  float4* Bs = smem_v4 + (D / 4) * kDenseRows;   // [D / 4][kDenseQ]
+  float* Cs = reinterpret_cast<float*>(smem_v4); // [kDenseRows][kDenseQ + 1] after the product
+  __shared__ float s_b[kDenseRows];
+  pdl_trigger();
+  pdl_wait();
+  int li = 0;
+  while (li + 1 < dl.count && int64_t(blockIdx.x) >= dl.tile0[li + 1]) ++li;
+  const int level = dl.level[li];
+  const int64_t n_nodes = dl.n_nodes[li];
+  const int R = G.nref, npt = kDenseRows / R, rows = npt * R;
+  const int g = blockIdx.y, qb = blockIdx.z;
+  const int64_t n0 = (int64_t(blockIdx.x) - dl.tile0[li]) * npt;
+  const int nn = int(min64(npt, n_nodes - n0));
+  const int qn = min(kDenseQ, batch * G.group - qb * kDenseQ);
+  const int tid = threadIdx.x;
+  const float* level_base = store + G.off[level] + int64_t(g) * G.cap[level] * G.node_floats;
+  auto head_of = [&](int q) -> int64_t {
+    const int qi = qb * kDenseQ + q;
+    return int64_t(qi / G.group) * G.hq + g * G.group + qi % G.group;
+  };
+
+  // Stage the tile's planes, bhat and the queries.
+  for (int v = tid; v < kDenseRows * (D / 4); v += kDenseThreads) {
+    const int row = v / (D / 4), kb = v % (D / 4);
+    const int j = row / R, r = row % R;
+    float4* dst = As + kb * kDenseRows + row;
+    if (row < rows && j < nn) {
+      const float* src = level_base + (n0 + j) * G.node_floats + r * D + 4 * kb;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" : : "r"(uint32_t(__cvta_generic_to_shared(dst))),
+                   "l"(src) : "memory");
+    } else {
+      *dst = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  for (int v = tid; v < kDenseQ * (D / 4); v += kDenseThreads) {
+    const int q = v / (D / 4), kb = v % (D / 4);
+    float4* dst = Bs + kb * kDenseQ + q;
+    if (q < qn) {
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" : : "r"(uint32_t(__cvta_generic_to_shared(dst))),
+                   "l"(Q + head_of(q) * D + 4 * kb) : "memory");
+    } else {
+      *dst = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  if (tid < kDenseRows) {
+    const int j = tid / R, r = tid % R;
+    s_b[tid] = (tid < rows && j < nn) ? level_base[(n0 + j) * G.node_floats + R * D + r] : 0.f;
+  }
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+
+  const int tx = tid & 15, ty = tid >> 4;
+  float acc[4][2] = {};
+#pragma unroll 4
+  for (int kb = 0; kb < D / 4; ++kb) {
+    float4 a[4], b[2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = As[kb * kDenseRows + ty + 16 * i];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) b[j] = Bs[kb * kDenseQ + tx + 16 * j];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        acc[i][j] += a[i].x * b[j].x + a[i].y * b[j].y + a[i].z * b[j].z + a[i].w * b[j].w;
+  }
+  __syncthreads();                               // the operands are read; Cs overwrites them
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int row = ty + 16 * i;
+      Cs[row * (kDenseQ + 1) + tx + 16 * j] = acc[i][j] * G.scale + s_b[row];
+    }
+  __syncthreads();
+  for (int o = tid; o < npt * kDenseQ; o += kDenseThreads) {
+    const int j = o / kDenseQ, q = o % kDenseQ;
+    if (j >= nn || q >= qn) continue;
+    float m = -INFINITY;
+    for (int r = 0; r < R; ++r) m = fmaxf(m, Cs[(j * R + r) * (kDenseQ + 1) + q]);
+    dl.sigma[li][head_of(q) * n_nodes + n0 + j] = m;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Block-wide helpers for the select kernel (blockDim = kSelectThreads).
 // ---------------------------------------------------------------------------
@@ -263,6 +391,25 @@ __device__ float block_sum(float v, float* tmp) {
 
 // ---------------------------------------------------------------------------
 // Selection for one query head at one level.
+//
+// Candidates in candidate order (ascending node index): the children of the
+// kept parents (compacted from the level above's bitmap), then the level's
+// orphans. With at most kFastMax candidates every candidate's order key (score
+// descending, then index ascending) and its softmax mass in 2^-32 fixed point
+// are computed once into shared memory:
+//  * up to kFastSmallN candidates: thread i counts the mass of every candidate
+//    ordered before it; i is kept iff that mass is below p (the minimal prefix
+//    holding mass p). No radix passes, a handful of barriers.
+//  * more: the cut key by a radix select over 8-bit digits with per-warp
+//    histograms of mass, starting at the first byte in which the candidates'
+//    keys differ; runs of equal buckets are summed in registers before the
+//    atomic add.
+// The rounding of the fixed-point masses adds at most n 2^-33 to any
+// cumulative mass (< 2e-6 at n = 16384). Wider candidate sets (generic path):
+// scores cached when they fit, masses recomputed per pass in 2^-40 fixed point,
+// four radix passes. The fixed-budget mode (top-k) runs the same cut with a
+// mass of exactly 1 per candidate and the threshold k, so it keeps the first
+// min(k, n) candidates of the order.
 // ---------------------------------------------------------------------------
 struct SelectArgs {
   int level;
@@ -274,9 +421,10 @@ struct SelectArgs {
   const float* sigma;        // [B*Hq][n_nodes]
   int32_t* kp;               // scratch [B*Hq][kp_stride]
   int64_t kp_stride;
-  unsigned long long p_fixed;    // p in units of 2^-40 (select_kernel)
-  unsigned long long p_fixed32;  // p in units of 2^-32 (select_fast_kernel)
+  unsigned long long p_fixed;    // p in units of 2^-40 (generic path); top-k: k
+  unsigned long long p_fixed31;  // p in units of 2^-31 (shared-memory path); top-k: k
   int keep_all;
+  int topk;                  // fixed budget: every candidate weighs 1, the threshold is k
   int32_t* chunk_ids;        // level 1 only
   int32_t* n_chunks;
   int32_t max_sel;
@@ -293,31 +441,63 @@ __device__ __forceinline__ void forward_tree_status(const SelectArgs& a) {
   }
 }
 
-__global__ void __launch_bounds__(kSelectThreads)
-select_kernel(Geom G, SelectArgs a) {
+constexpr int kFastMax = 16384;
+constexpr int kFastSmallN = kSelectThreads;
+constexpr int kHistBins = (kSelectThreads / 32) * 256;   // generic path: per-warp 256-bin histograms
+constexpr int kCutBins = 2048;                           // splitter histogram of the shared-memory path
+constexpr int kBitsSmem = 4096;                          // kept-bitmap words held in shared memory
+static_assert(kSelectCache <= kFastMax, "the generic path caches scores in the key array");
+static_assert(2 * kCutBins * 4 + kFastSmallN * 4 + (kFastMax / 32) * 4 <= kHistBins * 8,
+              "the splitter histograms, window list and flags share the histogram region");
+
+__host__ __device__ constexpr size_t select_smem_bytes() {
+  return size_t(2 * kFastMax) * sizeof(uint32_t) + size_t(kHistBins) * sizeof(unsigned long long) +
+         size_t(kSelectKpCache) * sizeof(int32_t) + size_t(kBitsSmem) * sizeof(uint32_t);
+}
+
+// Shared memory of a select CTA (dynamic, select_smem_bytes()).
+struct SelectSmem {
+  uint32_t* s_key;               // [kFastMax] keys; the generic path's cached scores
+  uint32_t* s_m;                 // [kFastMax] fixed-point masses
+  unsigned long long* hist;      // [kHistBins] generic path; the shared-memory path uses the
+                                 // region for hm, hc [kCutBins] u32, win [kFastSmallN] i32 and
+                                 // flags [kFastMax / 32] u32
+  int32_t* s_kp;                 // [kSelectKpCache] kept parents
+  uint32_t* s_bits;              // [kBitsSmem] this level's kept bitmap when it fits
+};
+
+__device__ __forceinline__ SelectSmem select_smem() {
   extern __shared__ float4 smem_v4[];
-  unsigned long long* hist = reinterpret_cast<unsigned long long*>(smem_v4);  // [nwarps][256]
-  float* s_sig = reinterpret_cast<float*>(hist + (kSelectThreads / 32) * 256);
-  int32_t* s_kp = reinterpret_cast<int32_t*>(s_sig + kSelectCache);           // [kSelectKpCache]
+  SelectSmem m;
+  m.s_key = reinterpret_cast<uint32_t*>(smem_v4);
+  m.s_m = m.s_key + kFastMax;
+  m.hist = reinterpret_cast<unsigned long long*>(m.s_m + kFastMax);
+  m.s_kp = reinterpret_cast<int32_t*>(m.hist + kHistBins);
+  m.s_bits = reinterpret_cast<uint32_t*>(m.s_kp + kSelectKpCache);
+  return m;
+}
+
+__device__ void select_level(const Geom& G, const SelectArgs& a, const SelectSmem& sm) {
   __shared__ float s_f[33];
   __shared__ unsigned long long s_u[33];
   __shared__ uint32_t s_w[33];
   __shared__ uint32_t s_bucket;
   __shared__ unsigned long long s_before;
-  pdl_trigger();
-  pdl_wait();
-  forward_tree_status(a);
 
   const int bh = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
   const int C = G.chunk;
-  uint32_t* bits = a.kept_here + int64_t(bh) * a.words_here;
+  // This level's kept bitmap: built in shared memory when it fits (written out
+  // once at the end), else cleared and set in place in global memory.
+  uint32_t* gbits = a.kept_here + int64_t(bh) * a.words_here;
+  const bool bits_in_smem = a.words_here <= kBitsSmem;
+  uint32_t* bits = bits_in_smem ? sm.s_bits : gbits;
   for (int64_t w = tid; w < a.words_here; w += blockDim.x) bits[w] = 0u;
 
   // Kept parents of this head, ascending (compaction of the level-(l+1) bitmap).
   // Parents fit in shared memory unless the level above is very wide.
   const bool kp_in_smem = a.words_up <= kSelectKpCache / 32;
-  int32_t* kp = kp_in_smem ? s_kp : a.kp + int64_t(bh) * a.kp_stride;
+  int32_t* kp = kp_in_smem ? sm.s_kp : a.kp + int64_t(bh) * a.kp_stride;
   uint32_t n_kp = 0;
   if (a.kept_up != nullptr && a.words_up > 0) {
     const uint32_t* up = a.kept_up + int64_t(bh) * a.words_up;
@@ -335,14 +515,13 @@ select_kernel(Geom G, SelectArgs a) {
       n_kp += tot;
     }
   }
-  __syncthreads();   // kp visible to the block
+  __syncthreads();   // kp and the cleared bitmap visible to the block
 
   const int64_t orphan0 = int64_t(C) * a.n_par;
-  const int64_t n_child = int64_t(n_kp) * C;
-  const int64_t n_c = n_child + (a.n_nodes - orphan0);
+  const int64_t n_c64 = int64_t(n_kp) * C + (a.n_nodes - orphan0);
   // Candidate i -> node: child (i % C) of kept parent i / C, or an orphan.
   // Candidate and node indices fit 32 bits; the division is 32-bit.
-  const uint32_t uC = uint32_t(C), u_nchild = uint32_t(n_child);
+  const uint32_t uC = uint32_t(C), u_nchild = n_kp * uC;
   auto node_of = [&](int64_t i) -> int64_t {
     const uint32_t ui = uint32_t(i);
     if (ui < u_nchild) {
@@ -352,151 +531,178 @@ select_kernel(Geom G, SelectArgs a) {
     return orphan0 + (ui - u_nchild);
   };
   const float* sig = a.sigma + int64_t(bh) * a.n_nodes;
-  const bool cached = n_c <= kSelectCache;
-  if (cached) {
-    // Eight independent loads in flight per thread.
-    for (int64_t i0 = tid; i0 < n_c; i0 += 8 * int64_t(blockDim.x)) {
+  uint32_t kept_total = 0;
+
+  if (n_c64 <= kFastMax) {
+    // ---------------- all candidates in shared memory ----------------
+    const int n_c = int(n_c64);
+    uint32_t* s_key = sm.s_key;
+    uint32_t* s_m = sm.s_m;
+    float* s_sig = reinterpret_cast<float*>(s_key);
+    for (int i0 = tid; i0 < n_c; i0 += 8 * kSelectThreads) {      // eight loads in flight
       float v[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int64_t i = i0 + int64_t(u) * blockDim.x;
+        const int i = i0 + u * kSelectThreads;
         v[u] = i < n_c ? sig[node_of(i)] : 0.f;
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int64_t i = i0 + int64_t(u) * blockDim.x;
+        const int i = i0 + u * kSelectThreads;
         if (i < n_c) s_sig[i] = v[u];
       }
     }
-  }
-  __syncthreads();
-  auto sigma_of = [&](int64_t i) -> float { return cached ? s_sig[i] : sig[node_of(i)]; };
+    __syncthreads();
 
-  // Softmax statistics over the candidates.
-  float mx = -INFINITY;
-  for (int64_t i = tid; i < n_c; i += blockDim.x) mx = fmaxf(mx, sigma_of(i));
-  mx = block_max(mx, s_f);
-  float z = 0.f;
-  for (int64_t i = tid; i < n_c; i += blockDim.x) z += expf(sigma_of(i) - mx);
-  z = block_sum(z, s_f);
-  const float inv_z = 1.f / z;
-  auto mass_of = [&](float s) -> unsigned long long {
-    return __float2ull_rn(expf(s - mx) * inv_z * float(kMassScale));
-  };
-
-  // Cut: smallest key (score desc, index asc) whose cumulative mass reaches p.
-  bool keep_all = a.keep_all != 0 || n_c == 0;
-  uint32_t key_cut = 0xffffffffu;
-  unsigned long long t_keep = 0;
-  if (!keep_all) {
+    // Softmax statistics, then keys and masses in 2^-31 fixed point (the same
+    // arithmetic for every use of a candidate's mass; one candidate holds at
+    // most 2^31, all of them together less than 2^32).
+    float mx = -INFINITY;
+    for (int i = tid; i < n_c; i += kSelectThreads) mx = fmaxf(mx, s_sig[i]);
+    mx = block_max(mx, s_f);
+    float z = 0.f;
+    for (int i = tid; i < n_c; i += kSelectThreads) z += expf(s_sig[i] - mx);
+    z = block_sum(z, s_f);
+    const float scale31 = 2147483648.f / z;
+    auto mass_of = [&](float s) -> uint32_t {
+      return a.topk ? 1u : __float2uint_rn(expf(s - mx) * scale31);
+    };
     unsigned long long tm = 0;
-    for (int64_t i = tid; i < n_c; i += blockDim.x) tm += mass_of(sigma_of(i));
+    uint32_t k_hi = 0u;
+    for (int i = tid; i < n_c; i += kSelectThreads) {
+      const float s = s_sig[i];
+      const uint32_t m = mass_of(s);
+      const uint32_t key = ~float_order_key(s);
+      s_m[i] = m;
+      s_key[i] = key;
+      k_hi = max(k_hi, key);
+      tm += m;
+    }
+    k_hi = __reduce_max_sync(0xffffffffu, k_hi);
+    if (lane == 0) s_w[warp] = k_hi;
     unsigned long long total;
-    block_excl_scan<unsigned long long>(tm, s_u, &total);
-    if (total < a.p_fixed) keep_all = true;
-  }
-  if (!keep_all) {
-    uint32_t prefix = 0, pmask = 0;
-    unsigned long long before = 0;
-    unsigned long long* wh = hist + warp * 256;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int k = lane; k < 256; k += 32) wh[k] = 0ull;
-      __syncthreads();
-      // Runs of equal buckets are summed in a register and flushed once: the
-      // leading digits of nearby scores coincide, and per-element atomics on
-      // one bucket would serialise the whole warp.
-      uint32_t cb = 0xffffffffu;
-      unsigned long long cs = 0ull;
-      for (int64_t i = tid; i < n_c; i += blockDim.x) {
-        const float s = sigma_of(i);
-        const uint32_t key = ~float_order_key(s);
-        if ((key & pmask) == prefix) {
-          const uint32_t b = (key >> shift) & 255u;
-          const unsigned long long mm = mass_of(s);
-          if (b == cb) {
-            cs += mm;
-          } else {
-            if (cs != 0ull) atomicAdd(&wh[cb], cs);
-            cb = b;
-            cs = mm;
+    block_excl_scan<unsigned long long>(tm, s_u, &total);      // its barriers publish s_key / s_m / s_w
+    for (int w = 0; w < nw; ++w) k_hi = max(k_hi, s_w[w]);
+    const uint32_t k_lo = ~float_order_key(mx);                 // the highest score has the lowest key
+    const unsigned long long p31 = a.p_fixed31;
+    const bool keep_all = a.keep_all != 0 || n_c == 0 || total < p31;
+    __syncthreads();                                            // s_w is reused below
+
+    // Kept predicate over candidate i, filled in below: key < lo keeps; a key
+    // inside the cut window [lo, lo + 2^span) keeps by its flag, or (span 0:
+    // one key, all tied) by its tie rank.
+    uint32_t lo = 0u;
+    int span = 0;
+    unsigned long long before = 0ull, t_keep = 0ull;
+    uint32_t* hm = reinterpret_cast<uint32_t*>(sm.hist);        // [kCutBins] mass per bin
+    uint32_t* hc = hm + kCutBins;                               // [kCutBins] candidates per bin
+    int32_t* win = reinterpret_cast<int32_t*>(hc + kCutBins);   // [kFastSmallN] window members
+    uint32_t* flag = reinterpret_cast<uint32_t*>(win + kFastSmallN);   // [kFastMax / 32]
+    if (!keep_all) {
+      lo = k_lo;
+      const uint32_t range = k_hi - k_lo;
+      span = range == 0u ? 0 : 32 - __clz(range);
+      uint32_t n_win = uint32_t(n_c);
+      // Narrow the window to the splitter bin that holds the cut until it holds
+      // few candidates (or one key). Every pass keeps before < p <= before +
+      // (mass in the window).
+      while (n_win > uint32_t(kFastSmallN) && span > 0) {
+        const int shift = span > 11 ? span - 11 : 0;
+        for (int b = tid; b < kCutBins; b += kSelectThreads) { hm[b] = 0u; hc[b] = 0u; }
+        __syncthreads();
+        for (int i = tid; i < n_c; i += kSelectThreads) {
+          const uint32_t d = s_key[i] - lo;
+          if (span == 32 || (d >> span) == 0u) {
+            const uint32_t b = d >> shift;
+            atomicAdd(&hm[b], s_m[i]);
+            atomicAdd(&hc[b], 1u);
           }
         }
-      }
-      if (cs != 0ull) atomicAdd(&wh[cb], cs);
-      __syncthreads();
-      // bucket totals into warp 0's histogram
-      for (int k = tid; k < 256; k += blockDim.x) {
-        unsigned long long v = 0;
-        for (int w = 0; w < nw; ++w) v += hist[w * 256 + k];
-        hist[k] = v;
-      }
-      __syncthreads();
-      if (warp == 0) {
-        // lane owns buckets [8*lane, 8*lane+8)
-        unsigned long long loc[8], run = 0;
-        for (int k = 0; k < 8; ++k) { loc[k] = hist[8 * lane + k]; run += loc[k]; }
-        unsigned long long incl = warp_incl_scan<unsigned long long>(run);
-        unsigned long long excl = incl - run;
-        // first bucket whose inclusive cumulative mass reaches p
-        int found = -1;
-        unsigned long long acc = before + excl, acc_before = 0;
-        for (int k = 0; k < 8; ++k) {
-          if (found < 0 && acc + loc[k] >= a.p_fixed) { found = 8 * lane + k; acc_before = acc; }
-          acc += loc[k];
+        __syncthreads();
+        // first bin whose cumulative mass (with `before`) reaches p: thread t
+        // owns bins [4t, 4t + 4)
+        unsigned long long loc = 0ull;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) loc += hm[4 * tid + j];
+        unsigned long long tot_bins;
+        unsigned long long acc = before + block_excl_scan<unsigned long long>(loc, s_u, &tot_bins);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t mj = hm[4 * tid + j];
+          if (acc < p31 && acc + mj >= p31) {
+            s_bucket = uint32_t(4 * tid + j);
+            s_before = acc;
+            s_w[32] = hc[4 * tid + j];
+          }
+          acc += mj;
         }
-        const unsigned ball = __ballot_sync(0xffffffffu, found >= 0);
-        const int src = ball ? __ffs(ball) - 1 : 31;
-        const int fb = __shfl_sync(0xffffffffu, found, src);
-        const unsigned long long ab = __shfl_sync(0xffffffffu, acc_before, src);
-        if (lane == 0) {
-          s_bucket = fb < 0 ? 255u : uint32_t(fb);
-          s_before = fb < 0 ? before : ab;
-        }
+        __syncthreads();
+        lo += s_bucket << shift;
+        before = s_before;
+        n_win = s_w[32];
+        span = shift;
+        __syncthreads();                                        // s_bucket / s_before / s_w reused
       }
-      __syncthreads();
-      prefix |= s_bucket << shift;
-      pmask |= 255u << shift;
-      before = s_before;
-      __syncthreads();
+      if (span == 0) {
+        // One key in the window: the cut falls among tied candidates, taken in
+        // candidate order.
+        const uint32_t m_cut = mass_of(order_key_float(~lo));
+        const unsigned long long need = p31 > before ? p31 - before : 0ull;
+        t_keep = m_cut > 0u ? (need + m_cut - 1ull) / m_cut : 0ull;
+      } else {
+        // Few candidates in the window: each one counts the mass ordered before
+        // it (key, then candidate index) among them.
+        if (tid == 0) s_w[32] = 0u;
+        for (int w = tid; w < (n_c + 31) / 32; w += kSelectThreads) flag[w] = 0u;
+        __syncthreads();
+        for (int i = tid; i < n_c; i += kSelectThreads) {
+          const uint32_t d = s_key[i] - lo;
+          if (span == 32 || (d >> span) == 0u) win[atomicAdd(&s_w[32], 1u)] = i;
+        }
+        __syncthreads();
+        const int nwin = int(s_w[32]);
+        if (tid < nwin) {
+          const int i = win[tid];
+          const uint32_t ki = s_key[i];
+          unsigned long long cb = before;
+          for (int j = 0; j < nwin; ++j) {
+            const int ij = win[j];
+            const uint32_t kj = s_key[ij];
+            if (kj < ki || (kj == ki && ij < i)) cb += s_m[ij];
+          }
+          if (cb < p31) atomicOr(&flag[i >> 5], 1u << (i & 31));
+        }
+        __syncthreads();
+      }
     }
-    key_cut = prefix;
-    const unsigned long long pi_cut = mass_of(order_key_float(~key_cut));
-    const unsigned long long need = a.p_fixed > before ? a.p_fixed - before : 0ull;
-    t_keep = pi_cut > 0 ? (need + pi_cut - 1) / pi_cut : 0ull;
-  }
 
-  // Keep flags in candidate order (ascending node index): thread-contiguous
-  // ranges so that ties at the cut are taken lowest index first.
-  const int64_t per = (n_c + blockDim.x - 1) / blockDim.x;
-  const int64_t i_lo = min64(n_c, per * tid), i_hi = min64(n_c, i_lo + per);
-  uint32_t my_ties = 0;
-  if (!keep_all)
-    for (int64_t i = i_lo; i < i_hi; ++i) my_ties += (~float_order_key(sigma_of(i)) == key_cut);
-  uint32_t tie_total;
-  uint32_t tie_rank = block_excl_scan<uint32_t>(my_ties, s_w, &tie_total);
-  uint32_t my_kept = 0;
-  {
-    uint32_t tr = tie_rank;
-    for (int64_t i = i_lo; i < i_hi; ++i) {
-      bool k = keep_all;
-      if (!k) {
-        const uint32_t key = ~float_order_key(sigma_of(i));
-        k = key < key_cut || (key == key_cut && tr++ < t_keep);
-      }
-      my_kept += k;
+    // Kept candidates in candidate order (ascending node index): thread-
+    // contiguous ranges, positions by a scan.
+    const int per = (n_c + kSelectThreads - 1) / kSelectThreads;
+    const int i_lo = min(n_c, per * tid), i_hi = min(n_c, i_lo + per);
+    uint32_t tie_rank = 0;
+    if (!keep_all && span == 0) {
+      uint32_t my_ties = 0, tie_total;
+      for (int i = i_lo; i < i_hi; ++i) my_ties += (s_key[i] == lo);
+      tie_rank = block_excl_scan<uint32_t>(my_ties, s_w, &tie_total);
     }
-  }
-  uint32_t kept_total;
-  uint32_t pos = block_excl_scan<uint32_t>(my_kept, s_w, &kept_total);
-  {
-    uint32_t tr = tie_rank;
-    for (int64_t i = i_lo; i < i_hi; ++i) {
-      bool k = keep_all;
-      if (!k) {
-        const uint32_t key = ~float_order_key(sigma_of(i));
-        k = key < key_cut || (key == key_cut && tr++ < t_keep);
-      }
-      if (k) {
+    auto kept = [&](int i, uint32_t& tr) -> bool {
+      if (keep_all) return true;
+      const uint32_t key = s_key[i];
+      if (key < lo) return true;
+      if (span == 0) return key == lo && tr++ < t_keep;
+      return (flag[i >> 5] >> (i & 31)) & 1u;
+    };
+    uint32_t my_kept = 0;
+    {
+      uint32_t tr = tie_rank;
+      for (int i = i_lo; i < i_hi; ++i) my_kept += kept(i, tr) ? 1u : 0u;
+    }
+    uint32_t pos = block_excl_scan<uint32_t>(my_kept, s_w, &kept_total);
+    {
+      uint32_t tr = tie_rank;
+      for (int i = i_lo; i < i_hi; ++i) {
+        if (!kept(i, tr)) continue;
         const int64_t node = node_of(i);
         atomicOr(&bits[node >> 5], 1u << (node & 31));
         if (a.chunk_ids != nullptr && pos < uint32_t(a.max_sel))
@@ -504,268 +710,153 @@ select_kernel(Geom G, SelectArgs a) {
         ++pos;
       }
     }
-  }
-  if (a.chunk_ids != nullptr && tid == 0) {
-    a.n_chunks[bh] = int32_t(kept_total);
-    if (kept_total > uint32_t(a.max_sel) && a.status != nullptr)
-      atomicOr(a.status, ZHA_DEV_SELECTION_TRUNCATED);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Selection for one query head at one level, all candidates in shared memory
-// (n_nodes <= kFastMax). Each candidate's order key (score descending, then
-// index ascending) and its softmax mass in 2^-32 fixed point are computed once.
-//  * up to kFastSmallN candidates: thread i counts the mass of every candidate
-//    ordered before it; i is kept iff that mass is below p (the minimal prefix
-//    holding mass p). No radix passes, a handful of barriers.
-//  * more: the cut key by a radix select over 8-bit digits with per-warp
-//    histograms of mass, starting at the first byte in which the candidates'
-//    keys differ; runs of equal buckets are summed in registers before the
-//    atomic add.
-// The rounding of the fixed-point masses adds at most n 2^-33 to any
-// cumulative mass (< 2e-6 at n = 16384).
-// ---------------------------------------------------------------------------
-constexpr int kFastMax = 16384;
-constexpr int kFastSmallN = kSelectThreads;
-constexpr int kHistBins = (kSelectThreads / 32) * 256;   // per-warp 256-bin histograms
-
-__global__ void __launch_bounds__(kSelectThreads)
-select_fast_kernel(Geom G, SelectArgs a) {
-  extern __shared__ float4 smem_v4[];
-  uint32_t* s_key = reinterpret_cast<uint32_t*>(smem_v4);                    // scores, then keys
-  uint32_t* s_m = s_key + kFastMax;                                           // masses
-  unsigned long long* hist = reinterpret_cast<unsigned long long*>(s_m + kFastMax);   // [kHistBins]
-  int32_t* s_kp = reinterpret_cast<int32_t*>(hist + kHistBins);               // [kSelectKpCache]
-  float* s_sig = reinterpret_cast<float*>(s_key);
-  __shared__ float s_f[33];
-  __shared__ unsigned long long s_u[33];
-  __shared__ uint32_t s_w[33];
-  __shared__ uint32_t s_bucket;
-  __shared__ unsigned long long s_before;
-  pdl_trigger();
-  pdl_wait();
-  forward_tree_status(a);
-
-  const int bh = blockIdx.x;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int C = G.chunk;
-  uint32_t* bits = a.kept_here + int64_t(bh) * a.words_here;
-  for (int64_t w = tid; w < a.words_here; w += blockDim.x) bits[w] = 0u;
-
-  // Kept parents of this head, ascending.
-  const bool kp_in_smem = a.words_up <= kSelectKpCache / 32;
-  int32_t* kp = kp_in_smem ? s_kp : a.kp + int64_t(bh) * a.kp_stride;
-  uint32_t n_kp = 0;
-  if (a.kept_up != nullptr && a.words_up > 0) {
-    const uint32_t* up = a.kept_up + int64_t(bh) * a.words_up;
-    for (int64_t w0 = 0; w0 < a.words_up; w0 += blockDim.x) {
-      const int64_t w = w0 + tid;
-      const uint32_t word = w < a.words_up ? up[w] : 0u;
-      uint32_t tot;
-      uint32_t pos = n_kp + block_excl_scan<uint32_t>(__popc(word), s_w, &tot);
-      uint32_t x = word;
-      while (x) {
-        const int bit = __ffs(x) - 1;
-        x &= x - 1u;
-        kp[pos++] = int32_t(w * 32 + bit);
-      }
-      n_kp += tot;
-    }
-  }
-  __syncthreads();
-
-  const int64_t orphan0 = int64_t(C) * a.n_par;
-  const uint32_t uC = uint32_t(C), n_child = n_kp * uC;
-  const int n_c = int(n_child + uint32_t(a.n_nodes - orphan0));
-  auto node_of = [&](int i) -> int64_t {
-    const uint32_t ui = uint32_t(i);
-    if (ui < n_child) {
-      const uint32_t par = ui / uC;
-      return int64_t(kp[par]) * C + (ui - par * uC);
-    }
-    return orphan0 + (ui - n_child);
-  };
-  const float* sig = a.sigma + int64_t(bh) * a.n_nodes;
-  for (int i0 = tid; i0 < n_c; i0 += 8 * kSelectThreads) {      // eight loads in flight
-    float v[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * kSelectThreads;
-      v[u] = i < n_c ? sig[node_of(i)] : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * kSelectThreads;
-      if (i < n_c) s_sig[i] = v[u];
-    }
-  }
-  __syncthreads();
-
-  // Softmax statistics, then keys and fixed-point masses (same arithmetic for
-  // every use of a candidate's mass).
-  float mx = -INFINITY;
-  for (int i = tid; i < n_c; i += kSelectThreads) mx = fmaxf(mx, s_sig[i]);
-  mx = block_max(mx, s_f);
-  float z = 0.f;
-  for (int i = tid; i < n_c; i += kSelectThreads) z += expf(s_sig[i] - mx);
-  z = block_sum(z, s_f);
-  const float scale32 = 4294967296.f / z;
-  auto mass_of = [&](float s) -> uint32_t { return __float2uint_rn(expf(s - mx) * scale32); };
-  unsigned long long tm = 0;
-  for (int i = tid; i < n_c; i += kSelectThreads) {
-    const float s = s_sig[i];
-    const uint32_t m = mass_of(s);
-    s_m[i] = m;
-    s_key[i] = ~float_order_key(s);
-    tm += m;
-  }
-  unsigned long long total;
-  block_excl_scan<unsigned long long>(tm, s_u, &total);      // its barriers publish s_key / s_m
-  const unsigned long long p32 = a.p_fixed32;
-  const bool keep_all = a.keep_all != 0 || n_c == 0 || total < p32;
-
-  uint32_t kept_total = 0;
-  auto emit = [&](int i, uint32_t pos) {
-    const int64_t node = node_of(i);
-    atomicOr(&bits[node >> 5], 1u << (node & 31));
-    if (a.chunk_ids != nullptr && pos < uint32_t(a.max_sel))
-      a.chunk_ids[int64_t(bh) * a.max_sel + pos] = int32_t(node);
-  };
-  if (keep_all || n_c <= kFastSmallN) {
-    // Thread i = candidate i (candidate order = ascending node index).
-    bool k = false;
-    if (tid < n_c) {
-      if (keep_all) {
-        k = true;
-      } else {
-        const uint32_t ki = s_key[tid];
-        unsigned long long cb = 0ull;
-        for (int j = 0; j < n_c; ++j) {
-          const uint32_t kj = s_key[j];
-          if (kj < ki || (kj == ki && j < tid)) cb += s_m[j];
-        }
-        k = cb < p32;
-      }
-    }
-    if (keep_all && n_c > kSelectThreads) {
-      // keep everything: thread-contiguous ranges, positions by a scan
-      const int per = (n_c + kSelectThreads - 1) / kSelectThreads;
-      const int i_lo = min(n_c, per * tid), i_hi = min(n_c, i_lo + per);
-      uint32_t pos = block_excl_scan<uint32_t>(uint32_t(i_hi - i_lo), s_w, &kept_total);
-      for (int i = i_lo; i < i_hi; ++i) emit(i, pos++);
-    } else {
-      const uint32_t pos = block_excl_scan<uint32_t>(k ? 1u : 0u, s_w, &kept_total);
-      if (k) emit(tid, pos);
-    }
   } else {
-    // Leading bytes shared by every candidate's key are fixed up front.
-    uint32_t k_and = 0xffffffffu, k_or = 0u;
-    for (int i = tid; i < n_c; i += kSelectThreads) { k_and &= s_key[i]; k_or |= s_key[i]; }
+    // ---------------- generic path: more candidates than kFastMax ----------------
+    const int64_t n_c = n_c64;
+    float* s_sig = reinterpret_cast<float*>(sm.s_key);
+    const bool cached = n_c <= kSelectCache;
+    if (cached) {
+      for (int64_t i0 = tid; i0 < n_c; i0 += 8 * int64_t(blockDim.x)) {
+        float v[8];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      k_and &= __shfl_xor_sync(0xffffffffu, k_and, o);
-      k_or |= __shfl_xor_sync(0xffffffffu, k_or, o);
+        for (int u = 0; u < 8; ++u) {
+          const int64_t i = i0 + int64_t(u) * blockDim.x;
+          v[u] = i < n_c ? sig[node_of(i)] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int64_t i = i0 + int64_t(u) * blockDim.x;
+          if (i < n_c) s_sig[i] = v[u];
+        }
+      }
     }
-    if (lane == 0) { s_w[warp] = k_and; s_w[16 + warp] = k_or; }
     __syncthreads();
-    if (tid == 0) {
-      uint32_t x = 0xffffffffu, y = 0u;
-      for (int w = 0; w < kSelectThreads / 32; ++w) { x &= s_w[w]; y |= s_w[16 + w]; }
-      s_w[32] = x;
-      s_bucket = y;
+    auto sigma_of = [&](int64_t i) -> float { return cached ? s_sig[i] : sig[node_of(i)]; };
+
+    float mx = -INFINITY;
+    for (int64_t i = tid; i < n_c; i += blockDim.x) mx = fmaxf(mx, sigma_of(i));
+    mx = block_max(mx, s_f);
+    float z = 0.f;
+    for (int64_t i = tid; i < n_c; i += blockDim.x) z += expf(sigma_of(i) - mx);
+    z = block_sum(z, s_f);
+    const float inv_z = 1.f / z;
+    auto mass_of = [&](float s) -> unsigned long long {
+      return a.topk ? 1ull : __float2ull_rn(expf(s - mx) * inv_z * float(kMassScale));
+    };
+
+    // Cut: smallest key (score desc, index asc) whose cumulative mass reaches p.
+    bool keep_all = a.keep_all != 0;
+    uint32_t key_cut = 0xffffffffu;
+    unsigned long long t_keep = 0;
+    if (!keep_all) {
+      unsigned long long tm = 0;
+      for (int64_t i = tid; i < n_c; i += blockDim.x) tm += mass_of(sigma_of(i));
+      unsigned long long total;
+      block_excl_scan<unsigned long long>(tm, s_u, &total);
+      if (total < a.p_fixed) keep_all = true;
     }
-    __syncthreads();
-    k_and = s_w[32];
-    k_or = s_bucket;
-    const int lead = (k_and ^ k_or) == 0u ? 32 : __clz(k_and ^ k_or);   // common leading bits
-    const int first_byte = min(lead / 8, 3);
-    uint32_t pmask = first_byte == 0 ? 0u : ~0u << (32 - 8 * first_byte);
-    uint32_t prefix = k_and & pmask;
-    unsigned long long before = 0ull;
-    unsigned long long* wh = hist + warp * 256;
-#pragma unroll 1
-    for (int shift = 24 - 8 * first_byte; shift >= 0; shift -= 8) {
-      for (int k = lane; k < 256; k += 32) wh[k] = 0ull;
-      __syncthreads();
-      uint32_t cb = 0xffffffffu;
-      unsigned long long cs = 0ull;
-      for (int i = tid; i < n_c; i += kSelectThreads) {
-        const uint32_t key = s_key[i];
-        if ((key & pmask) == prefix) {
-          const uint32_t bkt = (key >> shift) & 255u;
-          if (bkt == cb) {
-            cs += s_m[i];
-          } else {
-            if (cs != 0ull) atomicAdd(&wh[cb], cs);
-            cb = bkt;
-            cs = s_m[i];
+    if (!keep_all) {
+      uint32_t prefix = 0, pmask = 0;
+      unsigned long long before = 0;
+      unsigned long long* hist = sm.hist;
+      unsigned long long* wh = hist + warp * 256;
+      for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int k = lane; k < 256; k += 32) wh[k] = 0ull;
+        __syncthreads();
+        uint32_t cb = 0xffffffffu;
+        unsigned long long cs = 0ull;
+        for (int64_t i = tid; i < n_c; i += blockDim.x) {
+          const float s = sigma_of(i);
+          const uint32_t key = ~float_order_key(s);
+          if ((key & pmask) == prefix) {
+            const uint32_t b = (key >> shift) & 255u;
+            const unsigned long long mm = mass_of(s);
+            if (b == cb) {
+              cs += mm;
+            } else {
+              if (cs != 0ull) atomicAdd(&wh[cb], cs);
+              cb = b;
+              cs = mm;
+            }
           }
         }
-      }
-      if (cs != 0ull) atomicAdd(&wh[cb], cs);
-      __syncthreads();
-      for (int k = tid; k < 256; k += kSelectThreads) {     // bucket totals into warp 0's histogram
-        unsigned long long v = 0ull;
-        for (int w = 0; w < kSelectThreads / 32; ++w) v += hist[w * 256 + k];
-        hist[k] = v;
-      }
-      __syncthreads();
-      if (warp == 0) {
-        // lane owns buckets [8 lane, 8 lane + 8): first bucket whose cumulative
-        // mass (with `before`) reaches p
-        unsigned long long loc[8], run = 0ull;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) { loc[k] = hist[8 * lane + k]; run += loc[k]; }
-        const unsigned long long incl = warp_incl_scan<unsigned long long>(run);
-        unsigned long long acc = before + incl - run, acc_before = 0ull;
-        int found = -1;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (found < 0 && acc + loc[k] >= p32) { found = 8 * lane + k; acc_before = acc; }
-          acc += loc[k];
+        if (cs != 0ull) atomicAdd(&wh[cb], cs);
+        __syncthreads();
+        for (int k = tid; k < 256; k += blockDim.x) {
+          unsigned long long v = 0;
+          for (int w = 0; w < nw; ++w) v += hist[w * 256 + k];
+          hist[k] = v;
         }
-        const unsigned ball = __ballot_sync(0xffffffffu, found >= 0);
-        const int src = ball ? __ffs(ball) - 1 : 31;
-        const int fb = __shfl_sync(0xffffffffu, found, src);
-        const unsigned long long ab = __shfl_sync(0xffffffffu, acc_before, src);
-        if (lane == 0) {
-          s_bucket = fb < 0 ? 255u : uint32_t(fb);
-          s_before = fb < 0 ? before : ab;
+        __syncthreads();
+        if (warp == 0) {
+          unsigned long long loc[8], run = 0;
+          for (int k = 0; k < 8; ++k) { loc[k] = hist[8 * lane + k]; run += loc[k]; }
+          unsigned long long incl = warp_incl_scan<unsigned long long>(run);
+          unsigned long long excl = incl - run;
+          int found = -1;
+          unsigned long long acc = before + excl, acc_before = 0;
+          for (int k = 0; k < 8; ++k) {
+            if (found < 0 && acc + loc[k] >= a.p_fixed) { found = 8 * lane + k; acc_before = acc; }
+            acc += loc[k];
+          }
+          const unsigned ball = __ballot_sync(0xffffffffu, found >= 0);
+          const int src = ball ? __ffs(ball) - 1 : 31;
+          const int fb = __shfl_sync(0xffffffffu, found, src);
+          const unsigned long long ab = __shfl_sync(0xffffffffu, acc_before, src);
+          if (lane == 0) {
+            s_bucket = fb < 0 ? 255u : uint32_t(fb);
+            s_before = fb < 0 ? before : ab;
+          }
         }
+        __syncthreads();
+        prefix |= s_bucket << shift;
+        pmask |= 255u << shift;
+        before = s_before;
+        __syncthreads();
       }
-      __syncthreads();
-      prefix |= s_bucket << shift;
-      pmask |= 255u << shift;
-      before = s_before;
-      __syncthreads();                                      // s_bucket / s_before are reused
+      key_cut = prefix;
+      const unsigned long long pi_cut = mass_of(order_key_float(~key_cut));
+      const unsigned long long need = a.p_fixed > before ? a.p_fixed - before : 0ull;
+      t_keep = pi_cut > 0 ? (need + pi_cut - 1) / pi_cut : 0ull;
     }
-    const uint32_t key_cut = prefix;
-    const uint32_t m_cut = mass_of(order_key_float(~key_cut));
-    const unsigned long long need = p32 > before ? p32 - before : 0ull;
-    const unsigned long long t_keep = m_cut > 0u ? (need + m_cut - 1ull) / m_cut : 0ull;
-    // Kept flags in candidate order: thread-contiguous ranges so that ties at
-    // the cut are taken lowest index first.
-    const int per = (n_c + kSelectThreads - 1) / kSelectThreads;
-    const int i_lo = min(n_c, per * tid), i_hi = min(n_c, i_lo + per);
+
+    // Keep flags in candidate order (ascending node index): thread-contiguous
+    // ranges so that ties at the cut are taken lowest index first.
+    const int64_t per = (n_c + blockDim.x - 1) / blockDim.x;
+    const int64_t i_lo = min64(n_c, per * tid), i_hi = min64(n_c, i_lo + per);
     uint32_t my_ties = 0;
-    for (int i = i_lo; i < i_hi; ++i) my_ties += (s_key[i] == key_cut);
+    if (!keep_all)
+      for (int64_t i = i_lo; i < i_hi; ++i) my_ties += (~float_order_key(sigma_of(i)) == key_cut);
     uint32_t tie_total;
-    const uint32_t tie_rank = block_excl_scan<uint32_t>(my_ties, s_w, &tie_total);
+    uint32_t tie_rank = block_excl_scan<uint32_t>(my_ties, s_w, &tie_total);
     uint32_t my_kept = 0;
     {
       uint32_t tr = tie_rank;
-      for (int i = i_lo; i < i_hi; ++i) {
-        const uint32_t key = s_key[i];
-        my_kept += (key < key_cut || (key == key_cut && tr++ < t_keep)) ? 1u : 0u;
+      for (int64_t i = i_lo; i < i_hi; ++i) {
+        bool k = keep_all;
+        if (!k) {
+          const uint32_t key = ~float_order_key(sigma_of(i));
+          k = key < key_cut || (key == key_cut && tr++ < t_keep);
+        }
+        my_kept += k;
       }
     }
     uint32_t pos = block_excl_scan<uint32_t>(my_kept, s_w, &kept_total);
     {
       uint32_t tr = tie_rank;
-      for (int i = i_lo; i < i_hi; ++i) {
-        const uint32_t key = s_key[i];
-        if (key < key_cut || (key == key_cut && tr++ < t_keep)) emit(i, pos++);
+      for (int64_t i = i_lo; i < i_hi; ++i) {
+        bool k = keep_all;
+        if (!k) {
+          const uint32_t key = ~float_order_key(sigma_of(i));
+          k = key < key_cut || (key == key_cut && tr++ < t_keep);
+        }
+        if (k) {
+          const int64_t node = node_of(i);
+          atomicOr(&bits[node >> 5], 1u << (node & 31));
+          if (a.chunk_ids != nullptr && pos < uint32_t(a.max_sel))
+            a.chunk_ids[int64_t(bh) * a.max_sel + pos] = int32_t(node);
+          ++pos;
+        }
       }
     }
   }
@@ -774,11 +865,39 @@ select_fast_kernel(Geom G, SelectArgs a) {
     if (kept_total > uint32_t(a.max_sel) && a.status != nullptr)
       atomicOr(a.status, ZHA_DEV_SELECTION_TRUNCATED);
   }
+  if (bits_in_smem) {
+    __syncthreads();
+    for (int64_t w = tid; w < a.words_here; w += blockDim.x) gbits[w] = sm.s_bits[w];
+  }
 }
 
-size_t select_fast_smem_bytes() {
-  return size_t(2 * kFastMax) * sizeof(uint32_t) + size_t(kHistBins) * sizeof(unsigned long long) +
-         size_t(kSelectKpCache) * sizeof(int32_t);
+// One level, one CTA per query head.
+__global__ void __launch_bounds__(kSelectThreads)
+select_fast_kernel(Geom G, SelectArgs a) {
+  pdl_trigger();
+  pdl_wait();
+  forward_tree_status(a);
+  select_level(G, a, select_smem());
+}
+
+// Levels top..bottom of a block of consecutive levels in one launch (the small
+// top levels scored densely): each level's kept bitmap, written by this CTA,
+// gives the next level's candidates after a CTA barrier.
+struct SelectLevels {
+  int32_t count;
+  SelectArgs lv[ZHA_MAX_LEVELS];
+};
+
+__global__ void __launch_bounds__(kSelectThreads)
+select_top_kernel(Geom G, SelectLevels t) {
+  pdl_trigger();
+  pdl_wait();
+  forward_tree_status(t.lv[0]);
+  const SelectSmem sm = select_smem();
+  for (int i = 0; i < t.count; ++i) {
+    select_level(G, t.lv[i], sm);
+    __syncthreads();                 // this level's bitmap before the next level reads it
+  }
 }
 
 cudaError_t launch_score_tc(const Geom& G, int level, int64_t n_nodes, int64_t n_par, int32_t batch,
@@ -790,22 +909,40 @@ cudaError_t launch_score_tma(const Geom& G, int level, int64_t n_nodes, int64_t 
                              const float* store, int32_t* status, cudaStream_t s, bool* used);
 
 // ---------------------------------------------------------------------------
-// Host launcher: levels L..1, score then select.
+// Host launcher. Levels L..1. The small top levels (at most kDenseMaxNodes
+// nodes per KV head each, kDenseMaxTotal nodes over all KV heads together) are
+// scored densely in one launch and selected in one launch; every lower level is
+// scored over its candidates (score_tma_kernel, score_tc_kernel or
+// score_kernel) and then selected.
 // ---------------------------------------------------------------------------
+constexpr int64_t kDenseMaxNodes = 1024;
+constexpr int64_t kDenseMaxTotal = 8192;
+
+template <int D, int RP>
+static size_t score_smem_bytes(const Geom& G, int32_t batch) {
+  using S = ScoreShape<D, RP>;
+  const int qn = batch * G.group;
+  return (size_t(kScoreThreads / 32) * S::KBUF +
+          size_t(qn < kScoreQBlock ? qn : kScoreQBlock) * S::QROW) * 4;
+}
+
+// Nodes per CTA: enough CTAs to fill the GPU twice over, at most kScoreTile.
+static int score_tile_for(int64_t n_nodes, int hkv) {
+  int tile = kScoreTile;
+  while (tile > kScoreThreads / 32 && (n_nodes * hkv) / tile < 2 * 148) tile >>= 1;
+  return tile;
+}
+
 template <int D, int RP>
 static cudaError_t launch_score_t(const Geom& G, int level, int64_t n_nodes, int64_t n_par,
                                   int32_t batch, const float* Q, const uint32_t* kept_up,
                                   int64_t words_up, float* sigma, const float* store,
                                   cudaStream_t s) {
-  using S = ScoreShape<D, RP>;
   const int qn = batch * G.group;
-  // Nodes per CTA: enough CTAs to fill the GPU twice over, at most kScoreTile.
-  int tile = kScoreTile;
-  while (tile > kScoreThreads / 32 && (n_nodes * G.hkv) / tile < 2 * 148) tile >>= 1;
+  const int tile = score_tile_for(n_nodes, G.hkv);
   dim3 grid(unsigned((n_nodes + tile - 1) / tile), unsigned(G.hkv),
             unsigned((qn + kScoreQBlock - 1) / kScoreQBlock));
-  const size_t smem = (size_t(kScoreThreads / 32) * S::KBUF +
-                       size_t(qn < kScoreQBlock ? qn : kScoreQBlock) * S::QROW) * 4;
+  const size_t smem = score_smem_bytes<D, RP>(G, batch);
   cudaError_t e = ensure_dynamic_smem(score_kernel<D, RP>, smem);
   if (e != cudaSuccess) return e;
   TraceScope ts("score_kernel", level, s);
@@ -816,55 +953,138 @@ static cudaError_t launch_score_t(const Geom& G, int level, int64_t n_nodes, int
 }
 
 template <int D>
-static cudaError_t launch_score_d(const Geom& G, int level, int64_t n_nodes, int64_t n_par,
-                                  int32_t batch, const float* Q, const uint32_t* kept_up,
-                                  int64_t words_up, float* sigma, const float* store,
-                                  cudaStream_t s) {
-  // Planes are padded to a power of two RP >= 128 / D so that each lane holds
-  // at least one float4 of its plane's row.
-  const int R = G.nref;
-#define ZHA_SCORE_CASE(RP)                                                                      \
-  if (R <= RP && RP * D >= 128)                                                                 \
-    return launch_score_t<D, RP>(G, level, n_nodes, n_par, batch, Q, kept_up, words_up, sigma, \
-                                 store, s);
-  if constexpr (D >= 128) ZHA_SCORE_CASE(1)
-  ZHA_SCORE_CASE(2)
-  ZHA_SCORE_CASE(4)
-  ZHA_SCORE_CASE(8)
-  ZHA_SCORE_CASE(16)
-  ZHA_SCORE_CASE(32)
-#undef ZHA_SCORE_CASE
-  return cudaErrorInvalidValue;
-}
-
-size_t select_smem_bytes() {
-  return size_t(kSelectThreads / 32) * 256 * sizeof(unsigned long long) +
-         size_t(kSelectCache) * sizeof(float) + size_t(kSelectKpCache) * sizeof(int32_t);
-}
-
-cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n_tokens, float p,
-                         int32_t* chunk_ids, int32_t* n_chunks, int32_t max_sel, uint32_t* bits,
-                         float* sigma, int32_t* kp, const RouteLayout& lay, int32_t* status,
-                         const float* store, cudaStream_t s) {
-  const size_t smem = select_smem_bytes();
-  cudaError_t e = ensure_dynamic_smem(select_kernel, smem);
+static cudaError_t launch_dense_t(const Geom& G, const DenseLevels& dl, int32_t batch, const float* Q,
+                                  const float* store, cudaStream_t s) {
+  const int qn = batch * G.group;
+  dim3 grid(unsigned(dl.tile0[dl.count]), unsigned(G.hkv), unsigned((qn + kDenseQ - 1) / kDenseQ));
+  const size_t smem = dense_smem_bytes<D>();
+  cudaError_t e = ensure_dynamic_smem(score_dense_kernel<D>, smem);
   if (e != cudaSuccess) return e;
+  TraceScope ts("score_dense_kernel", dl.level[dl.count - 1], s);
+  e = launch_pdl(score_dense_kernel<D>, grid, dim3(kDenseThreads), smem, s, G, dl, batch, Q, store);
+  zha_count_launch();
+  return e;
+}
+
+// Planes are padded to a power of two RP >= 128 / D so that each lane holds at
+// least one float4 of its plane's row.
+#define ZHA_SCORE_DISPATCH(CALL)                      \
+  do {                                                \
+    const int R = G.nref;                             \
+    if (G.d == 128) {                                 \
+      constexpr int D = 128;                          \
+      if (R <= 1) { constexpr int RP = 1; CALL; }     \
+      if (R <= 2) { constexpr int RP = 2; CALL; }     \
+      if (R <= 4) { constexpr int RP = 4; CALL; }     \
+      if (R <= 8) { constexpr int RP = 8; CALL; }     \
+      if (R <= 16) { constexpr int RP = 16; CALL; }   \
+      if (R <= 32) { constexpr int RP = 32; CALL; }   \
+    } else {                                          \
+      constexpr int D = 64;                           \
+      if (R <= 2) { constexpr int RP = 2; CALL; }     \
+      if (R <= 4) { constexpr int RP = 4; CALL; }     \
+      if (R <= 8) { constexpr int RP = 8; CALL; }     \
+      if (R <= 16) { constexpr int RP = 16; CALL; }   \
+      if (R <= 32) { constexpr int RP = 32; CALL; }   \
+    }                                                 \
+    return cudaErrorInvalidValue;                     \
+  } while (0)
+
+static cudaError_t launch_score_simt(const Geom& G, int level, int64_t n_nodes, int64_t n_par,
+                                     int32_t batch, const float* Q, const uint32_t* kept_up,
+                                     int64_t words_up, float* sigma, const float* store,
+                                     cudaStream_t s) {
+  ZHA_SCORE_DISPATCH(return (launch_score_t<D, RP>(G, level, n_nodes, n_par, batch, Q, kept_up,
+                                                    words_up, sigma, store, s)));
+}
+
+#undef ZHA_SCORE_DISPATCH
+
+static cudaError_t launch_dense(const Geom& G, const DenseLevels& dl, int32_t batch, const float* Q,
+                                const float* store, cudaStream_t s) {
+  return G.d == 128 ? launch_dense_t<128>(G, dl, batch, Q, store, s)
+                    : launch_dense_t<64>(G, dl, batch, Q, store, s);
+}
+
+cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n_tokens,
+                         const RoutePolicy& pol, int32_t* chunk_ids, int32_t* n_chunks,
+                         int32_t max_sel, uint32_t* bits, float* sigma, int32_t* kp,
+                         const RouteLayout& lay, int32_t* status, const float* store,
+                         cudaStream_t s) {
+  const size_t smem = select_smem_bytes();
+  cudaError_t e = ensure_dynamic_smem(select_fast_kernel, smem);
+  if (e != cudaSuccess) return e;
+  if ((e = ensure_dynamic_smem(select_top_kernel, smem)) != cudaSuccess) return e;
   const int heads = batch * G.hq;
-  SelectArgs a{};
-  a.p_fixed = (unsigned long long)ceil(double(p) * kMassScale);
-  if (a.p_fixed == 0) a.p_fixed = 1;
-  a.p_fixed32 = (unsigned long long)ceil(double(p) * 4294967296.0);
-  if (a.p_fixed32 == 0) a.p_fixed32 = 1;
-  const size_t smem_fast = select_fast_smem_bytes();
-  if ((e = ensure_dynamic_smem(select_fast_kernel, smem_fast)) != cudaSuccess)
-    return e;
-  a.keep_all = p >= 1.0f;
-  a.kp = kp;
-  int64_t kp_stride = lay.kp_ints / (heads > 0 ? heads : 1);
-  a.kp_stride = kp_stride;
-  a.max_sel = max_sel;
-  a.status = status;
-  for (int level = G.levels; level >= 1; --level) {
+  SelectArgs base{};
+  base.kp = kp;
+  base.kp_stride = lay.kp_ints / (heads > 0 ? heads : 1);
+  base.max_sel = max_sel;
+  base.status = status;
+  auto args_for = [&](int level) {
+    SelectArgs a = base;
+    a.level = level;
+    if (pol.topk) {
+      a.topk = 1;
+      a.p_fixed = a.p_fixed31 = (unsigned long long)pol.k[level];
+      a.keep_all = 0;
+    } else {
+      const double p = double(pol.p[level]);
+      a.p_fixed = (unsigned long long)ceil(p * kMassScale);
+      if (a.p_fixed == 0) a.p_fixed = 1;
+      a.p_fixed31 = (unsigned long long)ceil(p * 2147483648.0);
+      if (a.p_fixed31 == 0) a.p_fixed31 = 1;
+      a.keep_all = pol.p[level] >= 1.0f;
+    }
+    a.n_nodes = lay.n[level];
+    a.n_par = level < G.levels ? lay.n[level + 1] : 0;
+    a.kept_up = level < G.levels ? bits + lay.bits_off[level + 1] : nullptr;
+    a.words_up = level < G.levels ? lay.words[level + 1] : 0;
+    a.kept_here = bits + lay.bits_off[level];
+    a.words_here = lay.words[level];
+    a.sigma = sigma + lay.sig_off[level];
+    a.chunk_ids = level == 1 ? chunk_ids : nullptr;
+    a.n_chunks = level == 1 ? n_chunks : nullptr;
+    a.tree_status = level == G.levels ? tree_status_word(G, const_cast<float*>(store)) : nullptr;
+    return a;
+  };
+
+  // The dense block: levels L..l0 (l0 >= 2).
+  int l0 = G.levels + 1;
+  {
+    int64_t total = 0;
+    for (int level = G.levels; level >= 2; --level) {
+      const int64_t n = lay.n[level];
+      if (n > kDenseMaxNodes || total + n * G.hkv > kDenseMaxTotal) break;
+      total += n * G.hkv;
+      l0 = level;
+    }
+  }
+  if (l0 <= G.levels) {
+    DenseLevels dl{};
+    int64_t t0 = 0;
+    for (int level = G.levels; level >= l0; --level) {
+      if (lay.n[level] == 0) continue;
+      const int i = dl.count++;
+      const int npt = kDenseRows / G.nref;              // nodes per tile
+      dl.level[i] = level;
+      dl.n_nodes[i] = lay.n[level];
+      dl.tile0[i] = t0;
+      dl.sigma[i] = sigma + lay.sig_off[level];
+      t0 += (lay.n[level] + npt - 1) / npt;
+    }
+    dl.tile0[dl.count] = t0;
+    if (dl.count > 0 && (e = launch_dense(G, dl, batch, Q, store, s)) != cudaSuccess) return e;
+    SelectLevels sl{};
+    for (int level = G.levels; level >= l0; --level) sl.lv[sl.count++] = args_for(level);
+    {
+      TraceScope ts("select_top_kernel", l0, s);
+      e = launch_pdl(select_top_kernel, dim3(heads), dim3(kSelectThreads), smem, s, G, sl);
+    }
+    if (e != cudaSuccess) return e;
+    zha_count_launch();
+  }
+  for (int level = l0 - 1; level >= 1; --level) {
     const int64_t n_nodes = lay.n[level];
     const int64_t n_par = level < G.levels ? lay.n[level + 1] : 0;
     const uint32_t* up = level < G.levels ? bits + lay.bits_off[level + 1] : nullptr;
@@ -882,29 +1102,13 @@ cudaError_t launch_route(const Geom& G, const float* Q, int32_t batch, int64_t n
       else if (G.d == 128 && G.nref <= 16)      // tensor cores (zha_score_tc.cu)
         e = launch_score_tc(G, level, n_nodes, n_par, batch, Q, up, words_up, sg, store, status, s);
       else
-        e = G.d == 128 ? launch_score_d<128>(G, level, n_nodes, n_par, batch, Q, up, words_up, sg,
-                                             store, s)
-                       : launch_score_d<64>(G, level, n_nodes, n_par, batch, Q, up, words_up, sg,
-                                            store, s);
+        e = launch_score_simt(G, level, n_nodes, n_par, batch, Q, up, words_up, sg, store, s);
       if (e != cudaSuccess) return e;
     }
-    a.level = level;
-    a.n_nodes = n_nodes;
-    a.n_par = n_par;
-    a.kept_up = up;
-    a.words_up = words_up;
-    a.kept_here = bits + lay.bits_off[level];
-    a.words_here = lay.words[level];
-    a.sigma = sg;
-    a.chunk_ids = level == 1 ? chunk_ids : nullptr;
-    a.n_chunks = level == 1 ? n_chunks : nullptr;
-    a.tree_status = level == G.levels ? tree_status_word(G, const_cast<float*>(store)) : nullptr;
-    if (n_nodes <= kFastMax) {
+    const SelectArgs a = args_for(level);
+    {
       TraceScope ts("select_fast_kernel", level, s);
-      e = launch_pdl(select_fast_kernel, dim3(heads), dim3(kSelectThreads), smem_fast, s, G, a);
-    } else {
-      TraceScope ts("select_kernel", level, s);
-      e = launch_pdl(select_kernel, dim3(heads), dim3(kSelectThreads), smem, s, G, a);
+      e = launch_pdl(select_fast_kernel, dim3(heads), dim3(kSelectThreads), smem, s, G, a);
     }
     if (e != cudaSuccess) return e;
     zha_count_launch();

@@ -59,9 +59,10 @@ extern "C" zha_status zha_route_noalloc(const zha_tree* tree, const float* d_Q, 
                                         int64_t n_tokens, float p, int32_t* d_chunk_ids,
                                         int32_t* d_n_chunks, int32_t max_sel,
                                         uint32_t* d_kept_bits, int32_t* d_status, void* stream) {
-  zha_status st = zha_check_route_args(tree, d_Q, batch, n_tokens, p, d_chunk_ids, d_n_chunks,
-                                       max_sel, "zha_route_noalloc");
+  zha_status st = zha_check_route_args(tree, d_Q, batch, n_tokens, d_chunk_ids, d_n_chunks, max_sel,
+                                       "zha_route_noalloc");
   if (st != ZHA_OK) return st;
+  if ((st = zha_check_p(p, "zha_route_noalloc")) != ZHA_OK) return st;
   const zha::Geom& G = tree->geom;
   const zha::RouteLayout lay = zha::route_layout(G, batch, n_tokens);
   const int64_t need = d_kept_bits ? lay.bytes_no_bits : lay.bytes;
@@ -83,7 +84,8 @@ extern "C" zha_status zha_route_noalloc(const zha_tree* tree, const float* d_Q, 
   float* sigma = reinterpret_cast<float*>(ws);
   int32_t* kp = reinterpret_cast<int32_t*>(ws + zha::round_up(lay.sig_floats * 4, 256));
   uint32_t* bits = d_kept_bits ? d_kept_bits : reinterpret_cast<uint32_t*>(ws + lay.bytes_no_bits);
-  cudaError_t e = zha::launch_route(G, d_Q, batch, n_tokens, p, d_chunk_ids, d_n_chunks, max_sel,
+  cudaError_t e = zha::launch_route(G, d_Q, batch, n_tokens, zha::uniform_top_p(p), d_chunk_ids,
+                                    d_n_chunks, max_sel,
                                     bits, sigma, kp, lay, d_status, tree->store,
                                     static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {

@@ -19,7 +19,7 @@
 //                           at a time: box = 32 columns x 16 planes x 8 nodes,
 //                           128-byte swizzled, rows (node, plane) = MMA rows.
 //   converters (warps 4-11) thread = (row, 32-column box): each fp32 value ->
-//                           three bf16 terms (x = t0 + t1 + t2 to fp32's 24 bits),
+//                           three truncated bf16 terms (x = t0 + t1 + t2 exactly),
 //                           stored from registers straight into tensor memory (three
 //                           half-buffers), where
 //                           the MMA reads its A operand (shared memory only carries
@@ -96,16 +96,23 @@ __device__ __forceinline__ int group_width(const Geom& G, int batch, int q_block
   return min(kQn, batch * G.group - (v % q_blocks) * kQn);
 }
 
-// Two fp32 values -> three packed bf16x2 terms (x = t0 + t1 + t2 per lane of
-// the pair; the widening back to fp32 for the residual is a shift or a mask).
+// Two fp32 values -> three packed bf16x2 terms with x = t0 + t1 + t2 exactly
+// (x0 in the low half of each term, x1 in the high half). Each term is the
+// upper 16 bits of the remaining residual (a truncated bf16): t0 keeps the sign,
+// exponent and first 7 mantissa bits of x, the residual x - t0 is exact in fp32
+// with at most 16 significant bits, its upper half t1 leaves an exact residual
+// of at most 8 significant bits, which a bf16 holds, so t2 is exact. Byte
+// permutes, masks and subtractions only: no conversion instructions.
 __device__ __forceinline__ void split3_x2(float x0, float x1, uint32_t& t0, uint32_t& t1, uint32_t& t2) {
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(t0) : "f"(x1), "f"(x0));
-  x0 -= __uint_as_float(t0 << 16);
-  x1 -= __uint_as_float(t0 & 0xffff0000u);
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(t1) : "f"(x1), "f"(x0));
-  x0 -= __uint_as_float(t1 << 16);
-  x1 -= __uint_as_float(t1 & 0xffff0000u);
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(t2) : "f"(x1), "f"(x0));
+  const uint32_t u0 = __float_as_uint(x0), u1 = __float_as_uint(x1);
+  t0 = __byte_perm(u0, u1, 0x7632);
+  const float r0 = x0 - __uint_as_float(u0 & 0xffff0000u);
+  const float r1 = x1 - __uint_as_float(u1 & 0xffff0000u);
+  const uint32_t v0 = __float_as_uint(r0), v1 = __float_as_uint(r1);
+  t1 = __byte_perm(v0, v1, 0x7632);
+  const float q0 = r0 - __uint_as_float(v0 & 0xffff0000u);
+  const float q1 = r1 - __uint_as_float(v1 & 0xffff0000u);
+  t2 = __byte_perm(__float_as_uint(q0), __float_as_uint(q1), 0x7632);
 }
 
 // Eight fp32 values -> three bf16x8 terms.

@@ -36,6 +36,33 @@ class ZhaError(RuntimeError):
         self.status = status
 
 
+ZHA_SELECT_TOP_P = 0
+ZHA_SELECT_TOP_K = 1
+
+
+class RoutePolicy(ctypes.Structure):
+    """zha_route_policy: per-level top-p masses or top-k budgets (level l at index l-1)."""
+    _fields_ = [("mode", c_int32), ("reserved", c_int32), ("p", c_float * 8), ("k", c_int32 * 8)]
+
+
+def top_p_policy(p_by_level) -> RoutePolicy:
+    """Top-p with p_by_level[l-1] at level l (a sequence of up to 8 masses)."""
+    pol = RoutePolicy()
+    pol.mode = ZHA_SELECT_TOP_P
+    for i, v in enumerate(p_by_level):
+        pol.p[i] = float(v)
+    return pol
+
+
+def top_k_policy(k_by_level) -> RoutePolicy:
+    """Fixed-budget top-K with k_by_level[l-1] nodes kept at level l."""
+    pol = RoutePolicy()
+    pol.mode = ZHA_SELECT_TOP_K
+    for i, v in enumerate(k_by_level):
+        pol.k[i] = int(v)
+    return pol
+
+
 class Config(ctypes.Structure):
     _fields_ = [
         ("n_kv_heads", c_int32), ("n_q_heads", c_int32), ("head_dim", c_int32),
@@ -69,6 +96,8 @@ def _load() -> ctypes.CDLL:
         "zha_route": (c_int32, [P, P, c_int32, c_int64, c_float, P, P, c_int32, P, P, c_size_t,
                                 P, P]),
         "zha_route_noalloc": (c_int32, [P, P, c_int32, c_int64, c_float, P, P, c_int32, P, P, P]),
+        "zha_route_ex": (c_int32, [P, P, c_int32, c_int64, POINTER(RoutePolicy), P, P, c_int32, P, P,
+                                   c_size_t, P, P]),
         "zha_attend_workspace_bytes": (c_size_t, [POINTER(Config), c_int32, c_int64]),
         "zha_sparse_attend": (c_int32, [P, P, P, P, c_int64, c_int64, c_int32, P, P, c_int32, P,
                                         P, P, c_size_t, P, P]),
@@ -222,7 +251,7 @@ class Tree:
         blk = self.store[off.value: off.value + H * cap.value * nf.value].view(H, cap.value, nf.value)
         return blk[:, :, : R * d].reshape(H, cap.value, R, d), blk[:, :, R * d: R * d + R]
 
-    def route(self, Q: torch.Tensor, n_tokens: int, p: float, max_sel: int,
+    def route(self, Q: torch.Tensor, n_tokens: int, p: "float | RoutePolicy", max_sel: int,
               chunk_ids: torch.Tensor | None = None, n_chunks: torch.Tensor | None = None,
               kept_bits: torch.Tensor | None = None, ws: torch.Tensor | None = None,
               status: torch.Tensor | None = None, stream=None):
@@ -233,9 +262,15 @@ class Tree:
             n_chunks = torch.empty(B, self.cfg.n_q_heads, dtype=torch.int32, device=self.device)
         if ws is None:
             ws = _bytes_tensor(route_workspace_bytes(self.cfg, B, n_tokens), self.device)
-        check(lib.zha_route(self.handle, ptr(Q), B, n_tokens, p, ptr(chunk_ids), ptr(n_chunks),
-                            max_sel, ptr(kept_bits), ptr(ws), ws.numel() * ws.element_size(),
-                            ptr(status), stream_ptr(stream)), "zha_route")
+        if isinstance(p, RoutePolicy):
+            check(lib.zha_route_ex(self.handle, ptr(Q), B, n_tokens, byref(p), ptr(chunk_ids),
+                                   ptr(n_chunks), max_sel, ptr(kept_bits), ptr(ws),
+                                   ws.numel() * ws.element_size(), ptr(status), stream_ptr(stream)),
+                  "zha_route_ex")
+        else:
+            check(lib.zha_route(self.handle, ptr(Q), B, n_tokens, p, ptr(chunk_ids), ptr(n_chunks),
+                                max_sel, ptr(kept_bits), ptr(ws), ws.numel() * ws.element_size(),
+                                ptr(status), stream_ptr(stream)), "zha_route")
         return chunk_ids, n_chunks
 
     def sparse_attend(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, n_tokens: int,

@@ -174,6 +174,33 @@ zha_status zha_route(const zha_tree* tree, const float* d_Q, int32_t batch, int6
                      uint32_t* d_kept_bits, void* d_ws, size_t ws_bytes, int32_t* d_status,
                      void* stream);
 
+/* Per-level selection rule of zha_route_ex [ZHA: 전제와 한계]. The pages route
+ * with top-p at every level and name its depth scaling: one fixed p per level
+ * gives an effective p^L, correcting with p^(1/L) drives p towards 1, so p has
+ * to follow depth; they also set top-p against a fixed-budget top-K, which
+ * keeps the same number of nodes whether the mass is concentrated or flat. */
+typedef enum { ZHA_SELECT_TOP_P = 0, ZHA_SELECT_TOP_K = 1 } zha_select_mode;
+
+typedef struct {
+    int32_t mode;      /* zha_select_mode */
+    int32_t reserved;  /* must be 0 */
+    float p[8];        /* ZHA_SELECT_TOP_P: mass of level l (1..L) at p[l-1]; > 0, finite; >= 1
+                          keeps every candidate of that level */
+    int32_t k[8];      /* ZHA_SELECT_TOP_K: nodes kept at level l at k[l-1], >= 1: the first
+                          min(k, candidates) in the order score descending, node index ascending */
+} zha_route_policy;
+
+/* zha_route with a per-level policy: top-p with its own p at each level (for
+ * instance p^(1/L) per level), or fixed-budget top-K. Candidates, scores,
+ * outputs, workspace and status are as for zha_route; only the cut of each
+ * level changes. zha_route(p) is zha_route_ex with mode ZHA_SELECT_TOP_P and p
+ * at every level. ZHA_ERR_INVALID for a NULL policy, an unknown mode, reserved
+ * != 0, or a p / k of levels 1..L out of range (entries past L are ignored). */
+zha_status zha_route_ex(const zha_tree* tree, const float* d_Q, int32_t batch, int64_t n_tokens,
+                        const zha_route_policy* policy, int32_t* d_chunk_ids, int32_t* d_n_chunks,
+                        int32_t max_sel, uint32_t* d_kept_bits, void* d_ws, size_t ws_bytes,
+                        int32_t* d_status, void* stream);
+
 /* Size of the routing scratch built into the library for zha_route_noalloc. */
 #define ZHA_ROUTE_NOALLOC_SCRATCH_BYTES (32u << 20) /* 32 MiB per GPU that loads the library */
 

@@ -22,6 +22,10 @@ from .zha_oracle import (  # noqa: F401
     OracleTree,
     build_tree,
     top_p_prefix,
+    top_k_prefix,
+    RoutePolicy,
+    depth_scaled_p,
+    select_level,
     TopP,
     route,
     RouteTrace,

@@ -40,12 +40,23 @@ class RouteReport:
                 "hard": len(self.hard), "exact_heads": len(self.exact_heads)}
 
 
+def _level_mass(p, level):
+    """The top-p mass of `level` under a number, a {level: p} dict or a
+    RoutePolicy; None for a fixed-budget (top-K) level."""
+    if isinstance(p, O.RoutePolicy):
+        return p.at(level) if p.mode == "top_p" else None
+    if isinstance(p, dict):
+        return p[level]
+    return p
+
+
 def compare_route_head(q, otree, p, kept_by_level: dict, report: RouteReport, key,
                        route_fn=None) -> None:
     """Compare one query head's kept sets {level: node ids} with the oracle,
     level by level (each level conditioned on the compared kept set one level
-    up). ``route_fn`` replaces ``zha_oracle.route`` (same signature) for routing
-    variants."""
+    up). ``p`` is what ``zha_oracle.route`` takes: a mass, a {level: p} dict or a
+    RoutePolicy (for top-K levels only score ties count). ``route_fn`` replaces
+    ``zha_oracle.route`` (same signature) for routing variants."""
     route = route_fn if route_fn is not None else O.route
     forced = {lvl: ids for lvl, ids in kept_by_level.items()}
     tr = route(q, otree, p, forced_kept=forced)
@@ -61,8 +72,10 @@ def compare_route_head(q, otree, p, kept_by_level: dict, report: RouteReport, ke
         sel = lt.topp
         m = sel.m
         sigma_cut = lt.sigma[sel.order[m - 1]] if m > 0 else math.inf
-        near_mass = (m >= 1 and abs(sel.cum[m - 1] - p) <= TIE_TOL) or \
-                    (m >= 2 and abs(sel.cum[m - 2] - p) <= TIE_TOL)
+        p_lvl = _level_mass(p, lvl)
+        near_mass = p_lvl is not None and (
+            (m >= 1 and abs(sel.cum[m - 1] - p_lvl) <= TIE_TOL) or
+            (m >= 2 and abs(sel.cum[m - 2] - p_lvl) <= TIE_TOL))
         for node in own ^ got:
             if node not in cand_pos:
                 report.hard.append((key, lvl, node, "not a candidate"))

@@ -42,7 +42,10 @@ causal example, the online-softmax table, the softmax-saturation numbers, tangen
 exactness, the convexity lower bound, the finite-difference gradient
 dF/dq = khat/sqrt(d), identical-key and single-key chunks, merge == direct
 summary over raw keys, brute-force minimal prefix over all subsets, hand-built
-routing trees, set invariants, and p=1 routed == dense attention.
+routing trees, set invariants, and p=1 routed == dense attention; for the
+routing policies, brute force over all subsets (top-K), the closed-form kept
+counts of a flat tree under a fixed p and under p**(1/L), and the product of
+the depth-scaled masses.
 ``captured_mass`` is a diagnostic only: parity unpinned.
 """
 
@@ -292,6 +295,63 @@ def top_p_prefix(sigma: np.ndarray, ids: np.ndarray, p: float) -> TopP:
     return TopP(kept=kept, order=order, pi=pi, cum=cum, m=m)
 
 
+def top_k_prefix(sigma: np.ndarray, ids: np.ndarray, k: int) -> TopP:
+    """Fixed-budget selection: the first min(k, n) candidates in the order
+    score descending, node index ascending. [ZHA: 전제와 한계] sets top-p
+    routing against a fixed-budget top-K, which keeps the same number of nodes
+    whether the mass is concentrated or flat; this is that comparison mode.
+    ``pi`` and ``cum`` are the softmax masses along the order, as for top-p.
+    """
+    sigma = np.asarray(sigma, np.float64)
+    ids = np.asarray(ids, np.int64)
+    n = sigma.shape[0]
+    if n == 0:
+        e = np.zeros(0, np.int64)
+        return TopP(kept=e, order=e, pi=np.zeros(0), cum=np.zeros(0), m=0)
+    order = np.lexsort((ids, -sigma))
+    pi = np.exp(sigma - logsumexp(sigma))
+    cum = np.cumsum(pi[order])
+    m = min(int(k), n)
+    return TopP(kept=np.sort(ids[order[:m]]), order=order, pi=pi, cum=cum, m=m)
+
+
+@dataclass
+class RoutePolicy:
+    """How each level's kept prefix is chosen. [ZHA: 전제와 한계]
+
+    mode "top_p": level l keeps the minimal prefix holding estimated mass
+    ``p[l]`` (one p for every level when ``p`` is a number).
+    mode "top_k": level l keeps the first ``k[l]`` candidates (fixed budget).
+    """
+    mode: str = "top_p"
+    p: object = 0.9
+    k: object = None
+
+    def at(self, level: int):
+        v = self.p if self.mode == "top_p" else self.k
+        return v[level] if isinstance(v, dict) else v
+
+
+def depth_scaled_p(p: float, levels: int) -> dict:
+    """Per-level mass p_l = p**(1/L) for l = 1..L, so that the product of the
+    per-level masses is p. [ZHA: 전제와 한계] names both ends of the depth
+    scaling: a fixed p per level gives an effective p**L, which goes to 0 with
+    depth, while correcting with p**(1/L) drives each level's p towards 1."""
+    return {lvl: float(p) ** (1.0 / levels) for lvl in range(1, levels + 1)}
+
+
+def select_level(sigma: np.ndarray, ids: np.ndarray, level: int, policy) -> TopP:
+    """One level's selection under ``policy`` (a number p, a {level: p} dict,
+    or a RoutePolicy)."""
+    if isinstance(policy, RoutePolicy):
+        if policy.mode == "top_k":
+            return top_k_prefix(sigma, ids, policy.at(level))
+        return top_p_prefix(sigma, ids, policy.at(level))
+    if isinstance(policy, dict):
+        return top_p_prefix(sigma, ids, policy[level])
+    return top_p_prefix(sigma, ids, policy)
+
+
 @dataclass
 class LevelTrace:
     candidates: np.ndarray      # node ids at this level, ascending
@@ -321,7 +381,7 @@ def leaf_token_set(leaf_chunks: np.ndarray, chunk: int, n_tokens: int) -> np.nda
     return np.unique(np.concatenate(parts))
 
 
-def route(q: np.ndarray, tree: OracleTree, p: float,
+def route(q: np.ndarray, tree: OracleTree, p,
           forced_kept: dict | None = None) -> RouteTrace:
     """Per-level top-p routing of one query head through one tree.
     [ZHA: 전제와 한계]
@@ -330,6 +390,8 @@ def route(q: np.ndarray, tree: OracleTree, p: float,
     candidates are scored (``node_score``), softmaxed and cut by
     ``top_p_prefix``; the next level's candidates are the children of the kept
     nodes plus that level's orphans (nodes whose parent does not exist).
+    ``p`` is one mass for every level, a {level: p_l} schedule, or a
+    RoutePolicy (per-level p, or the fixed-budget top-K comparison mode).
 
     ``forced_kept`` (level -> node ids) makes the expansion below that level use
     the given kept set instead of this oracle's own; each level still records its
@@ -347,7 +409,7 @@ def route(q: np.ndarray, tree: OracleTree, p: float,
         cand = np.concatenate([children.astype(np.int64), orphans])
         khat, bhat = tree.nodes[lvl]
         sigma = node_score(q, khat[cand], bhat[cand]) if cand.size else np.zeros(0)
-        sel = top_p_prefix(sigma, cand, p)
+        sel = select_level(sigma, cand, lvl, p)
         if forced_kept is not None and lvl in forced_kept:
             expanded = np.sort(np.asarray(forced_kept[lvl], np.int64))
         else:

@@ -179,3 +179,36 @@ def test_split_arithmetic_of_the_tensor_core_attention():
                 visited = {c for c in range(c_lo, c_hi + 1) if (c + 1) * T // n > c * T // n}
                 meets = {c for c in range(n) if max(start[c], lo) < min(start[c + 1], hi)}
                 assert visited == meets
+
+
+def test_route_ex_rejects_bad_policies_before_any_launch(zha):
+    """zha_route_ex checks its policy on the host: NULL, unknown mode, reserved
+    != 0, p <= 0 or not finite, k < 1 on a level of the tree; entries past the
+    tree's levels are ignored."""
+    cfg = _cfg(zha)
+    handle = ctypes.c_void_p()
+    assert zha.lib.zha_tree_create(ctypes.byref(cfg), ctypes.c_void_p(1 << 40), 1 << 34,
+                                   ctypes.c_void_p(1 << 41), ctypes.byref(handle)) == zha.ZHA_OK
+    P = ctypes.c_void_p
+    before = zha.launch_count()
+    try:
+        def call(pol):
+            return zha.lib.zha_route_ex(handle, P(1 << 42), 4, 10, pol, P(1 << 43), P(1 << 44), 16, None,
+                                        P(1 << 45), 16, None, None)
+        assert call(None) == zha.ZHA_ERR_INVALID and "policy" in zha.last_error()
+        bad_mode = zha.top_p_policy([0.9] * 3)
+        bad_mode.mode = 7
+        assert call(ctypes.byref(bad_mode)) == zha.ZHA_ERR_INVALID
+        res = zha.top_p_policy([0.9] * 3)
+        res.reserved = 1
+        assert call(ctypes.byref(res)) == zha.ZHA_ERR_INVALID
+        for ps in ([0.9, 0.0, 0.9], [0.9, 0.9, float("nan")], [-1.0, 0.9, 0.9]):
+            assert call(ctypes.byref(zha.top_p_policy(ps))) == zha.ZHA_ERR_INVALID
+        assert call(ctypes.byref(zha.top_k_policy([5, 0, 2]))) == zha.ZHA_ERR_INVALID
+        # valid policies (levels 4..8 unset) pass the policy checks and then
+        # fail on the tiny workspace
+        assert call(ctypes.byref(zha.top_p_policy([0.9, 0.9, 0.9]))) == zha.ZHA_ERR_CAPACITY
+        assert call(ctypes.byref(zha.top_k_policy([5, 3, 2]))) == zha.ZHA_ERR_CAPACITY
+        assert zha.launch_count() == before
+    finally:
+        zha.lib.zha_tree_destroy(handle)

@@ -62,11 +62,12 @@ def run_pipeline(zha, inp, n_tokens, p=None, max_sel=None, batch_index=0, stream
 
 
 def check_case(zha, inp, n_tokens, p=None, heads=None, all_nodes=True, batch_index=0, tree=None,
-               dev=None):
-    """Full comparison; returns the route report."""
+               dev=None, oracle_p=None):
+    """Full comparison; returns the route report. ``p`` goes to the GPU route
+    (a mass or a zha.RoutePolicy), ``oracle_p`` (default: ``p``) to the oracle's."""
     spec = inp.spec
     res = run_pipeline(zha, inp, n_tokens, p=p, batch_index=batch_index, tree=tree, dev=dev)
-    p = res["p"]
+    p = res["p"] if oracle_p is None else oracle_p
     assert res["status"] == 0
     G = spec.group
     B = spec.batch
@@ -472,3 +473,35 @@ def test_build_status_is_clean_and_reaches_the_route(zha):
     st = res["tree"].store.view(torch.int32)
     off = (zha.tree_bytes(res["tree"].cfg) - 256) // 4
     assert int(st[off].item()) == 0
+
+
+# ---------------------------------------------------------------------------
+# Routing policies: per-level p and fixed-budget top-K [ZHA: 전제와 한계]
+# ---------------------------------------------------------------------------
+
+POLICY_CASES = {
+    "depth_scaled_p": ("top_p", [0.75 ** (1 / 3)] * 3),
+    "per_level_p": ("top_p", [0.95, 0.8, 0.5]),          # levels 1, 2, 3
+    "top_k_small": ("top_k", [40, 12, 3]),               # counting path (<= 512 candidates)
+    "top_k_wide": ("top_k", [700, 150, 20]),             # radix path at level 1
+}
+
+
+@pytest.mark.parametrize("case", list(POLICY_CASES))
+def test_route_policies_match_the_oracle(zha, parity_log, case):
+    """zha_route_ex against the oracle's route under the same policy, every
+    level of every head (C = 16, L = 3, 65557 tokens, clustered keys)."""
+    mode, vals = POLICY_CASES[case]
+    spec = W.scaled("256k", n_kv_heads=2, n_q_heads=8, n_tokens=65536, stream_tokens=64)
+    inp = W.generate(spec)
+    if mode == "top_p":
+        gpu_p = zha.top_p_policy(vals)
+        oracle_p = O.RoutePolicy(mode="top_p", p={l + 1: float(np.float32(v)) for l, v in enumerate(vals)})
+    else:
+        gpu_p = zha.top_k_policy(vals)
+        oracle_p = O.RoutePolicy(mode="top_k", k={l + 1: v for l, v in enumerate(vals)})
+    rep = check_case(zha, inp, 65536 + 21, p=gpu_p, oracle_p=oracle_p)
+    parity_log(f"policy_{case}", rep)
+    if mode == "top_k":
+        res = run_pipeline(zha, inp, 65536 + 21, p=gpu_p)
+        assert (res["cnt"] <= vals[0]).all()

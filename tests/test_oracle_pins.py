@@ -381,3 +381,100 @@ def test_bf16_decode_is_exact():
     assert O.bf16_bits_to_f64(np.array([0x3F80], np.uint16))[0] == 1.0
     assert O.bf16_bits_to_f64(np.array([0xC020], np.uint16))[0] == -2.5
     assert O.bf16_bits_to_f64(np.array([0x0000], np.uint16))[0] == 0.0
+
+
+# ---------------------------------------------------------------------------
+# Routing policies: per-level p schedule and fixed-budget top-K
+# [ZHA: 전제와 한계]
+# ---------------------------------------------------------------------------
+
+def _precedes(sig, ids, a, b):
+    """Candidate a comes before candidate b: higher score, or equal score and
+    lower node index."""
+    return sig[a] > sig[b] or (sig[a] == sig[b] and ids[a] < ids[b])
+
+
+def test_top_k_is_the_upward_closed_subset_by_brute_force():
+    """Among all subsets of size min(k, n) exactly one contains, with each of
+    its members, every candidate that precedes it; top_k_prefix keeps it."""
+    rng = np.random.default_rng(21)
+    for _ in range(300):
+        n = int(rng.integers(0, 9))
+        sig = rng.integers(-3, 3, size=n).astype(float)          # many ties
+        ids = rng.permutation(40)[:n]
+        k = int(rng.integers(1, 11))
+        sel = O.top_k_prefix(sig, ids, k)
+        m = min(k, n)
+        closed = []
+        for S in itertools.combinations(range(n), m):
+            Sset = set(S)
+            if all(not _precedes(sig, ids, b, a) for a in Sset for b in range(n) if b not in Sset):
+                closed.append(sorted(ids[list(S)]))
+        assert len(closed) == 1
+        assert list(sel.kept) == closed[0] and sel.m == m
+
+
+def _flat_tree(C=4, L=3, n_tokens=256):
+    """Every key equal: every node of a level has the same summary, so the
+    candidates' estimated masses are uniform and ties go to the lower index."""
+    d = 8
+    K = np.tile(np.linspace(-1.0, 1.0, d), (n_tokens, 1))
+    qhat = np.random.default_rng(3).standard_normal((2, d))
+    return O.build_tree(K, qhat, C, L, n_tokens), np.random.default_rng(4).standard_normal(d)
+
+
+def _kept_counts(trace):
+    return {lvl: len(lt.topp.kept) for lvl, lt in trace.levels.items()}
+
+
+def test_flat_tree_kept_counts_under_fixed_and_depth_scaled_p():
+    """Uniform masses over n candidates: top-p keeps ceil(p n) of them. With
+    C = 4 and 4, 16, 64 nodes at levels 3, 2, 1: a fixed p = 0.7 keeps 3 of 4,
+    then 9 of 12, then 26 of 36 (26/64 = 0.41 of the chunks: the per-level
+    fractions multiply); p**(1/3) = 0.8879 per level keeps 4 of 4, 15 of 16,
+    54 of 60 (0.84 of the chunks)."""
+    tree, q = _flat_tree()
+    fixed = O.route(q, tree, 0.7)
+    assert _kept_counts(fixed) == {3: 3, 2: 9, 1: 26}
+    assert list(fixed.levels[3].topp.kept) == [0, 1, 2]           # ties: lower index first
+    assert [len(fixed.levels[l].candidates) for l in (3, 2, 1)] == [4, 12, 36]
+    scaled = O.route(q, tree, O.depth_scaled_p(0.7, 3))
+    assert _kept_counts(scaled) == {3: 4, 2: 15, 1: 54}
+    sched = O.route(q, tree, {3: 0.55, 2: 0.9, 1: 0.3})    # ceil(2.2), ceil(10.8), ceil(13.2)
+    assert _kept_counts(sched) == {3: 3, 2: 11, 1: 14}
+    pol = O.route(q, tree, O.RoutePolicy(mode="top_p", p={3: 0.55, 2: 0.9, 1: 0.3}))
+    assert _kept_counts(pol) == {3: 3, 2: 11, 1: 14}
+
+
+def test_depth_scaled_masses_multiply_to_p():
+    for p in (0.3, 0.75, 0.9, 0.99):
+        for L in (1, 2, 3, 6):
+            sched = O.depth_scaled_p(p, L)
+            assert sorted(sched) == list(range(1, L + 1))
+            assert abs(math.prod(sched.values()) - p) < 1e-12
+            assert all(v >= p for v in sched.values())
+
+
+def test_top_k_route_keeps_the_budget_at_every_level():
+    """Flat tree: top-K keeps exactly min(k_l, candidates) per level. Random
+    trees: each level's kept set is the upward-closed subset of that level's
+    candidates (checked pairwise) of size min(k_l, candidates)."""
+    tree, q = _flat_tree()
+    tr = O.route(q, tree, O.RoutePolicy(mode="top_k", k={3: 2, 2: 5, 1: 7}))
+    assert _kept_counts(tr) == {3: 2, 2: 5, 1: 7}
+    assert list(tr.levels[3].topp.kept) == [0, 1] and list(tr.leaf_chunks) == list(range(7))
+    rng = np.random.default_rng(8)
+    for n_tokens in (97, 300, 1000):
+        K = rng.standard_normal((n_tokens, 8))
+        t = O.build_tree(K, rng.standard_normal((3, 8)), 4, 3, n_tokens)
+        budget = {3: 3, 2: 6, 1: 9}
+        tr = O.route(rng.standard_normal(8) * 2, t, O.RoutePolicy(mode="top_k", k=budget))
+        for lvl, lt in tr.levels.items():
+            n = len(lt.candidates)
+            kept = set(lt.topp.kept.tolist())
+            assert len(kept) == min(budget[lvl], n)
+            pos = {int(c): i for i, c in enumerate(lt.candidates)}
+            for a in kept:
+                for b in lt.candidates:
+                    if int(b) not in kept:
+                        assert not _precedes(lt.sigma, lt.candidates, pos[int(b)], pos[a])
