@@ -21,6 +21,12 @@ from .zha_oracle import (  # noqa: F401
     merge_children,
     OracleTree,
     build_tree,
+    rope_angles,
+    rope_rotate,
+    node_position,
+    summarise_chunk_rope,
+    merge_children_rope,
+    build_tree_rope,
     top_p_prefix,
     top_k_prefix,
     RoutePolicy,

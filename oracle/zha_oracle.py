@@ -18,7 +18,8 @@ Citations
                   "토큰 세 개로 직접 계산하기" (3-token worked example),
                   "Causal mask 는 뒤에 오는 토큰을 가린다",
                   "같은 계산을 메모리 IO 를 줄여서 한다: FlashAttention 계열"
-                  (online-softmax table).
+                  (online-softmax table), "Attention 은 순서를 모르므로 위치
+                  정보를 따로 넣는다" (RoPE).
 [ASM: 방법론]     page "효율적인 긴 컨텍스트 생성을 위한 컨텍스트 기억화"
                   (aitrends.kr/articles/59378), section "방법론": the merge of two
                   attention states, used only as a second statement of the identity
@@ -247,6 +248,119 @@ def build_tree(K: np.ndarray, qhat: np.ndarray, chunk: int, levels: int,
         kh = kh[: n_here * chunk].reshape(n_here, chunk, *kh.shape[1:])
         bh = bh[: n_here * chunk].reshape(n_here, chunk, bh.shape[-1])
         tree.nodes[lvl] = merge_children(qhat, kh, bh)
+    return tree
+
+
+# ----------------------------------------------------------------------------
+# Rotary positions   [ZHA: 무엇과 다른가; Attention: "Attention 은 순서를 모르므로 위치 정보를 따로 넣는다"]
+# ----------------------------------------------------------------------------
+
+def rope_angles(d: int, base: float, pairs: int) -> np.ndarray:
+    """Rotation speed theta_i of each element pair i = (2i, 2i+1).
+
+    [Attention: "Attention 은 순서를 모르므로 위치 정보를 따로 넣는다"] pairs the
+    elements of a query or key two by
+    two, reads each pair as a point of a plane, and turns pair i of the token
+    at position m by the angle m * theta_i, a different speed per pair (Su et
+    al., 2021). Reading: theta_i = base**(-2i/d), the first ``pairs`` pairs
+    turn, the others (partial RoPE) stay as they are (theta = 0).
+    """
+    i = np.arange(d // 2, dtype=np.float64)
+    theta = np.power(float(base), -2.0 * i / d)
+    theta[int(pairs):] = 0.0
+    return theta
+
+
+def rope_rotate(x: np.ndarray, pos, base: float, pairs: int) -> np.ndarray:
+    """Turn pair i of x (elements 2i, 2i+1) by pos * theta_i. x: [..., d];
+    pos: a number or an array broadcasting against x[..., 0]."""
+    x = np.asarray(x, np.float64)
+    d = x.shape[-1]
+    ang = np.asarray(pos, np.float64)[..., None] * rope_angles(d, base, pairs)     # [..., d/2]
+    c, s = np.cos(ang), np.sin(ang)
+    a, b = x[..., 0::2], x[..., 1::2]
+    out = np.empty(np.broadcast_shapes(x.shape, ang.shape[:-1] + (d,)), np.float64)
+    out[..., 0::2] = a * c - b * s
+    out[..., 1::2] = a * s + b * c
+    return out
+
+
+def node_position(level: int, index, chunk: int):
+    """Position of node (level, index): its first token, index * chunk**level
+    (reading: a node's rotated reference query sits where its span starts)."""
+    return np.asarray(index, np.int64) * chunk ** level
+
+
+def summarise_chunk_rope(qhat: np.ndarray, Kc: np.ndarray, pos, base: float,
+                         pairs: int) -> tuple[np.ndarray, np.ndarray]:
+    """Level-1 summary with rotary positions: the tangent plane of F_C taken at
+    the chunk's rotated reference queries q_hat_{r,c} = rotate(q_hat_r, pos_c),
+    over the keys as the cache stores them (already rotated at their own
+    positions). [ZHA: 무엇과 다른가]
+
+    qhat: [R, d]; Kc: [..., C, d]; pos: [...] chunk positions.
+    """
+    qhat = np.asarray(qhat, np.float64)
+    Kc = np.asarray(Kc, np.float64)
+    pos = np.asarray(pos, np.float64)
+    q_rot = rope_rotate(qhat, pos[..., None], base, pairs)        # [..., R, d]
+    d = Kc.shape[-1]
+    u = np.einsum("...rd,...jd->...rj", q_rot, Kc) / np.sqrt(d)    # [..., R, C]
+    keys = np.broadcast_to(Kc[..., None, :, :], u.shape + (d,))
+    F, khat = combine_log_masses(u, keys)
+    bhat = F - np.sum(khat * q_rot, axis=-1) / np.sqrt(d)
+    return khat, bhat
+
+
+def merge_children_rope(qhat: np.ndarray, khat_ch: np.ndarray, bhat_ch: np.ndarray,
+                        pos_parent, pos_children, base: float,
+                        pairs: int) -> tuple[np.ndarray, np.ndarray]:
+    """Parent summary from its children's with rotary positions. [ZHA: 무엇과
+    다른가]: each child is re-evaluated at the parent's rotated reference query
+    q_hat_{r,P}; its log mass there is its tangent value at its own rotated
+    reference query, F_c(q_hat_{r,c}) = q_hat_{r,c}.khat_{r,c}/sqrt(d) + bhat_{r,c},
+    plus the correction 1/sqrt(d) <khat_{r,c}, q_hat_{r,P} - q_hat_{r,c}>; the
+    parent then combines these log masses and the children's compressed keys
+    as in the position-free merge.
+
+    khat_ch: [..., C, R, d]; bhat_ch: [..., C, R]; pos_parent: [...];
+    pos_children: [..., C].
+    """
+    qhat = np.asarray(qhat, np.float64)
+    khat_ch = np.asarray(khat_ch, np.float64)
+    bhat_ch = np.asarray(bhat_ch, np.float64)
+    d = qhat.shape[-1]
+    q_P = rope_rotate(qhat, np.asarray(pos_parent, np.float64)[..., None], base, pairs)     # [..., R, d]
+    q_c = rope_rotate(qhat, np.asarray(pos_children, np.float64)[..., None], base, pairs)   # [..., C, R, d]
+    F_c = np.sum(khat_ch * q_c, axis=-1) / np.sqrt(d) + bhat_ch                # [..., C, R]
+    corr = np.sum(khat_ch * (q_P[..., None, :, :] - q_c), axis=-1) / np.sqrt(d)
+    u = F_c + corr
+    F, khat = combine_log_masses(np.swapaxes(u, -1, -2), np.moveaxis(khat_ch, -3, -2))
+    bhat = F - np.sum(khat * q_P, axis=-1) / np.sqrt(d)
+    return khat, bhat
+
+
+def build_tree_rope(K: np.ndarray, qhat: np.ndarray, chunk: int, levels: int, n_tokens: int,
+                    base: float, pairs: int) -> OracleTree:
+    """``build_tree`` for a model with rotary positions: level-1 summaries at
+    each chunk's rotated reference queries, upper levels by
+    ``merge_children_rope``. [ZHA: 무엇과 다른가]"""
+    K = np.asarray(K, np.float64)
+    qhat = np.asarray(qhat, np.float64)
+    d = K.shape[1]
+    tree = OracleTree(chunk=chunk, levels=levels, n_tokens=int(n_tokens), qhat=qhat)
+    n1 = tree.n_nodes(1)
+    Kc = K[: n1 * chunk].reshape(n1, chunk, d)
+    tree.nodes[1] = summarise_chunk_rope(qhat, Kc, node_position(1, np.arange(n1), chunk), base, pairs)
+    for lvl in range(2, levels + 1):
+        n_here = tree.n_nodes(lvl)
+        kh, bh = tree.nodes[lvl - 1]
+        kh = kh[: n_here * chunk].reshape(n_here, chunk, *kh.shape[1:])
+        bh = bh[: n_here * chunk].reshape(n_here, chunk, bh.shape[-1])
+        par = np.arange(n_here)
+        ch = par[:, None] * chunk + np.arange(chunk)[None, :]
+        tree.nodes[lvl] = merge_children_rope(qhat, kh, bh, node_position(lvl, par, chunk),
+                                              node_position(lvl - 1, ch, chunk), base, pairs)
     return tree
 
 

@@ -478,3 +478,100 @@ def test_top_k_route_keeps_the_budget_at_every_level():
                 for b in lt.candidates:
                     if int(b) not in kept:
                         assert not _precedes(lt.sigma, lt.candidates, pos[int(b)], pos[a])
+
+
+# ---------------------------------------------------------------------------
+# Rotary positions: summaries at rotated reference queries and the merge's
+# correction term [ZHA: 무엇과 다른가; Attention: "Attention 은 순서를 모르므로
+# 위치 정보를 따로 넣는다"]
+# ---------------------------------------------------------------------------
+
+def test_rope_inner_product_depends_only_on_the_offset():
+    """The Attention page: rotating q by m theta and k by n theta leaves an
+    inner product that depends on (m - n) theta alone; rotations keep norms;
+    no rotated pair (or position 0) is the identity."""
+    rng = np.random.default_rng(31)
+    for d, pairs in ((8, 4), (16, 5), (64, 32)):
+        q, k = rng.standard_normal(d), rng.standard_normal(d)
+        for m, n in ((7, 3), (1000, 999), (5, 5), (0, 12)):
+            a = O.rope_rotate(q, m, 10000.0, pairs) @ O.rope_rotate(k, n, 10000.0, pairs)
+            b = O.rope_rotate(q, m - n, 10000.0, pairs) @ k
+            assert abs(a - b) < 1e-10 * (1 + abs(a))
+        assert abs(np.linalg.norm(O.rope_rotate(q, 123, 500.0, pairs)) - np.linalg.norm(q)) < 1e-12
+        assert np.array_equal(O.rope_rotate(q, 0, 10000.0, pairs), q)
+        assert np.allclose(O.rope_rotate(q, 77, 10000.0, 0), q, rtol=0, atol=0)
+    # partial rotation: pairs past `pairs` are untouched
+    x = rng.standard_normal(16)
+    y = O.rope_rotate(x, 9, 10000.0, 3)
+    assert np.array_equal(y[6:], x[6:]) and not np.allclose(y[:6], x[:6])
+
+
+def test_rope_tree_without_rotated_pairs_is_the_position_free_tree():
+    rng = np.random.default_rng(32)
+    K = rng.standard_normal((4 * 16 + 3, 8))
+    qhat = rng.standard_normal((3, 8))
+    a = O.build_tree_rope(K, qhat, 4, 3, K.shape[0], 10000.0, 0)
+    b = O.build_tree(K, qhat, 4, 3, K.shape[0])
+    for lvl in (1, 2, 3):
+        assert np.allclose(a.nodes[lvl][0], b.nodes[lvl][0], rtol=0, atol=1e-12)
+        assert np.allclose(a.nodes[lvl][1], b.nodes[lvl][1], rtol=0, atol=1e-12)
+
+
+def test_rope_level1_plane_is_exact_at_the_rotated_reference_query():
+    """t_{r,c}(q_hat_{r,c}) = F_c(q_hat_{r,c}) with q_hat_{r,c} = rotate(q_hat_r, pos_c),
+    and the summary equals the position-free one taken in the chunk's frame:
+    khat = rotate(khat', pos) for keys rotated back by -pos."""
+    rng = np.random.default_rng(33)
+    qhat = rng.standard_normal((4, 16)) * 2
+    Kc = rng.standard_normal((8, 16))
+    for pos in (0, 5, 4096, 1 << 20):
+        kh, bh = O.summarise_chunk_rope(qhat, Kc, pos, 10000.0, 8)
+        q_rot = O.rope_rotate(qhat, pos, 10000.0, 8)
+        t = np.sum(kh * q_rot, axis=-1) / 4.0 + bh
+        assert np.allclose(t, O.chunk_log_mass(q_rot, Kc), rtol=0, atol=1e-12)
+        kh0, bh0 = O.summarise_chunk(qhat, O.rope_rotate(Kc, -pos, 10000.0, 8))
+        assert np.allclose(kh, O.rope_rotate(kh0, pos, 10000.0, 8), rtol=0, atol=1e-10)
+        assert np.allclose(bh, bh0, rtol=0, atol=1e-10)
+
+
+def test_rope_merge_of_single_key_children_is_exact():
+    """A child whose keys are all the same key k has F_c(q) = log C + q.k/sqrt(d),
+    a linear function, so its plane is exact at every query and the corrected
+    merge equals the direct summary of all the parent's keys at the parent's
+    rotated reference query."""
+    rng = np.random.default_rng(34)
+    C, d, R = 4, 16, 3
+    qhat = rng.standard_normal((R, d))
+    for P in (0, 1, 37):
+        child_keys = rng.standard_normal((C, d)) * 2
+        K = np.repeat(child_keys, C, axis=0)                           # C children of C equal keys
+        pos_ch = O.node_position(1, P * C + np.arange(C), C)
+        kh_c, bh_c = O.summarise_chunk_rope(qhat, K.reshape(C, C, d), pos_ch, 10000.0, d // 2)
+        kh, bh = O.merge_children_rope(qhat, kh_c, bh_c, O.node_position(2, P, C), pos_ch, 10000.0, d // 2)
+        kd, bd = O.summarise_chunk_rope(qhat, K, O.node_position(2, P, C), 10000.0, d // 2)
+        assert np.allclose(kh, kd, rtol=0, atol=1e-10) and np.allclose(bh, bd, rtol=0, atol=1e-10)
+
+
+def test_rope_merge_correction_is_second_order_in_the_rotation():
+    """For a general child, the corrected log mass at the parent's rotated
+    reference query differs from the true F_c there by O(angle^2): halving the
+    position offset divides the error by ~4. Without the correction term the
+    error is first order (halving divides it by ~2)."""
+    rng = np.random.default_rng(35)
+    d, R = 16, 2
+    qhat = rng.standard_normal((R, d)) * 2
+    Kc = rng.standard_normal((8, d)) * 1.5
+    errs, errs_plain = [], []
+    for t in (0.02, 0.01, 0.005):
+        kh_c, bh_c = O.summarise_chunk_rope(qhat, Kc[None], np.array([t]), 1.0, d // 2)   # base 1: theta = 1
+        kh, bh = O.merge_children_rope(qhat, kh_c, bh_c, 0.0, np.array([t]), 1.0, d // 2)
+        F_P = bh + np.sum(kh * qhat, axis=-1) / 4.0                    # parent at position 0: q_hat_P = q_hat
+        true = O.chunk_log_mass(qhat, Kc)
+        errs.append(np.max(np.abs(F_P - true)))
+        q_c = O.rope_rotate(qhat, t, 1.0, d // 2)
+        plain = np.sum(kh_c[0] * q_c, axis=-1) / 4.0 + bh_c[0]          # F_c at its own query, uncorrected
+        errs_plain.append(np.max(np.abs(plain - true)))
+    for a, b in zip(errs, errs[1:]):
+        assert 3.5 < a / b < 4.5
+    for a, b in zip(errs_plain, errs_plain[1:]):
+        assert 1.7 < a / b < 2.3
