@@ -64,6 +64,10 @@ static zha_status make_geom(const zha_config* c, zha::Geom* g, size_t* bytes) {
   if (c->kv_dtype != ZHA_F32 && c->kv_dtype != ZHA_BF16)
     return fail(ZHA_ERR_INVALID, "kv_dtype %d unknown", c->kv_dtype);
   if (c->reserved != 0) return fail(ZHA_ERR_INVALID, "reserved must be 0");
+  if (c->rope_pairs < 0 || c->rope_pairs > c->head_dim / 2)
+    return fail(ZHA_ERR_INVALID, "rope_pairs %d outside [0, head_dim / 2]", c->rope_pairs);
+  if (c->rope_pairs > 0 && !(c->rope_base > 1.f && std::isfinite(c->rope_base)))
+    return fail(ZHA_ERR_INVALID, "rope_base must be finite and > 1 with rotary positions");
   if (c->max_tokens < 1 || c->max_tokens > (int64_t(1) << 34))
     return fail(ZHA_ERR_INVALID, "max_tokens %lld out of range", (long long)c->max_tokens);
   zha::Geom G{};
@@ -78,6 +82,8 @@ static zha_status make_geom(const zha_config* c, zha::Geom* g, size_t* bytes) {
   G.kv_bf16 = c->kv_dtype == ZHA_BF16;
   G.scale = float(1.0 / std::sqrt(double(c->head_dim)));
   G.max_tokens = c->max_tokens;
+  G.rope_pairs = c->rope_pairs;
+  G.rope_log2_base = c->rope_pairs > 0 ? std::log2(double(c->rope_base)) : 0.0;
   int64_t off = 0;
   for (int l = 1; l <= G.levels; ++l) {
     G.cap[l] = zha::nodes_at(c->max_tokens, c->chunk, l);

@@ -30,9 +30,10 @@ __host__ __device__ inline int l1_chunks_per_tile(int chunk) { return kL1Tokens 
 
 template <int D>
 __host__ __device__ inline size_t l1_smem_bytes(int nref) {
-  // keys [128][D+4], reference queries [R][D+4], scores [R][128], F [R][128/C] (<= R*64)
+  // keys [128][D+4], reference queries [R][D+4], scores [R][128], F [R][128/C] (<= R*64),
+  // rotations of the tile's chunks [128/C][D/2] (cos, sin) (<= 64 chunks)
   return sizeof(float) * (size_t(kL1Tokens) * (D + 4) + size_t(nref) * (D + 4) +
-                          size_t(nref) * kL1Tokens + size_t(nref) * 64);
+                          size_t(nref) * kL1Tokens + size_t(nref) * 64 + size_t(64) * D);
 }
 
 template <typename T, int D>
@@ -47,8 +48,10 @@ __device__ void summarise_tile(const Geom& G, int g, const T* __restrict__ K, in
   float* qs = ks + kL1Tokens * DP;        // [R][DP]
   float* ss = qs + R * DP;                // [R][128]
   float* fs = ss + R * kL1Tokens;         // [R][nch]
+  float2* rot = reinterpret_cast<float2*>(fs + R * 64);   // [nch][D/2] (cos, sin) of the chunk start
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nwarps = blockDim.x >> 5;
+  const int RP = G.rope_pairs;
 
   // Stage keys (16-byte vectors, coalesced) and reference queries.
   {
@@ -68,8 +71,28 @@ __device__ void summarise_tile(const Geom& G, int g, const T* __restrict__ K, in
       *reinterpret_cast<float4*>(qs + row * DP + col) =
           *reinterpret_cast<const float4*>(qb + int64_t(row) * D + col);
     }
+    for (int v = tid; v < nch * RP; v += blockDim.x) {
+      const int cl = v / RP, i = v % RP;
+      float c, s;
+      rope_cos_sin(G, (c0 + cl) * C, i, &c, &s);
+      rot[cl * (D / 2) + i] = make_float2(c, s);
+    }
   }
   __syncthreads();
+  // Rotary positions: the chunk's summaries at the reference queries turned to
+  // the chunk's position equal the position-free summaries of the keys turned
+  // back by that position (then khat is turned forward again, below).
+  if (RP > 0) {
+    for (int v = tid; v < TT * RP; v += blockDim.x) {
+      const int t = v / RP, i = v % RP;
+      const float2 cs = rot[(t / C) * (D / 2) + i];
+      float* k2 = ks + t * DP + 2 * i;
+      const float a = k2[0], b = k2[1];
+      k2[0] = a * cs.x + b * cs.y;
+      k2[1] = b * cs.x - a * cs.y;
+    }
+    __syncthreads();
+  }
 
   // Scores: warp w takes plane pairs (2w, 2w+1), lane takes tokens lane + 32i.
   for (int rp = warp; 2 * rp < R; rp += nwarps) {
@@ -129,6 +152,16 @@ __device__ void summarise_tile(const Geom& G, int g, const T* __restrict__ K, in
 #pragma unroll
     for (int e = 0; e < EPL; ++e) dot += acc[e] * qs[r * DP + EPL * lane + e];
     dot = warp_sum(dot);
+#pragma unroll
+    for (int e = 0; e < EPL; e += 2) {            // khat back into the keys' frame
+      const int i = (EPL * lane + e) / 2;
+      if (i < RP) {
+        const float2 cs = rot[cl * (D / 2) + i];
+        const float a = acc[e], b = acc[e + 1];
+        acc[e] = a * cs.x - b * cs.y;
+        acc[e + 1] = a * cs.y + b * cs.x;
+      }
+    }
     float* rec = store + G.off[1] + (int64_t(g) * G.cap[1] + c0 + cl) * G.node_floats;
 #pragma unroll
     for (int e = 0; e < EPL; ++e) rec[r * D + EPL * lane + e] = acc[e];
@@ -165,6 +198,20 @@ __device__ void merge_item(const Geom& G, int g, int level, int64_t parent, int 
   const int C = G.chunk, R = G.nref;
   float q[EPL];
   load_slice<EPL>(refq + (int64_t(g) * R + r) * D, EPL * lane, q);
+  // Rotary positions: the children are re-evaluated at the parent's rotated
+  // reference query (its plane at that query: the tangent value at the child's
+  // own rotated query plus the correction 1/sqrt(d) <khat_c, q_P - q_c>).
+#pragma unroll
+  for (int e = 0; e < EPL; e += 2) {
+    const int i = (EPL * lane + e) / 2;
+    if (i < G.rope_pairs) {
+      float c, s;
+      rope_cos_sin(G, parent * span_of(C, level), i, &c, &s);
+      const float a = q[e], b = q[e + 1];
+      q[e] = a * c - b * s;
+      q[e + 1] = a * s + b * c;
+    }
+  }
   const float* child0 = store + G.off[level - 1] +
                         (int64_t(g) * G.cap[level - 1] + parent * C) * G.node_floats;
   float m = -INFINITY, l = 0.f, acc[EPL] = {};

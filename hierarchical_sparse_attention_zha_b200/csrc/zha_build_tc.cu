@@ -302,7 +302,7 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
 cudaError_t launch_build_level1_tc(const Geom& G, const void* K, int64_t ld, int64_t c_begin,
                                    int64_t c_end, const float* refq, float* store, int32_t* status,
                                    cudaStream_t s) {
-  if (!(G.kv_bf16 && G.d == bD && G.nref == bR && G.chunk == 64))
+  if (!(G.kv_bf16 && G.d == bD && G.nref == bR && G.chunk == 64 && G.rope_pairs == 0))
     return cudaErrorNotSupported;
   if (c_end <= c_begin) return cudaSuccess;
   const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();

@@ -21,6 +21,8 @@ struct Geom {
   int32_t hkv, hq, group, d, chunk, levels, nref, node_floats;
   int32_t kv_bf16;
   float scale;                           // 1 / sqrt(d)
+  int32_t rope_pairs;                    // rotated element pairs (0: position-free)
+  double rope_log2_base;                 // log2 of the rotation base
   int64_t max_tokens;
   int64_t cap[ZHA_MAX_LEVELS + 2];       // node capacity per KV head, index by level
   int64_t off[ZHA_MAX_LEVELS + 2];       // float offset of level l's [hkv][cap][node] block
@@ -31,6 +33,25 @@ struct Geom {
 // 256-byte block that follows the summary levels in the store.
 __host__ __device__ inline int32_t* tree_status_word(const Geom& g, float* store) {
   return reinterpret_cast<int32_t*>(store + g.status_off);
+}
+
+// Rotation of element pair i at position pos: angle pos * base^(-2i/d),
+// formed and reduced modulo 2 pi in double precision (positions reach 2^34),
+// then turned into the cosine and sine. Pairs from G.rope_pairs on do not turn.
+__device__ __forceinline__ void rope_cos_sin(const Geom& G, int64_t pos, int pair, float* c, float* s) {
+  if (pair >= G.rope_pairs || pos == 0) {
+    *c = 1.f;
+    *s = 0.f;
+    return;
+  }
+  const double theta = exp2(-2.0 * double(pair) / double(G.d) * G.rope_log2_base);
+  const double two_pi = 6.283185307179586476925286766559;
+  double ang = double(pos) * theta;
+  ang -= two_pi * floor(ang / two_pi);
+  double sd, cd;
+  sincos(ang, &sd, &cd);
+  *c = float(cd);
+  *s = float(sd);
 }
 
 // C^l, saturating at a value above any token count.

@@ -67,7 +67,8 @@ class Config(ctypes.Structure):
     _fields_ = [
         ("n_kv_heads", c_int32), ("n_q_heads", c_int32), ("head_dim", c_int32),
         ("chunk", c_int32), ("levels", c_int32), ("n_ref", c_int32),
-        ("kv_dtype", c_int32), ("reserved", c_int32), ("max_tokens", c_int64),
+        ("kv_dtype", c_int32), ("rope_pairs", c_int32), ("max_tokens", c_int64),
+        ("rope_base", c_float), ("reserved", c_int32),
     ]
 
 
@@ -101,6 +102,8 @@ def _load() -> ctypes.CDLL:
         "zha_attend_workspace_bytes": (c_size_t, [POINTER(Config), c_int32, c_int64]),
         "zha_sparse_attend": (c_int32, [P, P, P, P, c_int64, c_int64, c_int32, P, P, c_int32, P,
                                         P, P, c_size_t, P, P]),
+        "zha_diagnostics_workspace_bytes": (c_size_t, [POINTER(Config), c_int32, c_int64]),
+        "zha_route_diagnostics": (c_int32, [P, P, P, c_int64, c_int32, c_int64, P, P, P, c_size_t, P]),
         "zha_trace_enable": (c_int32, [c_int32, c_char_p, c_int32]),
         "zha_trace_count": (c_int32, []),
         "zha_trace_dropped": (c_int32, []),
@@ -168,9 +171,12 @@ def trace_clear() -> None:
 
 
 def make_config(n_kv_heads: int, n_q_heads: int, head_dim: int, chunk: int, levels: int,
-                n_ref: int, kv_dtype: torch.dtype, max_tokens: int) -> Config:
+                n_ref: int, kv_dtype: torch.dtype, max_tokens: int, rope_pairs: int = 0,
+                rope_base: float = 10000.0) -> Config:
+    """zha_config; rope_pairs > 0 declares rotary positions (see zha.h)."""
     dt = {torch.float32: ZHA_F32, torch.bfloat16: ZHA_BF16}[kv_dtype]
-    return Config(n_kv_heads, n_q_heads, head_dim, chunk, levels, n_ref, dt, 0, max_tokens)
+    return Config(n_kv_heads, n_q_heads, head_dim, chunk, levels, n_ref, dt, rope_pairs, max_tokens,
+                  rope_base if rope_pairs > 0 else 0.0, 0)
 
 
 def tree_bytes(cfg: Config) -> int:
@@ -272,6 +278,21 @@ class Tree:
                                 max_sel, ptr(kept_bits), ptr(ws), ws.numel() * ws.element_size(),
                                 ptr(status), stream_ptr(stream)), "zha_route")
         return chunk_ids, n_chunks
+
+    def diagnostics(self, Q: torch.Tensor, K: torch.Tensor, n_tokens: int, usage: bool = True,
+                    stream=None):
+        """zha_route_diagnostics: (kl [L, B, Hq] float32, usage [L, R] int64 or None)."""
+        self._kv(K)
+        B = Q.shape[0]
+        L = self.cfg.levels
+        kl = torch.empty(L, B, self.cfg.n_q_heads, dtype=torch.float32, device=self.device)
+        use = torch.zeros(L, self.cfg.n_ref, dtype=torch.int32, device=self.device) if usage else None
+        ws = _bytes_tensor(int(lib.zha_diagnostics_workspace_bytes(byref(self.cfg), B, n_tokens)),
+                           self.device)
+        check(lib.zha_route_diagnostics(self.handle, ptr(Q), ptr(K), K.shape[1], B, n_tokens, ptr(kl),
+                                        ptr(use), ptr(ws), ws.numel() * 4, stream_ptr(stream)),
+              "zha_route_diagnostics")
+        return kl, (use.to(torch.int64) if use is not None else None)
 
     def sparse_attend(self, Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, n_tokens: int,
                       chunk_ids: torch.Tensor, n_chunks: torch.Tensor,

@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define ZHA_ABI_VERSION 1
+#define ZHA_ABI_VERSION 2
 
 typedef enum {
     ZHA_OK = 0,
@@ -71,9 +71,25 @@ typedef struct {
     int32_t levels;      /* L: summary levels, 1..8; level l covers C^l tokens */
     int32_t n_ref;       /* R: reference queries per tree, 1..32 */
     int32_t kv_dtype;    /* zha_dtype of the K and V caches */
-    int32_t reserved;    /* must be 0 */
+    int32_t rope_pairs;  /* rotary positions: 0 = none (position-free keys); else the number
+                            of leading element pairs (2i, 2i+1), 1..head_dim/2, that the
+                            model turns by position * rope_base^(-2i/head_dim) */
     int64_t max_tokens;  /* tokens the summary store must cover, >= 1 */
+    float rope_base;     /* rotation base (> 1) when rope_pairs > 0; ignored otherwise */
+    int32_t reserved;    /* must be 0 */
 } zha_config;
+
+/* Rotary positions [ZHA: 무엇과 다른가; Attention: "Attention 은 순서를 모르므로 위치
+ * 정보를 따로 넣는다"]: with rope_pairs > 0 the caches hold keys as the model
+ * rotates them (key of position m turned by m * theta_i per pair i) and decode
+ * queries come rotated at their own position. The summaries are then taken at
+ * rotated reference queries: node n of level l sits at the position of its
+ * first token, p_n = n * C^l, and its reference queries are q_hat_r rotated by
+ * p_n. A parent re-evaluates each child c at its own rotated reference query
+ * q_hat_{r,P}: u_c = F_c(q_hat_{r,c}) + 1/sqrt(d) <khat_{r,c}, q_hat_{r,P} -
+ * q_hat_{r,c}>, which is the child's plane evaluated at q_hat_{r,P}. khat is
+ * stored in the keys' (rotated) frame, so routing and attention use the
+ * decode queries as they come. */
 
 typedef struct zha_tree zha_tree; /* opaque host handle; holds no device memory */
 
@@ -256,6 +272,28 @@ zha_status zha_sparse_attend(const zha_tree* tree, const float* d_Q, const void*
                              const int32_t* d_chunk_ids, const int32_t* d_n_chunks,
                              int32_t max_sel, float* d_O, float* d_lse, void* d_ws,
                              size_t ws_bytes, int32_t* d_status, void* stream);
+
+/* ---- Routing diagnostics [ZHA: 어떻게 쓰나; 전제와 한계] -----------------------
+ * How well each level's estimate follows the dense attention mass, for
+ * `batch` queries d_Q [batch][n_q_heads][d] against the tree and the keys d_K
+ * [n_kv_heads][ld][d] at n_tokens (the tree must cover C*floor(n_tokens/C),
+ * else ZHA_ERR_STATE). For every level l and query head:
+ *   target p_{l}(n) = the dense softmax weights of q over the keys the level's
+ *     complete nodes cover, summed node by node (the reference queries' KL
+ *     training target [ZHA: 어떻게 쓰나]; the in-progress tail is in no node);
+ *   estimate p_hat_{l}(n) = softmax over the level's nodes of max_r t_r(q);
+ *   d_kl[l-1][batch][n_q_heads] = KL(p_l || p_hat_l) (float32, natural log).
+ * d_usage (nullable, uint32 [L][n_ref], ACCUMULATED -- the caller zeroes it):
+ * for every node of every level and every query head, +1 at the plane r that
+ * gives the node's score (lowest r on ties); [ZHA: 전제와 한계] reports that
+ * few reference queries serve the upper levels and that their use evens out
+ * towards the leaves. Every node of every level is scored and the dense mass of
+ * every complete chunk is formed, so this costs a dense pass over the keys: a
+ * diagnostic, not part of routing. d_ws: >= zha_diagnostics_workspace_bytes. */
+size_t zha_diagnostics_workspace_bytes(const zha_config* cfg, int32_t batch, int64_t n_tokens);
+zha_status zha_route_diagnostics(const zha_tree* tree, const float* d_Q, const void* d_K, int64_t ld,
+                                 int32_t batch, int64_t n_tokens, float* d_kl, uint32_t* d_usage,
+                                 void* d_ws, size_t ws_bytes, void* stream);
 
 /* ---- Kernel timing (profiling; the pages have no counterpart) ------------
  * While enabled, every kernel the library launches whose name contains

@@ -38,4 +38,8 @@ from .zha_oracle import (  # noqa: F401
     leaf_token_set,
     attend,
     captured_mass,
+    level_target_mass,
+    level_estimate,
+    level_kl,
+    plane_usage,
 )

@@ -556,6 +556,49 @@ def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray,
     return O[0], float(logsumexp(s))
 
 
+# ----------------------------------------------------------------------------
+# Routing diagnostics   [ZHA: 어떻게 쓰나; 전제와 한계]
+# ----------------------------------------------------------------------------
+
+def level_target_mass(q: np.ndarray, K: np.ndarray, tree: OracleTree, level: int) -> np.ndarray:
+    """Target distribution p_{l,C}(q) over the complete nodes of `level`:
+    the dense attention weights of q over the keys, summed node by node.
+    [ZHA: 어떻게 쓰나] (the target of the reference queries' KL training).
+    Reading: the weights are taken over the keys the level's nodes cover and
+    normalised over the nodes (keys of the in-progress tail are in no node)."""
+    n_l = tree.n_nodes(level)
+    span = tree.chunk ** level
+    A, _ = sdpa(np.asarray(q, np.float64)[None], np.asarray(K, np.float64)[: n_l * span],
+                np.zeros((n_l * span, 1)))
+    return A[0].reshape(n_l, span).sum(axis=1)
+
+
+def level_estimate(q: np.ndarray, tree: OracleTree, level: int) -> np.ndarray:
+    """Estimate p_hat_{l,C}(q): softmax over the level's nodes of their scores
+    max_r t_r(q). [ZHA: 어떻게 쓰나]"""
+    khat, bhat = tree.nodes[level]
+    sigma = node_score(q, khat, bhat)
+    return np.exp(sigma - logsumexp(sigma))
+
+
+def level_kl(q: np.ndarray, K: np.ndarray, tree: OracleTree, level: int) -> float:
+    """KL(p_{l,C}(q) || p_hat_{l,C}(q)) over the level's nodes. [ZHA: 어떻게 쓰나]"""
+    p = level_target_mass(q, K, tree, level)
+    ph = level_estimate(q, tree, level)
+    nz = p > 0
+    return float(np.sum(p[nz] * (np.log(p[nz]) - np.log(ph[nz]))))
+
+
+def plane_usage(q: np.ndarray, tree: OracleTree, level: int) -> np.ndarray:
+    """How often each reference query gives a node's score: for every node of
+    the level the plane r attaining max_r t_r(q) (lowest r on ties), counted
+    per r. [ZHA: 전제와 한계] reports that few reference queries serve the upper
+    levels and the use evens out towards the leaves."""
+    khat, bhat = tree.nodes[level]
+    t = tangent_planes(q, khat, bhat)                    # [n, R]
+    return np.bincount(np.argmax(t, axis=-1), minlength=khat.shape[-2])
+
+
 def captured_mass(q: np.ndarray, K: np.ndarray, tokens: np.ndarray,
                   n_tokens: int) -> float:
     """Share of the dense attention mass over [0, n_tokens) that S holds.

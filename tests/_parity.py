@@ -42,11 +42,12 @@ def to_device(inp: W.Inputs, device="cuda"):
     return K, V, torch.from_numpy(inp.ref_q).to(device), torch.from_numpy(inp.Q).to(device)
 
 
-def config_for(spec: W.Workload, max_tokens: int | None = None):
+def config_for(spec: W.Workload, max_tokens: int | None = None, rope_pairs: int = 0,
+               rope_base: float = 10000.0):
     from hierarchical_sparse_attention_zha_b200 import zha
     return zha.make_config(spec.n_kv_heads, spec.n_q_heads, spec.head_dim, spec.chunk, spec.levels,
                            spec.n_ref, torch.bfloat16 if spec.kv_dtype == "bf16" else torch.float32,
-                           max_tokens or spec.capacity)
+                           max_tokens or spec.capacity, rope_pairs=rope_pairs, rope_base=rope_base)
 
 
 def summary_errors(kh_gpu: np.ndarray, bh_gpu: np.ndarray, kh_ref: np.ndarray, bh_ref: np.ndarray):

@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(zha):
 
 
 def test_version_and_status_strings(zha):
-    assert zha.lib.zha_abi_version() == 1
+    assert zha.lib.zha_abi_version() == 2
     assert zha.status_str(0) == "ok"
     assert "state" in zha.status_str(zha.ZHA_ERR_STATE)
     assert zha.status_str(-99) == "unknown status"
@@ -212,3 +212,18 @@ def test_route_ex_rejects_bad_policies_before_any_launch(zha):
         assert zha.launch_count() == before
     finally:
         zha.lib.zha_tree_destroy(handle)
+
+
+def test_rotary_config_is_validated(zha):
+    """rope_pairs in [0, head_dim / 2]; a base > 1 (finite) when rope_pairs > 0;
+    the base is ignored without rotated pairs."""
+    assert zha.tree_bytes(_cfg(zha, rope_pairs=64, rope_base=10000.0)) > 0
+    assert zha.tree_bytes(_cfg(zha, rope_pairs=65, rope_base=10000.0)) == 0
+    assert zha.tree_bytes(_cfg(zha, rope_pairs=-1)) == 0
+    assert zha.tree_bytes(_cfg(zha, rope_pairs=8, rope_base=1.0)) == 0
+    assert zha.tree_bytes(_cfg(zha, rope_pairs=8, rope_base=float("inf"))) == 0
+    cfg = _cfg(zha)
+    cfg.rope_base = -3.0                  # no rotated pairs: not read
+    assert zha.tree_bytes(cfg) > 0
+    # the rotary fields do not change the store's size
+    assert zha.tree_bytes(_cfg(zha, rope_pairs=64, rope_base=10000.0)) == zha.tree_bytes(_cfg(zha))

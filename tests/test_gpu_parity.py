@@ -62,7 +62,7 @@ def run_pipeline(zha, inp, n_tokens, p=None, max_sel=None, batch_index=0, stream
 
 
 def check_case(zha, inp, n_tokens, p=None, heads=None, all_nodes=True, batch_index=0, tree=None,
-               dev=None, oracle_p=None):
+               dev=None, oracle_p=None, oracle_build=None):
     """Full comparison; returns the route report. ``p`` goes to the GPU route
     (a mass or a zha.RoutePolicy), ``oracle_p`` (default: ``p``) to the oracle's."""
     spec = inp.spec
@@ -76,7 +76,8 @@ def check_case(zha, inp, n_tokens, p=None, heads=None, all_nodes=True, batch_ind
     for g in range(spec.n_kv_heads):
         Kf = cache_f64(inp, g, n_tokens)
         Vf = values_f64(inp, g, n_tokens)
-        otree = O.build_tree(Kf, inp.ref_q[g], spec.chunk, spec.levels, n_tokens)
+        build = oracle_build or O.build_tree
+        otree = build(Kf, inp.ref_q[g], spec.chunk, spec.levels, n_tokens)
         # summaries, every level
         for lvl in range(1, spec.levels + 1):
             n_l = otree.n_nodes(lvl)
@@ -505,3 +506,110 @@ def test_route_policies_match_the_oracle(zha, parity_log, case):
     if mode == "top_k":
         res = run_pipeline(zha, inp, 65536 + 21, p=gpu_p)
         assert (res["cnt"] <= vals[0]).all()
+
+
+# ---------------------------------------------------------------------------
+# Rotary positions [ZHA: 무엇과 다른가]: summaries at rotated reference queries,
+# the merge's correction term; routing and attention unchanged
+# ---------------------------------------------------------------------------
+
+ROPE_CASES = {
+    "f32_d64_full": (W.scaled("tiny", n_tokens=3000, chunk=8, levels=3, n_ref=4, batch=3,
+                              n_needles=0), 2990, 32, 10000.0),
+    "bf16_d128_partial": (W.scaled("1m", n_kv_heads=2, n_q_heads=16, n_tokens=8192, stream_tokens=128,
+                                   levels=2, batch=2, n_needles=2), 8192 + 77, 16, 10000.0),
+    "bf16_c4_deep": (W.scaled("deep", n_kv_heads=1, n_q_heads=4, n_tokens=4096, levels=4, batch=2),
+                     4096 + 3, 64, 500000.0),
+    "bf16_262k_positions": (W.scaled("1m", n_kv_heads=1, n_q_heads=8, n_tokens=262144,
+                                     stream_tokens=128, n_needles=4), 262144 + 100, 64, 10000.0),
+}
+
+
+@pytest.mark.parametrize("name", list(ROPE_CASES))
+def test_rotary_positions_match_the_oracle(zha, parity_log, name):
+    """Every summary of every level against the oracle's build with rotated
+    reference queries (norm-wise 1e-4), then routing and attention on that tree."""
+    spec, n_tokens, pairs, base = ROPE_CASES[name]
+    inp = W.generate(spec)
+    dev = to_device(inp)
+    tree = zha.Tree(config_for(spec, rope_pairs=pairs, rope_base=base), dev[2])
+    tree.build(dev[0], n_tokens)
+    build = lambda K, q, C, L, n: O.build_tree_rope(K, q, C, L, n, base, pairs)
+    rep = check_case(zha, inp, n_tokens, tree=tree, dev=dev, oracle_build=build)
+    parity_log(f"rope_{name}", rep)
+
+
+def test_rotary_positions_append_matches_the_oracle(zha):
+    """Appends with rotary positions (one chunk per call across a level-2
+    boundary, then a bulk append) against the oracle's build."""
+    spec = W.scaled("1m", n_kv_heads=1, n_q_heads=8, n_tokens=64 * 70, stream_tokens=0, levels=2,
+                    batch=2, n_needles=0)
+    inp = W.generate(spec)
+    K, V, refq, Q = to_device(inp)
+    tree = zha.Tree(config_for(spec, rope_pairs=48, rope_base=10000.0), refq)
+    tree.build(K, 64 * 61 + 3)
+    for n in range(64 * 61 + 4, 64 * 66 + 1):
+        tree.append_chunk(K, n)
+    tree.append_chunk(K, 64 * 70)                     # 4 chunks in one call
+    torch.cuda.synchronize()
+    otree = O.build_tree_rope(cache_f64(inp, 0, 64 * 70), inp.ref_q[0], 64, 2, 64 * 70, 10000.0, 48)
+    for lvl in (1, 2):
+        n_l = otree.n_nodes(lvl)
+        kh, bh = tree.level(lvl)
+        ek, eb = summary_errors(kh[0, :n_l].cpu().numpy().astype(np.float64),
+                                bh[0, :n_l].cpu().numpy().astype(np.float64), *otree.nodes[lvl])
+        assert ek <= SUMMARY_RTOL and eb <= SUMMARY_RTOL, (lvl, ek, eb)
+
+
+# ---------------------------------------------------------------------------
+# Routing diagnostics [ZHA: 어떻게 쓰나; 전제와 한계]
+# ---------------------------------------------------------------------------
+
+DIAG_CASES = {
+    "f32_d64": (W.scaled("tiny", n_tokens=2048, n_needles=2, batch=4), 2048 - 3, 0),
+    "bf16_c64": (W.scaled("1m", n_kv_heads=2, n_q_heads=16, n_tokens=8192, stream_tokens=128, levels=2,
+                          batch=2, n_needles=2), 8192 + 77, 0),
+    "bf16_rope_c4": (W.scaled("deep", n_kv_heads=1, n_q_heads=4, n_tokens=4096, levels=4, batch=2),
+                     4096 + 3, 64),
+}
+
+
+@pytest.mark.parametrize("name", list(DIAG_CASES))
+def test_route_diagnostics_match_the_oracle(zha, name):
+    """KL(target || estimate) per level and head against the oracle's fp64
+    value: |dKL| <= 2e-4 + 2e-3 KL (fp32 log-masses and scores, each within
+    ~1e-5 of the oracle's, move KL by a few 1e-5). Plane-usage counts per
+    level: identical except for nodes whose two best planes lie within 1e-5
+    (counted; each may move one count)."""
+    spec, n_tokens, pairs = DIAG_CASES[name]
+    inp = W.generate(spec)
+    K, V, refq, Q = to_device(inp)
+    tree = zha.Tree(config_for(spec, rope_pairs=pairs, rope_base=10000.0), refq)
+    tree.build(K, n_tokens)
+    kl, usage = tree.diagnostics(Q[0].contiguous(), K, n_tokens)
+    torch.cuda.synchronize()
+    kl, usage = kl.cpu().numpy(), usage.cpu().numpy()
+    G = spec.group
+    want = np.zeros_like(usage)
+    near = np.zeros(spec.levels, int)
+    for g in range(spec.n_kv_heads):
+        Kf = cache_f64(inp, g, n_tokens)
+        if pairs:
+            otree = O.build_tree_rope(Kf, inp.ref_q[g], spec.chunk, spec.levels, n_tokens, 10000.0, pairs)
+        else:
+            otree = O.build_tree(Kf, inp.ref_q[g], spec.chunk, spec.levels, n_tokens)
+        for b in range(spec.batch):
+            for h in range(g * G, (g + 1) * G):
+                q = inp.Q[0, b, h].astype(np.float64)
+                for lvl in range(1, spec.levels + 1):
+                    if otree.n_nodes(lvl) == 0:
+                        continue
+                    ref = O.level_kl(q, Kf, otree, lvl)
+                    assert abs(kl[lvl - 1, b, h] - ref) <= 2e-4 + 2e-3 * ref, (lvl, b, h, kl[lvl - 1, b, h], ref)
+                    want[lvl - 1] += O.plane_usage(q, otree, lvl)
+                    t = np.sort(O.tangent_planes(q, *otree.nodes[lvl]), axis=-1)
+                    if t.shape[-1] > 1:
+                        near[lvl - 1] += int(np.sum(t[:, -1] - t[:, -2] <= 1e-5))
+    for lvl in range(spec.levels):
+        assert np.abs(usage[lvl] - want[lvl]).sum() <= 2 * near[lvl], (lvl, usage[lvl], want[lvl], near[lvl])
+    assert usage.sum(axis=1)[0] == spec.batch * spec.n_q_heads * (n_tokens // spec.chunk)

@@ -575,3 +575,57 @@ def test_rope_merge_correction_is_second_order_in_the_rotation():
         assert 3.5 < a / b < 4.5
     for a, b in zip(errs_plain, errs_plain[1:]):
         assert 1.7 < a / b < 2.3
+
+
+# ---------------------------------------------------------------------------
+# Routing diagnostics [ZHA: 어떻게 쓰나; 전제와 한계]
+# ---------------------------------------------------------------------------
+
+def test_target_mass_sums_dense_weights_per_node_by_a_plain_loop():
+    """p_{l,C}: the dense softmax weights summed node by node (a loop over
+    nodes and keys with math.exp), normalised over the level's nodes."""
+    rng = np.random.default_rng(41)
+    K = rng.standard_normal((4 * 16 + 5, 6))
+    q = rng.standard_normal(6) * 2
+    tree = O.build_tree(K, rng.standard_normal((2, 6)), 4, 2, K.shape[0])
+    for lvl in (1, 2):
+        span = 4 ** lvl
+        n_l = tree.n_nodes(lvl)
+        w = [sum(math.exp(float(q @ K[j]) / math.sqrt(6)) for j in range(i * span, (i + 1) * span))
+             for i in range(n_l)]
+        ref = np.array(w) / sum(w)
+        assert np.allclose(O.level_target_mass(q, K, tree, lvl), ref, rtol=1e-12, atol=0)
+
+
+def test_kl_is_zero_when_every_chunk_repeats_one_key():
+    """A chunk of C copies of one key has F(q) = log C + q.k/sqrt(d), a linear
+    function: every plane is exact, the estimate equals the target at every
+    level, KL = 0. Random chunks give KL > 0."""
+    rng = np.random.default_rng(42)
+    keys = rng.standard_normal((4, 8)) * 2
+    K = np.repeat(keys, 16, axis=0)                    # every level-2 node (16 tokens) one key
+    qhat = rng.standard_normal((3, 8))
+    tree = O.build_tree(K, qhat, 4, 2, 64)
+    for _ in range(5):
+        q = rng.standard_normal(8) * 3
+        for lvl in (1, 2):
+            assert abs(O.level_kl(q, K, tree, lvl)) < 1e-12
+    K2 = rng.standard_normal((64, 8)) * 2
+    tree2 = O.build_tree(K2, qhat, 4, 2, 64)
+    assert O.level_kl(rng.standard_normal(8) * 3, K2, tree2, 1) > 1e-6
+
+
+def test_plane_usage_by_hand():
+    """Equal reference queries give equal planes: every node counts for r = 0.
+    A query equal to reference query r makes plane r exact (tangent) and the
+    others lower (convexity): at level 1 every node counts for r."""
+    rng = np.random.default_rng(43)
+    K = rng.standard_normal((64, 8))
+    same = np.repeat(rng.standard_normal((1, 8)), 3, axis=0)
+    tree = O.build_tree(K, same, 4, 2, 64)
+    assert list(O.plane_usage(rng.standard_normal(8), tree, 1)) == [16, 0, 0]
+    qhat = rng.standard_normal((3, 8)) * 2
+    tree = O.build_tree(K, qhat, 4, 2, 64)
+    for r in range(3):
+        u = O.plane_usage(qhat[r], tree, 1)
+        assert u[r] == 16 and u.sum() == 16
