@@ -518,8 +518,8 @@ ROPE_CASES = {
                               n_needles=0), 2990, 32, 10000.0),
     "bf16_d128_partial": (W.scaled("1m", n_kv_heads=2, n_q_heads=16, n_tokens=8192, stream_tokens=128,
                                    levels=2, batch=2, n_needles=2), 8192 + 77, 16, 10000.0),
-    "bf16_c4_deep": (W.scaled("deep", n_kv_heads=1, n_q_heads=4, n_tokens=4096, levels=4, batch=2),
-                     4096 + 3, 64, 500000.0),
+    "bf16_c4_deep": (W.scaled("deep", n_kv_heads=1, n_q_heads=4, n_tokens=4096, levels=4, batch=2,
+                              stream_tokens=16), 4096 + 3, 64, 500000.0),
     "bf16_262k_positions": (W.scaled("1m", n_kv_heads=1, n_q_heads=8, n_tokens=262144,
                                      stream_tokens=128, n_needles=4), 262144 + 100, 64, 10000.0),
 }
@@ -569,8 +569,8 @@ DIAG_CASES = {
     "f32_d64": (W.scaled("tiny", n_tokens=2048, n_needles=2, batch=4), 2048 - 3, 0),
     "bf16_c64": (W.scaled("1m", n_kv_heads=2, n_q_heads=16, n_tokens=8192, stream_tokens=128, levels=2,
                           batch=2, n_needles=2), 8192 + 77, 0),
-    "bf16_rope_c4": (W.scaled("deep", n_kv_heads=1, n_q_heads=4, n_tokens=4096, levels=4, batch=2),
-                     4096 + 3, 64),
+    "bf16_rope_c4": (W.scaled("deep", n_kv_heads=1, n_q_heads=4, n_tokens=4096, levels=4, batch=2,
+                              stream_tokens=16), 4096 + 3, 64),
 }
 
 
