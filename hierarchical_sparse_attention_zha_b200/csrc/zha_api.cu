@@ -9,19 +9,18 @@
 #include "zha_internal.cuh"
 
 namespace zha {
-cudaError_t launch_build(const Geom& G, const void* K, int64_t ld, int64_t nb_old, int64_t nb_new,
+cudaError_t launch_build(const Geom& G, const KvView& kv, int64_t nb_old, int64_t nb_new,
                          const float* refq, float* store, cudaStream_t s);
-cudaError_t launch_append(const Geom& G, const void* K, int64_t ld, int64_t nb_old, int64_t nb_new,
+cudaError_t launch_append(const Geom& G, const KvView& kv, int64_t nb_old, int64_t nb_new,
                           const float* refq, float* store, cudaStream_t s);
-cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const void* V, int64_t ld,
-                             int64_t n_tokens, int32_t batch, const int32_t* chunk_ids,
-                             const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
-                             void* ws, const TcAttendLayout& lay, int32_t* status, cudaStream_t s);
-cudaError_t launch_attend(const Geom& G, const float* Q, const void* K, const void* V, int64_t ld,
-                          int64_t n_tokens, int32_t batch, const int32_t* chunk_ids,
-                          const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
-                          float* partial, const AttendLayout& lay, int32_t* status,
-                          cudaStream_t s);
+cudaError_t launch_attend_tc(const Geom& G, const float* Q, const KvView& kv, int64_t n_tokens,
+                             int32_t batch, const int32_t* chunk_ids, const int32_t* n_chunks,
+                             int32_t max_sel, float* O, float* lse, void* ws, const TcAttendLayout& lay,
+                             int32_t* status, cudaStream_t s);
+cudaError_t launch_attend(const Geom& G, const float* Q, const KvView& kv, int64_t n_tokens,
+                          int32_t batch, const int32_t* chunk_ids, const int32_t* n_chunks,
+                          int32_t max_sel, float* O, float* lse, float* partial,
+                          const AttendLayout& lay, int32_t* status, cudaStream_t s);
 }  // namespace zha
 
 static std::atomic<uint64_t> g_launches{0};
@@ -160,36 +159,76 @@ zha_status zha_tree_level_layout(const zha_tree* tree, int32_t level, int64_t* o
   return ZHA_OK;
 }
 
-static zha_status check_cache(const zha_tree* tree, const void* d_K, int64_t ld, int64_t n_tokens,
-                              const char* what) {
+}  // extern "C"
+
+// A zha_kv_cache checked against the tree and turned into the kernels' view.
+// `need_v`: the call reads values too. Contiguous: ld rows per KV head, at
+// least n_tokens; paged: ld pages, a block table with >= ceil(n_tokens / C)
+// entries per KV head.
+static zha_status kv_view(const zha_tree* tree, const zha_kv_cache* kv, int64_t n_tokens, bool need_v,
+                          const char* what, zha::KvView* out) {
   if (tree == nullptr) return fail(ZHA_ERR_INVALID, "%s: tree is NULL", what);
-  if (d_K == nullptr || !aligned(d_K, 16))
-    return fail(ZHA_ERR_INVALID, "%s: K must be a non-NULL 16-byte aligned device pointer", what);
-  if (ld < 1) return fail(ZHA_ERR_INVALID, "%s: ld must be >= 1", what);
-  if (n_tokens < 0 || n_tokens > ld || n_tokens > tree->geom.max_tokens)
-    return fail(ZHA_ERR_INVALID, "%s: n_tokens %lld outside [0, min(ld, max_tokens)]", what,
-                (long long)n_tokens);
+  if (kv == nullptr) return fail(ZHA_ERR_INVALID, "%s: cache is NULL", what);
+  if (kv->k == nullptr || !aligned(kv->k, 16) || (need_v && (kv->v == nullptr || !aligned(kv->v, 16))))
+    return fail(ZHA_ERR_INVALID, "%s: K%s must be non-NULL 16-byte aligned device pointers", what,
+                need_v ? " and V" : "");
+  if (kv->ld < 1) return fail(ZHA_ERR_INVALID, "%s: ld must be >= 1", what);
+  if (n_tokens < 0 || n_tokens > tree->geom.max_tokens)
+    return fail(ZHA_ERR_INVALID, "%s: n_tokens %lld outside [0, max_tokens]", what, (long long)n_tokens);
+  if (kv->block_table == nullptr) {
+    if (n_tokens > kv->ld)
+      return fail(ZHA_ERR_INVALID, "%s: n_tokens %lld outside [0, min(ld, max_tokens)]", what,
+                  (long long)n_tokens);
+  } else {
+    const int64_t blocks = (n_tokens + tree->geom.chunk - 1) / tree->geom.chunk;
+    if (!aligned(kv->block_table, 4) || kv->max_blocks < blocks)
+      return fail(ZHA_ERR_INVALID, "%s: the block table needs >= %lld entries per KV head", what,
+                  (long long)blocks);
+    if (kv->ld > (int64_t(1) << 31) / tree->geom.chunk)
+      return fail(ZHA_ERR_UNSUPPORTED, "%s: more than 2^31 token slots in the page pool", what);
+  }
+  out->k = kv->k;
+  out->v = kv->v;
+  out->ld = kv->ld;
+  out->table = kv->block_table;
+  out->max_blocks = kv->block_table ? kv->max_blocks : 0;
   return ZHA_OK;
 }
 
-zha_status zha_build(zha_tree* tree, const void* d_K, int64_t ld, int64_t n_tokens, void* stream) {
-  zha_status st = check_cache(tree, d_K, ld, n_tokens, "zha_build");
+static zha_kv_cache contiguous(const void* k, const void* v, int64_t ld) {
+  zha_kv_cache c{};
+  c.k = k;
+  c.v = v;
+  c.ld = ld;
+  return c;
+}
+
+extern "C" {
+
+zha_status zha_build_kv(zha_tree* tree, const zha_kv_cache* kv, int64_t n_tokens, void* stream) {
+  zha::KvView view{};
+  zha_status st = kv_view(tree, kv, n_tokens, false, "zha_build", &view);
   if (st != ZHA_OK) return st;
   const int64_t nb = int64_t(tree->geom.chunk) * (n_tokens / tree->geom.chunk);
   // A full build starts the tree's status afresh.
   cudaError_t e = cudaMemsetAsync(zha::tree_status_word(tree->geom, tree->store), 0, sizeof(int32_t),
                                   static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "zha_build");
-  e = zha::launch_build(tree->geom, d_K, ld, 0, nb, tree->ref_q, tree->store,
+  e = zha::launch_build(tree->geom, view, 0, nb, tree->ref_q, tree->store,
                         static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "zha_build");
   tree->nb = nb;
   return ZHA_OK;
 }
 
-zha_status zha_append_chunk(zha_tree* tree, const void* d_K, int64_t ld, int64_t n_tokens,
-                            void* stream) {
-  zha_status st = check_cache(tree, d_K, ld, n_tokens, "zha_append_chunk");
+zha_status zha_build(zha_tree* tree, const void* d_K, int64_t ld, int64_t n_tokens, void* stream) {
+  const zha_kv_cache kv = contiguous(d_K, nullptr, ld);
+  return zha_build_kv(tree, &kv, n_tokens, stream);
+}
+
+zha_status zha_append_chunk_kv(zha_tree* tree, const zha_kv_cache* kv, int64_t n_tokens, void* stream) {
+  zha::KvView view{};
+  zha_status st = kv_view(tree, kv, n_tokens, false, "zha_append_chunk", &view);
   if (st != ZHA_OK) return st;
   const int64_t nb_new = int64_t(tree->geom.chunk) * (n_tokens / tree->geom.chunk);
   if (nb_new < tree->nb)
@@ -198,13 +237,19 @@ zha_status zha_append_chunk(zha_tree* tree, const void* d_K, int64_t ld, int64_t
   if (nb_new == tree->nb) return ZHA_OK;
   const int64_t new_chunks = (nb_new - tree->nb) / tree->geom.chunk;
   cudaError_t e = new_chunks <= 8
-                      ? zha::launch_append(tree->geom, d_K, ld, tree->nb, nb_new, tree->ref_q,
-                                           tree->store, static_cast<cudaStream_t>(stream))
-                      : zha::launch_build(tree->geom, d_K, ld, tree->nb, nb_new, tree->ref_q,
-                                          tree->store, static_cast<cudaStream_t>(stream));
+                      ? zha::launch_append(tree->geom, view, tree->nb, nb_new, tree->ref_q, tree->store,
+                                           static_cast<cudaStream_t>(stream))
+                      : zha::launch_build(tree->geom, view, tree->nb, nb_new, tree->ref_q, tree->store,
+                                          static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "zha_append_chunk");
   tree->nb = nb_new;
   return ZHA_OK;
+}
+
+zha_status zha_append_chunk(zha_tree* tree, const void* d_K, int64_t ld, int64_t n_tokens,
+                            void* stream) {
+  const zha_kv_cache kv = contiguous(d_K, nullptr, ld);
+  return zha_append_chunk_kv(tree, &kv, n_tokens, stream);
 }
 
 size_t zha_route_workspace_bytes(const zha_config* cfg, int32_t batch, int64_t n_tokens) {
@@ -319,21 +364,20 @@ size_t zha_attend_workspace_bytes(const zha_config* cfg, int32_t batch, int64_t 
   return size_t(zha::attend_layout(G, batch, n_tokens).bytes);
 }
 
-zha_status zha_sparse_attend(const zha_tree* tree, const float* d_Q, const void* d_K,
-                             const void* d_V, int64_t ld, int64_t n_tokens, int32_t batch,
-                             const int32_t* d_chunk_ids, const int32_t* d_n_chunks,
-                             int32_t max_sel, float* d_O, float* d_lse, void* d_ws,
-                             size_t ws_bytes, int32_t* d_status, void* stream) {
-  if (tree == nullptr) return fail(ZHA_ERR_INVALID, "zha_sparse_attend: tree is NULL");
+zha_status zha_sparse_attend_kv(const zha_tree* tree, const float* d_Q, const zha_kv_cache* kv,
+                                int64_t n_tokens, int32_t batch, const int32_t* d_chunk_ids,
+                                const int32_t* d_n_chunks, int32_t max_sel, float* d_O, float* d_lse,
+                                void* d_ws, size_t ws_bytes, int32_t* d_status, void* stream) {
+  zha::KvView view{};
+  zha_status st = kv_view(tree, kv, n_tokens, true, "zha_sparse_attend", &view);
+  if (st != ZHA_OK) return st;
   const zha::Geom& G = tree->geom;
-  if (d_Q == nullptr || d_K == nullptr || d_V == nullptr || d_O == nullptr ||
-      !aligned(d_Q, 16) || !aligned(d_K, 16) || !aligned(d_V, 16) || !aligned(d_O, 16))
+  if (d_Q == nullptr || d_O == nullptr || !aligned(d_Q, 16) || !aligned(d_O, 16))
     return fail(ZHA_ERR_INVALID,
                 "zha_sparse_attend: Q, K, V, O must be non-NULL 16-byte aligned device pointers");
   if (batch < 1 || batch > 65535)
     return fail(ZHA_ERR_INVALID, "zha_sparse_attend: batch must be 1..65535");
-  if (ld < 1 || n_tokens < 1 || n_tokens > ld)
-    return fail(ZHA_ERR_INVALID, "zha_sparse_attend: need 1 <= n_tokens <= ld");
+  if (n_tokens < 1) return fail(ZHA_ERR_INVALID, "zha_sparse_attend: need 1 <= n_tokens <= ld");
   if (d_chunk_ids == nullptr || d_n_chunks == nullptr || max_sel < 1)
     return fail(ZHA_ERR_INVALID, "zha_sparse_attend: chunk_ids / n_chunks NULL or max_sel < 1");
   if (zha::use_tc_attend(G)) {
@@ -346,9 +390,8 @@ zha_status zha_sparse_attend(const zha_tree* tree, const float* d_Q, const void*
       return fail(ZHA_ERR_CAPACITY,
                   "zha_sparse_attend: workspace must be 256-byte aligned with %lld bytes",
                   (long long)lay.bytes);
-    cudaError_t e = zha::launch_attend_tc(G, d_Q, d_K, d_V, ld, n_tokens, batch, d_chunk_ids,
-                                          d_n_chunks, max_sel, d_O, d_lse, d_ws, lay, d_status,
-                                          static_cast<cudaStream_t>(stream));
+    cudaError_t e = zha::launch_attend_tc(G, d_Q, view, n_tokens, batch, d_chunk_ids, d_n_chunks, max_sel,
+                                          d_O, d_lse, d_ws, lay, d_status, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "zha_sparse_attend");
     return ZHA_OK;
   }
@@ -359,11 +402,23 @@ zha_status zha_sparse_attend(const zha_tree* tree, const float* d_Q, const void*
     return fail(ZHA_ERR_CAPACITY,
                 "zha_sparse_attend: workspace must be 256-byte aligned with %lld bytes",
                 (long long)lay.bytes);
-  cudaError_t e = zha::launch_attend(G, d_Q, d_K, d_V, ld, n_tokens, batch, d_chunk_ids,
-                                     d_n_chunks, max_sel, d_O, d_lse, static_cast<float*>(d_ws),
-                                     lay, d_status, static_cast<cudaStream_t>(stream));
+  cudaError_t e = zha::launch_attend(G, d_Q, view, n_tokens, batch, d_chunk_ids, d_n_chunks, max_sel, d_O,
+                                     d_lse, static_cast<float*>(d_ws), lay, d_status,
+                                     static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "zha_sparse_attend");
   return ZHA_OK;
+}
+
+zha_status zha_sparse_attend(const zha_tree* tree, const float* d_Q, const void* d_K,
+                             const void* d_V, int64_t ld, int64_t n_tokens, int32_t batch,
+                             const int32_t* d_chunk_ids, const int32_t* d_n_chunks,
+                             int32_t max_sel, float* d_O, float* d_lse, void* d_ws,
+                             size_t ws_bytes, int32_t* d_status, void* stream) {
+  if (tree != nullptr && d_K != nullptr && d_V != nullptr && (ld < 1 || n_tokens < 1 || n_tokens > ld))
+    return fail(ZHA_ERR_INVALID, "zha_sparse_attend: need 1 <= n_tokens <= ld");
+  const zha_kv_cache kv = contiguous(d_K, d_V, ld);
+  return zha_sparse_attend_kv(tree, d_Q, &kv, n_tokens, batch, d_chunk_ids, d_n_chunks, max_sel, d_O,
+                              d_lse, d_ws, ws_bytes, d_status, stream);
 }
 
 }  // extern "C"

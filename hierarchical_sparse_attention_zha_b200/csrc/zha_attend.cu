@@ -32,10 +32,7 @@ cudaError_t launch_combine(const Geom& G, int32_t batch, const int32_t* chunk_id
                            const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
                            const float* partial, const AttendLayout& lay, int32_t* status,
                            cudaStream_t s);
-cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const void* V, int64_t ld,
-                             int64_t n_tokens, int32_t batch, const int32_t* chunk_ids,
-                             const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
-                             void* ws, const TcAttendLayout& lay, int32_t* status, cudaStream_t s);
+
 
 template <int D>
 __host__ __device__ inline size_t attend_smem_bytes(int range_chunks) {
@@ -56,10 +53,11 @@ __device__ __forceinline__ int lower_bound_i32(const int32_t* a, int n, int64_t 
 template <typename T, int D>
 __global__ void __launch_bounds__(kAttThreads)
 attend_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const float* __restrict__ Q,
-              const T* __restrict__ K, const T* __restrict__ V, int64_t ld,
-              const int32_t* __restrict__ chunk_ids, const int32_t* __restrict__ n_chunks,
+              KvView kv, const int32_t* __restrict__ chunk_ids, const int32_t* __restrict__ n_chunks,
               int32_t max_sel, int32_t range_chunks, int64_t n_ranges,
-              float* __restrict__ partial, int64_t slots_per_head) {
+              float* __restrict__ partial, int64_t slots_per_head, int32_t* status) {
+  const T* __restrict__ K = static_cast<const T*>(kv.k);
+  const T* __restrict__ V = static_cast<const T*>(kv.v);
   constexpr int DP = D + 4;
   constexpr int VEC = 16 / sizeof(T);
   constexpr int NV = D / 32;            // float4 groups per thread in the output update
@@ -189,16 +187,22 @@ attend_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const float* 
           msk = s_mask0;
         }
       }
+      if (tid < nt && kv.table != nullptr && kv_row(kv, g, tok, C) < 0) {
+        msk = 0u;                     // page outside the pool: not read, not attended
+        if (status != nullptr) atomicOr(status, ZHA_DEV_BAD_PAGE);
+      }
       s_tok[tid] = tok;
       s_tmask[tid] = msk;
     }
     __syncthreads();
-    // Stage K and V rows of the tile (16-byte vectors).
+    // Stage K and V rows of the tile (16-byte vectors); a token on a page the
+    // block table does not hold reads as zeros and no head attends it.
     for (int v = tid; v < kAttT * (D / VEC); v += blockDim.x) {
       const int row = v / (D / VEC), col = (v % (D / VEC)) * VEC;
       float kt[VEC], vt[VEC];
-      if (row < nt) {
-        const int64_t off = (int64_t(g) * ld + s_tok[row]) * D;
+      const int64_t kr = row < nt ? kv_row(kv, g, s_tok[row], C) : -1;
+      if (kr >= 0) {
+        const int64_t off = kr * D;
         load_slice<VEC>(K + off, col, kt);
         load_slice<VEC>(V + off, col, vt);
       } else {
@@ -298,9 +302,8 @@ attend_kernel(Geom G, int32_t batch, int64_t n_tokens, int64_t nb, const float* 
 }
 
 template <typename T, int D>
-static cudaError_t launch_attend_t(const Geom& G, const float* Q, const void* K, const void* V,
-                                   int64_t ld, int64_t n_tokens, int32_t batch,
-                                   const int32_t* chunk_ids, const int32_t* n_chunks,
+static cudaError_t launch_attend_t(const Geom& G, const float* Q, const KvView& kv, int64_t n_tokens,
+                                   int32_t batch, const int32_t* chunk_ids, const int32_t* n_chunks,
                                    int32_t max_sel, float* O, float* lse, float* partial,
                                    const AttendLayout& lay, int32_t* status, cudaStream_t s) {
   const size_t smem = attend_smem_bytes<D>(lay.range_chunks);
@@ -311,9 +314,9 @@ static cudaError_t launch_attend_t(const Geom& G, const float* Q, const void* K,
   dim3 grid(unsigned(lay.n_ranges + 1), unsigned(G.hkv), unsigned((qn + kAttQ - 1) / kAttQ));
   {
     TraceScope ts("attend_kernel", 0, s);
-    attend_kernel<T, D><<<grid, kAttThreads, smem, s>>>(
-        G, batch, n_tokens, nb, Q, static_cast<const T*>(K), static_cast<const T*>(V), ld, chunk_ids,
-        n_chunks, max_sel, lay.range_chunks, lay.n_ranges, partial, lay.slots_per_head);
+    attend_kernel<T, D><<<grid, kAttThreads, smem, s>>>(G, batch, n_tokens, nb, Q, kv, chunk_ids, n_chunks,
+                                                        max_sel, lay.range_chunks, lay.n_ranges, partial,
+                                                        lay.slots_per_head, status);
   }
   zha_count_launch();
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -455,22 +458,19 @@ cudaError_t launch_combine(const Geom& G, int32_t batch, const int32_t* chunk_id
   return cudaGetLastError();
 }
 
-cudaError_t launch_attend(const Geom& G, const float* Q, const void* K, const void* V, int64_t ld,
-                          int64_t n_tokens, int32_t batch, const int32_t* chunk_ids,
-                          const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
-                          float* partial, const AttendLayout& lay, int32_t* status,
-                          cudaStream_t s) {
+cudaError_t launch_attend(const Geom& G, const float* Q, const KvView& kv, int64_t n_tokens,
+                          int32_t batch, const int32_t* chunk_ids, const int32_t* n_chunks,
+                          int32_t max_sel, float* O, float* lse, float* partial,
+                          const AttendLayout& lay, int32_t* status, cudaStream_t s) {
   if (G.kv_bf16)
-    return G.d == 128 ? launch_attend_t<__nv_bfloat16, 128>(G, Q, K, V, ld, n_tokens, batch,
-                                                            chunk_ids, n_chunks, max_sel, O, lse,
-                                                            partial, lay, status, s)
-                      : launch_attend_t<__nv_bfloat16, 64>(G, Q, K, V, ld, n_tokens, batch,
-                                                           chunk_ids, n_chunks, max_sel, O, lse,
-                                                           partial, lay, status, s);
-  return G.d == 128 ? launch_attend_t<float, 128>(G, Q, K, V, ld, n_tokens, batch, chunk_ids,
-                                                  n_chunks, max_sel, O, lse, partial, lay, status, s)
-                    : launch_attend_t<float, 64>(G, Q, K, V, ld, n_tokens, batch, chunk_ids,
-                                                 n_chunks, max_sel, O, lse, partial, lay, status, s);
+    return G.d == 128 ? launch_attend_t<__nv_bfloat16, 128>(G, Q, kv, n_tokens, batch, chunk_ids, n_chunks,
+                                                            max_sel, O, lse, partial, lay, status, s)
+                      : launch_attend_t<__nv_bfloat16, 64>(G, Q, kv, n_tokens, batch, chunk_ids, n_chunks,
+                                                           max_sel, O, lse, partial, lay, status, s);
+  return G.d == 128 ? launch_attend_t<float, 128>(G, Q, kv, n_tokens, batch, chunk_ids, n_chunks, max_sel,
+                                                  O, lse, partial, lay, status, s)
+                    : launch_attend_t<float, 64>(G, Q, kv, n_tokens, batch, chunk_ids, n_chunks, max_sel,
+                                                 O, lse, partial, lay, status, s);
 }
 
 }  // namespace zha

@@ -77,6 +77,7 @@ struct Misc {
   float mrun[2][kQ];                      // running maxima per head, by group parity
   float scl[kQ];                          // rescale factors of the current tile
   int32_t tok0[kStages][kMaxEntries];
+  int32_t page[kStages][kMaxEntries];     // paged caches: pool page of the entry's chunk
   int32_t nvalid[kStages][kMaxEntries];
   uint32_t emask[kStages][kMaxEntries];
   uint16_t rowj[kTok];                    // (entry << 8) | row in chunk, 0xffff = unused row
@@ -326,8 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     Geom G, int32_t batch, int32_t q_blocks, int32_t n_blocks, int64_t block_chunks,
                     int32_t units, int64_t n_tokens, int64_t nb, const float* __restrict__ Q,
-                    const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
-                    int64_t ld, const int32_t* __restrict__ ids, const uint32_t* __restrict__ masks,
+                    KvView kv, const int32_t* __restrict__ ids, const uint32_t* __restrict__ masks,
                     int64_t cap, const int32_t* __restrict__ counts, int32_t* __restrict__ split,
                     float* __restrict__ slots, int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
@@ -340,6 +340,9 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int C = G.chunk;
   const int cpt = chunks_per_tile(C);
+  const bool paged = kv.table != nullptr;
+  const __nv_bfloat16* __restrict__ K = static_cast<const __nv_bfloat16*>(kv.k);
+  const __nv_bfloat16* __restrict__ V = static_cast<const __nv_bfloat16*>(kv.v);
   const int64_t n_tail = n_tokens - nb;
   const int has_tail = n_tail > 0 ? 1 : 0;
   // Tiles of unit u: its entries, plus the tail in a group's last block.
@@ -425,11 +428,13 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     // stage is free.
     const int ptid = tid, piece = ptid & 15, rs = ptid >> 4;
     SpanWalk wk{s_toff, n_blocks, u0};
-    int32_t pf_tok0[2] = {-1, -1}, pf_nv[2] = {0, 0};
+    int32_t pf_tok0[2] = {-1, -1}, pf_nv[2] = {0, 0}, pf_pg[2] = {0, 0};
     uint32_t pf_m[2] = {0u, 0u};
+    bool bad_page = false;
     auto prefetch = [&](int64_t t) {
       wk.seek(t);
       const int uu = wk.u, v = uu / n_blocks, blk = uu % n_blocks;
+      const int gkv = v / q_blocks;
       const int E = counts[uu];
       const bool tail_here = has_tail && blk == n_blocks - 1;
       const int nq = group_width(G, batch, q_blocks, v);
@@ -450,6 +455,16 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             pf_tok0[h] = int32_t(nb);
             pf_nv[h] = int32_t(n_tail);
             pf_m[h] = allq;
+          }
+          // Paged cache: the entry's page; one outside the pool drops the entry.
+          if (paged && pf_tok0[h] >= 0) {
+            const int64_t row = kv_row(kv, gkv, pf_tok0[h], C);
+            if (row < 0) {
+              pf_tok0[h] = -1; pf_nv[h] = 0; pf_m[h] = 0u;
+              bad_page = true;
+            } else {
+              pf_pg[h] = int32_t(row / C);
+            }
           }
         }
       }
@@ -473,6 +488,7 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             const int j = lane + 32 * h;
             if (j < cpt) {
               ms.tok0[st][j] = pf_tok0[h];
+              ms.page[st][j] = pf_pg[h];
               ms.nvalid[st][j] = pf_nv[h];
               ms.emask[st][j] = pf_m[h];
             }
@@ -487,16 +503,20 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
               const int32_t tok0 = ms.tok0[st][j];
               if (tok0 < 0) continue;
               const uint32_t roff = uint32_t(j * C * 128);
-              tc::tma_load_3d(sK + roff, &tmK, 0, tok0, g, &ms.full[st]);
-              tc::tma_load_3d(sK + 16384 + roff, &tmK, 64, tok0, g, &ms.full[st]);
-              tc::tma_load_3d(sV + roff, &tmV, 0, tok0, g, &ms.full[st]);
-              tc::tma_load_3d(sV + 16384 + roff, &tmV, 64, tok0, g, &ms.full[st]);
+              // contiguous: {d, tokens, KV head}; paged: {d, row in page, page}
+              const int32_t y = paged ? 0 : tok0, z = paged ? ms.page[st][j] : g;
+              tc::tma_load_3d(sK + roff, &tmK, 0, y, z, &ms.full[st]);
+              tc::tma_load_3d(sK + 16384 + roff, &tmK, 64, y, z, &ms.full[st]);
+              tc::tma_load_3d(sV + roff, &tmV, 0, y, z, &ms.full[st]);
+              tc::tma_load_3d(sV + 16384 + roff, &tmV, 64, y, z, &ms.full[st]);
             }
           }
           __syncwarp();
           if (t + 1 < t1) prefetch(t + 1);
         }
         if (failed && lane == 0) atomicOr(&ms.err, 1u);
+        if (__any_sync(0xffffffffu, bad_page) && lane == 0 && status != nullptr)
+          atomicOr(status, ZHA_DEV_BAD_PAGE);
       }
     } else {
     for (int64_t t = t0; t < t1; ++t, ++li) {
@@ -512,6 +532,7 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           const int j = lane + 32 * h;
           if (j < cpt) {
             ms.tok0[st][j] = pf_tok0[h];
+            ms.page[st][j] = pf_pg[h];
             ms.nvalid[st][j] = pf_nv[h];
             ms.emask[st][j] = pf_m[h];
           }
@@ -519,29 +540,33 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       }
       if (tc::named_sync_or(2, kProducers, bad)) { failed = true; break; }
       if (warp == 0 && t + 1 < t1) prefetch(t + 1);
-      const __nv_bfloat16* kb = K + g * ld * kD;
-      const __nv_bfloat16* vb = V + g * ld * kD;
       const uint32_t sK = tc::smem_u32(smem + st * kStageBytes), sV = sK + 32768;
 #pragma unroll 4
       for (int k = 0; k < kTok / 4; ++k) {
         const int r = rs + 4 * k;
         const uint32_t jr = ms.rowj[r];
         bool valid = false;
-        int64_t tok = 0;
+        int64_t row = 0;
         if (jr != 0xffffu) {
           const int j = int(jr >> 8), rr = int(jr & 255u);
           const int32_t tok0 = ms.tok0[st][j];
-          if (tok0 >= 0 && rr < ms.nvalid[st][j]) { valid = true; tok = int64_t(tok0) + rr; }
+          if (tok0 >= 0 && rr < ms.nvalid[st][j]) {
+            // contiguous: row of KV head g; paged: row rr of the entry's page
+            row = paged ? int64_t(ms.page[st][j]) * C + rr : g * kv.ld + int64_t(tok0) + rr;
+            valid = true;
+          }
         }
         const uint32_t off = tc::sw128_offset(r, 8 * piece, kTok);
-        tc::cp_async16(sK + off, kb + tok * kD + 8 * piece, valid ? 16u : 0u);
-        tc::cp_async16(sV + off, vb + tok * kD + 8 * piece, valid ? 16u : 0u);
+        tc::cp_async16(sK + off, K + row * kD + 8 * piece, valid ? 16u : 0u);
+        tc::cp_async16(sV + off, V + row * kD + 8 * piece, valid ? 16u : 0u);
       }
       tc::cp_async_arrive_noinc(&ms.full[st]);
       if (ptid == 0) tc::mbar_arrive(&ms.full[st]);
     }
     tc::cp_async_wait_pending0();
     if (failed && ptid == 0) atomicOr(&ms.err, 1u);
+    if (warp == 0 && __any_sync(0xffffffffu, bad_page) && lane == 0 && status != nullptr)
+      atomicOr(status, ZHA_DEV_BAD_PAGE);
     }
   } else if (warp == 2) {
     // ---------------- MMA issuer ----------------
@@ -708,7 +733,19 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         if (jr != 0xffffu) {
           const int j = int(jr >> 8), rr = int(jr & 255u);
           const int32_t tok0 = ms.tok0[st][j];
-          if (tok0 >= 0 && rr < ms.nvalid[st][j]) rmask = (tok0 + rr == 0) ? allq : ms.emask[st][j];
+          if (tok0 >= 0 && rr < ms.nvalid[st][j]) {
+            rmask = (tok0 + rr == 0) ? allq : ms.emask[st][j];
+          } else if (kTma && paged && wg == 0 && tok0 >= 0) {
+            // A tensor copy brings whole pages: this row of the in-progress
+            // chunk's page holds no token yet, and its V must not carry
+            // non-finite bytes into the P.V product (P is 0 there).
+            uint8_t* vrow = smem + st * kStageBytes + 32768 + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+              for (int c16 = 0; c16 < 8; ++c16)
+                *reinterpret_cast<uint4*>(vrow + h * 16384 + c16 * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
         }
         rmask >>= q0;
       }
@@ -958,12 +995,26 @@ bool kv_tensor_map(CUtensorMap* m, const void* base, int64_t n_tokens, int64_t l
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// A bf16 page pool [n_pages][C][d] as a 3-D tensor {d, C, n_pages}: box = 64
+// columns x the C rows of one page; a page id outside the pool reads as zeros.
+bool page_tensor_map(CUtensorMap* m, const void* base, int64_t n_pages, int chunk) {
+  const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[3] = {cuuint64_t(kD), cuuint64_t(chunk), cuuint64_t(n_pages)};
+  const cuuint64_t strides[2] = {cuuint64_t(kD) * 2, cuuint64_t(chunk) * kD * 2};
+  const cuuint32_t box[3] = {64u, cuuint32_t(chunk), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
-cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const void* V, int64_t ld,
-                             int64_t n_tokens, int32_t batch, const int32_t* chunk_ids,
-                             const int32_t* n_chunks, int32_t max_sel, float* O, float* lse,
-                             void* ws, const TcAttendLayout& lay, int32_t* status, cudaStream_t s) {
+cudaError_t launch_attend_tc(const Geom& G, const float* Q, const KvView& kv, int64_t n_tokens,
+                             int32_t batch, const int32_t* chunk_ids, const int32_t* n_chunks,
+                             int32_t max_sel, float* O, float* lse, void* ws, const TcAttendLayout& lay,
+                             int32_t* status, cudaStream_t s) {
   char* base = static_cast<char*>(ws);
   int32_t* ids = reinterpret_cast<int32_t*>(base + lay.ids_off);
   uint32_t* masks = reinterpret_cast<uint32_t*>(base + lay.masks_off);
@@ -987,8 +1038,12 @@ cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const
 
   // Tensor copies when every chunk box starts on a swizzle atom (C % 8 == 0).
   CUtensorMap mk{}, mv{};
-  const bool tma = G.chunk % 8 == 0 && kv_tensor_map(&mk, K, n_tokens, ld, G.hkv, G.chunk) &&
-                   kv_tensor_map(&mv, V, n_tokens, ld, G.hkv, G.chunk);
+  const bool tma = G.chunk % 8 == 0 &&
+                   (kv.table == nullptr
+                        ? kv_tensor_map(&mk, kv.k, n_tokens, kv.ld, G.hkv, G.chunk) &&
+                              kv_tensor_map(&mv, kv.v, n_tokens, kv.ld, G.hkv, G.chunk)
+                        : page_tensor_map(&mk, kv.k, kv.ld, G.chunk) &&
+                              page_tensor_map(&mv, kv.v, kv.ld, G.chunk));
   auto kern = tma ? attend_split_kernel<true> : attend_split_kernel<false>;
   const size_t smem = split_smem_bytes(units);
   if ((e = ensure_dynamic_smem(kern, smem)) != cudaSuccess) return e;
@@ -998,9 +1053,8 @@ cudaError_t launch_attend_tc(const Geom& G, const float* Q, const void* K, const
   {
     TraceScope ts("attend_split_kernel", 0, s);
     e = launch_pdl(kern, dim3(ctas), dim3(kThreads), smem, s, mk, mv, G, batch, lay.q_blocks,
-                   lay.n_blocks, lay.block_chunks, units, n_tokens, nb, Q,
-                   static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V), ld, ids,
-                   masks, lay.cap, counts, split, slots, status);
+                   lay.n_blocks, lay.block_chunks, units, n_tokens, nb, Q, kv, ids, masks, lay.cap,
+                   counts, split, slots, status);
   }
   if (e != cudaSuccess) return e;
   zha_count_launch();

@@ -37,9 +37,9 @@ __host__ __device__ inline size_t l1_smem_bytes(int nref) {
 }
 
 template <typename T, int D>
-__device__ void summarise_tile(const Geom& G, int g, const T* __restrict__ K, int64_t ld,
-                               int64_t c0, int nch, const float* __restrict__ refq,
-                               float* __restrict__ store, float* smem) {
+__device__ void summarise_tile(const Geom& G, int g, const KvView& kv, int64_t c0, int nch,
+                               const float* __restrict__ refq, float* __restrict__ store,
+                               float* smem) {
   constexpr int DP = D + 4;
   constexpr int EPL = D / 32;
   const int C = G.chunk, R = G.nref;
@@ -53,18 +53,28 @@ __device__ void summarise_tile(const Geom& G, int g, const T* __restrict__ K, in
   const int nwarps = blockDim.x >> 5;
   const int RP = G.rope_pairs;
 
-  // Stage keys (16-byte vectors, coalesced) and reference queries.
+  // Stage keys (16-byte vectors, coalesced) and reference queries. A key whose
+  // page the block table does not hold reads as zeros and marks the tree.
   {
     constexpr int VEC = 16 / sizeof(T);
-    const T* base = K + (int64_t(g) * ld + c0 * C) * D;
+    const T* K = static_cast<const T*>(kv.k);
     const int nvec = TT * (D / VEC);
+    bool bad = false;
     for (int v = tid; v < nvec; v += blockDim.x) {
       const int row = v / (D / VEC), col = (v % (D / VEC)) * VEC;
+      const int64_t kr = kv_row(kv, g, c0 * C + row, C);
       float tmp[VEC];
-      load_slice<VEC>(base + int64_t(row) * D, col, tmp);
+      if (kr >= 0) {
+        load_slice<VEC>(K + kr * D, col, tmp);
+      } else {
+        bad = true;
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) tmp[i] = 0.f;
+      }
 #pragma unroll
       for (int i = 0; i < VEC; ++i) ks[row * DP + col + i] = tmp[i];
     }
+    if (bad) atomicOr(tree_status_word(G, store), ZHA_DEV_BAD_PAGE);
     const float* qb = refq + int64_t(g) * R * D;
     for (int v = tid; v < R * (D / 4); v += blockDim.x) {
       const int row = v / (D / 4), col = (v % (D / 4)) * 4;
@@ -171,15 +181,14 @@ __device__ void summarise_tile(const Geom& G, int g, const T* __restrict__ K, in
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kBuildThreads)
-build_level1_kernel(Geom G, const T* __restrict__ K, int64_t ld, int64_t c_begin,
-                    int64_t c_end, const float* __restrict__ refq, float* __restrict__ store) {
+build_level1_kernel(Geom G, KvView kv, int64_t c_begin, int64_t c_end,
+                    const float* __restrict__ refq, float* __restrict__ store) {
   extern __shared__ float4 smem_v4[];
   const int cpt = l1_chunks_per_tile(G.chunk);
   const int64_t c0 = c_begin + int64_t(blockIdx.x) * cpt;
   if (c0 >= c_end) return;
   const int nch = int(min64(cpt, c_end - c0));
-  summarise_tile<T, D>(G, blockIdx.y, K, ld, c0, nch, refq, store,
-                       reinterpret_cast<float*>(smem_v4));
+  summarise_tile<T, D>(G, blockIdx.y, kv, c0, nch, refq, store, reinterpret_cast<float*>(smem_v4));
 }
 
 // ---------------------------------------------------------------------------
@@ -284,8 +293,8 @@ merge_level_kernel(Geom G, int level, int64_t parent0, int64_t n_parents,
 // ---------------------------------------------------------------------------
 template <typename T, int D>
 __global__ void __launch_bounds__(kBuildThreads)
-append_kernel(Geom G, const T* __restrict__ K, int64_t ld, int64_t nb_old, int64_t nb_new,
-              const float* __restrict__ refq, float* __restrict__ store) {
+append_kernel(Geom G, KvView kv, int64_t nb_old, int64_t nb_new, const float* __restrict__ refq,
+              float* __restrict__ store) {
   extern __shared__ float4 smem_v4[];
   float* smem = reinterpret_cast<float*>(smem_v4);
   const int g = blockIdx.x;
@@ -294,7 +303,7 @@ append_kernel(Geom G, const T* __restrict__ K, int64_t ld, int64_t nb_old, int64
   const int64_t c_begin = nb_old / C, c_end = nb_new / C;
   for (int64_t c0 = c_begin; c0 < c_end; c0 += cpt) {
     const int nch = int(min64(cpt, c_end - c0));
-    summarise_tile<T, D>(G, g, K, ld, c0, nch, refq, store, smem);
+    summarise_tile<T, D>(G, g, kv, c0, nch, refq, store, smem);
     __syncthreads();
   }
   const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
@@ -313,24 +322,24 @@ append_kernel(Geom G, const T* __restrict__ K, int64_t ld, int64_t nb_old, int64
 // Summarise chunks [nb_old/C, nb_new/C) and merge the parents they complete:
 // one level-1 launch and one launch per upper level that gains nodes.
 template <typename T, int D>
-static cudaError_t launch_build_t(const Geom& G, const void* K, int64_t ld, int64_t nb_old,
-                                  int64_t nb_new, const float* refq, float* store,
-                                  cudaStream_t s) {
+static cudaError_t launch_build_t(const Geom& G, const KvView& kv, int64_t nb_old, int64_t nb_new,
+                                  const float* refq, float* store, cudaStream_t s) {
   const size_t smem = l1_smem_bytes<D>(G.nref);
   cudaError_t e = ensure_dynamic_smem(build_level1_kernel<T, D>, smem);
   if (e != cudaSuccess) return e;
   const int64_t c_begin = nb_old / G.chunk, c_end = nb_new / G.chunk;
-  // bf16, d = 128, R = 16, C = 64: the tensor-core level 1 (zha_build_tc.cu).
+  // bf16, d = 128, R = 16, C = 64, contiguous cache: the tensor-core level 1 (zha_build_tc.cu).
   const cudaError_t etc =
-      launch_build_level1_tc(G, K, ld, c_begin, c_end, refq, store, tree_status_word(G, store), s);
+      kv.table != nullptr
+          ? cudaErrorNotSupported
+          : launch_build_level1_tc(G, kv.k, kv.ld, c_begin, c_end, refq, store, tree_status_word(G, store), s);
   if (etc != cudaSuccess && etc != cudaErrorNotSupported) return etc;
   if (etc != cudaSuccess && c_end > c_begin) {
     const int cpt = l1_chunks_per_tile(G.chunk);
     dim3 grid(unsigned((c_end - c_begin + cpt - 1) / cpt), unsigned(G.hkv));
     {
       TraceScope ts("build_level1_kernel", 1, s);
-      build_level1_kernel<T, D><<<grid, kBuildThreads, smem, s>>>(
-          G, static_cast<const T*>(K), ld, c_begin, c_end, refq, store);
+      build_level1_kernel<T, D><<<grid, kBuildThreads, smem, s>>>(G, kv, c_begin, c_end, refq, store);
     }
     zha_count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -355,35 +364,33 @@ static cudaError_t launch_build_t(const Geom& G, const void* K, int64_t ld, int6
 }
 
 template <typename T, int D>
-static cudaError_t launch_append_t(const Geom& G, const void* K, int64_t ld, int64_t nb_old,
-                                   int64_t nb_new, const float* refq, float* store,
-                                   cudaStream_t s) {
+static cudaError_t launch_append_t(const Geom& G, const KvView& kv, int64_t nb_old, int64_t nb_new,
+                                   const float* refq, float* store, cudaStream_t s) {
   const size_t smem = l1_smem_bytes<D>(G.nref);
   cudaError_t e = ensure_dynamic_smem(append_kernel<T, D>, smem);
   if (e != cudaSuccess) return e;
   TraceScope ts("append_kernel", 0, s);
-  append_kernel<T, D><<<G.hkv, kBuildThreads, smem, s>>>(G, static_cast<const T*>(K), ld, nb_old,
-                                                          nb_new, refq, store);
+  append_kernel<T, D><<<G.hkv, kBuildThreads, smem, s>>>(G, kv, nb_old, nb_new, refq, store);
   zha_count_launch();
   return cudaGetLastError();
 }
 
-cudaError_t launch_build(const Geom& G, const void* K, int64_t ld, int64_t nb_old, int64_t nb_new,
+cudaError_t launch_build(const Geom& G, const KvView& kv, int64_t nb_old, int64_t nb_new,
                          const float* refq, float* store, cudaStream_t s) {
   if (G.kv_bf16)
-    return G.d == 128 ? launch_build_t<__nv_bfloat16, 128>(G, K, ld, nb_old, nb_new, refq, store, s)
-                      : launch_build_t<__nv_bfloat16, 64>(G, K, ld, nb_old, nb_new, refq, store, s);
-  return G.d == 128 ? launch_build_t<float, 128>(G, K, ld, nb_old, nb_new, refq, store, s)
-                    : launch_build_t<float, 64>(G, K, ld, nb_old, nb_new, refq, store, s);
+    return G.d == 128 ? launch_build_t<__nv_bfloat16, 128>(G, kv, nb_old, nb_new, refq, store, s)
+                      : launch_build_t<__nv_bfloat16, 64>(G, kv, nb_old, nb_new, refq, store, s);
+  return G.d == 128 ? launch_build_t<float, 128>(G, kv, nb_old, nb_new, refq, store, s)
+                    : launch_build_t<float, 64>(G, kv, nb_old, nb_new, refq, store, s);
 }
 
-cudaError_t launch_append(const Geom& G, const void* K, int64_t ld, int64_t nb_old, int64_t nb_new,
+cudaError_t launch_append(const Geom& G, const KvView& kv, int64_t nb_old, int64_t nb_new,
                           const float* refq, float* store, cudaStream_t s) {
   if (G.kv_bf16)
-    return G.d == 128 ? launch_append_t<__nv_bfloat16, 128>(G, K, ld, nb_old, nb_new, refq, store, s)
-                      : launch_append_t<__nv_bfloat16, 64>(G, K, ld, nb_old, nb_new, refq, store, s);
-  return G.d == 128 ? launch_append_t<float, 128>(G, K, ld, nb_old, nb_new, refq, store, s)
-                    : launch_append_t<float, 64>(G, K, ld, nb_old, nb_new, refq, store, s);
+    return G.d == 128 ? launch_append_t<__nv_bfloat16, 128>(G, kv, nb_old, nb_new, refq, store, s)
+                      : launch_append_t<__nv_bfloat16, 64>(G, kv, nb_old, nb_new, refq, store, s);
+  return G.d == 128 ? launch_append_t<float, 128>(G, kv, nb_old, nb_new, refq, store, s)
+                    : launch_append_t<float, 64>(G, kv, nb_old, nb_new, refq, store, s);
 }
 
 }  // namespace zha

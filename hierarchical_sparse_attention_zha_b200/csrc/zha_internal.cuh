@@ -54,6 +54,30 @@ __device__ __forceinline__ void rope_cos_sin(const Geom& G, int64_t pos, int pai
   *s = float(sd);
 }
 
+// ---------------------------------------------------------------------------
+// A K/V cache as the kernels see it: contiguous [Hkv][ld][d], or paged -- a
+// pool of pages of C tokens [n_pages][C][d] and a block table [Hkv][max_blocks]
+// giving the page of each chunk of each KV head (ld then counts the pages).
+// ---------------------------------------------------------------------------
+struct KvView {
+  const void* k;
+  const void* v;
+  int64_t ld;                  // contiguous: tokens per KV head block; paged: pages in the pool
+  const int32_t* table;        // nullptr: contiguous
+  int64_t max_blocks;
+};
+
+// Row (token slot) of token `tok` of KV head g in the cache's row space, or -1
+// when the block table names a page outside the pool (nothing is read then).
+__host__ __device__ inline int64_t kv_row(const KvView& kv, int g, int64_t tok, int chunk) {
+  if (kv.table == nullptr) return int64_t(g) * kv.ld + tok;
+  const int64_t c = tok / chunk;
+  if (c >= kv.max_blocks) return -1;
+  const int32_t page = kv.table[int64_t(g) * kv.max_blocks + c];
+  if (page < 0 || int64_t(page) >= kv.ld) return -1;
+  return int64_t(page) * chunk + (tok - c * chunk);
+}
+
 // C^l, saturating at a value above any token count.
 __host__ __device__ inline int64_t span_of(int32_t chunk, int32_t level) {
   int64_t s = 1;

@@ -28,6 +28,7 @@ ZHA_BF16 = 1
 ZHA_DEV_SELECTION_TRUNCATED = 1
 ZHA_DEV_BAD_SELECTION = 2
 ZHA_DEV_TIMEOUT = 4
+ZHA_DEV_BAD_PAGE = 8
 
 
 class ZhaError(RuntimeError):
@@ -61,6 +62,30 @@ def top_k_policy(k_by_level) -> RoutePolicy:
     for i, v in enumerate(k_by_level):
         pol.k[i] = int(v)
     return pol
+
+
+class KvCache(ctypes.Structure):
+    """zha_kv_cache: a contiguous [Hkv, ld, d] cache, or page pools [n_pages, C, d]
+    with a block table [Hkv, max_blocks] (int32 page ids)."""
+    _fields_ = [("k", c_void_p), ("v", c_void_p), ("ld", c_int64), ("block_table", c_void_p),
+                ("max_blocks", c_int64)]
+
+
+def kv_cache(K: torch.Tensor, V: torch.Tensor | None = None,
+             block_table: torch.Tensor | None = None) -> KvCache:
+    """A zha_kv_cache over torch tensors: contiguous when block_table is None
+    (K [Hkv, ld, d]), else page pools K, V [n_pages, C, d] and block_table
+    [Hkv, max_blocks] int32."""
+    c = KvCache()
+    c.k = K.data_ptr()
+    c.v = V.data_ptr() if V is not None else None
+    c.ld = K.shape[0] if block_table is not None else K.shape[1]
+    if block_table is not None:
+        if not (block_table.is_cuda and block_table.dtype == torch.int32 and block_table.is_contiguous()):
+            raise ValueError("block_table must be a contiguous int32 CUDA tensor [Hkv, max_blocks]")
+        c.block_table = block_table.data_ptr()
+        c.max_blocks = block_table.shape[1]
+    return c
 
 
 class Config(ctypes.Structure):
@@ -102,6 +127,10 @@ def _load() -> ctypes.CDLL:
         "zha_attend_workspace_bytes": (c_size_t, [POINTER(Config), c_int32, c_int64]),
         "zha_sparse_attend": (c_int32, [P, P, P, P, c_int64, c_int64, c_int32, P, P, c_int32, P,
                                         P, P, c_size_t, P, P]),
+        "zha_build_kv": (c_int32, [P, POINTER(KvCache), c_int64, P]),
+        "zha_append_chunk_kv": (c_int32, [P, POINTER(KvCache), c_int64, P]),
+        "zha_sparse_attend_kv": (c_int32, [P, P, POINTER(KvCache), c_int64, c_int32, P, P, c_int32, P, P,
+                                           P, c_size_t, P, P]),
         "zha_diagnostics_workspace_bytes": (c_size_t, [POINTER(Config), c_int32, c_int64]),
         "zha_route_diagnostics": (c_int32, [P, P, P, c_int64, c_int32, c_int64, P, P, P, c_size_t, P]),
         "zha_trace_enable": (c_int32, [c_int32, c_char_p, c_int32]),
@@ -247,6 +276,32 @@ class Tree:
         self._kv(K)
         check(lib.zha_append_chunk(self.handle, ptr(K), K.shape[1], n_tokens, stream_ptr(stream)),
               "zha_append_chunk")
+
+    def build_kv(self, kv: KvCache, n_tokens: int, stream=None) -> None:
+        """zha_build_kv over a zha_kv_cache (see kv_cache())."""
+        check(lib.zha_build_kv(self.handle, byref(kv), n_tokens, stream_ptr(stream)), "zha_build_kv")
+
+    def append_chunk_kv(self, kv: KvCache, n_tokens: int, stream=None) -> None:
+        check(lib.zha_append_chunk_kv(self.handle, byref(kv), n_tokens, stream_ptr(stream)),
+              "zha_append_chunk_kv")
+
+    def sparse_attend_kv(self, Q: torch.Tensor, kv: KvCache, n_tokens: int, chunk_ids: torch.Tensor,
+                         n_chunks: torch.Tensor, out: torch.Tensor | None = None,
+                         lse: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                         status: torch.Tensor | None = None, stream=None):
+        B = Q.shape[0]
+        if out is None:
+            out = torch.empty(B, self.cfg.n_q_heads, self.cfg.head_dim, dtype=torch.float32,
+                              device=self.device)
+        if lse is None:
+            lse = torch.empty(B, self.cfg.n_q_heads, dtype=torch.float32, device=self.device)
+        if ws is None:
+            ws = _bytes_tensor(attend_workspace_bytes(self.cfg, B, n_tokens), self.device)
+        check(lib.zha_sparse_attend_kv(self.handle, ptr(Q), byref(kv), n_tokens, B, ptr(chunk_ids),
+                                       ptr(n_chunks), chunk_ids.shape[-1], ptr(out), ptr(lse), ptr(ws),
+                                       ws.numel() * ws.element_size(), ptr(status), stream_ptr(stream)),
+              "zha_sparse_attend_kv")
+        return out, lse
 
     def level(self, level: int) -> tuple[torch.Tensor, torch.Tensor]:
         """Views of level `level`'s summaries: khat [Hkv, cap, R, d], bhat [Hkv, cap, R]."""

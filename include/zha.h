@@ -60,6 +60,7 @@ typedef enum {
 #define ZHA_DEV_SELECTION_TRUNCATED 1 /* zha_route: a head kept more than max_sel chunks; its list holds the first max_sel (ascending) and d_n_chunks the true count */
 #define ZHA_DEV_BAD_SELECTION 2       /* zha_sparse_attend: a chunk list had an id out of range, was not strictly ascending, or a count outside [0, max_sel]; out-of-range ids are never read, and which in-range entries of such a list are attended is unspecified */
 #define ZHA_DEV_TIMEOUT 4             /* a kernel's bounded wait for its tensor-core work ran out; its outputs are not valid (it released its resources and returned) */
+#define ZHA_DEV_BAD_PAGE 8            /* a paged cache's block table named a page outside the pool (or lacked an entry); those keys were not read (treated as absent) and the outputs that needed them are not valid */
 
 typedef enum { ZHA_F32 = 0, ZHA_BF16 = 1 } zha_dtype;
 
@@ -272,6 +273,36 @@ zha_status zha_sparse_attend(const zha_tree* tree, const float* d_Q, const void*
                              const int32_t* d_chunk_ids, const int32_t* d_n_chunks,
                              int32_t max_sel, float* d_O, float* d_lse, void* d_ws,
                              size_t ws_bytes, int32_t* d_status, void* stream);
+
+/* ---- Paged K/V caches [Attention: "KV cache 를 담는 방식을 바꾼다: PagedAttention,
+ * 양자화"] ---------------------------------------------------------------------
+ * A cache held in pages of C tokens (block size = the tree's chunk): a pool
+ * [n_pages][C][head_dim] for K and one for V (element type kv_dtype), and a
+ * block table: page of chunk c (tokens [cC, (c+1)C)) of KV head g at
+ * block_table[g * max_blocks + c]. The in-progress chunk lives in its page too.
+ * Summaries, routing and attention are the same as over the contiguous cache
+ * holding the same keys and values; only the addresses differ. A table entry
+ * outside [0, n_pages) is never dereferenced: ZHA_DEV_BAD_PAGE is set (in the
+ * call's d_status, or for builds in the tree's status word, which the next
+ * zha_route reports) and those keys count as absent. */
+typedef struct {
+    const void* k;              /* contiguous: [n_kv_heads][ld][head_dim]; paged: K page pool */
+    const void* v;              /* same layout as k; not read by builds (may be NULL there) */
+    int64_t ld;                 /* contiguous: token rows per KV head (>= n_tokens); paged: n_pages */
+    const int32_t* block_table; /* NULL: contiguous; else [n_kv_heads][max_blocks] int32 page ids */
+    int64_t max_blocks;         /* paged: table entries per KV head, >= ceil(n_tokens / C) */
+} zha_kv_cache;
+
+/* zha_build / zha_append_chunk / zha_sparse_attend over a zha_kv_cache. The
+ * contiguous entry points above are these calls with block_table = NULL. The
+ * tensor-core level-1 build serves contiguous caches; paged caches are built
+ * by the CUDA-core kernels (same summaries within rounding). */
+zha_status zha_build_kv(zha_tree* tree, const zha_kv_cache* kv, int64_t n_tokens, void* stream);
+zha_status zha_append_chunk_kv(zha_tree* tree, const zha_kv_cache* kv, int64_t n_tokens, void* stream);
+zha_status zha_sparse_attend_kv(const zha_tree* tree, const float* d_Q, const zha_kv_cache* kv,
+                                int64_t n_tokens, int32_t batch, const int32_t* d_chunk_ids,
+                                const int32_t* d_n_chunks, int32_t max_sel, float* d_O, float* d_lse,
+                                void* d_ws, size_t ws_bytes, int32_t* d_status, void* stream);
 
 /* ---- Routing diagnostics [ZHA: 어떻게 쓰나; 전제와 한계] -----------------------
  * How well each level's estimate follows the dense attention mass, for

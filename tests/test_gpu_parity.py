@@ -613,3 +613,112 @@ def test_route_diagnostics_match_the_oracle(zha, name):
     for lvl in range(spec.levels):
         assert np.abs(usage[lvl] - want[lvl]).sum() <= 2 * near[lvl], (lvl, usage[lvl], want[lvl], near[lvl])
     assert usage.sum(axis=1)[0] == spec.batch * spec.n_q_heads * (n_tokens // spec.chunk)
+
+
+# ---------------------------------------------------------------------------
+# Paged K/V caches [Attention: "KV cache 를 담는 방식을 바꾼다: PagedAttention,
+# 양자화"]: pages of C tokens in a shuffled pool, a block table per KV head
+# ---------------------------------------------------------------------------
+
+def _paged(K, V, C, n_visible, seed, extra_pages=7):
+    """Pools [n_pages, C, d] holding the first n_visible tokens of each KV head
+    in shuffled pages (every other slot, unused pages included, is NaN), and the
+    block table [Hkv, max_blocks]."""
+    Hkv, cap, d = K.shape
+    blocks = -(-cap // C)
+    n_pages = Hkv * blocks + extra_pages
+    rng = np.random.default_rng(seed)
+    table = rng.permutation(n_pages)[: Hkv * blocks].reshape(Hkv, blocks).astype(np.int32)
+    Kp = torch.full((n_pages, C, d), float("nan"), dtype=K.dtype, device=K.device)
+    Vp = torch.full_like(Kp, float("nan"))
+    for g in range(Hkv):
+        for b in range(blocks):
+            rows = min(C, n_visible - b * C)
+            if rows <= 0:
+                break
+            Kp[int(table[g, b]), :rows] = K[g, b * C: b * C + rows]
+            Vp[int(table[g, b]), :rows] = V[g, b * C: b * C + rows]
+    return Kp, Vp, torch.from_numpy(table).to(K.device), table
+
+
+PAGED_CASES = {
+    "bf16_c64_tma": (W.scaled("1m", n_kv_heads=2, n_q_heads=16, n_tokens=8192, stream_tokens=128, levels=2,
+                              batch=2, n_needles=2), 8192 + 77),
+    "bf16_c4_cp_async": (W.scaled("deep", n_kv_heads=1, n_q_heads=4, n_tokens=4096, levels=4, batch=2,
+                                  stream_tokens=16), 4096 + 3),
+    "f32_d64": (W.scaled("tiny", n_tokens=2048, n_needles=2, batch=4), 2048 - 3),
+}
+
+
+@pytest.mark.parametrize("name", list(PAGED_CASES))
+def test_paged_cache_matches_the_oracle_and_the_contiguous_cache(zha, parity_log, name):
+    """Tree built from the pages: every summary and the routing against the
+    oracle; attention over the pages against the oracle and against the
+    contiguous cache's attention on the same selection (same arithmetic)."""
+    spec, n_tokens = PAGED_CASES[name]
+    inp = W.generate(spec)
+    dev = to_device(inp)
+    K, V, refq, Q = dev
+    Kp, Vp, table, _ = _paged(K, V, spec.chunk, n_tokens, seed=3)
+    kv = zha.kv_cache(Kp, Vp, table)
+    tree = zha.Tree(config_for(spec), refq)
+    tree.build_kv(kv, n_tokens)
+    rep = check_case(zha, inp, n_tokens, tree=tree, dev=dev)
+    parity_log(f"paged_{name}", rep)
+    res = run_pipeline(zha, inp, n_tokens, tree=tree, dev=dev)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ids = torch.from_numpy(res["ids"]).cuda()
+    cnt = torch.from_numpy(res["cnt"]).cuda()
+    out, lse = tree.sparse_attend_kv(Q[0].contiguous(), kv, n_tokens, ids, cnt, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    out, lse = out.cpu().numpy(), lse.cpu().numpy()
+    assert np.isfinite(out).all() and np.isfinite(lse).all()
+    assert np.max(np.abs(out - res["out"])) <= 1e-6 and np.max(np.abs(lse - res["lse"])) <= 1e-5
+
+
+def test_paged_append_and_a_page_outside_the_pool(zha):
+    """Appends through the block table as pages fill (one chunk per call), then
+    an entry naming a page outside the pool: the build marks the tree (the next
+    route reports ZHA_DEV_BAD_PAGE), attention over it reports the bit too, and
+    every output stays finite."""
+    C = 64
+    spec = W.scaled("1m", n_kv_heads=1, n_q_heads=8, n_tokens=C * 40, stream_tokens=C * 4, levels=2,
+                    batch=2, n_needles=0)
+    inp = W.generate(spec)
+    K, V, refq, Q = to_device(inp)
+    n0, n1 = C * 40 + 5, C * 43 + 9
+    Kp, Vp, table_t, table = _paged(K, V, C, n1, seed=8)
+    kv = zha.kv_cache(Kp, Vp, table_t)
+    tree = zha.Tree(config_for(spec), refq)
+    tree.build_kv(kv, n0)
+    for n in range(n0 + 1, n1 + 1):
+        tree.append_chunk_kv(kv, n)
+    fresh = zha.Tree(config_for(spec), refq)
+    fresh.build(K, n1)
+    torch.cuda.synchronize()
+    otree = O.build_tree(cache_f64(inp, 0, n1), inp.ref_q[0], C, 2, n1)
+    for lvl in (1, 2):
+        n_l = otree.n_nodes(lvl)
+        kh, bh = tree.level(lvl)
+        ek, eb = summary_errors(kh[0, :n_l].cpu().numpy().astype(np.float64),
+                                bh[0, :n_l].cpu().numpy().astype(np.float64), *otree.nodes[lvl])
+        assert ek <= SUMMARY_RTOL and eb <= SUMMARY_RTOL, (lvl, ek, eb)
+    # a table entry outside the pool
+    bad = table_t.clone()
+    bad[0, 3] = Kp.shape[0] + 10
+    kv_bad = zha.kv_cache(Kp, Vp, bad)
+    t2 = zha.Tree(config_for(spec), refq)
+    t2.build_kv(kv_bad, n1)
+    q = Q[0].contiguous()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ids, cnt = t2.route(q, n1, 0.9, n1 // C, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) & zha.ZHA_DEV_BAD_PAGE
+    all_ids = torch.arange(n1 // C, dtype=torch.int32, device="cuda").repeat(spec.batch, spec.n_q_heads, 1)
+    all_cnt = torch.full((spec.batch, spec.n_q_heads), n1 // C, dtype=torch.int32, device="cuda")
+    st2 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse = fresh.sparse_attend_kv(q, kv_bad, n1, all_ids.contiguous(), all_cnt, status=st2)
+    torch.cuda.synchronize()
+    assert int(st2.item()) & zha.ZHA_DEV_BAD_PAGE
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
