@@ -25,13 +25,15 @@
 //                           the MMA reads its A operand (shared memory only carries
 //                           the raw tiles and Q)
 //   MMA issuer (warp 1)     S^T[(node, plane)][head] over the half's 4 K-steps:
-//                           A_t0 . [q0 | q1 | q2]^T (N = 96), A_t1 . [q0 | q1]^T
-//                           (N = 64), A_t2 . q0^T (N = 32) into one of two TMEM
-//                           buffers -- the six products with term indices summing
-//                           to <= 2, the dropped ones are below fp32 rounding
-//   epilogue (warps 12-15)  thread = (node, plane) row: sum of the three column
-//                           groups, x 1/sqrt(d) + bhat, maximum over the node's 16
+//                           the six products A_ti . q_j^T with i + j <= 2 (the
+//                           dropped ones are below fp32 rounding), each N = 32,
+//                           accumulated into one 32-column TMEM buffer (of two):
+//                           the terms are stacked along K, not along N
+//   epilogue (warps 12-15)  thread = (node, plane) row: one 32-column load,
+//                           x 1/sqrt(d) + bhat, maximum over the node's 16
 //                           planes, scores of the candidate (node, head) pairs
+// The converters pace themselves on the mbarriers alone (no CTA-wide barrier
+// in their loop).
 // Every wait is bounded; a time-out sets ZHA_DEV_TIMEOUT and the roles stop.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -57,9 +59,9 @@ constexpr int kThreads = 512;             // warps: 0 producer, 1 MMA, 2-3 idle,
 constexpr int kConv = 256;                // converter threads (warps 4-11)
 constexpr int kEpiWarp0 = 12;
 constexpr uint32_t kWaitTries = tc::kWaitPolls;
-constexpr uint32_t kTmemCols = 512;       // D buffers (96 columns) at 0 and 128; A half-buffers
-constexpr uint32_t kTmemA = 224;          // (3 terms x 32 columns) at 224, 320 and 416
-constexpr int kABufs = 3;
+constexpr uint32_t kTmemCols = 512;       // D buffers (32 columns) at 0 and 32; A half-buffers
+constexpr uint32_t kTmemA = 64;           // (3 terms x 32 columns) at 64, 160, 256 and 352
+constexpr int kABufs = 4;
 
 struct Meta {                             // one half-tile, producer -> converters
   int32_t node0, group, half, flags;      // flags: 1 = first tile of a group, 2 = end
@@ -155,7 +157,7 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&ms.d_full[b], 1);
       tc::mbar_init(&ms.d_free[b], 128);
-      tc::mbar_init(&emeta_full[b], 1);
+      tc::mbar_init(&emeta_full[b], 128);      // the converter threads that write the tile's bhat
     }
     tc::mbar_init(&ms.q_ready, kConv);
   }
@@ -253,8 +255,6 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      constexpr uint32_t idesc96 = tc::idesc_bf16(128, 96, 0, 0);
-      constexpr uint32_t idesc64 = tc::idesc_bf16(128, 64, 0, 0);
       constexpr uint32_t idesc32 = tc::idesc_bf16(128, 32, 0, 0);
       int64_t k = 0, tile_i = 0;
       int seg = 0;
@@ -280,15 +280,21 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
           ++seg;
         }
         tc::fence_after_sync();
-        const uint32_t d = tbase + uint32_t(tile_i & 1) * 128;
+        const uint32_t d = tbase + uint32_t(tile_i & 1) * 32;
         const uint32_t tA = tbase + kTmemA + uint32_t(ab) * 96;      // term t at + 32 t
-        const uint32_t sQ = tc::smem_u32(smem + kOffQ) + uint32_t(cm.half) * 12288;
+        const uint32_t sQ = tc::smem_u32(smem + kOffQ) + uint32_t(cm.half) * 12288;   // term j rows at + 4096 j
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {           // K-step = 16 bf16 = 8 TMEM columns
-          const uint64_t b = tc::desc_sw128(sQ + ks * 32, 16, 1024);
-          tc::mma_bf16_ta(d, tA + ks * 8, b, idesc96, (cm.half == 0 && ks == 0) ? 0u : 1u);
-          tc::mma_bf16_ta(d, tA + 32 + ks * 8, b, idesc64, 1u);
-          tc::mma_bf16_ta(d, tA + 64 + ks * 8, b, idesc32, 1u);
+          const uint64_t q0 = tc::desc_sw128(sQ + ks * 32, 16, 1024);
+          const uint64_t q1 = tc::desc_sw128(sQ + 4096 + ks * 32, 16, 1024);
+          const uint64_t q2 = tc::desc_sw128(sQ + 8192 + ks * 32, 16, 1024);
+          const uint32_t a0 = tA + ks * 8, a1 = tA + 32 + ks * 8, a2 = tA + 64 + ks * 8;
+          tc::mma_bf16_ta(d, a0, q0, idesc32, (cm.half == 0 && ks == 0) ? 0u : 1u);
+          tc::mma_bf16_ta(d, a0, q1, idesc32, 1u);
+          tc::mma_bf16_ta(d, a0, q2, idesc32, 1u);
+          tc::mma_bf16_ta(d, a1, q0, idesc32, 1u);
+          tc::mma_bf16_ta(d, a1, q1, idesc32, 1u);
+          tc::mma_bf16_ta(d, a2, q0, idesc32, 1u);
         }
         tc::mma_commit(&ms.a_free[ab]);
         if (cm.half == 1) {
@@ -311,13 +317,14 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
       const int slot = int(k % kRawSlots);
       const int64_t use = k / kRawSlots;
       const int ab = int(k % kABufs);
-      bool bad = !tc::mbar_wait(&ms.raw_full[slot], uint32_t(use & 1), kWaitTries);
-      if (tc::named_sync_or(1, kConv, bad)) { failed = true; break; }
+      if (!tc::mbar_wait(&ms.raw_full[slot], uint32_t(use & 1), kWaitTries)) { failed = true; break; }
       const Meta mt = ms.meta[slot];
+      bool bad = false;
       const bool end = (mt.flags & 2) != 0;
-      // A half-buffer ab was last read by the MMAs of half k - 2; the tile's
-      // metadata slot by the epilogue of tile_i - 2.
-      // (also before the end marker: the MMA issuer reads cmeta[ab] of half k - 3 first)
+      // A half-buffer ab was last read by the MMAs of half k - kABufs; the
+      // tile's metadata slot by the epilogue of tile_i - 2 (also before the end
+      // marker: the MMA issuer reads cmeta[ab] of half k - kABufs first). Each
+      // thread waits for itself; the arrivals count every converter thread.
       if (k >= kABufs)
         bad |= !tc::mbar_wait(&ms.a_free[ab], uint32_t(((k / kABufs) - 1) & 1), kWaitTries);
       if ((end || mt.half == 0) && tile_i >= 2)
@@ -327,14 +334,14 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
       const bool new_q = !end && mt.half == 0 && (mt.flags & 1);
       if (new_q && k >= 1)
         bad |= !tc::mbar_wait(&ms.a_free[(k - 1) % kABufs], uint32_t(((k - 1) / kABufs) & 1), kWaitTries);
-      if (tc::named_sync_or(1, kConv, bad)) { failed = true; break; }
+      if (bad) { failed = true; break; }
       if (end) {
         if (ctid == 0) {
           ms.cmeta[ab].half = 0;
           ms.cmeta[ab].flags = 2;
           ms.emeta[tile_i & 1].flags = 2;
-          tc::mbar_arrive(&emeta_full[tile_i & 1]);
         }
+        if (ctid < kNodes * kR) tc::mbar_arrive(&emeta_full[tile_i & 1]);
         tc::mbar_arrive(&ms.conv_done[ab]);
         break;
       }
@@ -375,10 +382,9 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
 #pragma unroll
         for (int j = 0; j < kNodes; ++j) em.mask[j] = mt.mask[j];
       }
-      if (mt.half == 0) {
-        if (ctid < kNodes * kR) ms.emeta[tile_i & 1].bhat[ctid] = ms.bhat_raw[slot][ctid];
-        tc::named_sync(1, kConv);
-        if (ctid == 0) tc::mbar_arrive(&emeta_full[tile_i & 1]);
+      if (mt.half == 0 && ctid < kNodes * kR) {
+        ms.emeta[tile_i & 1].bhat[ctid] = ms.bhat_raw[slot][ctid];
+        tc::mbar_arrive(&emeta_full[tile_i & 1]);      // after this thread's writes (thread 0: the header)
       }
       // Raw half: [2 boxes of 32 columns][128 rows][128 B] fp32, 128-byte
       // swizzled. Thread = (row cr, box cb): its 32 values -> three terms of 16
@@ -431,14 +437,7 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
       const float bhat_r = ms.emeta[b].bhat[r];
       if (em_flags & 2) break;
       float v[kQn];
-      tc::tmem_ld32(tbase + t_lane + uint32_t(b) * 128, v);
-#pragma unroll
-      for (int g4 = 0; g4 < 4; ++g4) {            // + column groups 32..63 and 64..95, 16 at a time
-        float w[16];
-        tc::tmem_ld16(tbase + t_lane + uint32_t(b) * 128 + 32 + 16 * g4, w);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[16 * (g4 & 1) + i] += w[i];
-      }
+      tc::tmem_ld32(tbase + t_lane + uint32_t(b) * 32, v);
       tc::fence_before_sync();
       tc::mbar_arrive(&ms.d_free[b]);
       const int64_t node = int64_t(em_node0) + nj;
