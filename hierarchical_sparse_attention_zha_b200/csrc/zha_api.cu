@@ -81,6 +81,8 @@ static zha_status make_geom(const zha_config* c, zha::Geom* g, size_t* bytes) {
   G.kv_bf16 = c->kv_dtype == ZHA_BF16;
   G.scale = float(1.0 / std::sqrt(double(c->head_dim)));
   G.max_tokens = c->max_tokens;
+  G.wait_polls = 1u << 15;                     // ~2 s with the waits' suspend hint
+  G.debug_withhold = 0;
   G.rope_pairs = c->rope_pairs;
   G.rope_log2_base = c->rope_pairs > 0 ? std::log2(double(c->rope_base)) : 0.0;
   int64_t off = 0;
@@ -146,6 +148,13 @@ zha_status zha_tree_create(const zha_config* cfg, void* d_store, size_t store_by
 }
 
 void zha_tree_destroy(zha_tree* tree) { delete tree; }
+
+zha_status zha_tree_debug(zha_tree* tree, uint32_t wait_polls, int32_t withhold) {
+  if (tree == nullptr) return fail(ZHA_ERR_INVALID, "zha_tree_debug: tree is NULL");
+  tree->geom.wait_polls = wait_polls == 0 ? 1u << 15 : wait_polls;
+  tree->geom.debug_withhold = withhold != 0;
+  return ZHA_OK;
+}
 
 int64_t zha_tree_built_tokens(const zha_tree* tree) { return tree ? tree->nb : -1; }
 

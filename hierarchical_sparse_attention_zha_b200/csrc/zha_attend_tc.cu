@@ -514,6 +514,10 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           __syncwarp();
           if (t + 1 < t1) prefetch(t + 1);
         }
+        // Every tensor copy issued into the stages lands before the CTA may exit.
+        if (lane == 0)
+          for (int64_t j = li > kStages ? li - kStages : 0; j < li; ++j)
+            if (!tc::mbar_wait(&ms.full[j % kStages], uint32_t((j / kStages) & 1), kWaitTries)) failed = true;
         if (failed && lane == 0) atomicOr(&ms.err, 1u);
         if (__any_sync(0xffffffffu, bad_page) && lane == 0 && status != nullptr)
           atomicOr(status, ZHA_DEV_BAD_PAGE);

@@ -40,7 +40,7 @@ constexpr uint32_t bTmemCols = 256;                  // S at 0 (48 cols), khat a
 constexpr uint32_t bTmemK = 128;
 
 struct BMisc {
-  uint64_t full[bStages], empty[bStages], s_full, s_free, w_ready, k_full, k_free, q_ready;
+  uint64_t full[bStages], empty[bStages], s_full, s_free, w_ready, k_full, k_free, q_ready, drain;
   uint32_t tmem_base, err;
   float red[4][bR];
   float F[4][bR];                                    // per chunk of the tile (<= 4 chunks)
@@ -90,6 +90,7 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
     tc::mbar_init(&ms.k_full, 1);
     tc::mbar_init(&ms.k_free, 128);
     tc::mbar_init(&ms.q_ready, 128);
+    tc::mbar_init(&ms.drain, 1);
   }
   if (warp == 1) tc::tmem_alloc(&ms.tmem_base, bTmemCols);
   tc::fence_before_sync();
@@ -101,7 +102,8 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int64_t li = 0; li < my_tiles; ++li) {
+      int64_t li = 0;
+      for (; li < my_tiles; ++li) {
         const int64_t t = blockIdx.x + li * gridDim.x;
         const int st = int(li % bStages);
         const int64_t use = li / bStages;
@@ -115,6 +117,9 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
         tc::tma_load_3d(dst, &tmK, 0, tok0, g, &ms.full[st]);
         tc::tma_load_3d(dst + 16384, &tmK, 64, tok0, g, &ms.full[st]);
       }
+      // Every tensor copy issued lands before the CTA may exit.
+      for (int64_t j = li > bStages ? li - bStages : 0; j < li; ++j)
+        if (!tc::mbar_wait(&ms.full[j % bStages], uint32_t((j / bStages) & 1), kTries)) atomicOr(&ms.err, 1u);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -151,6 +156,9 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
         tc::mma_commit(&ms.k_full);
         tc::mma_commit(&ms.empty[st]);
       }
+      // Every MMA issued completes before TMEM is released.
+      tc::mma_commit(&ms.drain);
+      if (!tc::mbar_wait(&ms.drain, 0u, kTries)) failed = true;
       if (failed) atomicOr(&ms.err, 1u);
     }
   } else {

@@ -23,6 +23,8 @@ struct Geom {
   float scale;                           // 1 / sqrt(d)
   int32_t rope_pairs;                    // rotated element pairs (0: position-free)
   double rope_log2_base;                 // log2 of the rotation base
+  uint32_t wait_polls;                   // polls of a bounded mbarrier wait before it gives up
+  int32_t debug_withhold;                // test hook: the level scoring's producer sends nothing
   int64_t max_tokens;
   int64_t cap[ZHA_MAX_LEVELS + 2];       // node capacity per KV head, index by level
   int64_t off[ZHA_MAX_LEVELS + 2];       // float offset of level l's [hkv][cap][node] block

@@ -7,18 +7,20 @@
 // prefix holding estimated mass p, pass the kept nodes' children and the
 // parentless chunks down (전제와 한계).
 //
-// Per level l = L..1 the host launches two kernels:
+// The small top levels (a few hundred nodes per KV head) are scored densely,
+// every node for every query head, by score_dense_kernel (zha_dense.cuh) in one
+// launch and selected level after level by select_top_kernel in one launch.
+// Every lower level l takes two launches:
 //   scoring -- head_dim 128 with R = 16: score_tma_kernel (zha_score_tma.cu,
 //              tensor copies + tcgen05); head_dim 128 with R < 16:
 //              score_tc_kernel (zha_score_tc.cu); otherwise score_kernel here
 //              (one warp per candidate node -- the union over the query heads of
 //              a KV head -- its R planes in registers, one score per query head
 //              that has the node as candidate);
-//   selection -- one CTA per query head: softmax over its candidates, the cut
-//              on the key (score desc, node index asc) by fixed-point mass, kept
-//              bitmap (and at level 1 the ascending chunk list).
-//              select_fast_kernel when the level fits in shared memory
-//              (<= 16384 nodes), select_kernel otherwise.
+//   selection -- select_fast_kernel, one CTA per query head: softmax over its
+//              candidates, the cut on the key (score desc, node index asc) by
+//              fixed-point mass, kept bitmap (and at level 1 the ascending
+//              chunk list).
 // Both kinds are launched with programmatic dependent launch.
 #include "zha_host.cuh"
 #include "zha_internal.cuh"
@@ -279,20 +281,21 @@ __device__ float block_sum(float v, float* tmp) {
 // Candidates in candidate order (ascending node index): the children of the
 // kept parents (compacted from the level above's bitmap), then the level's
 // orphans. With at most kFastMax candidates every candidate's order key (score
-// descending, then index ascending) and its softmax mass in 2^-32 fixed point
-// are computed once into shared memory:
-//  * up to kFastSmallN candidates: thread i counts the mass of every candidate
-//    ordered before it; i is kept iff that mass is below p (the minimal prefix
-//    holding mass p). No radix passes, a handful of barriers.
-//  * more: the cut key by a radix select over 8-bit digits with per-warp
-//    histograms of mass, starting at the first byte in which the candidates'
-//    keys differ; runs of equal buckets are summed in registers before the
-//    atomic add.
-// The rounding of the fixed-point masses adds at most n 2^-33 to any
-// cumulative mass (< 2e-6 at n = 16384). Wider candidate sets (generic path):
-// scores cached when they fit, masses recomputed per pass in 2^-40 fixed point,
-// four radix passes. The fixed-budget mode (top-k) runs the same cut with a
-// mass of exactly 1 per candidate and the threshold k, so it keeps the first
+// descending, then index ascending) and its softmax mass in 2^-31 fixed point
+// are computed once into shared memory. The cut is then found in a window of
+// keys [lo, lo + 2^span), narrowed pass by pass: a 2048-bin histogram of mass
+// (and count) over the window's keys, the bin where the cumulative mass
+// (with everything before the window) reaches p becomes the next window. Once
+// the window holds at most kFastSmallN candidates, each of them counts the mass
+// ordered before it among them (keys, then candidate index) and is kept iff
+// that mass is below p -- the minimal prefix holding mass p. A window of one
+// key (all tied) keeps its first candidates in candidate order. The rounding
+// of the fixed-point masses adds at most n 2^-32 to any cumulative mass
+// (< 4e-6 at n = 16384). Wider candidate sets (generic path): scores cached
+// when they fit, masses recomputed per pass in 2^-40 fixed point, four radix
+// passes of 8 bits with per-warp histograms. The fixed-budget mode (top-k)
+// runs the same cut with a mass of exactly 1 per candidate and the threshold
+// k, so it keeps the first
 // min(k, n) candidates of the order.
 // ---------------------------------------------------------------------------
 struct SelectArgs {

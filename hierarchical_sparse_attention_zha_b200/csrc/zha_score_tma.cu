@@ -25,15 +25,13 @@
 //                           the MMA reads its A operand (shared memory only carries
 //                           the raw tiles and Q)
 //   MMA issuer (warp 1)     S^T[(node, plane)][head] over the half's 4 K-steps:
-//                           the six products A_ti . q_j^T with i + j <= 2 (the
-//                           dropped ones are below fp32 rounding), each N = 32,
-//                           accumulated into one 32-column TMEM buffer (of two):
-//                           the terms are stacked along K, not along N
-//   epilogue (warps 12-15)  thread = (node, plane) row: one 32-column load,
-//                           x 1/sqrt(d) + bhat, maximum over the node's 16
+//                           A_t0 . [q0 | q1 | q2]^T (N = 96), A_t1 . [q0 | q1]^T
+//                           (N = 64), A_t2 . q0^T (N = 32) into one of two TMEM
+//                           buffers -- the six products with term indices summing
+//                           to <= 2, the dropped ones are below fp32 rounding
+//   epilogue (warps 12-15)  thread = (node, plane) row: sum of the three column
+//                           groups, x 1/sqrt(d) + bhat, maximum over the node's 16
 //                           planes, scores of the candidate (node, head) pairs
-// The converters pace themselves on the mbarriers alone (no CTA-wide barrier
-// in their loop).
 // Every wait is bounded; a time-out sets ZHA_DEV_TIMEOUT and the roles stop.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -58,10 +56,9 @@ constexpr int kOffMisc = kOffQ + 2 * 12288;
 constexpr int kThreads = 512;             // warps: 0 producer, 1 MMA, 2-3 idle, 4-11 convert, 12-15 epilogue
 constexpr int kConv = 256;                // converter threads (warps 4-11)
 constexpr int kEpiWarp0 = 12;
-constexpr uint32_t kWaitTries = tc::kWaitPolls;
-constexpr uint32_t kTmemCols = 512;       // D buffers (32 columns) at 0 and 32; A half-buffers
-constexpr uint32_t kTmemA = 64;           // (3 terms x 32 columns) at 64, 160, 256 and 352
-constexpr int kABufs = 4;
+constexpr uint32_t kTmemCols = 512;       // D buffers (96 columns) at 0 and 128; A half-buffers
+constexpr uint32_t kTmemA = 224;          // (3 terms x 32 columns) at 224, 320 and 416
+constexpr int kABufs = 3;
 
 struct Meta {                             // one half-tile, producer -> converters
   int32_t node0, group, half, flags;      // flags: 1 = first tile of a group, 2 = end
@@ -78,7 +75,7 @@ struct EMeta {                            // converters -> epilogue, per tile
 
 struct Misc {
   uint64_t raw_full[kRawSlots], raw_empty[kRawSlots];
-  uint64_t conv_done[kABufs], a_free[kABufs], d_full[2], d_free[2], q_ready;
+  uint64_t conv_done[kABufs], a_free[kABufs], d_full[2], d_free[2], q_ready, drain;
   uint32_t tmem_base, err;
   Meta meta[kRawSlots];
   alignas(128) float bhat_raw[kRawSlots][kNodes * kR];  // tensor-copied with the first half of a tile
@@ -157,9 +154,10 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&ms.d_full[b], 1);
       tc::mbar_init(&ms.d_free[b], 128);
-      tc::mbar_init(&emeta_full[b], 128);      // the converter threads that write the tile's bhat
+      tc::mbar_init(&emeta_full[b], 1);
     }
     tc::mbar_init(&ms.q_ready, kConv);
+    tc::mbar_init(&ms.drain, 1);
   }
   pdl_trigger();
   if (warp == 1) tc::tmem_alloc(&ms.tmem_base, kTmemCols);
@@ -193,7 +191,9 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
     };
     uint32_t nw0 = 0u, nw1 = 0u;
     if (t0 < t1) load_words(int32_t(t0), nw0, nw1);
-    for (int32_t t = int32_t(t0); int64_t(t) < t1 && !failed; ++t) {
+    // Test hook: send nothing, so that every consumer's bounded wait runs out.
+    const int32_t t_stop = G.debug_withhold ? int32_t(t0) : int32_t(t1);
+    for (int32_t t = int32_t(t0); t < t_stop && !failed; ++t) {
       const uint32_t w0 = nw0, w1 = nw1;
       load_words(t + 1, nw0, nw1);
       const int v = t / nt32;
@@ -220,7 +220,7 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
         const int slot = int(k % kRawSlots);
         const int64_t use = k / kRawSlots;
         bool bad = false;
-        if (use > 0) bad = !tc::mbar_wait(&ms.raw_empty[slot], uint32_t((use - 1) & 1), kWaitTries);
+        if (use > 0) bad = !tc::mbar_wait(&ms.raw_empty[slot], uint32_t((use - 1) & 1), G.wait_polls);
         if (__any_sync(0xffffffffu, bad)) { failed = true; break; }
         if (lane == 0) {
           Meta& mt = ms.meta[slot];
@@ -239,34 +239,51 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
         __syncwarp();
       }
     }
-    if (!failed) {                                 // end of the stream
+    bool sent_end = false;
+    if (!failed && !G.debug_withhold) {            // end of the stream
       const int slot = int(k % kRawSlots);
       const int64_t use = k / kRawSlots;
       bool bad = false;
-      if (use > 0) bad = !tc::mbar_wait(&ms.raw_empty[slot], uint32_t((use - 1) & 1), kWaitTries);
+      if (use > 0) bad = !tc::mbar_wait(&ms.raw_empty[slot], uint32_t((use - 1) & 1), G.wait_polls);
       if (__any_sync(0xffffffffu, bad)) {
         failed = true;
-      } else if (lane == 0) {
-        ms.meta[slot].flags = 2;
-        tc::mbar_arrive(&ms.raw_full[slot]);
+      } else {
+        sent_end = true;
+        if (lane == 0) {
+          ms.meta[slot].flags = 2;
+          tc::mbar_arrive(&ms.raw_full[slot]);
+        }
       }
+    }
+    // Before the CTA may exit, every tensor copy issued into shared memory has
+    // landed: wait for the last copy of each slot (already complete when the
+    // converters consumed it). The end marker reused the slot of copy k - 5
+    // only after the converters had taken that copy, and moved that slot's
+    // phase on, so that copy is not waited for again.
+    if (lane == 0) {
+      const int64_t j0 = (k > kRawSlots ? k - kRawSlots : 0) + (sent_end && k >= kRawSlots ? 1 : 0);
+      for (int64_t j = j0; j < k; ++j)
+        if (!tc::mbar_wait(&ms.raw_full[j % kRawSlots], uint32_t((j / kRawSlots) & 1), G.wait_polls))
+          failed = true;
     }
     if (failed && lane == 0) atomicOr(&ms.err, 1u);
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
+      constexpr uint32_t idesc96 = tc::idesc_bf16(128, 96, 0, 0);
+      constexpr uint32_t idesc64 = tc::idesc_bf16(128, 64, 0, 0);
       constexpr uint32_t idesc32 = tc::idesc_bf16(128, 32, 0, 0);
       int64_t k = 0, tile_i = 0;
       int seg = 0;
       bool failed = false;
       while (true) {
         const int ab = int(k % kABufs);
-        if (!tc::mbar_wait(&ms.conv_done[ab], uint32_t((k / kABufs) & 1), kWaitTries)) { failed = true; break; }
+        if (!tc::mbar_wait(&ms.conv_done[ab], uint32_t((k / kABufs) & 1), G.wait_polls)) { failed = true; break; }
         const CMeta cm = ms.cmeta[ab];
         if (cm.half == 0 || (cm.flags & 2)) {
           // The D buffer of this tile must have been read by the epilogue.
           if (tile_i >= 2 &&
-              !tc::mbar_wait(&ms.d_free[tile_i & 1], uint32_t(((tile_i >> 1) - 1) & 1), kWaitTries)) {
+              !tc::mbar_wait(&ms.d_free[tile_i & 1], uint32_t(((tile_i >> 1) - 1) & 1), G.wait_polls)) {
             failed = true;
             break;
           }
@@ -276,25 +293,19 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
           break;
         }
         if (cm.half == 0 && (cm.flags & 1)) {
-          if (!tc::mbar_wait(&ms.q_ready, uint32_t(seg & 1), kWaitTries)) { failed = true; break; }
+          if (!tc::mbar_wait(&ms.q_ready, uint32_t(seg & 1), G.wait_polls)) { failed = true; break; }
           ++seg;
         }
         tc::fence_after_sync();
-        const uint32_t d = tbase + uint32_t(tile_i & 1) * 32;
+        const uint32_t d = tbase + uint32_t(tile_i & 1) * 128;
         const uint32_t tA = tbase + kTmemA + uint32_t(ab) * 96;      // term t at + 32 t
-        const uint32_t sQ = tc::smem_u32(smem + kOffQ) + uint32_t(cm.half) * 12288;   // term j rows at + 4096 j
+        const uint32_t sQ = tc::smem_u32(smem + kOffQ) + uint32_t(cm.half) * 12288;
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {           // K-step = 16 bf16 = 8 TMEM columns
-          const uint64_t q0 = tc::desc_sw128(sQ + ks * 32, 16, 1024);
-          const uint64_t q1 = tc::desc_sw128(sQ + 4096 + ks * 32, 16, 1024);
-          const uint64_t q2 = tc::desc_sw128(sQ + 8192 + ks * 32, 16, 1024);
-          const uint32_t a0 = tA + ks * 8, a1 = tA + 32 + ks * 8, a2 = tA + 64 + ks * 8;
-          tc::mma_bf16_ta(d, a0, q0, idesc32, (cm.half == 0 && ks == 0) ? 0u : 1u);
-          tc::mma_bf16_ta(d, a0, q1, idesc32, 1u);
-          tc::mma_bf16_ta(d, a0, q2, idesc32, 1u);
-          tc::mma_bf16_ta(d, a1, q0, idesc32, 1u);
-          tc::mma_bf16_ta(d, a1, q1, idesc32, 1u);
-          tc::mma_bf16_ta(d, a2, q0, idesc32, 1u);
+          const uint64_t b = tc::desc_sw128(sQ + ks * 32, 16, 1024);
+          tc::mma_bf16_ta(d, tA + ks * 8, b, idesc96, (cm.half == 0 && ks == 0) ? 0u : 1u);
+          tc::mma_bf16_ta(d, tA + 32 + ks * 8, b, idesc64, 1u);
+          tc::mma_bf16_ta(d, tA + 64 + ks * 8, b, idesc32, 1u);
         }
         tc::mma_commit(&ms.a_free[ab]);
         if (cm.half == 1) {
@@ -303,6 +314,9 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
         }
         ++k;
       }
+      // Every MMA issued so far completes before TMEM is released.
+      tc::mma_commit(&ms.drain);
+      if (!tc::mbar_wait(&ms.drain, 0u, G.wait_polls)) failed = true;
       if (failed) atomicOr(&ms.err, 1u);
     }
   } else if (warp >= 4 && warp < kEpiWarp0) {
@@ -317,31 +331,30 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
       const int slot = int(k % kRawSlots);
       const int64_t use = k / kRawSlots;
       const int ab = int(k % kABufs);
-      if (!tc::mbar_wait(&ms.raw_full[slot], uint32_t(use & 1), kWaitTries)) { failed = true; break; }
+      bool bad = !tc::mbar_wait(&ms.raw_full[slot], uint32_t(use & 1), G.wait_polls);
+      if (tc::named_sync_or(1, kConv, bad)) { failed = true; break; }
       const Meta mt = ms.meta[slot];
-      bool bad = false;
       const bool end = (mt.flags & 2) != 0;
-      // A half-buffer ab was last read by the MMAs of half k - kABufs; the
-      // tile's metadata slot by the epilogue of tile_i - 2 (also before the end
-      // marker: the MMA issuer reads cmeta[ab] of half k - kABufs first). Each
-      // thread waits for itself; the arrivals count every converter thread.
+      // A half-buffer ab was last read by the MMAs of half k - 2; the tile's
+      // metadata slot by the epilogue of tile_i - 2.
+      // (also before the end marker: the MMA issuer reads cmeta[ab] of half k - 3 first)
       if (k >= kABufs)
-        bad |= !tc::mbar_wait(&ms.a_free[ab], uint32_t(((k / kABufs) - 1) & 1), kWaitTries);
+        bad |= !tc::mbar_wait(&ms.a_free[ab], uint32_t(((k / kABufs) - 1) & 1), G.wait_polls);
       if ((end || mt.half == 0) && tile_i >= 2)
-        bad |= !tc::mbar_wait(&ms.d_free[tile_i & 1], uint32_t(((tile_i >> 1) - 1) & 1), kWaitTries);
+        bad |= !tc::mbar_wait(&ms.d_free[tile_i & 1], uint32_t(((tile_i >> 1) - 1) & 1), G.wait_polls);
       // A new group's Q replaces the old one once every MMA that reads it (the
       // previous half's) is complete.
       const bool new_q = !end && mt.half == 0 && (mt.flags & 1);
       if (new_q && k >= 1)
-        bad |= !tc::mbar_wait(&ms.a_free[(k - 1) % kABufs], uint32_t(((k - 1) / kABufs) & 1), kWaitTries);
-      if (bad) { failed = true; break; }
+        bad |= !tc::mbar_wait(&ms.a_free[(k - 1) % kABufs], uint32_t(((k - 1) / kABufs) & 1), G.wait_polls);
+      if (tc::named_sync_or(1, kConv, bad)) { failed = true; break; }
       if (end) {
         if (ctid == 0) {
           ms.cmeta[ab].half = 0;
           ms.cmeta[ab].flags = 2;
           ms.emeta[tile_i & 1].flags = 2;
+          tc::mbar_arrive(&emeta_full[tile_i & 1]);
         }
-        if (ctid < kNodes * kR) tc::mbar_arrive(&emeta_full[tile_i & 1]);
         tc::mbar_arrive(&ms.conv_done[ab]);
         break;
       }
@@ -382,9 +395,10 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
 #pragma unroll
         for (int j = 0; j < kNodes; ++j) em.mask[j] = mt.mask[j];
       }
-      if (mt.half == 0 && ctid < kNodes * kR) {
-        ms.emeta[tile_i & 1].bhat[ctid] = ms.bhat_raw[slot][ctid];
-        tc::mbar_arrive(&emeta_full[tile_i & 1]);      // after this thread's writes (thread 0: the header)
+      if (mt.half == 0) {
+        if (ctid < kNodes * kR) ms.emeta[tile_i & 1].bhat[ctid] = ms.bhat_raw[slot][ctid];
+        tc::named_sync(1, kConv);
+        if (ctid == 0) tc::mbar_arrive(&emeta_full[tile_i & 1]);
       }
       // Raw half: [2 boxes of 32 columns][128 rows][128 B] fp32, 128-byte
       // swizzled. Thread = (row cr, box cb): its 32 values -> three terms of 16
@@ -428,8 +442,8 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
     while (true) {
       const int b = int(tile_i & 1);
       const uint32_t ph = uint32_t((tile_i >> 1) & 1);
-      bool bad = !tc::mbar_wait(&emeta_full[b], ph, kWaitTries);
-      bad |= !tc::mbar_wait(&ms.d_full[b], ph, kWaitTries);
+      bool bad = !tc::mbar_wait(&emeta_full[b], ph, G.wait_polls);
+      bad |= !tc::mbar_wait(&ms.d_full[b], ph, G.wait_polls);
       if (tc::named_sync_or(3, 128, bad)) { failed = true; break; }
       tc::fence_after_sync();
       const int32_t em_flags = ms.emeta[b].flags, em_node0 = ms.emeta[b].node0, em_group = ms.emeta[b].group;
@@ -437,7 +451,14 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
       const float bhat_r = ms.emeta[b].bhat[r];
       if (em_flags & 2) break;
       float v[kQn];
-      tc::tmem_ld32(tbase + t_lane + uint32_t(b) * 32, v);
+      tc::tmem_ld32(tbase + t_lane + uint32_t(b) * 128, v);
+#pragma unroll
+      for (int g4 = 0; g4 < 4; ++g4) {            // + column groups 32..63 and 64..95, 16 at a time
+        float w[16];
+        tc::tmem_ld16(tbase + t_lane + uint32_t(b) * 128 + 32 + 16 * g4, w);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[16 * (g4 & 1) + i] += w[i];
+      }
       tc::fence_before_sync();
       tc::mbar_arrive(&ms.d_free[b]);
       const int64_t node = int64_t(em_node0) + nj;

@@ -133,6 +133,7 @@ def _load() -> ctypes.CDLL:
                                            P, c_size_t, P, P]),
         "zha_diagnostics_workspace_bytes": (c_size_t, [POINTER(Config), c_int32, c_int64]),
         "zha_route_diagnostics": (c_int32, [P, P, P, c_int64, c_int32, c_int64, P, P, P, c_size_t, P]),
+        "zha_tree_debug": (c_int32, [P, ctypes.c_uint32, c_int32]),
         "zha_trace_enable": (c_int32, [c_int32, c_char_p, c_int32]),
         "zha_trace_count": (c_int32, []),
         "zha_trace_dropped": (c_int32, []),

@@ -326,6 +326,16 @@ zha_status zha_route_diagnostics(const zha_tree* tree, const float* d_Q, const v
                                  int32_t batch, int64_t n_tokens, float* d_kl, uint32_t* d_usage,
                                  void* d_ws, size_t ws_bytes, void* stream);
 
+/* ---- Test hook (the pages have no counterpart) ------------------------------
+ * For tests of the bounded waits of this tree's tensor-core level scoring
+ * (head_dim 128, R = 16): wait_polls = polls of each of its mbarrier waits
+ * before the wait gives up (0 restores the default, about 2 s; each poll lets
+ * the thread sleep up to about 65 us); withhold != 0 makes its producer send
+ * nothing, so that the consumers' waits run out with nothing in flight: the
+ * kernel releases its tensor memory, returns, and the route reports
+ * ZHA_DEV_TIMEOUT (its outputs are then not valid). Not for production use. */
+zha_status zha_tree_debug(zha_tree* tree, uint32_t wait_polls, int32_t withhold);
+
 /* ---- Kernel timing (profiling; the pages have no counterpart) ------------
  * While enabled, every kernel the library launches whose name contains
  * `name_filter` (NULL or "" = all) and whose tag equals `tag_filter` (-1 = all;

@@ -722,3 +722,32 @@ def test_paged_append_and_a_page_outside_the_pool(zha):
     torch.cuda.synchronize()
     assert int(st2.item()) & zha.ZHA_DEV_BAD_PAGE
     assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+
+
+def test_bounded_wait_times_out_cleanly_and_the_next_call_is_clean(zha, parity_log):
+    """The level scoring's producer withholds everything (test hook), so its
+    consumers' bounded waits (16 polls, ~1 ms) run out with nothing in flight:
+    the route returns within the bound with ZHA_DEV_TIMEOUT set. With the hook
+    cleared, the next route on the same tree is clean and matches the oracle."""
+    import time
+    spec = W.scaled("1m", n_kv_heads=1, n_q_heads=8, n_tokens=8192, stream_tokens=64, batch=2,
+                    n_needles=0)
+    inp = W.generate(spec)
+    dev = to_device(inp)
+    K, V, refq, Q = dev
+    n_tokens = 8192 + 5
+    tree = zha.Tree(config_for(spec), refq)
+    tree.build(K, n_tokens)
+    q = Q[0].contiguous()
+    torch.cuda.synchronize()
+    assert zha.lib.zha_tree_debug(tree.handle, 16, 1) == zha.ZHA_OK
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    tree.route(q, n_tokens, spec.p, n_tokens // spec.chunk, status=st)
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    assert int(st.item()) & zha.ZHA_DEV_TIMEOUT
+    assert elapsed < 5.0
+    assert zha.lib.zha_tree_debug(tree.handle, 0, 0) == zha.ZHA_OK
+    rep = check_case(zha, inp, n_tokens, tree=tree, dev=dev)       # asserts a zero status
+    parity_log("after_timeout", rep)
