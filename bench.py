@@ -65,10 +65,14 @@ def parse():
     return ap.parse_args()
 
 
-def measured_traffic(workload: str, kernel_key: str):
+def measured_traffic(workload: str, kernel_key: str, alg_bytes: float):
     """DRAM bytes per launch of `kernel_key` measured by ncu on this workload
     (profiles/traffic_<workload>.json), or None. The record names the kernel's
-    source file and its SHA-256 when captured; a changed source voids it."""
+    source file and its SHA-256 when captured; a changed source voids it. A
+    record taken on a smaller context of the same configuration holds the ratio
+    of DRAM bytes to the launch's algorithmic bytes instead, and the traffic of
+    a full launch is that ratio times `alg_bytes` (the launch's algorithmic
+    bytes here)."""
     import hashlib
     path = os.path.join(ROOT, "profiles", f"traffic_{workload.lower().replace(' ', '_')}.json")
     if not os.path.exists(path):
@@ -81,6 +85,11 @@ def measured_traffic(workload: str, kernel_key: str):
     src = os.path.join(ROOT, rec["source"])
     if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["source_sha256"]:
         return None, f"ncu traffic of {kernel_key} predates the current {rec['source']}"
+    if "dram_per_algorithmic" in rec:
+        return float(rec["dram_per_algorithmic"]) * alg_bytes, (
+            f"ncu dram__bytes_read.sum + dram__bytes_write.sum of one {kernel_key} launch = "
+            f"{rec['dram_per_algorithmic']:.4f} x its algorithmic bytes, scaled to this launch's "
+            f"algorithmic bytes ({rec.get('note', 'see profiles/')})")
     return float(rec["dram_bytes_per_launch"]), (
         f"ncu dram__bytes_read.sum + dram__bytes_write.sum of one {kernel_key} launch "
         f"({rec.get('note', 'see profiles/')})")
@@ -574,7 +583,7 @@ def run_zha(args, world, rank, local):
     roofline = None
     if len(dom_ms) == K_steps and all(b is not None for b in dom_b) and sum(dom_ms) > 0:
         ach = sum(dom_b) / (sum(dom_ms) * 1e-3) / 1e9
-        traffic, traffic_note = measured_traffic(spec.name, dom_key)
+        traffic, traffic_note = measured_traffic(spec.name, dom_key, float(np.mean(dom_b)))
         roofline = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                     "traffic": traffic, "traffic_note": traffic_note, "kernel": dom_key,
                     "bytes_per_launch": float(np.mean(dom_b)), "mean_us": float(np.mean(dom_ms)) * 1e3,

@@ -1,5 +1,5 @@
 // zha_build_tc.cu -- level-1 tree build on the sm_100a tensor cores (bf16
-// caches, head_dim 128, R = 16, C = 64).
+// caches, head_dim 128, R = 16, C = 16, 32, 64 or 128).
 //
 // Citations: [ZHA: 무엇과 다른가] = page "ZHA는 KV 캐시를 트리로 요약해 어텐션 비용을
 // 준(sub)이차로 낮춘다" (onedev.kr/papers/1556), section "무엇과 다른가": the chunk's
@@ -10,14 +10,19 @@
 //   S[t][r]  = k_t . q_r / sqrt(d)          tcgen05.mma, A = K tile (K-major),
 //                                           B = q in three bf16 terms stacked
 //                                           along N (N = 48), TMEM [128][48]
-//   per (chunk, plane): F = LSE_t S, W[t][r] = exp(S - F)   (softmax warps)
+//   per (chunk, plane): F = LSE_t S, W[t][r] = exp(S - F)   (softmax warps; a
+//                                           chunk's rows are half a warp (C = 16),
+//                                           one warp or several)
 //   khat^T[d][r] = sum_t K[t][d] W[t][r]    tcgen05.mma per chunk, A = the same
 //                                           K tile read MN-major (M = d), B = W
 //                                           in two bf16 terms (N = 32)
 //   bhat_r = F - q_r . khat_r / sqrt(d)     epilogue (thread = d row)
 // Roles: warp 0 tensor copies of K (2 stages; rows past the built prefix read
-// as zeros), warp 1 MMA issuer, warps 2-5 softmax + epilogue (TMEM lane
-// quadrants 2, 3, 0, 1). Every wait is bounded.
+// as zeros), warp 1 MMA issuer, warps 2-5 softmax (thread = token row), warps
+// 6-9 epilogue (thread = d row); each group covers the TMEM lane quadrants 2,
+// 3, 0, 1. W, F and the khat accumulators are double-buffered (khat when two
+// buffers fit in TMEM), so the epilogue of one tile overlaps the softmax of
+// the next. Every wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -33,20 +38,34 @@ constexpr int bTok = 128, bD = 128, bR = 16;
 constexpr int bStages = 2;
 constexpr int bStageBytes = 32768;                   // K tile [2 halves][128 rows][128 B]
 constexpr int bOffQ = bStages * bStageBytes;         // [2 halves][48 rows][128 B]
-constexpr int bOffW = bOffQ + 2 * 6144;              // W [128 tokens][32 = 16 planes x 2 terms] SW64
-constexpr int bOffMisc = bOffW + 8192;
-constexpr int bThreads = 192;
-constexpr uint32_t bTmemCols = 256;                  // S at 0 (48 cols), khat at 128 (<= 4 x 32)
-constexpr uint32_t bTmemK = 128;
+constexpr int bWBytes = 8192;                        // W [128 tokens][32 = 16 planes x 2 terms] SW64
+constexpr int bOffW = bOffQ + 2 * 6144;              // two W buffers
+constexpr int bOffMisc = bOffW + 2 * bWBytes;
+constexpr int bThreads = 320;                        // warps: 0 copies, 1 MMA, 2-5 softmax, 6-9 epilogue
+constexpr uint32_t bTmemK = 64;                      // S at 0 (48 cols), khat buffers from 64 (32 per chunk)
+constexpr int bMaxChunks = bTok / 16;                // chunks per tile at C = 16
+
+// khat buffers in TMEM: two when they fit in 256 columns after S, else one.
+__host__ __device__ inline int build_khat_bufs(int chunk) {
+  return bTmemK + 2u * uint32_t(bTok / chunk) * 32u <= 256u ? 2 : 1;
+}
+// TMEM columns of a CTA.
+__host__ __device__ inline uint32_t build_tmem_cols(int chunk) {
+  return bTmemK + uint32_t(build_khat_bufs(chunk) * (bTok / chunk)) * 32u <= 256u ? 256u : 512u;
+}
 
 struct BMisc {
-  uint64_t full[bStages], empty[bStages], s_full, s_free, w_ready, k_full, k_free, q_ready, drain;
+  uint64_t full[bStages], empty[bStages], s_full, s_free, w_ready[2], k_full[2], k_free[2], q_ready, drain;
   uint32_t tmem_base, err;
-  float red[4][bR];
-  float F[4][bR];                                    // per chunk of the tile (<= 4 chunks)
+  float red_max[bMaxChunks][bR];                     // softmax: per reduction unit (half-warp, warp)
+  float red_sum[bMaxChunks][bR];
+  float F[2][bMaxChunks][bR];                        // per W buffer and chunk of the tile
+  float red_e[2][bMaxChunks][4][bR];                 // epilogue: q_r . khat partial sums per warp
 };
 
-__device__ __forceinline__ float tr16(float (&v)[16], bool is_max) {
+// Reduction of 16 values (one per plane) over lanes: afterwards lane L holds
+// plane L & 15 reduced over its half-warp, or over the whole warp (full).
+__device__ __forceinline__ float tr16(float (&v)[16], bool is_max, bool full = true) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int o = 8, half = 8; o > 0; o >>= 1, half >>= 1) {
@@ -59,13 +78,25 @@ __device__ __forceinline__ float tr16(float (&v)[16], bool is_max) {
       v[i] = is_max ? fmaxf(keep, got) : keep + got;
     }
   }
+  if (!full) return v[0];
   const float other = __shfl_xor_sync(0xffffffffu, v[0], 16);
   return is_max ? fmaxf(v[0], other) : v[0] + other;
 }
 
 }  // namespace
 
-__global__ void __launch_bounds__(bThreads, 1)
+// Tiles li = 0, 1, ... of the CTA; W and F buffer wb = li & 1, khat buffer
+// kb = li % kbufs. Barrier waits and the phases they expect:
+//   MMA       S(li + 1): full[stage] and s_free (li);  khat(li): w_ready[wb] (li)
+//             and k_free (tile li - kbufs: the epilogue has read that buffer)
+//   softmax   s_full (li); k_free (li - kbufs: W[wb], F[wb] and the khat buffer
+//             of tile li - 2 or li - 1 are read)
+//   epilogue  w_ready[wb] (li: F of the tile), k_full[kb] (li)
+// None of these barriers can complete the phase after the awaited one before
+// its waiter has passed (each later completion depends on the waiter), so
+// parity waits are unambiguous. The MMA order S(0), S(1), khat(0), S(2),
+// khat(1), ... waits only on work issued before it.
+__global__ void __launch_bounds__(bThreads, 2)
 build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_begin, int64_t c_end,
                    const float* __restrict__ refq, float* __restrict__ store, int32_t* status) {
   extern __shared__ uint8_t smem_raw[];
@@ -75,8 +106,10 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = blockIdx.y;
   const int C = G.chunk, cpt = bTok / C;
+  const int kbufs = build_khat_bufs(C);
   const int64_t n_tiles = (c_end - c_begin + cpt - 1) / cpt;
-  const uint32_t kTries = tc::kWaitPolls;
+  const uint32_t kTries = G.wait_polls;
+  const uint32_t tmem_cols = build_tmem_cols(C);
 
   if (tid == 0) {
     ms.err = 0u;
@@ -86,19 +119,24 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
     }
     tc::mbar_init(&ms.s_full, 1);
     tc::mbar_init(&ms.s_free, 128);
-    tc::mbar_init(&ms.w_ready, 128);
-    tc::mbar_init(&ms.k_full, 1);
-    tc::mbar_init(&ms.k_free, 128);
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&ms.w_ready[b], 128);
+      tc::mbar_init(&ms.k_full[b], 1);
+      tc::mbar_init(&ms.k_free[b], 128);
+    }
     tc::mbar_init(&ms.q_ready, 128);
     tc::mbar_init(&ms.drain, 1);
   }
-  if (warp == 1) tc::tmem_alloc(&ms.tmem_base, bTmemCols);
+  if (warp == 1) tc::tmem_alloc(&ms.tmem_base, tmem_cols);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tbase = ms.tmem_base;
   // this CTA's tiles of head g: t = blockIdx.x, blockIdx.x + gridDim.x, ...
   const int64_t my_tiles = n_tiles > blockIdx.x ? (n_tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  auto khat_col = [&](int64_t li) -> uint32_t {
+    return bTmemK + uint32_t(li % kbufs) * uint32_t(cpt) * 32u;
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -125,13 +163,13 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
     if (lane == 0) {
       constexpr uint32_t idesc_s = tc::idesc_bf16(bTok, 3 * bR, 0, 0);
       constexpr uint32_t idesc_k = tc::idesc_bf16(bD, 2 * bR, 1, 1);
-      const uint32_t sQ = tc::smem_u32(smem + bOffQ), sW = tc::smem_u32(smem + bOffW);
-      bool failed = !tc::mbar_wait(&ms.q_ready, 0u, kTries);
-      for (int64_t li = 0; li < my_tiles && !failed; ++li) {
-        const int st = int(li % bStages);
-        const uint32_t ph = uint32_t(li & 1);
-        if (!tc::mbar_wait(&ms.full[st], uint32_t((li / bStages) & 1), kTries)) { failed = true; break; }
-        if (li > 0 && !tc::mbar_wait(&ms.s_free, ph ^ 1u, kTries)) { failed = true; break; }
+      const uint32_t sQ = tc::smem_u32(smem + bOffQ);
+      bool failed = my_tiles > 0 && !tc::mbar_wait(&ms.q_ready, 0u, kTries);
+      int64_t ns = 0;                                // next tile to score
+      auto issue_s = [&]() -> bool {
+        const int st = int(ns % bStages);
+        if (!tc::mbar_wait(&ms.full[st], uint32_t((ns / bStages) & 1), kTries)) return false;
+        if (ns > 0 && !tc::mbar_wait(&ms.s_free, uint32_t((ns - 1) & 1), kTries)) return false;
         tc::fence_after_sync();
         const uint32_t sK = tc::smem_u32(smem + st * bStageBytes);
 #pragma unroll
@@ -141,30 +179,47 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
           tc::mma_bf16(tbase, a, b, idesc_s, ks != 0 ? 1u : 0u);
         }
         tc::mma_commit(&ms.s_full);
-        // khat per chunk once W is written (and the previous khat was read)
-        if (!tc::mbar_wait(&ms.w_ready, ph, kTries)) { failed = true; break; }
-        if (li > 0 && !tc::mbar_wait(&ms.k_free, ph ^ 1u, kTries)) { failed = true; break; }
+        ++ns;
+        return true;
+      };
+      auto issue_k = [&](int64_t li) -> bool {
+        const int wb = int(li & 1);
+        if (!tc::mbar_wait(&ms.w_ready[wb], uint32_t((li >> 1) & 1), kTries)) return false;
+        if (li >= kbufs) {
+          const int64_t lp = li - kbufs;
+          if (!tc::mbar_wait(&ms.k_free[lp % kbufs], uint32_t((lp / kbufs) & 1), kTries)) return false;
+        }
         tc::fence_after_sync();
+        const int st = int(li % bStages);
+        const uint32_t sK = tc::smem_u32(smem + st * bStageBytes);
+        const uint32_t sW = tc::smem_u32(smem + bOffW + wb * bWBytes);
+        const uint32_t dk = tbase + khat_col(li);
         for (int c = 0; c < cpt; ++c) {
           for (int kk = 0; kk < C / 16; ++kk) {
             const int ks = c * (C / 16) + kk;              // 16-token K-step of the tile
             const uint64_t a = tc::desc_sw128(sK + ks * 2048, 16384, 1024);
             const uint64_t b = tc::desc_sw64(sW + ks * 1024, 8192, 512);
-            tc::mma_bf16(tbase + bTmemK + uint32_t(c) * 32, a, b, idesc_k, kk != 0 ? 1u : 0u);
+            tc::mma_bf16(dk + uint32_t(c) * 32, a, b, idesc_k, kk != 0 ? 1u : 0u);
           }
         }
-        tc::mma_commit(&ms.k_full);
+        tc::mma_commit(&ms.k_full[li % kbufs]);
         tc::mma_commit(&ms.empty[st]);
+        return true;
+      };
+      if (!failed && my_tiles > 0) failed = !issue_s();
+      for (int64_t li = 0; li < my_tiles && !failed; ++li) {
+        if (ns < my_tiles && !issue_s()) { failed = true; break; }
+        if (!issue_k(li)) failed = true;
       }
       // Every MMA issued completes before TMEM is released.
       tc::mma_commit(&ms.drain);
       if (!tc::mbar_wait(&ms.drain, 0u, kTries)) failed = true;
       if (failed) atomicOr(&ms.err, 1u);
     }
-  } else {
-    // ---------------- softmax + epilogue (warps 2-5) ----------------
+  } else if (warp < 6) {
+    // ---------------- softmax (warps 2-5): thread = token row ----------------
     const int q4 = warp & 3;                        // TMEM lane quadrant
-    const int r = q4 * 32 + lane;                   // token row / output dim
+    const int r = q4 * 32 + lane;                   // token row of the tile
     const uint32_t t_lane = uint32_t(q4 * 32) << 16;
     const int stid = tid - 64;                      // 0..127
     const float* qg = refq + int64_t(g) * bR * bD;
@@ -190,16 +245,15 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
     }
     tc::fence_async_smem();
     tc::mbar_arrive(&ms.q_ready);
-    float qd[bR];                                   // q_r[d] for this thread's d row
-#pragma unroll
-    for (int pl = 0; pl < bR; ++pl) qd[pl] = qg[pl * bD + r];
-    const int chunk_of_row = r / C, warps_per_chunk = C / 32;
+    // Reduction units: a chunk of C >= 32 rows spans C / 32 warps (unit = warp),
+    // a chunk of 16 rows is half a warp (unit = half-warp).
+    const bool half_units = C < 32;
+    const int chunk_of_row = r / C, units = half_units ? 1 : C / 32;
+    const int unit = half_units ? 2 * q4 + (lane >> 4) : q4, unit0 = chunk_of_row * units;
     bool failed = false;
-    for (int64_t li = 0; li < my_tiles && !failed; ++li) {
-      const int64_t t = blockIdx.x + li * gridDim.x;
-      const int64_t chunk0 = c_begin + t * cpt;
-      const uint32_t ph = uint32_t(li & 1);
-      bool bad = !tc::mbar_wait(&ms.s_full, ph, kTries);
+    for (int64_t li = 0; li < my_tiles; ++li) {
+      const int wb = int(li & 1);
+      bool bad = !tc::mbar_wait(&ms.s_full, uint32_t(li & 1), kTries);
       tc::fence_after_sync();
       float s[bR];
       {
@@ -212,38 +266,41 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
       }
       tc::fence_before_sync();
       tc::mbar_arrive(&ms.s_free);
-      // previous tile's khat MMA (reads W) must be complete before W is rewritten
-      if (li > 0) bad |= !tc::mbar_wait(&ms.k_full, ph ^ 1u, kTries);
+      // W[wb] and F[wb] are free once the epilogue of tile li - kbufs is done
+      // (it waited for the khat MMA that read W[wb]).
+      if (li >= kbufs) {
+        const int64_t lp = li - kbufs;
+        bad |= !tc::mbar_wait(&ms.k_free[lp % kbufs], uint32_t((lp / kbufs) & 1), kTries);
+      }
       // per (chunk, plane) maximum and sum over the chunk's rows
       float tmp[bR];
 #pragma unroll
       for (int i = 0; i < bR; ++i) tmp[i] = s[i];
-      const float wm = tr16(tmp, true);
-      if (lane < bR) ms.red[q4][lane] = wm;
+      const float wm = tr16(tmp, true, !half_units);
+      if (half_units || lane < bR) ms.red_max[unit][lane & 15] = wm;
       if (tc::named_sync_or(1, 128, bad)) { failed = true; break; }
       float m[bR];
 #pragma unroll
       for (int i = 0; i < bR; ++i) {
         float x = -INFINITY;
-        for (int w = 0; w < warps_per_chunk; ++w) x = fmaxf(x, ms.red[chunk_of_row * warps_per_chunk + w][i]);
+        for (int w = 0; w < units; ++w) x = fmaxf(x, ms.red_max[unit0 + w][i]);
         m[i] = x;
       }
-      tc::named_sync(1, 128);
 #pragma unroll
       for (int i = 0; i < bR; ++i) tmp[i] = expf(s[i] - m[i]);
-      const float wl = tr16(tmp, false);
-      if (lane < bR) ms.red[q4][lane] = wl;
+      const float wl = tr16(tmp, false, !half_units);
+      if (half_units || lane < bR) ms.red_sum[unit][lane & 15] = wl;
       tc::named_sync(1, 128);
       float F[bR];
 #pragma unroll
       for (int i = 0; i < bR; ++i) {
         float l = 0.f;
-        for (int w = 0; w < warps_per_chunk; ++w) l += ms.red[chunk_of_row * warps_per_chunk + w][i];
+        for (int w = 0; w < units; ++w) l += ms.red_sum[unit0 + w][i];
         F[i] = m[i] + logf(l);
       }
       if (r % C == 0) {
 #pragma unroll
-        for (int i = 0; i < bR; ++i) ms.F[chunk_of_row][i] = F[i];
+        for (int i = 0; i < bR; ++i) ms.F[wb][chunk_of_row][i] = F[i];
       }
       // W = exp(S - F) in two bf16 terms, MN-major: token row, 16 planes hi then lo (64 B)
       {
@@ -254,7 +311,7 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
           hi[i] = __float2bfloat16_rn(w);
           lo[i] = __float2bfloat16_rn(w - __bfloat162float(hi[i]));
         }
-        uint8_t* sW = smem + bOffW;
+        uint8_t* sW = smem + bOffW + wb * bWBytes;
         *reinterpret_cast<uint4*>(sW + tc::sw64_mn_chunk(r, 0)) = *reinterpret_cast<const uint4*>(hi);
         *reinterpret_cast<uint4*>(sW + tc::sw64_mn_chunk(r, 1)) = *reinterpret_cast<const uint4*>(hi + 8);
         *reinterpret_cast<uint4*>(sW + tc::sw64_mn_chunk(r, 2)) = *reinterpret_cast<const uint4*>(lo);
@@ -262,17 +319,34 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
       }
       tc::fence_async_smem();
       tc::fence_before_sync();
-      tc::mbar_arrive(&ms.w_ready);
-      // epilogue: khat (thread = d row) and bhat per chunk
-      bad = !tc::mbar_wait(&ms.k_full, ph, kTries);
+      tc::mbar_arrive(&ms.w_ready[wb]);
+    }
+    if (failed && stid == 0) atomicOr(&ms.err, 1u);
+  } else {
+    // ---------------- epilogue (warps 6-9): thread = output dim d ----------------
+    const int q4 = warp & 3;                        // TMEM lane quadrant
+    const int r = q4 * 32 + lane;                   // d row
+    const uint32_t t_lane = uint32_t(q4 * 32) << 16;
+    const int etid = tid - 192;                     // 0..127
+    const float* qg = refq + int64_t(g) * bR * bD;
+    float qd[bR];                                   // q_r[d] for this thread's d row
+#pragma unroll
+    for (int pl = 0; pl < bR; ++pl) qd[pl] = qg[pl * bD + r];
+    bool failed = false;
+    for (int64_t li = 0; li < my_tiles; ++li) {
+      const int64_t t = blockIdx.x + li * gridDim.x;
+      const int64_t chunk0 = c_begin + t * cpt;
+      const int wb = int(li & 1), kb = int(li % kbufs);
+      bool bad = !tc::mbar_wait(&ms.w_ready[wb], uint32_t((li >> 1) & 1), kTries);   // F of the tile
+      bad |= !tc::mbar_wait(&ms.k_full[kb], uint32_t((li / kbufs) & 1), kTries);
       tc::fence_after_sync();
-      tc::named_sync(1, 128);                      // ms.F visible
+      const uint32_t dk = tbase + t_lane + khat_col(li);
       for (int c = 0; c < cpt; ++c) {
-        float kh[bR], kl[bR];
-        tc::tmem_ld16(tbase + t_lane + bTmemK + uint32_t(c) * 32, kh);
-        tc::tmem_ld16(tbase + t_lane + bTmemK + uint32_t(c) * 32 + 16, kl);
+        float kh[bR], kl[bR], tmp[bR];
+        tc::tmem_ld16(dk + uint32_t(c) * 32, kh);
+        tc::tmem_ld16(dk + uint32_t(c) * 32 + 16, kl);
         const int64_t node = chunk0 + c;
-        const bool live = node < c_end;
+        const bool live = !bad && node < c_end;
         float* rec = store + G.off[1] + (int64_t(g) * G.cap[1] + node) * G.node_floats;
 #pragma unroll
         for (int i = 0; i < bR; ++i) {
@@ -281,25 +355,30 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
           tmp[i] = kh[i] * qd[i];
         }
         const float dsum = tr16(tmp, false);
-        if (lane < bR) ms.red[q4][lane] = dsum;
-        tc::named_sync(1, 128);
-        if (stid < bR && live) {
-          const float dot = ms.red[0][stid] + ms.red[1][stid] + ms.red[2][stid] + ms.red[3][stid];
-          rec[bR * bD + stid] = ms.F[c][stid] - dot * G.scale;
+        if (lane < bR) ms.red_e[wb][c][q4][lane] = dsum;
+      }
+      if (tc::named_sync_or(2, 128, bad)) { failed = true; break; }
+      // bhat_r = F - q_r . khat_r / sqrt(d) for every (chunk, plane) of the tile
+      for (int v = etid; v < cpt * bR; v += 128) {
+        const int c = v / bR, i = v % bR;
+        const int64_t node = chunk0 + c;
+        if (node < c_end) {
+          const float dot = ms.red_e[wb][c][0][i] + ms.red_e[wb][c][1][i] + ms.red_e[wb][c][2][i] +
+                            ms.red_e[wb][c][3][i];
+          store[G.off[1] + (int64_t(g) * G.cap[1] + node) * G.node_floats + bR * bD + i] =
+              ms.F[wb][c][i] - dot * G.scale;
         }
-        tc::named_sync(1, 128);
       }
       tc::fence_before_sync();
-      tc::mbar_arrive(&ms.k_free);
-      if (tc::named_sync_or(1, 128, bad)) failed = true;   // same decision in every thread
+      tc::mbar_arrive(&ms.k_free[kb]);
     }
-    if (failed && stid == 0) atomicOr(&ms.err, 1u);
+    if (failed && etid == 0) atomicOr(&ms.err, 1u);
   }
   tc::fence_before_sync();
   __syncthreads();
   if (warp == 1) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(tbase, bTmemCols);
+    tc::tmem_dealloc(tbase, tmem_cols);
   }
   if (tid == 0 && ms.err != 0u && status != nullptr) atomicOr(status, ZHA_DEV_TIMEOUT);
 }
@@ -310,7 +389,8 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
 cudaError_t launch_build_level1_tc(const Geom& G, const void* K, int64_t ld, int64_t c_begin,
                                    int64_t c_end, const float* refq, float* store, int32_t* status,
                                    cudaStream_t s) {
-  if (!(G.kv_bf16 && G.d == bD && G.nref == bR && G.chunk == 64 && G.rope_pairs == 0))
+  const bool chunk_ok = G.chunk == 16 || G.chunk == 32 || G.chunk == 64 || G.chunk == 128;
+  if (!(G.kv_bf16 && G.d == bD && G.nref == bR && chunk_ok && G.rope_pairs == 0))
     return cudaErrorNotSupported;
   if (c_end <= c_begin) return cudaSuccess;
   const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
@@ -331,7 +411,9 @@ cudaError_t launch_build_level1_tc(const Geom& G, const void* K, int64_t ld, int
   if ((e = device_sm_count(&sms)) != cudaSuccess) return e;
   const int cpt = bTok / G.chunk;
   const int64_t tiles = (c_end - c_begin + cpt - 1) / cpt;
-  int64_t per_head = (2 * int64_t(sms) + G.hkv - 1) / G.hkv;
+  // two CTAs per SM when both fit in tensor memory, else one
+  const int per_sm = build_tmem_cols(G.chunk) <= 256u ? 2 : 1;
+  int64_t per_head = (per_sm * int64_t(sms) + G.hkv - 1) / G.hkv;
   if (per_head > tiles) per_head = tiles;
   TraceScope ts("build_l1_tc_kernel", 1, s);
   build_l1_tc_kernel<<<dim3(unsigned(per_head), unsigned(G.hkv)), bThreads, smem, s>>>(

@@ -329,7 +329,7 @@ __device__ __forceinline__ void forward_tree_status(const SelectArgs& a) {
 }
 
 constexpr int kFastMax = 16384;
-constexpr int kFastSmallN = kSelectThreads;
+constexpr int kFastSmallN = kSelectThreads / 4;       // window size of the exact count
 constexpr int kHistBins = (kSelectThreads / 32) * 256;   // generic path: per-warp 256-bin histograms
 constexpr int kCutBins = 2048;                           // splitter histogram of the shared-memory path
 constexpr int kBitsSmem = 4096;                          // kept-bitmap words held in shared memory
@@ -548,15 +548,24 @@ __device__ void select_level(const Geom& G, const SelectArgs& a, const SelectSme
         }
         __syncthreads();
         const int nwin = int(s_w[32]);
-        if (tid < nwin) {
-          const int i = win[tid];
+        // Four threads per window member (lanes 4m .. 4m + 3 of one warp), each
+        // over every fourth other member, their partial masses summed by shuffles.
+        const int mi = tid >> 2, part = tid & 3;
+        unsigned long long cb = 0ull;
+        int i = 0;
+        if (mi < nwin) {
+          i = win[mi];
           const uint32_t ki = s_key[i];
-          unsigned long long cb = before;
-          for (int j = 0; j < nwin; ++j) {
+          for (int j = part; j < nwin; j += 4) {
             const int ij = win[j];
             const uint32_t kj = s_key[ij];
             if (kj < ki || (kj == ki && ij < i)) cb += s_m[ij];
           }
+        }
+        cb += __shfl_xor_sync(0xffffffffu, cb, 1);
+        cb += __shfl_xor_sync(0xffffffffu, cb, 2);
+        if (mi < nwin && part == 0) {
+          cb += before;
           if (cb < p31) atomicOr(&flag[i >> 5], 1u << (i & 31));
         }
         __syncthreads();

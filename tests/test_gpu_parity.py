@@ -463,6 +463,44 @@ def test_append_bf16_d128_c64_r16_matches_the_oracle(zha, parity_log):
     parity_log("append_bf16_c64", rep)
 
 
+@pytest.mark.parametrize("C,levels,c0", [(16, 3, 261), (32, 2, 101), (128, 2, 131)])
+def test_tensor_core_build_other_chunk_sizes(zha, parity_log, C, levels, c0):
+    """The tensor-core level-1 build at C = 16 (a chunk is half a warp's rows),
+    32 (one warp) and 128 (a whole tile), bf16 keys, head_dim 128, R = 16: a
+    prefill to an odd chunk count, then 13 chunks in one call from that odd
+    chunk (c_begin > 0, a tile partly past the new prefix). Every node of every
+    level against the oracle (norm-wise relative 1e-4), then routing and
+    attention at the final length. The kernel must have run."""
+    spec = W.scaled("1m", n_kv_heads=2, n_q_heads=16, n_tokens=C * (c0 + 14), stream_tokens=0, chunk=C,
+                    levels=levels, batch=2, n_needles=2)
+    inp = W.generate(spec)
+    dev = to_device(inp)
+    K, V, refq, Q = dev
+    tree = zha.Tree(config_for(spec), refq)
+    zha.trace_enable(64, "build_l1_tc")
+    try:
+        tree.build(K, C * c0 + 3)
+        tree.append_chunk(K, C * (c0 + 13) + 7)    # 13 chunks from chunk c0 (odd)
+        torch.cuda.synchronize()
+        launched = len(zha.trace_records())
+    finally:
+        zha.trace_enable(0)
+    assert launched == 2
+    n_final = C * (c0 + 13) + 7
+    assert tree.built_tokens == C * (c0 + 13)
+    for g in range(spec.n_kv_heads):
+        otree = O.build_tree(cache_f64(inp, g, n_final), inp.ref_q[g], C, levels, n_final)
+        for lvl in range(1, levels + 1):
+            n_l = otree.n_nodes(lvl)
+            assert n_l > 0
+            kh, bh = tree.level(lvl)
+            ek, eb = summary_errors(kh[g, :n_l].cpu().numpy().astype(np.float64),
+                                    bh[g, :n_l].cpu().numpy().astype(np.float64), *otree.nodes[lvl])
+            assert ek <= SUMMARY_RTOL and eb <= SUMMARY_RTOL, (g, lvl, ek, eb)
+    rep = check_case(zha, inp, n_final, tree=tree, dev=dev)
+    parity_log(f"build_tc_c{C}", rep)
+
+
 def test_build_status_is_clean_and_reaches_the_route(zha):
     """The tree's device status word (build time-outs) starts at zero after a
     build and a route over it reports no bit."""
