@@ -322,6 +322,23 @@ struct SpanWalk {
 // and 64-column half, issued by one thread); needs C % 8 == 0 so that every box
 // starts on a 1024-byte swizzle atom. Otherwise two warps stage rows with
 // cp.async (zero-filling rows without a token).
+// 2^x by the hardware approximation (a few ulp; results below 2^-126 are 0).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Two fp32 values -> their bf16x2 rounding and the bf16x2 rounding of the
+// remainders (x0 in the low halves).
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+  const float2 f = __bfloat1622float2(h);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - f.x, x1 - f.y);
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
 template <bool kTma>
 __global__ void __launch_bounds__(kThreads, 1)
 attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -657,6 +674,9 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 #pragma unroll
     for (int i = 0; i < kHalfQ; ++i) lrow[i] = 0.f;
     int gp = 0;                                    // group parity: ms.mrun[gp] is live
+    float mr[kHalfQ];                              // this warpgroup's running maxima (= ms.mrun[gp])
+#pragma unroll
+    for (int i = 0; i < kHalfQ; ++i) mr[i] = -INFINITY;
 
     // Q of group vq -> two bf16 terms, K-major 128-byte-swizzled rows: row q the
     // high term of head q, row 32 + q its low term (both warpgroups share it).
@@ -705,6 +725,7 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       return ok;
     };
     uint32_t allq = 0u;
+    const uint32_t jr = ms.rowj[r];                // this row's (chunk entry, row in chunk)
     if (t0 < t1) write_q(u0 / n_blocks);
     int64_t li = 0;
     for (int64_t t = t0; t < t1; ++t, ++li) {
@@ -733,7 +754,6 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       }
       uint32_t rmask = 0u;
       {
-        const uint32_t jr = ms.rowj[r];
         if (jr != 0xffffu) {
           const int j = int(jr >> 8), rr = int(jr & 255u);
           const int32_t tok0 = ms.tok0[st][j];
@@ -753,12 +773,11 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         }
         rmask >>= q0;
       }
-      const float* mrun = ms.mrun[gp] + q0;
       bool fire = false;
 #pragma unroll
       for (int i = 0; i < kHalfQ; ++i) {
         s[i] = ((rmask >> i) & 1u) ? s[i] * scale2 : -INFINITY;
-        fire |= s[i] > mrun[i] + kRescaleSlack;
+        fire |= s[i] > mr[i] + kRescaleSlack;
       }
       const uint32_t word = (__any_sync(0xffffffffu, fire) ? 1u : 0u) |
                             (__any_sync(0xffffffffu, bad) ? 2u : 0u);
@@ -788,7 +807,10 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         tc::named_sync(bar_id, 128);
         const float* scl = ms.scl + q0;
 #pragma unroll
-        for (int i = 0; i < kHalfQ; ++i) lrow[i] *= scl[i];
+        for (int i = 0; i < kHalfQ; ++i) {
+          lrow[i] *= scl[i];
+          mr[i] = ms.mrun[gp][q0 + i];
+        }
         if (!start) {                    // O holds earlier tiles of this group
           pending_bad |= !wait_pv(li - 1);
           tc::fence_after_sync();
@@ -805,22 +827,26 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       // p = 2^(s - m), stored MN-major over the stage's consumed K rows: row =
       // token, 64 bf16 (the high terms of the 32 heads, then the low terms),
       // 128-byte swizzled; this warpgroup writes its 16 heads of each half.
+      // The exponent is at most kRescaleSlack; ex2.approx (flushing results
+      // below 2^-126 to zero) is accurate to a few ulp there. Pairs of heads
+      // are rounded to bf16x2 in one conversion.
       uint8_t* sP = smem + st * kStageBytes;
 #pragma unroll
       for (int c = 0; c < kHalfQ / 8; ++c) {
-        __align__(16) __nv_bfloat16 hi[8], lo[8];
+        uint32_t hi[4], lo[4];
 #pragma unroll
-        for (int jq = 0; jq < 8; ++jq) {
-          const int i = 8 * c + jq;
-          const float p = mrun[i] == -INFINITY ? 0.f : exp2f(s[i] - mrun[i]);
-          lrow[i] += p;
-          hi[jq] = __float2bfloat16_rn(p);
-          lo[jq] = __float2bfloat16_rn(p - __bfloat162float(hi[jq]));
+        for (int jp = 0; jp < 4; ++jp) {
+          const int i = 8 * c + 2 * jp;
+          const float p0 = mr[i] == -INFINITY ? 0.f : fast_exp2(s[i] - mr[i]);
+          const float p1 = mr[i + 1] == -INFINITY ? 0.f : fast_exp2(s[i + 1] - mr[i + 1]);
+          lrow[i] += p0;
+          lrow[i + 1] += p1;
+          split_bf16x2(p0, p1, hi[jp], lo[jp]);
         }
         *reinterpret_cast<uint4*>(sP + tc::sw128_offset(r, q0 + 8 * c, kTok)) =
-            *reinterpret_cast<const uint4*>(hi);
+            make_uint4(hi[0], hi[1], hi[2], hi[3]);
         *reinterpret_cast<uint4*>(sP + tc::sw128_offset(r, kQ + q0 + 8 * c, kTok)) =
-            *reinterpret_cast<const uint4*>(lo);
+            make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
       // PV of the previous tile must be complete before p_full of this one
       // (it usually is by now); a time-out is reported at the next barrier.
@@ -862,7 +888,10 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
               make_float4(mq * 0.6931471805599453f, L, 0.f, 0.f);
         }
 #pragma unroll
-        for (int i = 0; i < kHalfQ; ++i) lrow[i] = 0.f;
+        for (int i = 0; i < kHalfQ; ++i) {
+          lrow[i] = 0.f;
+          mr[i] = -INFINITY;             // the next group's maxima (set above)
+        }
         gp ^= 1;
       }
     }
