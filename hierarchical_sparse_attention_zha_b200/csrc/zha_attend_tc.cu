@@ -305,16 +305,24 @@ struct SpanWalk {
   const int32_t* toff;       // tile offsets of the units (shared memory)
   int n_blocks;
   int u;                     // current unit
+  int g = -1;                // its group, and the group's first and end tile
+  int32_t g_lo = 0, g_hi = 0;
   // Advance to the unit holding tile t (t is non-decreasing between calls).
   __device__ __forceinline__ void seek(int64_t t) {
     while (t >= toff[u + 1]) ++u;
+    const int gu = u / n_blocks;
+    if (gu != g) {
+      g = gu;
+      g_lo = toff[gu * n_blocks];
+      g_hi = toff[(gu + 1) * n_blocks];
+    }
   }
-  __device__ __forceinline__ int group() const { return u / n_blocks; }
+  __device__ __forceinline__ int group() const { return g; }
   __device__ __forceinline__ bool group_start(int64_t t, int64_t t0) const {
-    return t == t0 || t == toff[(u / n_blocks) * n_blocks];
+    return t == t0 || t == g_lo;
   }
   __device__ __forceinline__ bool group_end(int64_t t, int64_t t1) const {
-    return t + 1 == t1 || t + 1 == toff[(u / n_blocks + 1) * n_blocks];
+    return t + 1 == t1 || t + 1 == g_hi;
   }
 };
 
@@ -712,10 +720,16 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     };
 
     SpanWalk wk{s_toff, n_blocks, u0};
-    int od = 0;                    // PV completions (o_done phases) consumed
+    int64_t od = 0;                // PV completions of o_done known to this thread
     bool failed = false, pending_bad = false;
-    // Wait for the PV of tile k. Called only before this thread arrives on
-    // p_full of tile k + 1, so at most one completion is ahead of `od`.
+    // Wait for the PV of tile k (k = li - 1 before this thread's P of tile li
+    // is signalled, or k = li after it at a group's last tile, once PV of
+    // li - 1 is known complete). Once s_full of tile li is observed, the PVs of
+    // tiles < li - 1 are complete: S of tile li was issued after them, and its
+    // commit tracks every earlier MMA. So before P of tile li, o_done has
+    // completed li - 1 or li times; after it, with PV of li - 1 waited for, li
+    // or li + 1 times (PV of li + 1 needs this thread's next P). Each phase
+    // waited for (in order, from od) is therefore unambiguous.
     auto wait_pv = [&](int64_t k) -> bool {
       bool ok = true;
       while (od <= k) {
@@ -728,7 +742,13 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     const uint32_t jr = ms.rowj[r];                // this row's (chunk entry, row in chunk)
     if (t0 < t1) write_q(u0 / n_blocks);
     int64_t li = 0;
+    int st = 0;                                    // li % kStages
+    uint32_t st_ph = 0u;                           // (li / kStages) & 1
     for (int64_t t = t0; t < t1; ++t, ++li) {
+      if (li > 0 && ++st == kStages) {
+        st = 0;
+        st_ph ^= 1u;
+      }
       wk.seek(t);
       const int v = wk.group();
       const bool start = wk.group_start(t, t0);
@@ -737,11 +757,11 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         const int nq = group_width(G, batch, q_blocks, v);
         allq = nq == 32 ? 0xffffffffu : ((1u << nq) - 1u);
       }
-      const int st = int(li % kStages);
-      bool bad = !tc::mbar_wait(&ms.full[st], uint32_t((li / kStages) & 1), kWaitTries);
+      bool bad = !tc::mbar_wait(&ms.full[st], st_ph, kWaitTries);
       bad |= !tc::mbar_wait(&ms.s_full[li & 1], uint32_t((li >> 1) & 1), kWaitTries);
       bad |= pending_bad;
       pending_bad = false;
+      if (od < li - 1) od = li - 1;                // PVs before tile li - 1 are complete
       tc::fence_after_sync();
       float s[kHalfQ];
       {
@@ -848,9 +868,9 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         *reinterpret_cast<uint4*>(sP + tc::sw128_offset(r, kQ + q0 + 8 * c, kTok)) =
             make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
-      // PV of the previous tile must be complete before p_full of this one
-      // (it usually is by now); a time-out is reported at the next barrier.
-      if (li > 0) pending_bad |= !wait_pv(li - 1);
+      // At a group's last tile PV of the previous tile completes first, so that
+      // the wait for this tile's PV below starts from a known phase.
+      if (end && li > 0) pending_bad |= !wait_pv(li - 1);
       tc::fence_async_smem();
       tc::fence_before_sync();
       tc::mbar_arrive(&ms.p_full[li & 1]);

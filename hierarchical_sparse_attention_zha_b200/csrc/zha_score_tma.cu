@@ -19,21 +19,27 @@
 //                           at a time: box = 32 columns x 16 planes x 8 nodes,
 //                           128-byte swizzled, rows (node, plane) = MMA rows.
 //   converters (warps 4-11) thread = (row, 32-column box): each fp32 value ->
-//                           three truncated bf16 terms (x = t0 + t1 + t2 exactly),
-//                           stored from registers straight into tensor memory (three
-//                           half-buffers), where
-//                           the MMA reads its A operand (shared memory only carries
-//                           the raw tiles and Q)
+//                           two fp16 terms, t0 = x rounded to fp16 and t1 = the
+//                           remainder rounded to fp16 (x = t0 + t1 to about 2^-24
+//                           |x|), stored from registers straight into tensor memory,
+//                           where the MMA reads its A operand (shared memory only
+//                           carries the raw tiles and Q, split the same way)
 //   MMA issuer (warp 1)     S^T[(node, plane)][head] over the half's 4 K-steps:
-//                           A_t0 . [q0 | q1 | q2]^T (N = 96), A_t1 . [q0 | q1]^T
-//                           (N = 64), A_t2 . q0^T (N = 32) into one of two TMEM
-//                           buffers -- the six products with term indices summing
-//                           to <= 2, the dropped ones are below fp32 rounding
-//   epilogue (warps 12-15)  thread = (node, plane) row: sum of the three column
+//                           A_t0 . [q0 | q1]^T (N = 64) and A_t1 . q0^T (N = 32)
+//                           into one of two TMEM buffers -- the three products
+//                           above 2^-24 of the result; A and B are both fp16
+//   epilogue (warps 12-15)  thread = (node, plane) row: sum of the two column
 //                           groups, x 1/sqrt(d) + bhat, maximum over the node's 16
-//                           planes, scores of the candidate (node, head) pairs
+//                           planes, scores of the candidate (node, head) pairs.
+//                           An element beyond the fp16 range (|x| >= 65520) makes
+//                           its products non-finite; a row that shows one is
+//                           recomputed in fp32 from the node record and Q
+// The fp16 terms keep the products exact to fp32 rounding for every element of
+// magnitude up to 65504; smaller than 2^-14 they lose relative, not absolute,
+// precision (an absolute error below 2^-25 per element).
 // Every wait is bounded; a time-out sets ZHA_DEV_TIMEOUT and the roles stop.
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
 #include "zha_host.cuh"
@@ -51,13 +57,15 @@ constexpr int kD = 128;
 constexpr int kRawSlots = 5;              // raw fp32 half-tiles in flight
 constexpr int kRawBytes = 32768;          // [2 boxes][128 rows][128 B]
 constexpr int kOffRaw = 0;
-constexpr int kOffQ = kRawSlots * kRawBytes;          // 2 halves x [96 rows][128 B]
-constexpr int kOffMisc = kOffQ + 2 * 12288;
+constexpr int kQHalf = 2 * kQn * 128;                 // [64 rows = term x 32 heads][128 B]
+constexpr int kOffQ = kRawSlots * kRawBytes;          // 2 halves x kQHalf
+constexpr int kOffMisc = kOffQ + 2 * kQHalf;
 constexpr int kThreads = 512;             // warps: 0 producer, 1 MMA, 2-3 idle, 4-11 convert, 12-15 epilogue
 constexpr int kConv = 256;                // converter threads (warps 4-11)
 constexpr int kEpiWarp0 = 12;
-constexpr uint32_t kTmemCols = 512;       // D buffers (96 columns) at 0 and 128; A half-buffers
-constexpr uint32_t kTmemA = 224;          // (3 terms x 32 columns) at 224, 320 and 416
+constexpr uint32_t kTmemCols = 512;       // D buffers (64 columns) at 0 and 64; A half-buffers
+constexpr uint32_t kTmemA = 128;          // (2 terms x 32 columns) at 128, 192 and 256
+constexpr uint32_t kDCols = 64, kACols = 64;
 constexpr int kABufs = 3;
 
 struct Meta {                             // one half-tile, producer -> converters
@@ -95,32 +103,24 @@ __device__ __forceinline__ int group_width(const Geom& G, int batch, int q_block
   return min(kQn, batch * G.group - (v % q_blocks) * kQn);
 }
 
-// Two fp32 values -> three packed bf16x2 terms with x = t0 + t1 + t2 exactly
-// (x0 in the low half of each term, x1 in the high half). Each term is the
-// upper 16 bits of the remaining residual (a truncated bf16): t0 keeps the sign,
-// exponent and first 7 mantissa bits of x, the residual x - t0 is exact in fp32
-// with at most 16 significant bits, its upper half t1 leaves an exact residual
-// of at most 8 significant bits, which a bf16 holds, so t2 is exact. Byte
-// permutes, masks and subtractions only: no conversion instructions.
-__device__ __forceinline__ void split3_x2(float x0, float x1, uint32_t& t0, uint32_t& t1, uint32_t& t2) {
-  const uint32_t u0 = __float_as_uint(x0), u1 = __float_as_uint(x1);
-  t0 = __byte_perm(u0, u1, 0x7632);
-  const float r0 = x0 - __uint_as_float(u0 & 0xffff0000u);
-  const float r1 = x1 - __uint_as_float(u1 & 0xffff0000u);
-  const uint32_t v0 = __float_as_uint(r0), v1 = __float_as_uint(r1);
-  t1 = __byte_perm(v0, v1, 0x7632);
-  const float q0 = r0 - __uint_as_float(v0 & 0xffff0000u);
-  const float q1 = r1 - __uint_as_float(v1 & 0xffff0000u);
-  t2 = __byte_perm(__float_as_uint(q0), __float_as_uint(q1), 0x7632);
+// Two fp32 values -> two packed fp16x2 terms, x = t0 + t1 + e (x0 in the low
+// halves): t0 rounds x to fp16 (11 significant bits), the remainder x - t0 is
+// exact in fp32 and t1 rounds it to fp16, so |e| <= 2^-24 |x| while x and the
+// remainder are normal fp16 numbers.
+__device__ __forceinline__ void split2_x2(float x0, float x1, uint32_t& t0, uint32_t& t1) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const float2 f = __half22float2(h);
+  const __half2 l = __floats2half2_rn(x0 - f.x, x1 - f.y);
+  t0 = *reinterpret_cast<const uint32_t*>(&h);
+  t1 = *reinterpret_cast<const uint32_t*>(&l);
 }
 
-// Eight fp32 values -> three bf16x8 terms.
-__device__ __forceinline__ void split3_x8(const float4& a, const float4& b, uint4& t0, uint4& t1,
-                                          uint4& t2) {
-  split3_x2(a.x, a.y, t0.x, t1.x, t2.x);
-  split3_x2(a.z, a.w, t0.y, t1.y, t2.y);
-  split3_x2(b.x, b.y, t0.z, t1.z, t2.z);
-  split3_x2(b.z, b.w, t0.w, t1.w, t2.w);
+// Eight fp32 values -> two fp16x8 terms.
+__device__ __forceinline__ void split2_x8(const float4& a, const float4& b, uint4& t0, uint4& t1) {
+  split2_x2(a.x, a.y, t0.x, t1.x);
+  split2_x2(a.z, a.w, t0.y, t1.y);
+  split2_x2(b.x, b.y, t0.z, t1.z);
+  split2_x2(b.z, b.w, t0.w, t1.w);
 }
 
 }  // namespace
@@ -154,7 +154,7 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&ms.d_full[b], 1);
       tc::mbar_init(&ms.d_free[b], 128);
-      tc::mbar_init(&emeta_full[b], 1);
+      tc::mbar_init(&emeta_full[b], kNodes * kR);
     }
     tc::mbar_init(&ms.q_ready, kConv);
     tc::mbar_init(&ms.drain, 1);
@@ -270,9 +270,8 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      constexpr uint32_t idesc96 = tc::idesc_bf16(128, 96, 0, 0);
-      constexpr uint32_t idesc64 = tc::idesc_bf16(128, 64, 0, 0);
-      constexpr uint32_t idesc32 = tc::idesc_bf16(128, 32, 0, 0);
+      constexpr uint32_t idesc64 = tc::idesc_f16(128, 64, 0, 0);
+      constexpr uint32_t idesc32 = tc::idesc_f16(128, 32, 0, 0);
       int64_t k = 0, tile_i = 0;
       int seg = 0;
       bool failed = false;
@@ -297,15 +296,14 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
           ++seg;
         }
         tc::fence_after_sync();
-        const uint32_t d = tbase + uint32_t(tile_i & 1) * 128;
-        const uint32_t tA = tbase + kTmemA + uint32_t(ab) * 96;      // term t at + 32 t
-        const uint32_t sQ = tc::smem_u32(smem + kOffQ) + uint32_t(cm.half) * 12288;
+        const uint32_t d = tbase + uint32_t(tile_i & 1) * kDCols;
+        const uint32_t tA = tbase + kTmemA + uint32_t(ab) * kACols;   // term t at + 32 t
+        const uint32_t sQ = tc::smem_u32(smem + kOffQ) + uint32_t(cm.half) * kQHalf;
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {           // K-step = 16 bf16 = 8 TMEM columns
-          const uint64_t b = tc::desc_sw128(sQ + ks * 32, 16, 1024);
-          tc::mma_bf16_ta(d, tA + ks * 8, b, idesc96, (cm.half == 0 && ks == 0) ? 0u : 1u);
-          tc::mma_bf16_ta(d, tA + 32 + ks * 8, b, idesc64, 1u);
-          tc::mma_bf16_ta(d, tA + 64 + ks * 8, b, idesc32, 1u);
+        for (int ks = 0; ks < 4; ++ks) {           // K-step = 16 fp16 = 8 TMEM columns
+          const uint64_t b = tc::desc_sw128(sQ + ks * 32, 16, 1024);   // rows: q0 heads, then q1
+          tc::mma_f16_ta(d, tA + ks * 8, b, idesc64, (cm.half == 0 && ks == 0) ? 0u : 1u);
+          tc::mma_f16_ta(d, tA + 32 + ks * 8, b, idesc32, 1u);
         }
         tc::mma_commit(&ms.a_free[ab]);
         if (cm.half == 1) {
@@ -332,7 +330,8 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
       const int64_t use = k / kRawSlots;
       const int ab = int(k % kABufs);
       bool bad = !tc::mbar_wait(&ms.raw_full[slot], uint32_t(use & 1), G.wait_polls);
-      if (tc::named_sync_or(1, kConv, bad)) { failed = true; break; }
+      // (after a failed wait mt is stale: it then only steers bounded waits
+      // before the converters agree to stop)
       const Meta mt = ms.meta[slot];
       const bool end = (mt.flags & 2) != 0;
       // A half-buffer ab was last read by the MMAs of half k - 2; the tile's
@@ -353,14 +352,14 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
           ms.cmeta[ab].half = 0;
           ms.cmeta[ab].flags = 2;
           ms.emeta[tile_i & 1].flags = 2;
-          tc::mbar_arrive(&emeta_full[tile_i & 1]);
         }
+        if (ctid < kNodes * kR) tc::mbar_arrive(&emeta_full[tile_i & 1]);
         tc::mbar_arrive(&ms.conv_done[ab]);
         break;
       }
       if (new_q) {
-        // Q of group mt.group -> three bf16 terms, rows term * 32 + q of a
-        // [2 halves][96 rows][128 B] K-major 128-byte-swizzled operand.
+        // Q of group mt.group -> two fp16 terms, rows term * 32 + q of a
+        // [2 halves][64 rows][128 B] K-major 128-byte-swizzled operand.
         const int v = mt.group;
         const int nq = group_width(G, batch, q_blocks, v);
         const int q = ctid >> 3, part = ctid & 7;
@@ -373,13 +372,13 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
             a = *reinterpret_cast<const float4*>(src);
             b = *reinterpret_cast<const float4*>(src + 4);
           }
-          uint4 t[3];
-          split3_x8(a, b, t[0], t[1], t[2]);
+          uint4 t[2];
+          split2_x8(a, b, t[0], t[1]);
           const int half = col >> 6, c16 = (col & 63) >> 3;
 #pragma unroll
-          for (int term = 0; term < 3; ++term) {
+          for (int term = 0; term < 2; ++term) {
             const int row = term * kQn + q;
-            const uint32_t off = uint32_t(half * 12288 + (row >> 3) * 1024 + (row & 7) * 128 +
+            const uint32_t off = uint32_t(half * kQHalf + (row >> 3) * 1024 + (row & 7) * 128 +
                                           ((c16 ^ (row & 7)) << 4));
             *reinterpret_cast<uint4*>(smem + kOffQ + off) = t[term];
           }
@@ -395,30 +394,30 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
 #pragma unroll
         for (int j = 0; j < kNodes; ++j) em.mask[j] = mt.mask[j];
       }
-      if (mt.half == 0) {
-        if (ctid < kNodes * kR) ms.emeta[tile_i & 1].bhat[ctid] = ms.bhat_raw[slot][ctid];
-        tc::named_sync(1, kConv);
-        if (ctid == 0) tc::mbar_arrive(&emeta_full[tile_i & 1]);
+      // The tile's metadata and bhat reach the epilogue through 128 arrivals
+      // (thread 0's after it wrote the fields above).
+      if (mt.half == 0 && ctid < kNodes * kR) {
+        ms.emeta[tile_i & 1].bhat[ctid] = ms.bhat_raw[slot][ctid];
+        tc::mbar_arrive(&emeta_full[tile_i & 1]);
       }
       // Raw half: [2 boxes of 32 columns][128 rows][128 B] fp32, 128-byte
-      // swizzled. Thread = (row cr, box cb): its 32 values -> three terms of 16
-      // packed bf16 pairs -> TMEM columns [term * 32 + cb * 16, + 16) of the A
+      // swizzled. Thread = (row cr, box cb): its 32 values -> two terms of 16
+      // packed fp16 pairs -> TMEM columns [term * 32 + cb * 16, + 16) of the A
       // half-buffer, lane cr.
       tc::fence_after_sync();                      // after a_free: the MMAs that read this A are done
       {
         const int sw = cr & 7;
         const uint8_t* rrow = smem + kOffRaw + slot * kRawBytes + cb * 16384 + (cr >> 3) * 1024 + sw * 128;
-        uint32_t t0[16], t1[16], t2[16];
+        uint32_t t0[16], t1[16];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const float4 x = *reinterpret_cast<const float4*>(rrow + ((c ^ sw) << 4));
-          split3_x2(x.x, x.y, t0[2 * c], t1[2 * c], t2[2 * c]);
-          split3_x2(x.z, x.w, t0[2 * c + 1], t1[2 * c + 1], t2[2 * c + 1]);
+          split2_x2(x.x, x.y, t0[2 * c], t1[2 * c]);
+          split2_x2(x.z, x.w, t0[2 * c + 1], t1[2 * c + 1]);
         }
-        const uint32_t tA = tbase + (uint32_t(cq * 32) << 16) + kTmemA + uint32_t(ab) * 96 + cb * 16;
+        const uint32_t tA = tbase + (uint32_t(cq * 32) << 16) + kTmemA + uint32_t(ab) * kACols + cb * 16;
         tc::tmem_st16u(tA, t0);
         tc::tmem_st16u(tA + 32, t1);
-        tc::tmem_st16u(tA + 64, t2);
         tc::tmem_wait_st();
       }
       if (ctid == 0) {
@@ -451,18 +450,38 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
       const float bhat_r = ms.emeta[b].bhat[r];
       if (em_flags & 2) break;
       float v[kQn];
-      tc::tmem_ld32(tbase + t_lane + uint32_t(b) * 128, v);
+      tc::tmem_ld32(tbase + t_lane + uint32_t(b) * kDCols, v);
 #pragma unroll
-      for (int g4 = 0; g4 < 4; ++g4) {            // + column groups 32..63 and 64..95, 16 at a time
+      for (int g2 = 0; g2 < 2; ++g2) {            // + column group 32..63, 16 at a time
         float w[16];
-        tc::tmem_ld16(tbase + t_lane + uint32_t(b) * 128 + 32 + 16 * g4, w);
+        tc::tmem_ld16(tbase + t_lane + uint32_t(b) * kDCols + 32 + 16 * g2, w);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[16 * (g4 & 1) + i] += w[i];
+        for (int i = 0; i < 16; ++i) v[16 * g2 + i] += w[i];
       }
       tc::fence_before_sync();
       tc::mbar_arrive(&ms.d_free[b]);
       const int64_t node = int64_t(em_node0) + nj;
       const bool live = node < n_nodes;
+      // A non-finite product means an element beyond the fp16 range (or a
+      // non-finite input): this row's dot products are recomputed in fp32.
+      bool finite = true;
+#pragma unroll
+      for (int q = 0; q < kQn; ++q) finite &= isfinite(v[q]);
+      if (!finite && live) {
+        const int gq = em_group / q_blocks;
+        const float* krow = level_base + (int64_t(gq) * G.cap[level] + node) * G.node_floats + plane * kD;
+        const int nq = group_width(G, batch, q_blocks, em_group);
+#pragma unroll
+        for (int q = 0; q < kQn; ++q) {
+          float acc = 0.f;
+          if (q < nq) {
+            const float* qrow = Q + head_of(G, q_blocks, em_group, q) * kD;
+#pragma unroll 1
+            for (int dd = 0; dd < kD; ++dd) acc = fmaf(qrow[dd], krow[dd], acc);
+          }
+          v[q] = acc;
+        }
+      }
       const float bh_ = bhat_r;
 #pragma unroll
       for (int q = 0; q < kQn; ++q) v[q] = live ? v[q] * G.scale + bh_ : -INFINITY;

@@ -254,7 +254,8 @@ class Tree:
 
     def __del__(self):
         h = getattr(self, "handle", None)
-        if h is not None and h.value:
+        # (at interpreter exit the module's globals may already be gone)
+        if h is not None and h.value and lib is not None:
             lib.zha_tree_destroy(h)
             self.handle = None
 
