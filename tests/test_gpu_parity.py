@@ -501,6 +501,52 @@ def test_tensor_core_build_other_chunk_sizes(zha, parity_log, C, levels, c0):
     parity_log(f"build_tc_c{C}", rep)
 
 
+def test_scores_beyond_the_fp16_range_are_recomputed_in_fp32(zha, parity_log):
+    """Level scoring on the tensor cores splits each value into two fp16 terms;
+    an element of magnitude >= 65520 (fp16 overflow) makes a row's products
+    non-finite and the kernel recomputes that row in fp32. Plant such elements
+    in level-1 summaries and in one query, route, and compare every level's
+    kept set with the oracle's routing over the same summaries."""
+    spec = W.scaled("1m", n_kv_heads=1, n_q_heads=8, n_tokens=8192, stream_tokens=64, levels=2, batch=2,
+                    n_needles=0)
+    inp = W.generate(spec)
+    K, V, refq, Q = to_device(inp)
+    n_tokens = 8192 + 5
+    tree = zha.Tree(config_for(spec), refq)
+    tree.build(K, n_tokens)
+    kh, _ = tree.level(1)
+    kh[0, 3, 2, 5] = 7.0e4                 # one element of one plane
+    kh[0, 40, 0, 100] = -2.0e5
+    kh[0, 77, :, 17] = 9.0e4               # every plane of a node
+    Qm = Q.clone()
+    Qm[0, 1, 5] = 1.0e5                    # a query head with an element beyond the range
+    torch.cuda.synchronize()
+    q = Qm[0].contiguous()
+    B = q.shape[0]
+    max_sel = n_tokens // spec.chunk
+    bits = torch.zeros(zha.route_kept_words(tree.cfg, B, n_tokens) + 1, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ids, cnt = tree.route(q, n_tokens, spec.p, max_sel, kept_bits=bits, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    kept = kept_from_bits(bits.cpu().numpy().view(np.uint32), spec, B, n_tokens)
+    otree = O.OracleTree(chunk=spec.chunk, levels=spec.levels, n_tokens=n_tokens, qhat=inp.ref_q[0])
+    for lvl in range(1, spec.levels + 1):
+        k_l, b_l = tree.level(lvl)
+        n_l = otree.n_nodes(lvl)
+        otree.nodes[lvl] = (k_l[0, :n_l].cpu().numpy().astype(np.float64),
+                            b_l[0, :n_l].cpu().numpy().astype(np.float64))
+    qh = Qm[0].cpu().numpy().astype(np.float64)
+    report = RouteReport()
+    for b in range(B):
+        for h in range(spec.n_q_heads):
+            compare_route_head(qh[b, h], otree, spec.p, {lvl: kept[lvl][(b, h)] for lvl in kept}, report,
+                               (b, h))
+    assert not report.hard, report.hard[:10]
+    assert report.heads == B * spec.n_q_heads
+    parity_log("fp16_range_fallback", report)
+
+
 def test_build_status_is_clean_and_reaches_the_route(zha):
     """The tree's device status word (build time-outs) starts at zero after a
     build and a route over it reports no bit."""
