@@ -145,18 +145,18 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
     ms.err = 0u;
     for (int s = 0; s < kRawSlots; ++s) {
       tc::mbar_init(&ms.raw_full[s], 1);
-      tc::mbar_init(&ms.raw_empty[s], kConv);
+      tc::mbar_init(&ms.raw_empty[s], kConv / 32);      // one arrival per converter warp
     }
     for (int b = 0; b < kABufs; ++b) {
-      tc::mbar_init(&ms.conv_done[b], kConv);
+      tc::mbar_init(&ms.conv_done[b], kConv / 32);
       tc::mbar_init(&ms.a_free[b], 1);
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&ms.d_full[b], 1);
       tc::mbar_init(&ms.d_free[b], 128);
-      tc::mbar_init(&emeta_full[b], kNodes * kR);
+      tc::mbar_init(&emeta_full[b], kNodes * kR / 32);  // the warps copying bhat
     }
-    tc::mbar_init(&ms.q_ready, kConv);
+    tc::mbar_init(&ms.q_ready, kConv / 32);
     tc::mbar_init(&ms.drain, 1);
   }
   pdl_trigger();
@@ -346,15 +346,19 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
       const bool new_q = !end && mt.half == 0 && (mt.flags & 1);
       if (new_q && k >= 1)
         bad |= !tc::mbar_wait(&ms.a_free[(k - 1) % kABufs], uint32_t(((k - 1) / kABufs) & 1), G.wait_polls);
-      if (tc::named_sync_or(1, kConv, bad)) { failed = true; break; }
+      // A warp stops as a whole; the other roles' bounded waits then run out.
+      if (__any_sync(0xffffffffu, bad)) { failed = true; break; }
       if (end) {
         if (ctid == 0) {
           ms.cmeta[ab].half = 0;
           ms.cmeta[ab].flags = 2;
           ms.emeta[tile_i & 1].flags = 2;
         }
-        if (ctid < kNodes * kR) tc::mbar_arrive(&emeta_full[tile_i & 1]);
-        tc::mbar_arrive(&ms.conv_done[ab]);
+        __syncwarp();
+        if (lane == 0) {
+          if (ctid < kNodes * kR) tc::mbar_arrive(&emeta_full[tile_i & 1]);
+          tc::mbar_arrive(&ms.conv_done[ab]);
+        }
         break;
       }
       if (new_q) {
@@ -384,7 +388,8 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
           }
         }
         tc::fence_async_smem();
-        tc::mbar_arrive(&ms.q_ready);
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&ms.q_ready);
       }
       if (mt.half == 0 && ctid == 0) {
         EMeta& em = ms.emeta[tile_i & 1];
@@ -394,11 +399,12 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
 #pragma unroll
         for (int j = 0; j < kNodes; ++j) em.mask[j] = mt.mask[j];
       }
-      // The tile's metadata and bhat reach the epilogue through 128 arrivals
-      // (thread 0's after it wrote the fields above).
+      // The tile's metadata and bhat reach the epilogue through one arrival per
+      // copying warp (warp 4's after thread 0 wrote the fields above).
       if (mt.half == 0 && ctid < kNodes * kR) {
         ms.emeta[tile_i & 1].bhat[ctid] = ms.bhat_raw[slot][ctid];
-        tc::mbar_arrive(&emeta_full[tile_i & 1]);
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&emeta_full[tile_i & 1]);
       }
       // Raw half: [2 boxes of 32 columns][128 rows][128 B] fp32, 128-byte
       // swizzled. Thread = (row cr, box cb): its 32 values -> two terms of 16
@@ -425,12 +431,15 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
         ms.cmeta[ab].flags = mt.flags & 1;
       }
       tc::fence_before_sync();
-      tc::mbar_arrive(&ms.raw_empty[slot]);
-      tc::mbar_arrive(&ms.conv_done[ab]);
+      __syncwarp();
+      if (lane == 0) {                             // for the warp's 32 threads
+        tc::mbar_arrive(&ms.raw_empty[slot]);
+        tc::mbar_arrive(&ms.conv_done[ab]);
+      }
       if (mt.half == 1) ++tile_i;
       ++k;
     }
-    if (failed && ctid == 0) atomicOr(&ms.err, 1u);
+    if (failed && lane == 0) atomicOr(&ms.err, 1u);
   } else if (warp >= kEpiWarp0) {
     // ---------------- epilogue: thread = TMEM lane = (node, plane) row ----------------
     const int eq = warp & 3;
@@ -438,6 +447,8 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
     const uint32_t t_lane = uint32_t(eq * 32) << 16;
     int64_t tile_i = 0;
     bool failed = false;
+    int row_group = -1;                            // group of the cached score rows
+    int64_t srow[2] = {0, 0};                      // sigma rows of heads 2 plane, 2 plane + 1
     while (true) {
       const int b = int(tile_i & 1);
       const uint32_t ph = uint32_t((tile_i >> 1) & 1);
@@ -464,10 +475,12 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
       const bool live = node < n_nodes;
       // A non-finite product means an element beyond the fp16 range (or a
       // non-finite input): this row's dot products are recomputed in fp32.
-      bool finite = true;
+      // (Finite products stay far below the fp32 range, so the sum of the
+      // row's values is finite exactly when every value is.)
+      float vsum = 0.f;
 #pragma unroll
-      for (int q = 0; q < kQn; ++q) finite &= isfinite(v[q]);
-      if (!finite && live) {
+      for (int q = 0; q < kQn; ++q) vsum += v[q];
+      if (!isfinite(vsum) && live) {
         const int gq = em_group / q_blocks;
         const float* krow = level_base + (int64_t(gq) * G.cap[level] + node) * G.node_floats + plane * kD;
         const int nq = group_width(G, batch, q_blocks, em_group);
@@ -497,12 +510,15 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
         }
       }
       if (live) {
+        if (em_group != row_group) {
+          row_group = em_group;
+#pragma unroll
+          for (int kk = 0; kk < 2; ++kk) srow[kk] = head_of(G, q_blocks, em_group, 2 * plane + kk) * n_nodes;
+        }
         const uint32_t m = node_mask;
 #pragma unroll
-        for (int kk = 0; kk < 2; ++kk) {
-          const int q = 2 * plane + kk;
-          if ((m >> q) & 1u) sigma[head_of(G, q_blocks, em_group, q) * n_nodes + node] = v[kk];
-        }
+        for (int kk = 0; kk < 2; ++kk)
+          if ((m >> (2 * plane + kk)) & 1u) sigma[srow[kk] + node] = v[kk];
       }
       ++tile_i;
     }
