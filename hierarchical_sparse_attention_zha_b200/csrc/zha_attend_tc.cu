@@ -72,7 +72,6 @@ constexpr int kRowWords = kWinWords + 1;  // padded bitmap row (bank-conflict-fr
 struct Misc {
   uint64_t full[kStages], empty[kStages], s_full[2], p_full[2], o_done, q_ready, drain;
   uint32_t tmem_base, err;
-  uint32_t flags[2][2][4];
   float red[2][2][4][16];
   float mrun[2][kQ];                      // running maxima per head, by group parity
   float scl[kQ];                          // rescale factors of the current tile
@@ -408,10 +407,10 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     }
     for (int bb = 0; bb < 2; ++bb) {
       tc::mbar_init(&ms.s_full[bb], 1);
-      tc::mbar_init(&ms.p_full[bb], 256);
+      tc::mbar_init(&ms.p_full[bb], 8);           // one arrival per softmax warp
     }
     tc::mbar_init(&ms.o_done, 1);
-    tc::mbar_init(&ms.q_ready, 256);
+    tc::mbar_init(&ms.q_ready, 8);
     tc::mbar_init(&ms.drain, 1);
   }
   if (kTma) {
@@ -716,7 +715,8 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
             *reinterpret_cast<const uint4*>(lo);
       }
       tc::fence_async_smem();
-      tc::mbar_arrive(&ms.q_ready);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&ms.q_ready);
     };
 
     SpanWalk wk{s_toff, n_blocks, u0};
@@ -799,16 +799,17 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
         s[i] = ((rmask >> i) & 1u) ? s[i] * scale2 : -INFINITY;
         fire |= s[i] > mr[i] + kRescaleSlack;
       }
-      const uint32_t word = (__any_sync(0xffffffffu, fire) ? 1u : 0u) |
-                            (__any_sync(0xffffffffu, bad) ? 2u : 0u);
-      if (lane == 0) ms.flags[li & 1][wg][sw] = word;
-      tc::named_sync(bar_id, 128);
-      const uint32_t all = ms.flags[li & 1][wg][0] | ms.flags[li & 1][wg][1] |
-                           ms.flags[li & 1][wg][2] | ms.flags[li & 1][wg][3];
-      if (all & 2u) { failed = true; break; }
+      // One barrier tells the warpgroup whether any thread saw a score past its
+      // running maximum plus the slack, or a failed wait; only then a second
+      // one tells the two apart.
+      bool rescale = false;
+      if (tc::named_sync_or(bar_id, 128, fire || bad)) {
+        if (tc::named_sync_or(bar_id, 128, bad)) { failed = true; break; }
+        rescale = true;
+      }
       // S of this tile is complete, so Q may be replaced for the next group now.
       if (end && t + 1 < t1) write_q(v + 1);
-      if (all & 1u) {
+      if (rescale) {
         // Raise this warpgroup's running maxima to the tile's, rescale l and O.
         float tmp[kHalfQ];
 #pragma unroll
@@ -873,7 +874,8 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
       if (end && li > 0) pending_bad |= !wait_pv(li - 1);
       tc::fence_async_smem();
       tc::fence_before_sync();
-      tc::mbar_arrive(&ms.p_full[li & 1]);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&ms.p_full[li & 1]);   // for the warp's 32 rows
       if (end) {
         // The group's piece of this span is done: write one state per head.
         const bool bad2 = !wait_pv(li) || pending_bad;

@@ -118,13 +118,13 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
       tc::mbar_init(&ms.empty[s], 1);
     }
     tc::mbar_init(&ms.s_full, 1);
-    tc::mbar_init(&ms.s_free, 128);
+    tc::mbar_init(&ms.s_free, 4);                   // one arrival per warp of a warpgroup
     for (int b = 0; b < 2; ++b) {
-      tc::mbar_init(&ms.w_ready[b], 128);
+      tc::mbar_init(&ms.w_ready[b], 4);
       tc::mbar_init(&ms.k_full[b], 1);
-      tc::mbar_init(&ms.k_free[b], 128);
+      tc::mbar_init(&ms.k_free[b], 4);
     }
-    tc::mbar_init(&ms.q_ready, 128);
+    tc::mbar_init(&ms.q_ready, 4);
     tc::mbar_init(&ms.drain, 1);
   }
   if (warp == 1) tc::tmem_alloc(&ms.tmem_base, tmem_cols);
@@ -244,7 +244,8 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
       }
     }
     tc::fence_async_smem();
-    tc::mbar_arrive(&ms.q_ready);
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(&ms.q_ready);
     // Reduction units: a chunk of C >= 32 rows spans C / 32 warps (unit = warp),
     // a chunk of 16 rows is half a warp (unit = half-warp).
     const bool half_units = C < 32;
@@ -265,7 +266,8 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
         for (int i = 0; i < bR; ++i) s[i] = (s[i] + w1[i] + w2[i]) * G.scale;
       }
       tc::fence_before_sync();
-      tc::mbar_arrive(&ms.s_free);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&ms.s_free);
       // W[wb] and F[wb] are free once the epilogue of tile li - kbufs is done
       // (it waited for the khat MMA that read W[wb]).
       if (li >= kbufs) {
@@ -319,7 +321,8 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
       }
       tc::fence_async_smem();
       tc::fence_before_sync();
-      tc::mbar_arrive(&ms.w_ready[wb]);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&ms.w_ready[wb]);
     }
     if (failed && stid == 0) atomicOr(&ms.err, 1u);
   } else {
@@ -370,7 +373,8 @@ build_l1_tc_kernel(const __grid_constant__ CUtensorMap tmK, Geom G, int64_t c_be
         }
       }
       tc::fence_before_sync();
-      tc::mbar_arrive(&ms.k_free[kb]);
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&ms.k_free[kb]);
     }
     if (failed && etid == 0) atomicOr(&ms.err, 1u);
   }
