@@ -268,10 +268,16 @@ union_prep_kernel(Geom G, int32_t batch, int32_t q_blocks, int32_t n_blocks, int
     }
     if (lane == 0) s_scan[q] = warp_cnt;
     __syncthreads();
-    if (tid == 0) {
-      uint32_t run = 0;
-      for (int w = 0; w < 32; ++w) { const uint32_t t = s_scan[w]; s_scan[w] = run; run += t; }
-      s_scan[32] = run;
+    if (q == 0) {                                  // exclusive scan of the 32 warp counts
+      const uint32_t c = s_scan[lane];
+      uint32_t incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+      }
+      s_scan[lane] = incl - c;
+      if (lane == 31) s_scan[32] = incl;
     }
     __syncthreads();
     int64_t pos = total + s_scan[q];

@@ -324,28 +324,25 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
     const int cr = cq * 32 + lane;                  // MMA row = (node, plane)
     const int cb = (warp - 4) >> 2;                 // 32-column box of the half
     int64_t k = 0, tile_i = 0;
+    int slot = 0, ab = 0, prev_ab = kABufs - 1;    // k % kRawSlots, k % kABufs, (k - 1) % kABufs
+    uint32_t slot_par = 0u, ab_par = 0u, prev_par = 1u;   // the matching (k / n) & 1
     bool failed = false;
     while (true) {
-      const int slot = int(k % kRawSlots);
-      const int64_t use = k / kRawSlots;
-      const int ab = int(k % kABufs);
-      bool bad = !tc::mbar_wait(&ms.raw_full[slot], uint32_t(use & 1), G.wait_polls);
-      // (after a failed wait mt is stale: it then only steers bounded waits
-      // before the converters agree to stop)
-      const Meta mt = ms.meta[slot];
-      const bool end = (mt.flags & 2) != 0;
-      // A half-buffer ab was last read by the MMAs of half k - 2; the tile's
-      // metadata slot by the epilogue of tile_i - 2.
-      // (also before the end marker: the MMA issuer reads cmeta[ab] of half k - 3 first)
-      if (k >= kABufs)
-        bad |= !tc::mbar_wait(&ms.a_free[ab], uint32_t(((k / kABufs) - 1) & 1), G.wait_polls);
-      if ((end || mt.half == 0) && tile_i >= 2)
+      bool bad = !tc::mbar_wait(&ms.raw_full[slot], slot_par, G.wait_polls);
+      // (after a failed wait these fields are stale: they then only steer
+      // bounded waits before the warp stops)
+      const int32_t m_flags = ms.meta[slot].flags, m_half = ms.meta[slot].half;
+      const bool end = (m_flags & 2) != 0;
+      // A half-buffer ab was last read by the MMAs of half k - kABufs; the
+      // tile's metadata slot by the epilogue of tile_i - 2.
+      // (also before the end marker: the MMA issuer reads cmeta[ab] first)
+      if (k >= kABufs) bad |= !tc::mbar_wait(&ms.a_free[ab], ab_par ^ 1u, G.wait_polls);
+      if ((end || m_half == 0) && tile_i >= 2)
         bad |= !tc::mbar_wait(&ms.d_free[tile_i & 1], uint32_t(((tile_i >> 1) - 1) & 1), G.wait_polls);
       // A new group's Q replaces the old one once every MMA that reads it (the
       // previous half's) is complete.
-      const bool new_q = !end && mt.half == 0 && (mt.flags & 1);
-      if (new_q && k >= 1)
-        bad |= !tc::mbar_wait(&ms.a_free[(k - 1) % kABufs], uint32_t(((k - 1) / kABufs) & 1), G.wait_polls);
+      const bool new_q = !end && m_half == 0 && (m_flags & 1);
+      if (new_q && k >= 1) bad |= !tc::mbar_wait(&ms.a_free[prev_ab], prev_par, G.wait_polls);
       // A warp stops as a whole; the other roles' bounded waits then run out.
       if (__any_sync(0xffffffffu, bad)) { failed = true; break; }
       if (end) {
@@ -362,9 +359,9 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
         break;
       }
       if (new_q) {
-        // Q of group mt.group -> two fp16 terms, rows term * 32 + q of a
+        // Q of the slot's group -> two fp16 terms, rows term * 32 + q of a
         // [2 halves][64 rows][128 B] K-major 128-byte-swizzled operand.
-        const int v = mt.group;
+        const int v = ms.meta[slot].group;
         const int nq = group_width(G, batch, q_blocks, v);
         const int q = ctid >> 3, part = ctid & 7;
 #pragma unroll
@@ -391,18 +388,15 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&ms.q_ready);
       }
-      if (mt.half == 0 && ctid == 0) {
+      // The tile's metadata (lanes of warp 4, one field each) and bhat (warps
+      // 4-7) reach the epilogue through one arrival per copying warp.
+      if (m_half == 0 && ctid < kNodes * kR) {
         EMeta& em = ms.emeta[tile_i & 1];
-        em.node0 = mt.node0;
-        em.group = mt.group;
-        em.flags = mt.flags;
-#pragma unroll
-        for (int j = 0; j < kNodes; ++j) em.mask[j] = mt.mask[j];
-      }
-      // The tile's metadata and bhat reach the epilogue through one arrival per
-      // copying warp (warp 4's after thread 0 wrote the fields above).
-      if (mt.half == 0 && ctid < kNodes * kR) {
-        ms.emeta[tile_i & 1].bhat[ctid] = ms.bhat_raw[slot][ctid];
+        if (ctid < kNodes) em.mask[ctid] = ms.meta[slot].mask[ctid];
+        else if (ctid == kNodes) em.node0 = ms.meta[slot].node0;
+        else if (ctid == kNodes + 1) em.group = ms.meta[slot].group;
+        else if (ctid == kNodes + 2) em.flags = m_flags;
+        em.bhat[ctid] = ms.bhat_raw[slot][ctid];
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&emeta_full[tile_i & 1]);
       }
@@ -427,8 +421,8 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
         tc::tmem_wait_st();
       }
       if (ctid == 0) {
-        ms.cmeta[ab].half = mt.half;
-        ms.cmeta[ab].flags = mt.flags & 1;
+        ms.cmeta[ab].half = m_half;
+        ms.cmeta[ab].flags = m_flags & 1;
       }
       tc::fence_before_sync();
       __syncwarp();
@@ -436,8 +430,12 @@ score_tma_kernel(const __grid_constant__ CUtensorMap tmS, const __grid_constant_
         tc::mbar_arrive(&ms.raw_empty[slot]);
         tc::mbar_arrive(&ms.conv_done[ab]);
       }
-      if (mt.half == 1) ++tile_i;
+      if (m_half == 1) ++tile_i;
       ++k;
+      prev_ab = ab;
+      prev_par = ab_par;
+      if (++slot == kRawSlots) { slot = 0; slot_par ^= 1u; }
+      if (++ab == kABufs) { ab = 0; ab_par ^= 1u; }
     }
     if (failed && lane == 0) atomicOr(&ms.err, 1u);
   } else if (warp >= kEpiWarp0) {
