@@ -461,11 +461,16 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     int32_t pf_tok0[2] = {-1, -1}, pf_nv[2] = {0, 0}, pf_pg[2] = {0, 0};
     uint32_t pf_m[2] = {0u, 0u};
     bool bad_page = false;
+    int e_unit = -1, e_count = 0;                  // the unit whose entry count is held
     auto prefetch = [&](int64_t t) {
       wk.seek(t);
       const int uu = wk.u, v = uu / n_blocks, blk = uu % n_blocks;
       const int gkv = v / q_blocks;
-      const int E = counts[uu];
+      if (uu != e_unit) {                          // a load only when the unit changes
+        e_unit = uu;
+        e_count = counts[uu];
+      }
+      const int E = e_count;
       const bool tail_here = has_tail && blk == n_blocks - 1;
       const int nq = group_width(G, batch, q_blocks, v);
       const uint32_t allq = nq == 32 ? 0xffffffffu : ((1u << nq) - 1u);
@@ -526,19 +531,24 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
           const uint32_t n_ok = __popc(__ballot_sync(0xffffffffu, pf_tok0[0] >= 0 && lane < cpt)) +
                                 __popc(__ballot_sync(0xffffffffu, pf_tok0[1] >= 0 && lane + 32 < cpt));
           __syncwarp();
-          if (lane == 0) {
+          // The stage's byte count first (after the entries above), then each
+          // lane issues the copies of its own entries.
+          if (lane == 0) tc::mbar_arrive_expect_tx(&ms.full[st], n_ok * 512u * uint32_t(C));
+          __syncwarp();
+          {
             const uint32_t sK = tc::smem_u32(smem + st * kStageBytes), sV = sK + 32768;
-            tc::mbar_arrive_expect_tx(&ms.full[st], n_ok * 512u * uint32_t(C));
-            for (int j = 0; j < cpt; ++j) {
-              const int32_t tok0 = ms.tok0[st][j];
-              if (tok0 < 0) continue;
-              const uint32_t roff = uint32_t(j * C * 128);
-              // contiguous: {d, tokens, KV head}; paged: {d, row in page, page}
-              const int32_t y = paged ? 0 : tok0, z = paged ? ms.page[st][j] : g;
-              tc::tma_load_3d(sK + roff, &tmK, 0, y, z, &ms.full[st]);
-              tc::tma_load_3d(sK + 16384 + roff, &tmK, 64, y, z, &ms.full[st]);
-              tc::tma_load_3d(sV + roff, &tmV, 0, y, z, &ms.full[st]);
-              tc::tma_load_3d(sV + 16384 + roff, &tmV, 64, y, z, &ms.full[st]);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int j = lane + 32 * h;
+              if (j < cpt && pf_tok0[h] >= 0) {
+                const uint32_t roff = uint32_t(j * C * 128);
+                // contiguous: {d, tokens, KV head}; paged: {d, row in page, page}
+                const int32_t y = paged ? 0 : pf_tok0[h], z = paged ? pf_pg[h] : g;
+                tc::tma_load_3d(sK + roff, &tmK, 0, y, z, &ms.full[st]);
+                tc::tma_load_3d(sK + 16384 + roff, &tmK, 64, y, z, &ms.full[st]);
+                tc::tma_load_3d(sV + roff, &tmV, 0, y, z, &ms.full[st]);
+                tc::tma_load_3d(sV + 16384 + roff, &tmV, 64, y, z, &ms.full[st]);
+              }
             }
           }
           __syncwarp();
