@@ -366,7 +366,6 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
   Misc& ms = *reinterpret_cast<Misc*>(smem + kOffMisc);
   int32_t* s_toff = reinterpret_cast<int32_t*>(smem + kOffMisc + sizeof(Misc));   // [units + 1]
   pdl_trigger();
-  pdl_wait();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int C = G.chunk;
   const int cpt = chunks_per_tile(C);
@@ -381,25 +380,8 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     return (e + cpt - 1) / cpt;
   };
 
-  // Tile offsets of the units: warp 0, a blocked scan.
-  if (warp == 0) {
-    const int per = (units + 31) / 32;
-    const int b0 = min(units, lane * per), b1 = min(units, b0 + per);
-    int sum = 0;
-    for (int uu = b0; uu < b1; ++uu) sum += unit_tiles(uu);
-    int incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    int run = incl - sum;
-    for (int uu = b0; uu < b1; ++uu) {
-      s_toff[uu] = run;
-      run += unit_tiles(uu);
-    }
-    if (lane == 31) s_toff[units] = incl;
-  }
+  // Setup that reads nothing the previous kernel writes runs before the
+  // dependency wait (programmatic dependent launch).
   if (tid < kTok) {
     const int j = C >= kTok ? 0 : tid / C, rr = C >= kTok ? tid : tid % C;
     ms.rowj[tid] = (j < cpt && rr < C) ? uint16_t((j << 8) | rr) : uint16_t(0xffff);
@@ -429,6 +411,26 @@ attend_split_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
     tc::fence_async_smem();
   }
   if (warp == 2) tc::tmem_alloc(&ms.tmem_base, kTmemCols);
+  pdl_wait();                                    // counts of the union prep from here on
+  // Tile offsets of the units: warp 0, a blocked scan.
+  if (warp == 0) {
+    const int per = (units + 31) / 32;
+    const int b0 = min(units, lane * per), b1 = min(units, b0 + per);
+    int sum = 0;
+    for (int uu = b0; uu < b1; ++uu) sum += unit_tiles(uu);
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - sum;
+    for (int uu = b0; uu < b1; ++uu) {
+      s_toff[uu] = run;
+      run += unit_tiles(uu);
+    }
+    if (lane == 31) s_toff[units] = incl;
+  }
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();

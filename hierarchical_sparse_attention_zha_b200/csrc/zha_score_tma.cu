@@ -20,22 +20,23 @@
 //                           128-byte swizzled, rows (node, plane) = MMA rows.
 //   converters (warps 4-11) thread = (row, 32-column box): each fp32 value ->
 //                           two fp16 terms, t0 = x rounded to fp16 and t1 = the
-//                           remainder rounded to fp16 (x = t0 + t1 to about 2^-24
-//                           |x|), stored from registers straight into tensor memory,
+//                           remainder rounded to fp16 (x = t0 + t1 to 2^-22 |x|,
+//                           rounded to nearest), stored from registers into tensor memory,
 //                           where the MMA reads its A operand (shared memory only
 //                           carries the raw tiles and Q, split the same way)
 //   MMA issuer (warp 1)     S^T[(node, plane)][head] over the half's 4 K-steps:
 //                           A_t0 . [q0 | q1]^T (N = 64) and A_t1 . q0^T (N = 32)
 //                           into one of two TMEM buffers -- the three products
-//                           above 2^-24 of the result; A and B are both fp16
+//                           above 2^-22 of the result; A and B are both fp16
 //   epilogue (warps 12-15)  thread = (node, plane) row: sum of the two column
 //                           groups, x 1/sqrt(d) + bhat, maximum over the node's 16
 //                           planes, scores of the candidate (node, head) pairs.
 //                           An element beyond the fp16 range (|x| >= 65520) makes
 //                           its products non-finite; a row that shows one is
 //                           recomputed in fp32 from the node record and Q
-// The fp16 terms keep the products exact to fp32 rounding for every element of
-// magnitude up to 65504; smaller than 2^-14 they lose relative, not absolute,
+// The fp16 terms keep each product to about 2^-21 relative (unbiased), the
+// order of the fp32 accumulation's own rounding, for every element of
+// magnitude up to 65504; below 2^-14 they lose relative, not absolute,
 // precision (an absolute error below 2^-25 per element).
 // Every wait is bounded; a time-out sets ZHA_DEV_TIMEOUT and the roles stop.
 #include <cuda.h>
@@ -105,7 +106,7 @@ __device__ __forceinline__ int group_width(const Geom& G, int batch, int q_block
 
 // Two fp32 values -> two packed fp16x2 terms, x = t0 + t1 + e (x0 in the low
 // halves): t0 rounds x to fp16 (11 significant bits), the remainder x - t0 is
-// exact in fp32 and t1 rounds it to fp16, so |e| <= 2^-24 |x| while x and the
+// exact in fp32 and t1 rounds it to fp16, so |e| <= 2^-22 |x| while x and the
 // remainder are normal fp16 numbers.
 __device__ __forceinline__ void split2_x2(float x0, float x1, uint32_t& t0, uint32_t& t1) {
   const __half2 h = __floats2half2_rn(x0, x1);
