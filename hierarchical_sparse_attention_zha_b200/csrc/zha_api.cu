@@ -92,8 +92,16 @@ static zha_status make_geom(const zha_config* c, zha::Geom* g, size_t* bytes) {
     off += int64_t(G.hkv) * G.cap[l] * G.node_floats;
   }
   G.status_off = zha::round_up(off, 64);           // 256-byte aligned, one 256-byte block
+  int64_t end = G.status_off * 4 + 256;            // bytes
+  for (int l = 0; l <= ZHA_MAX_LEVELS + 1; ++l) G.split_off[l] = 0;
+  if (zha::has_plane_terms(G)) {
+    for (int l = 1; l <= G.levels; ++l) {
+      G.split_off[l] = end;                        // multiples of 8 KiB after a 256-byte boundary
+      end += int64_t(G.hkv) * 2 * G.cap[l] * G.nref * G.d * 2;
+    }
+  }
   *g = G;
-  if (bytes) *bytes = size_t(G.status_off * 4 + 256);
+  if (bytes) *bytes = size_t(end);
   return ZHA_OK;
 }
 

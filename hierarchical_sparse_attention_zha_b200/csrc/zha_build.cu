@@ -14,6 +14,7 @@ namespace zha {
 cudaError_t launch_build_level1_tc(const Geom& G, const void* K, int64_t ld, int64_t c_begin,
                                    int64_t c_end, const float* refq, float* store, int32_t* status,
                                    cudaStream_t s);
+cudaError_t launch_plane_terms(const Geom& G, float* store, int64_t nb_old, int64_t nb_new, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
 // Level 1. One CTA summarises a tile of `nch` consecutive chunks (nch*C <= 128
@@ -377,20 +378,26 @@ static cudaError_t launch_append_t(const Geom& G, const KvView& kv, int64_t nb_o
 
 cudaError_t launch_build(const Geom& G, const KvView& kv, int64_t nb_old, int64_t nb_new,
                          const float* refq, float* store, cudaStream_t s) {
+  cudaError_t e;
   if (G.kv_bf16)
-    return G.d == 128 ? launch_build_t<__nv_bfloat16, 128>(G, kv, nb_old, nb_new, refq, store, s)
-                      : launch_build_t<__nv_bfloat16, 64>(G, kv, nb_old, nb_new, refq, store, s);
-  return G.d == 128 ? launch_build_t<float, 128>(G, kv, nb_old, nb_new, refq, store, s)
-                    : launch_build_t<float, 64>(G, kv, nb_old, nb_new, refq, store, s);
+    e = G.d == 128 ? launch_build_t<__nv_bfloat16, 128>(G, kv, nb_old, nb_new, refq, store, s)
+                   : launch_build_t<__nv_bfloat16, 64>(G, kv, nb_old, nb_new, refq, store, s);
+  else
+    e = G.d == 128 ? launch_build_t<float, 128>(G, kv, nb_old, nb_new, refq, store, s)
+                   : launch_build_t<float, 64>(G, kv, nb_old, nb_new, refq, store, s);
+  return e == cudaSuccess ? launch_plane_terms(G, store, nb_old, nb_new, s) : e;
 }
 
 cudaError_t launch_append(const Geom& G, const KvView& kv, int64_t nb_old, int64_t nb_new,
                           const float* refq, float* store, cudaStream_t s) {
+  cudaError_t e;
   if (G.kv_bf16)
-    return G.d == 128 ? launch_append_t<__nv_bfloat16, 128>(G, kv, nb_old, nb_new, refq, store, s)
-                      : launch_append_t<__nv_bfloat16, 64>(G, kv, nb_old, nb_new, refq, store, s);
-  return G.d == 128 ? launch_append_t<float, 128>(G, kv, nb_old, nb_new, refq, store, s)
-                    : launch_append_t<float, 64>(G, kv, nb_old, nb_new, refq, store, s);
+    e = G.d == 128 ? launch_append_t<__nv_bfloat16, 128>(G, kv, nb_old, nb_new, refq, store, s)
+                   : launch_append_t<__nv_bfloat16, 64>(G, kv, nb_old, nb_new, refq, store, s);
+  else
+    e = G.d == 128 ? launch_append_t<float, 128>(G, kv, nb_old, nb_new, refq, store, s)
+                   : launch_append_t<float, 64>(G, kv, nb_old, nb_new, refq, store, s);
+  return e == cudaSuccess ? launch_plane_terms(G, store, nb_old, nb_new, s) : e;
 }
 
 }  // namespace zha

@@ -29,7 +29,14 @@ struct Geom {
   int64_t cap[ZHA_MAX_LEVELS + 2];       // node capacity per KV head, index by level
   int64_t off[ZHA_MAX_LEVELS + 2];       // float offset of level l's [hkv][cap][node] block
   int64_t status_off;                    // float offset of the tree's device status word
+  // Byte offset of level l's planes as two fp16 terms, [hkv][2][cap][R][d]
+  // (t0 = x rounded to fp16, t1 = x - t0 rounded to fp16), for the tensor-core
+  // scoring of head_dim 128, R = 16; 0 when the store has no such copy.
+  int64_t split_off[ZHA_MAX_LEVELS + 2];
 };
+
+// Whether the store carries fp16 plane terms (the tensor-core scoring's operand).
+__host__ __device__ inline bool has_plane_terms(const Geom& g) { return g.d == 128 && g.nref == 16; }
 
 // The tree's device status word (ZHA_DEV_* bits of the build kernels), in the
 // 256-byte block that follows the summary levels in the store.

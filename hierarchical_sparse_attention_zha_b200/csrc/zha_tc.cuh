@@ -74,6 +74,13 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b
       : "r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
 }
 
+// kind::f16 with fp16 operands, both from shared memory (the instruction is the
+// one above; the instruction descriptor selects fp16).
+__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t accumulate) {
+  mma_bf16(d_tmem, a, b, idesc, accumulate);
+}
+
 // The same with A read from tensor memory: a_tmem = TMEM address of A's first
 // column (lane = row, two bf16 of consecutive K per 32-bit column).
 __device__ __forceinline__ void mma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
@@ -308,6 +315,18 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, int3
       " [%0], [%1, {%2, %3, %4}], [%5];"
       :
       : "r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Tiled 4-D tensor copy global -> shared (no multicast), bytes counted on `bar`.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, int32_t x, int32_t y,
+                                            int32_t z, int32_t w, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];"
+      :
+      : "r"(dst), "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(z), "r"(w),
+        "r"(smem_u32(bar))
       : "memory");
 }
 

@@ -113,7 +113,14 @@ uint64_t zha_launch_count(void);
  * n_ref*head_dim + round_up(n_ref, 4) [ZHA: 무엇과 다른가]; then, at the next
  * 256-byte boundary, one 256-byte block whose first int32 is the tree's
  * device status word (ZHA_DEV_TIMEOUT set by a build kernel whose bounded wait
- * ran out; zha_build clears it, zha_route passes it on to its d_status). */
+ * ran out; zha_build clears it, zha_route passes it on to its d_status).
+ * With head_dim 128 and n_ref 16, a second copy of the planes follows, the
+ * operand of the tensor-core scoring: for l = 1..L, fp16
+ * [n_kv_heads][2][floor(max_tokens / C^l)][n_ref][head_dim], term 0 = khat
+ * rounded to fp16 and term 1 = the remainder rounded to fp16. zha_build and
+ * zha_append_chunk write it together with the float32 planes; the routing
+ * scores from the terms, so a caller that writes planes into the store itself
+ * writes their terms as well. */
 size_t zha_tree_bytes(const zha_config* cfg);
 
 /* Create a host handle over a caller-owned store (>= zha_tree_bytes bytes,

@@ -68,8 +68,10 @@ def test_tree_bytes_matches_the_documented_layout(zha):
         node = R * d + (R + 3) // 4 * 4
         floats = sum(H * (T // C ** l) * node for l in range(1, L + 1))
         # the levels, then a 256-byte block (the tree's device status word) at
-        # the next 256-byte boundary
-        assert zha.tree_bytes(cfg) == (floats * 4 + 255) // 256 * 256 + 256
+        # the next 256-byte boundary, then (head_dim 128, R = 16) the planes
+        # again as two fp16 terms
+        terms = sum(H * 2 * (T // C ** l) * R * d * 2 for l in range(1, L + 1)) if (d, R) == (128, 16) else 0
+        assert zha.tree_bytes(cfg) == (floats * 4 + 255) // 256 * 256 + 256 + terms
 
 
 @pytest.mark.parametrize("field,value", [("head_dim", 96), ("chunk", 1), ("chunk", 129),

@@ -421,6 +421,40 @@ def test_levels_wider_than_16384_nodes(zha, parity_log, levels, p):
     parity_log(f"wide_L{levels}_p{p}", rep)
 
 
+def plane_terms(zha, tree):
+    """Views [H, 2, cap, R, d] fp16 of the store's second copy of each level's
+    planes (head_dim 128, R = 16; the operand of the tensor-core scoring),
+    laid out after the status block as the header documents."""
+    cfg = tree.cfg
+    H, R, d, C, L = cfg.n_kv_heads, cfg.n_ref, cfg.head_dim, cfg.chunk, cfg.levels
+    caps = [cfg.max_tokens // C ** lvl for lvl in range(1, L + 1)]
+    sizes = [H * 2 * cap * R * d * 2 for cap in caps]
+    off = zha.tree_bytes(cfg) - sum(sizes)
+    raw = tree.store.view(torch.uint8)
+    out = {}
+    for lvl, cap, size in zip(range(1, L + 1), caps, sizes):
+        out[lvl] = raw[off: off + size].view(torch.float16).view(H, 2, cap, R, d)
+        off += size
+    return out
+
+
+def split_terms(x):
+    """Term 0 = x rounded to fp16, term 1 = (x - term 0) rounded to fp16."""
+    t0 = x.half()
+    return t0, (x - t0.float()).half()
+
+
+def check_plane_terms(zha, tree, n_tokens):
+    """Both fp16 terms of every built node of every level, bit for bit."""
+    C = tree.cfg.chunk
+    nb = C * (n_tokens // C)
+    for lvl, terms in plane_terms(zha, tree).items():
+        n_l = nb // C ** lvl
+        t0, t1 = split_terms(tree.level(lvl)[0][:, :n_l])
+        assert torch.equal(terms[:, 0, :n_l].view(torch.int16), t0.view(torch.int16)), lvl
+        assert torch.equal(terms[:, 1, :n_l].view(torch.int16), t1.view(torch.int16)), lvl
+
+
 def test_append_bf16_d128_c64_r16_matches_the_oracle(zha, parity_log):
     """The incremental build of the 1M-context configuration (bf16 keys,
     head_dim 128, R = 16, C = 64): a tensor-core prefill to an odd chunk count,
@@ -459,6 +493,8 @@ def test_append_bf16_d128_c64_r16_matches_the_oracle(zha, parity_log):
                 ek, eb = summary_errors(kh[g, :n_l].cpu().numpy().astype(np.float64),
                                         bh[g, :n_l].cpu().numpy().astype(np.float64), *otree.nodes[lvl])
                 assert ek <= SUMMARY_RTOL and eb <= SUMMARY_RTOL, (g, lvl, ek, eb)
+    for t in (inc, fresh):
+        check_plane_terms(zha, t, n_final)
     rep = check_case(zha, inp, n_final, tree=inc, dev=dev)
     parity_log("append_bf16_c64", rep)
 
@@ -497,6 +533,7 @@ def test_tensor_core_build_other_chunk_sizes(zha, parity_log, C, levels, c0):
             ek, eb = summary_errors(kh[g, :n_l].cpu().numpy().astype(np.float64),
                                     bh[g, :n_l].cpu().numpy().astype(np.float64), *otree.nodes[lvl])
             assert ek <= SUMMARY_RTOL and eb <= SUMMARY_RTOL, (g, lvl, ek, eb)
+    check_plane_terms(zha, tree, n_final)
     rep = check_case(zha, inp, n_final, tree=tree, dev=dev)
     parity_log(f"build_tc_c{C}", rep)
 
@@ -518,6 +555,11 @@ def test_scores_beyond_the_fp16_range_are_recomputed_in_fp32(zha, parity_log):
     kh[0, 3, 2, 5] = 7.0e4                 # one element of one plane
     kh[0, 40, 0, 100] = -2.0e5
     kh[0, 77, :, 17] = 9.0e4               # every plane of a node
+    # (a caller that writes planes itself rewrites their fp16 terms too)
+    t0, t1 = split_terms(kh)
+    terms = plane_terms(zha, tree)[1]
+    terms[:, 0] = t0
+    terms[:, 1] = t1
     Qm = Q.clone()
     Qm[0, 1, 5] = 1.0e5                    # a query head with an element beyond the range
     torch.cuda.synchronize()
@@ -556,7 +598,11 @@ def test_build_status_is_clean_and_reaches_the_route(zha):
     res = run_pipeline(zha, inp, 4096 + 3)
     assert res["status"] == 0
     st = res["tree"].store.view(torch.int32)
-    off = (zha.tree_bytes(res["tree"].cfg) - 256) // 4
+    # the 256-byte block after the levels (the fp16 plane terms follow it)
+    cfg = res["tree"].cfg
+    terms = sum(cfg.n_kv_heads * 2 * (cfg.max_tokens // cfg.chunk ** lvl) * cfg.n_ref * cfg.head_dim * 2
+                for lvl in range(1, cfg.levels + 1)) if (cfg.head_dim, cfg.n_ref) == (128, 16) else 0
+    off = (zha.tree_bytes(cfg) - terms - 256) // 4
     assert int(st[off].item()) == 0
 
 
