@@ -45,7 +45,7 @@
 extern "C" {
 #endif
 
-#define ZHA_ABI_VERSION 2
+#define ZHA_ABI_VERSION 3
 
 typedef enum {
     ZHA_OK = 0,

@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(zha):
 
 
 def test_version_and_status_strings(zha):
-    assert zha.lib.zha_abi_version() == 2
+    assert zha.lib.zha_abi_version() == 3
     assert zha.status_str(0) == "ok"
     assert "state" in zha.status_str(zha.ZHA_ERR_STATE)
     assert zha.status_str(-99) == "unknown status"
