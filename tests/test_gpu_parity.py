@@ -793,6 +793,8 @@ def test_paged_cache_matches_the_oracle_and_the_contiguous_cache(zha, parity_log
     kv = zha.kv_cache(Kp, Vp, table)
     tree = zha.Tree(config_for(spec), refq)
     tree.build_kv(kv, n_tokens)
+    if (tree.cfg.head_dim, tree.cfg.n_ref) == (128, 16):
+        check_plane_terms(zha, tree, n_tokens)
     rep = check_case(zha, inp, n_tokens, tree=tree, dev=dev)
     parity_log(f"paged_{name}", rep)
     res = run_pipeline(zha, inp, n_tokens, tree=tree, dev=dev)
